@@ -1,0 +1,234 @@
+/*
+ * isd.h -- C ABI of libisd.so, one Introspective Strided Decoding (ISD) step
+ * on an NVIDIA B200 (sm_100a).
+ *
+ * The method comes from "Introspective Diffusion Language Models"
+ * (arXiv 2604.11035).  Its project summary (hada.io pages) describes one
+ * forward pass that verifies the previous stride and drafts the next one
+ * ("Introspective Strided Decoding (ISD)"), new tokens proposed from q at
+ * MASK positions and verified with p at clean positions, kept with
+ * probability min(1, p(x)/q(x)) ("Inference & ISD"), strict causal
+ * attention with a logit shift ("Méthodologie d'I-DLM"), and a paged KV
+ * cache read by a paged-only attention kernel ("Serving (SGLang)").
+ *
+ * One step is three calls, in this order, on one stream:
+ *   isd_attn_strided     strided-query causal GQA attention, paged KV
+ *   isd_accept_resample  vocab softmax stats, ratio test, resample / bonus /
+ *                        draft sampling
+ *   isd_kv_commit        commit of the accepted prefix, rollback of the rest
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every pointer is a DEVICE pointer into memory the caller owns and keeps
+ *   alive until the enqueued work has finished.  The library never
+ *   allocates, frees or synchronises; all work is enqueued on `stream`
+ *   (0 = the legacy default stream) of the current device.
+ * - Arrays are dense, row-major, in the layouts stated below, 16-byte
+ *   aligned.
+ * - Stride rows: sequence b holds K = 2N query rows at absolute positions
+ *   L_b .. L_b + K - 1 (L_b = seq_len[b], its committed length).  Rows
+ *   0 .. n_b - 1 hold the pending tokens (row 0 the stride's exact token,
+ *   rows 1.. drafts under verification); rows n_b .. K - 1 are MASK rows.
+ *   Row r's logits score position L_b + r + 1 (logit shift).
+ * - Paged KV: page_size = 16 token slots; cache layout
+ *   [num_pages][Hkv][16][d]; logical page i of sequence b is physical page
+ *   page_table[b * page_table_stride + i].
+ * - Return value: ISD_OK when the work was enqueued.  Invalid arguments are
+ *   rejected on the host before anything is launched (ISD_ERR_INVALID_ARG,
+ *   ISD_ERR_UNSUPPORTED, ISD_ERR_WORKSPACE).  A failed launch returns
+ *   ISD_ERR_CUDA.  Conditions only the device can see (pool exhausted,
+ *   page-table row full, malformed state, page id out of range) are written
+ *   as an ISD_ERR_* code to the caller's `status` word, and the affected
+ *   work is skipped; no kernel traps and no kernel waits on another.
+ * - The calls are asynchronous and capture into CUDA graphs: they read no
+ *   device memory on the host and launch a fixed set of kernels.
+ */
+#ifndef ISD_H_
+#define ISD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ISD_ABI_VERSION 1
+#define ISD_PAGE_SIZE 16
+
+/* Return / status codes. */
+enum {
+  ISD_OK = 0,
+  ISD_ERR_INVALID_ARG = 1,     /* null pointer, bad size, aliasing       */
+  ISD_ERR_UNSUPPORTED = 2,     /* valid but outside the built kernels    */
+  ISD_ERR_CUDA = 3,            /* a CUDA runtime call or launch failed   */
+  ISD_ERR_WORKSPACE = 4,       /* workspace missing or too small         */
+  /* written by the device into *status */
+  ISD_ERR_POOL_EXHAUSTED = 16, /* commit needs more pages than are free  */
+  ISD_ERR_PAGE_TABLE_FULL = 17,/* a sequence outgrew its page-table row  */
+  ISD_ERR_BAD_STATE = 18,      /* n_pending, token or q row out of range */
+  ISD_ERR_BAD_PAGE = 19        /* page id outside [0, num_pages)         */
+};
+
+/* Element types. */
+enum { ISD_BF16 = 0, ISD_F32 = 1 };
+
+/* Uniform streams of the sampler (Philox counter word 3). */
+enum { ISD_STREAM_ACCEPT = 0, ISD_STREAM_RESAMPLE = 1, ISD_STREAM_DRAFT = 2 };
+
+/* ------------------------------------------------------------------------
+ * isd_attn_strided -- strided-query causal GQA attention over a paged KV
+ * cache (the "paged-only attention kernel" of the pages' serving stack).
+ *
+ * For sequence b, KV head h, stride row r and group member j (query head
+ * hq = h * g + j, g = Hq / Hkv):
+ *   keys   = cached positions [0, L_b) of head h, then k_new[b, 0..r, h]
+ *   O[b, r, hq] = sum_t softmax(softmax_scale * q[b, r, hq] . key_t) value_t
+ *   lse[b, r, hq] = log(sum_t exp(softmax_scale * q . key_t))   (natural)
+ * Strict causal: row r never sees stride rows > r; no window, no bias; Q/K
+ * arrive post-rotary.  Every row, including MASK and spare rows, is computed.
+ *
+ * Layouts: q, out [B][K][Hq][d]; k_new, v_new [B][K][Hkv][d];
+ * k_cache, v_cache [num_pages][Hkv][16][d]; page_table int32
+ * [B][page_table_stride]; seq_len int32 [B]; lse f32 [B][K][Hq] or NULL.
+ * dtype ISD_BF16 (tensor-core path; d = 128 or 64, K * g a multiple of 16
+ * and at most 128) or ISD_F32 (exact-fp32 SIMT path; d a multiple of 32,
+ * at most 128).  `out` may not alias any input.
+ * Workspace: isd_attn_workspace_bytes(args) bytes (split-KV partials);
+ * its contents need no initialisation.  `status` (optional) receives
+ * ISD_ERR_BAD_PAGE / ISD_ERR_PAGE_TABLE_FULL for malformed page tables;
+ * pages out of range read as zeros.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int32_t B, Hq, Hkv, d, K;
+  int32_t num_pages, page_table_stride;
+  int32_t dtype;
+  float softmax_scale;
+  int32_t num_ctas;            /* 0: one CTA per SM                       */
+  const void* q;
+  const void* k_new;
+  const void* v_new;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* page_table;
+  const int32_t* seq_len;
+  void* out;
+  float* lse;                  /* optional                                */
+  int32_t* status;             /* optional                                */
+  void* workspace;
+  size_t workspace_bytes;
+} isd_attn_args;
+
+size_t isd_attn_workspace_bytes(const isd_attn_args* a);
+int isd_attn_strided(const isd_attn_args* a, void* stream);
+
+/* ------------------------------------------------------------------------
+ * isd_accept_resample -- vocab softmax of p and q, the min(1, p/q) ratio
+ * test, and the residual / bonus / draft draws.
+ *
+ * Per sequence b with n = n_pending_in[b] (1 or N), L = seq_len[b]:
+ *  1. Row statistics m = max_v l_v, s = sum_v exp(l_v - m) (fp32) of
+ *     logits_cur rows 0 .. n + N - 2 (p rows 0..n-1, draft rows n..n+N-2).
+ *  2. Drafts i = 1 .. n-1 in order: p_i(x) from row i-1 of logits_cur,
+ *     q_i(x) from row q_row_in[b][i] of logits_prev with the stored
+ *     (m, s) = q_stats_in[b][i]; u_i = U(seed, b, step, L + i, ACCEPT);
+ *     accept iff u_i < p_i(x)/q_i(x).  a_b = drafts accepted before the
+ *     first rejection; n_commit[b] = 1 + a_b; commit_tokens[b][0..a_b] =
+ *     pending_in[b][0..a_b] (the rest -1).
+ *  3. Rejected at draft a+1: the exact token at L + a + 1 is drawn from
+ *     normalise(max(0, p - q)) (p from row a, q of draft a+1; p if that
+ *     mass is zero), stream RESAMPLE; next n = 1.
+ *     All accepted: the exact token at L + n is drawn from p of row n-1
+ *     (stream RESAMPLE), and drafts j = 1..N-1 at L + n + j from q of row
+ *     n + j - 1 (stream DRAFT), whose (m, s) go to q_stats_out[b][j] and
+ *     row index to q_row_out[b][j]; next n = N.
+ *  A draw with uniform u from masses w returns the smallest index v whose
+ *  running sum (ascending vocabulary order) exceeds u * sum(w).
+ *  U(seed, b, step, pos, stream) = (x0 >> 8) * 2^-24 with x0 the first word
+ *  of Philox4x32-10(key = (seed lo, seed hi), counter = (b, step, pos,
+ *  stream)) (Salmon et al., SC'11).
+ *
+ * Layouts: logits_cur, logits_prev [B][K][V] (dtype); pending_*, q_row_*
+ * int32 [B][N]; n_pending_* int32 [B]; q_stats_* f32 [B][N][2] (entry 0
+ * unused); n_commit int32 [B]; commit_tokens int32 [B][N]; row_stats f32
+ * [B][K][2] or NULL (m, s of the rows used, others untouched); ratio f32
+ * [B][N] or NULL (p/q of each verified draft, others untouched).
+ * The *_out state arrays must not alias the *_in ones.  A sequence whose
+ * state is malformed gets ISD_ERR_BAD_STATE in *status (if given),
+ * n_commit 0 and its state copied through unchanged.
+ * Workspace: isd_accept_workspace_bytes(args) bytes; no initialisation.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int32_t B, N, K, V;
+  int32_t dtype;
+  uint32_t step;
+  uint64_t seed;
+  const void* logits_cur;
+  const void* logits_prev;
+  const int32_t* seq_len;
+  const int32_t* pending_in;
+  const int32_t* n_pending_in;
+  const int32_t* q_row_in;
+  const float* q_stats_in;
+  int32_t* pending_out;
+  int32_t* n_pending_out;
+  int32_t* q_row_out;
+  float* q_stats_out;
+  int32_t* n_commit;
+  int32_t* commit_tokens;
+  float* row_stats;            /* optional                                */
+  float* ratio;                /* optional                                */
+  int32_t* status;             /* optional                                */
+  void* workspace;
+  size_t workspace_bytes;
+} isd_accept_args;
+
+size_t isd_accept_workspace_bytes(const isd_accept_args* a);
+int isd_accept_resample(const isd_accept_args* a, void* stream);
+
+/* ------------------------------------------------------------------------
+ * isd_kv_commit -- copy the staged K/V of rows 0 .. n_commit[b]-1 to cache
+ * positions L_b .. L_b + n_commit[b] - 1 and grow seq_len[b] by n_commit[b].
+ * Rows >= n_commit[b] (rejected drafts, MASK rows) are never written: that
+ * is the rollback.  When a committed position enters a new page, pages are
+ * popped from the free stack (entries [0, *free_top) are free, the top is
+ * free_stack[*free_top - 1]), sequence 0 first, and recorded in the page
+ * table; no page is freed.  All-or-nothing: if the pool or a page-table row
+ * is too small, *status gets the code and nothing changes.
+ *
+ * Layouts: k_new, v_new [B][K][Hkv][d]; k_cache, v_cache
+ * [num_pages][Hkv][16][d]; page_table int32 [B][page_table_stride];
+ * seq_len, n_commit int32 [B] (0 <= n_commit <= K); free_stack int32
+ * [num_pages]; free_top int32 [1]; status int32 [1] (required; set to
+ * ISD_OK on success).  Workspace: isd_commit_workspace_bytes(args) bytes.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int32_t B, K, Hkv, d;
+  int32_t num_pages, page_table_stride;
+  int32_t dtype;
+  const void* k_new;
+  const void* v_new;
+  void* k_cache;
+  void* v_cache;
+  int32_t* page_table;
+  int32_t* seq_len;
+  const int32_t* n_commit;
+  const int32_t* free_stack;
+  int32_t* free_top;
+  int32_t* status;
+  void* workspace;
+  size_t workspace_bytes;
+} isd_commit_args;
+
+size_t isd_commit_workspace_bytes(const isd_commit_args* a);
+int isd_kv_commit(const isd_commit_args* a, void* stream);
+
+/* Utilities. */
+int isd_abi_version(void);
+const char* isd_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ISD_H_ */

@@ -1,0 +1,711 @@
+// isd_attn_strided kernels: strided-query causal GQA attention over a paged
+// KV cache.
+//
+// Method: "Introspective Diffusion Language Models", project summary
+// (hada.io): strict causal attention with a logit shift ("Méthodologie"),
+// a paged KV cache and a paged-only attention kernel ("Serving (SGLang)"),
+// one forward pass carrying the verify rows and the MASK rows of a stride
+// ("Introspective Strided Decoding").  Row r of sequence b (position
+// L_b + r) attends to cached positions [0, L_b) and stride rows 0..r.
+//
+// bf16 path (tensor cores).  Work is a flat list of "units": for every
+// (sequence b, KV head h), one unit per cached page plus one tail unit for
+// the stride's own rows.  Each persistent CTA takes an equal contiguous
+// range of that list (no per-sequence imbalance, whatever the lengths).
+// Inside a CTA one producer warp walks the range and issues TMA loads of
+// each unit's K and V tiles (16 tokens x d, 128-byte swizzle) into a ring
+// of mbarrier-guarded stages; four consumer warps compute S = Q K^T and
+// O += P V with mma.sync m16n8k16 (bf16 in, fp32 accumulate) and an online
+// softmax in base 2.  All K*g query rows of a KV head share every K/V tile,
+// which is read from HBM exactly once.  Consumer warps split the rows into
+// groups of 16*MW and, when rows are few, split the units of a segment
+// round-robin and merge through shared memory at the segment's end.  A
+// (b, h) whose units straddle CTAs leaves fp32 partials (unnormalised O,
+// running max, running sum) that a combine kernel merges in CTA order.
+//
+// fp32 path (SIMT, exact fp32 arithmetic): one warp per query row.
+#include "common.cuh"
+
+namespace isd {
+
+constexpr int kCWarps = 4;                      // consumer warps
+constexpr int kAttnThreads = (kCWarps + 1) * 32;
+constexpr int kStages = 12;
+constexpr uint64_t kWaitCycles = 4000000000ull; // ~2 s at boost clock
+
+struct AttnDev {
+  int B, Hq, Hkv, K, g, M, P, stride, RG, KS;
+  float scale_log2;
+  const __nv_bfloat16* q;
+  __nv_bfloat16* out;
+  float* lse;
+  const int32_t* page_table;
+  const int32_t* seq_len;
+  int32_t* status;
+  float* part;        // [G][2][M][D + 2]
+  int32_t* ws_int;    // [B + 1] unit prefix, then G
+};
+
+// Bounded mbarrier wait (clock deadline); false on timeout.
+ISD_DEV bool wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if ((uint64_t)(clock64() - t0) > kWaitCycles) return false;
+  return true;
+}
+
+ISD_DEV int pages_of(const AttnDev& p, int b, bool* bad) {
+  int L = p.seq_len[b];
+  if (L < 0) { *bad = true; L = 0; }
+  int n = (L + kPage - 1) / kPage;
+  if (n > p.stride) { *bad = true; n = p.stride; }
+  return n;
+}
+
+// Position of unit u: sequence b (prefix[b] <= u < prefix[b+1]).
+ISD_DEV int find_seq(const int* prefix, int B, int u) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= u) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int D>
+ISD_DEV uint32_t swz(uint32_t base, int key, int chunk) {
+  // 128-byte swizzle of a [16 rows][64 cols] bf16 box; boxes of the d
+  // dimension are 2048 bytes apart.
+  return base + (chunk >> 3) * 2048 + key * 128 + (((chunk & 7) ^ (key & 7)) << 4);
+}
+
+template <int D, int MW>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_kc,
+                     const __grid_constant__ CUtensorMap tm_vc,
+                     const __grid_constant__ CUtensorMap tm_kn,
+                     const __grid_constant__ CUtensorMap tm_vn, AttnDev p) {
+  constexpr int kTile = 16 * D * 2;            // one K or V tile, bytes
+  constexpr int kStage = 2 * kTile;
+  constexpr int RW = 16 * MW;                  // rows per consumer warp
+  constexpr int kRedRow = D + 4;
+  constexpr int kRedWarp = RW * kRedRow + 2 * RW;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages * kStage);
+  uint64_t* empty = full + kStages;
+  float* red = reinterpret_cast<float*>(empty + kStages);
+  int* prefix = reinterpret_cast<int*>(red + kCWarps * kRedWarp);
+  __shared__ int scan_sh[33];
+  __shared__ int s_bad;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int B = p.B, Hkv = p.Hkv;
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  const int T = block_exclusive_scan_int(
+      B,
+      [&](int b) {
+        bool bad = false;
+        const int n = pages_of(p, b, &bad);
+        if (bad) s_bad = 1;
+        return Hkv * (n + 1);
+      },
+      prefix, scan_sh);
+  if (tid == 0) prefix[B] = T;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int u0 = (int)(((long long)c * T) / G);
+  const int u1 = (int)(((long long)(c + 1) * T) / G);
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], p.RG);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (c == 0) {
+    for (int i = tid; i <= B; i += blockDim.x) p.ws_int[i] = prefix[i];
+    if (tid == 0) {
+      p.ws_int[B + 1] = G;
+      if (s_bad && p.status) *p.status = ISD_ERR_PAGE_TABLE_FULL;
+    }
+  }
+  if (u0 >= u1) return;
+
+  // ------------------------------------------------------------- producer
+  // The whole warp resolves 32 units at a time (sequence, head, page id:
+  // one coalesced page-table load), prefetching the next 32 while lane 0
+  // issues the current ones, so no TMA waits on a dependent global load.
+  if (warp == kCWarps) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_kc);
+      tma_prefetch_desc(&tm_vc);
+      tma_prefetch_desc(&tm_kn);
+      tma_prefetch_desc(&tm_vn);
+    }
+    auto resolve = [&](int u, int& bb, int& hh, int& page) {
+      // page >= 0: cached page id; page == -1 - b marks the tail unit.
+      if (u >= u1) { bb = 0; hh = 0; page = 0; return; }
+      bb = find_seq(prefix, B, u);
+      const int units = (prefix[bb + 1] - prefix[bb]) / Hkv;
+      const int rel = u - prefix[bb];
+      hh = rel / units;
+      const int idx = rel % units;
+      if (idx == units - 1) {
+        page = -1;
+      } else {
+        page = p.page_table[(size_t)bb * p.stride + idx];
+        if (page < 0 || page >= p.P) {
+          if (p.status) *p.status = ISD_ERR_BAD_PAGE;
+          page = p.P;  // out of range: TMA fills zeros, no fault
+        }
+      }
+    };
+    int cb, ch, cp, nb, nh, np;
+    resolve(u0 + lane, cb, ch, cp);
+    bool failed = false;
+    for (int base = u0; base < u1; base += 32) {
+      resolve(base + 32 + lane, nb, nh, np);
+      const int cnt = min(32, u1 - base);
+      for (int j = 0; j < cnt; ++j) {
+        const int b = __shfl_sync(0xffffffffu, cb, j);
+        const int h = __shfl_sync(0xffffffffu, ch, j);
+        const int page = __shfl_sync(0xffffffffu, cp, j);
+        if (lane == 0) {
+          const int it = base - u0 + j;
+          const int s = it % kStages;
+          if (!failed && !wait_bounded(&empty[s], ((it / kStages) & 1) ^ 1)) {
+            failed = true;
+            if (p.status) *p.status = ISD_ERR_CUDA;
+          }
+          uint8_t* kdst = ring + s * kStage;
+          uint8_t* vdst = kdst + kTile;
+          mbar_arrive_expect_tx(&full[s], kStage);
+          if (page < 0) {  // tail: the stride's own rows (TMA zero-fills
+                           // rows >= K)
+#pragma unroll
+            for (int bi = 0; bi < D / 64; ++bi) {
+              tma_load_4d(kdst + bi * 2048, &tm_kn, &full[s], bi * 64, h, 0, b);
+              tma_load_4d(vdst + bi * 2048, &tm_vn, &full[s], bi * 64, h, 0, b);
+            }
+          } else {
+#pragma unroll
+            for (int bi = 0; bi < D / 64; ++bi) {
+              tma_load_4d(kdst + bi * 2048, &tm_kc, &full[s], bi * 64, 0, h,
+                          page);
+              tma_load_4d(vdst + bi * 2048, &tm_vc, &full[s], bi * 64, 0, h,
+                          page);
+            }
+          }
+        }
+        __syncwarp();
+      }
+      cb = nb; ch = nh; cp = np;
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  const int KS = p.KS;
+  const int rg = warp / KS, ks = warp % KS;
+  const int g = p.g, K = p.K, Hq = p.Hq;
+  float* my_red = red + warp * kRedWarp;
+  bool failed = false;
+  int u = u0, it = 0;
+  while (u < u1) {
+    const int b = find_seq(prefix, B, u);
+    const int units = (prefix[b + 1] - prefix[b]) / Hkv;
+    const int rel = u - prefix[b];
+    const int h = rel / units, idx0 = rel % units;
+    const int bh_end = prefix[b] + (h + 1) * units;
+    const int seg_end = min(u1, bh_end);
+    const int nseg = seg_end - u;
+    const bool complete = idx0 == 0 && seg_end == bh_end;
+    const int npg = units - 1;
+    const int L = p.seq_len[b];
+
+    // Q fragments of this warp's rows.
+    uint32_t qa[MW][D / 16][4];
+    int rrow[MW][2];
+#pragma unroll
+    for (int mt = 0; mt < MW; ++mt) {
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int m = rg * RW + mt * 16 + (lane >> 2) + hf * 8;
+        rrow[mt][hf] = m / g;
+      }
+      const int m0 = rg * RW + mt * 16 + (lane >> 2);
+      const int m1 = m0 + 8;
+      const __nv_bfloat16* q0 =
+          p.q + (((size_t)b * K + m0 / g) * Hq + h * g + m0 % g) * D;
+      const __nv_bfloat16* q1 =
+          p.q + (((size_t)b * K + m1 / g) * Hq + h * g + m1 % g) * D;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int col = kk * 16 + 2 * (lane & 3);
+        qa[mt][kk][0] = *reinterpret_cast<const uint32_t*>(q0 + col);
+        qa[mt][kk][1] = *reinterpret_cast<const uint32_t*>(q1 + col);
+        qa[mt][kk][2] = *reinterpret_cast<const uint32_t*>(q0 + col + 8);
+        qa[mt][kk][3] = *reinterpret_cast<const uint32_t*>(q1 + col + 8);
+      }
+    }
+    float acc[MW][D / 8][4];
+    float mrow[MW][2], lrow[MW][2];
+#pragma unroll
+    for (int mt = 0; mt < MW; ++mt) {
+#pragma unroll
+      for (int nt = 0; nt < D / 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.0f;
+      mrow[mt][0] = mrow[mt][1] = -INFINITY;
+      lrow[mt][0] = lrow[mt][1] = 0.0f;
+    }
+
+    for (int k = 0; k < nseg; ++k) {
+      const int itk = it + k;
+      if (itk % KS != ks) continue;
+      const int s = itk % kStages;
+      if (!failed && !wait_bounded(&full[s], (itk / kStages) & 1)) {
+        failed = true;
+        if (p.status) *p.status = ISD_ERR_CUDA;
+      }
+      const int uidx = idx0 + k;
+      const bool tail = uidx == npg;
+      const int valid = tail ? K : min(kPage, L - uidx * kPage);
+      const uint32_t kb = smem_u32(ring + s * kStage);
+      const uint32_t vb = kb + kTile;
+
+      // S = Q K^T over this tile's 16 keys.
+      float sc[MW][2][4];
+#pragma unroll
+      for (int mt = 0; mt < MW; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[mt][nt][e] = 0.0f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int key = ((lane >> 4) << 3) + (lane & 7);
+        const int chunk = 2 * kk + ((lane >> 3) & 1);
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4(swz<D>(kb, key, chunk), b0, b1, b2, b3);
+#pragma unroll
+        for (int mt = 0; mt < MW; ++mt) {
+          mma_bf16_16816(sc[mt][0], qa[mt][kk], b0, b1);
+          mma_bf16_16816(sc[mt][1], qa[mt][kk], b2, b3);
+        }
+      }
+      // Mask, online softmax (base 2), P as bf16 A fragments.
+      uint32_t pa[MW][4];
+#pragma unroll
+      for (int mt = 0; mt < MW; ++mt) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int r = rrow[mt][hf];
+          float mx = -INFINITY;
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int key = nt * 8 + 2 * (lane & 3) + e;
+              const bool ok = key < valid && (!tail || key <= r);
+              float& x = sc[mt][nt][hf * 2 + e];
+              x = ok ? x * p.scale_log2 : -INFINITY;
+              mx = fmaxf(mx, x);
+            }
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          const float mnew = fmaxf(mrow[mt][hf], mx);
+          const float alpha = ex2(mrow[mt][hf] - mnew);
+          mrow[mt][hf] = mnew;
+          float ls = 0.0f;
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              float& x = sc[mt][nt][hf * 2 + e];
+              x = ex2(x - mnew);
+              ls += x;
+            }
+          lrow[mt][hf] = lrow[mt][hf] * alpha + ls;
+#pragma unroll
+          for (int nt = 0; nt < D / 8; ++nt) {
+            acc[mt][nt][hf * 2] *= alpha;
+            acc[mt][nt][hf * 2 + 1] *= alpha;
+          }
+        }
+        pa[mt][0] = pack_bf16(sc[mt][0][0], sc[mt][0][1]);
+        pa[mt][1] = pack_bf16(sc[mt][0][2], sc[mt][0][3]);
+        pa[mt][2] = pack_bf16(sc[mt][1][0], sc[mt][1][1]);
+        pa[mt][3] = pack_bf16(sc[mt][1][2], sc[mt][1][3]);
+      }
+      // Invalid V rows (unwritten slots of a partial page) may hold any
+      // bits; zero them in the fragments so 0 * NaN cannot reach O.
+      const int k0 = 2 * (lane & 3);
+      const uint32_t mlo = (k0 < valid ? 0x0000FFFFu : 0u) |
+                           (k0 + 1 < valid ? 0xFFFF0000u : 0u);
+      const uint32_t mhi = (k0 + 8 < valid ? 0x0000FFFFu : 0u) |
+                           (k0 + 9 < valid ? 0xFFFF0000u : 0u);
+      // O += P V.
+#pragma unroll
+      for (int np = 0; np < D / 16; ++np) {
+        const int key = (((lane >> 3) & 1) << 3) + (lane & 7);
+        const int chunk = 2 * np + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4_trans(swz<D>(vb, key, chunk), b0, b1, b2, b3);
+        b0 &= mlo; b1 &= mhi; b2 &= mlo; b3 &= mhi;
+#pragma unroll
+        for (int mt = 0; mt < MW; ++mt) {
+          mma_bf16_16816(acc[mt][2 * np], pa[mt], b0, b1);
+          mma_bf16_16816(acc[mt][2 * np + 1], pa[mt], b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    // Row sums across the quad of threads sharing a row.
+#pragma unroll
+    for (int mt = 0; mt < MW; ++mt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        float l = lrow[mt][hf];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        lrow[mt][hf] = l;
+      }
+
+    const int slot = (u == u0) ? 0 : 1;
+    float* part = p.part + ((size_t)(c * 2 + slot)) * p.M * (D + 2);
+    if (KS == 1) {
+      // Write this warp's rows straight from registers.
+#pragma unroll
+      for (int mt = 0; mt < MW; ++mt)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int m = rg * RW + mt * 16 + (lane >> 2) + hf * 8;
+          const int r = m / g, j = m % g;
+          const float mr = mrow[mt][hf], l = lrow[mt][hf];
+          if (complete) {
+            const float inv = 1.0f / l;
+            __nv_bfloat16* o =
+                p.out + (((size_t)b * K + r) * Hq + h * g + j) * D;
+#pragma unroll
+            for (int nt = 0; nt < D / 8; ++nt) {
+              const int col = nt * 8 + 2 * (lane & 3);
+              *reinterpret_cast<uint32_t*>(o + col) =
+                  pack_bf16(acc[mt][nt][hf * 2] * inv,
+                            acc[mt][nt][hf * 2 + 1] * inv);
+            }
+            if (p.lse && (lane & 3) == 0)
+              p.lse[((size_t)b * K + r) * Hq + h * g + j] =
+                  (mr + log2f(l)) * kLn2;
+          } else {
+#pragma unroll
+            for (int nt = 0; nt < D / 8; ++nt) {
+              const int col = nt * 8 + 2 * (lane & 3);
+              *reinterpret_cast<float2*>(part + (size_t)m * D + col) =
+                  make_float2(acc[mt][nt][hf * 2], acc[mt][nt][hf * 2 + 1]);
+            }
+            if ((lane & 3) == 0) {
+              part[(size_t)p.M * D + m] = mr;
+              part[(size_t)p.M * D + p.M + m] = l;
+            }
+          }
+        }
+    } else {
+      // Merge the KS key splits of each row group through shared memory.
+#pragma unroll
+      for (int mt = 0; mt < MW; ++mt)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int rl = mt * 16 + (lane >> 2) + hf * 8;
+#pragma unroll
+          for (int nt = 0; nt < D / 8; ++nt) {
+            const int col = nt * 8 + 2 * (lane & 3);
+            *reinterpret_cast<float2*>(my_red + rl * kRedRow + col) =
+                make_float2(acc[mt][nt][hf * 2], acc[mt][nt][hf * 2 + 1]);
+          }
+          if ((lane & 3) == 0) {
+            my_red[RW * kRedRow + rl] = mrow[mt][hf];
+            my_red[RW * kRedRow + RW + rl] = lrow[mt][hf];
+          }
+        }
+      asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32));
+      const int cols = D / KS;
+      for (int e = lane; e < RW * cols; e += 32) {
+        const int rl = e / cols, col = ks * cols + e % cols;
+        float mstar = -INFINITY;
+        for (int q2 = 0; q2 < KS; ++q2) {
+          const float* rw = red + (rg * KS + q2) * kRedWarp;
+          mstar = fmaxf(mstar, rw[RW * kRedRow + rl]);
+        }
+        float o = 0.0f, l = 0.0f;
+        for (int q2 = 0; q2 < KS; ++q2) {
+          const float* rw = red + (rg * KS + q2) * kRedWarp;
+          const float mq = rw[RW * kRedRow + rl];
+          const float wgt = mq == -INFINITY ? 0.0f : ex2(mq - mstar);
+          o += rw[rl * kRedRow + col] * wgt;
+          l += rw[RW * kRedRow + RW + rl] * wgt;
+        }
+        const int m = rg * RW + rl;
+        const int r = m / g, j = m % g;
+        if (complete) {
+          p.out[(((size_t)b * K + r) * Hq + h * g + j) * D + col] =
+              __float2bfloat16_rn(o / l);
+          if (p.lse && col == 0)
+            p.lse[((size_t)b * K + r) * Hq + h * g + j] =
+                (mstar + log2f(l)) * kLn2;
+        } else {
+          part[(size_t)m * D + col] = o;
+          if (col == ks * cols) {
+            part[(size_t)p.M * D + m] = mstar;
+            part[(size_t)p.M * D + p.M + m] = l;
+          }
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32));
+    }
+    it += nseg;
+    u = seg_end;
+  }
+}
+
+// Merge the partials of every (b, h) whose units straddled CTAs.
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_kernel(AttnDev p) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int B = p.B;
+  const int* prefix = p.ws_int;
+  const long long T = prefix[B];
+  const long long G = p.ws_int[B + 1];
+  const int units = (prefix[b + 1] - prefix[b]) / p.Hkv;
+  const long long s = prefix[b] + (long long)h * units;
+  const long long e = s + units;
+  auto cta_of = [&](long long uu) { return (int)(((uu + 1) * G - 1) / T); };
+  const int cf = cta_of(s), cl = cta_of(e - 1);
+  if (cf == cl) return;
+  const int M = p.M, g = p.g, K = p.K, Hq = p.Hq;
+  for (int i = threadIdx.x; i < M * D; i += blockDim.x) {
+    const int m = i / D, col = i % D;
+    float mstar = -INFINITY;
+    for (int cc = cf; cc <= cl; ++cc) {
+      const long long u0 = ((long long)cc * T) / G;
+      if (u0 == ((long long)(cc + 1) * T) / G) continue;  // empty range
+      const int slot = (cc == cf && u0 != s) ? 1 : 0;
+      const float* part = p.part + ((size_t)(cc * 2 + slot)) * M * (D + 2);
+      mstar = fmaxf(mstar, part[(size_t)M * D + m]);
+    }
+    float o = 0.0f, l = 0.0f;
+    for (int cc = cf; cc <= cl; ++cc) {
+      const long long u0 = ((long long)cc * T) / G;
+      if (u0 == ((long long)(cc + 1) * T) / G) continue;  // empty range
+      const int slot = (cc == cf && u0 != s) ? 1 : 0;
+      const float* part = p.part + ((size_t)(cc * 2 + slot)) * M * (D + 2);
+      const float mq = part[(size_t)M * D + m];
+      const float w = mq == -INFINITY ? 0.0f : ex2(mq - mstar);
+      o += part[(size_t)m * D + col] * w;
+      l += part[(size_t)M * D + M + m] * w;
+    }
+    const int r = m / g, j = m % g;
+    p.out[(((size_t)b * K + r) * Hq + h * g + j) * D + col] =
+        __float2bfloat16_rn(o / l);
+    if (p.lse && col == 0)
+      p.lse[((size_t)b * K + r) * Hq + h * g + j] = (mstar + log2f(l)) * kLn2;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// fp32 SIMT path: one warp per (b, r, hq) query row, exact fp32 arithmetic.
+template <int DPL>  // d / 32 elements per lane
+__global__ void __launch_bounds__(128)
+    attn_f32_kernel(int B, int Hq, int Hkv, int K, int stride, int P,
+                    float scale, const float* q, const float* k_new,
+                    const float* v_new, const float* k_cache,
+                    const float* v_cache, const int32_t* page_table,
+                    const int32_t* seq_len, float* out, float* lse,
+                    int32_t* status) {
+  constexpr int D = DPL * 32;
+  const int lane = threadIdx.x & 31;
+  const int wg = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (wg >= B * K * Hq) return;
+  const int hq = wg % Hq, r = (wg / Hq) % K, b = wg / (Hq * K);
+  const int g = Hq / Hkv, h = hq / g;
+  int L = seq_len[b];
+  if (L < 0 || (L + kPage - 1) / kPage > stride) {
+    if (status && lane == 0) *status = ISD_ERR_PAGE_TABLE_FULL;
+    L = max(0, min(L, stride * kPage));
+  }
+  float qv[DPL], o[DPL];
+  const float* qp = q + (((size_t)b * K + r) * Hq + hq) * D;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) { qv[i] = qp[lane + 32 * i]; o[i] = 0.0f; }
+  float m = -INFINITY, l = 0.0f;
+  const int total = L + r + 1;
+  for (int t = 0; t < total; ++t) {
+    const float *kp, *vp;
+    if (t < L) {
+      const int page = page_table[(size_t)b * stride + t / kPage];
+      if (page < 0 || page >= P) {
+        if (status && lane == 0) *status = ISD_ERR_BAD_PAGE;
+        continue;
+      }
+      const size_t off = (((size_t)page * Hkv + h) * kPage + t % kPage) * D;
+      kp = k_cache + off;
+      vp = v_cache + off;
+    } else {
+      const size_t off = (((size_t)b * K + (t - L)) * Hkv + h) * D;
+      kp = k_new + off;
+      vp = v_new + off;
+    }
+    float dot = 0.0f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) dot = fmaf(qv[i], kp[lane + 32 * i], dot);
+    dot = warp_sum(dot) * scale;
+    const float mn = fmaxf(m, dot);
+    const float alpha = expf(m - mn);
+    const float pr = expf(dot - mn);
+    l = l * alpha + pr;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) o[i] = fmaf(o[i], alpha, pr * vp[lane + 32 * i]);
+    m = mn;
+  }
+  float* op = out + (((size_t)b * K + r) * Hq + hq) * D;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) op[lane + 32 * i] = o[i] / l;
+  if (lse && lane == 0) lse[((size_t)b * K + r) * Hq + hq] = m + logf(l);
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+
+size_t attn_smem_bytes(int D, int MW, int B) {
+  const int RW = 16 * MW;
+  const size_t red = (size_t)kCWarps * (RW * (D + 4) + 2 * RW) * 4;
+  return 1024 + (size_t)kStages * 2 * (16 * D * 2) + 2 * kStages * 8 + red +
+         (size_t)(B + 1) * 4;
+}
+
+size_t attn_workspace_bytes_impl(int B, int M, int D, int G) {
+  const size_t ints = ((size_t)(B + 2) * 4 + 255) & ~size_t(255);
+  return ints + (size_t)G * 2 * M * (D + 2) * 4;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
+                                  void*, const cuuint64_t*, const cuuint64_t*,
+                                  const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr,
+                                cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+static bool encode_4d(CUtensorMap* m, const void* base, const uint64_t dims[4],
+                      const uint64_t strides_bytes[3], const uint32_t box[4]) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
+  cuuint64_t gs[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
+  cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), gd,
+            gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int MW>
+static int launch_bf16(const isd_attn_args* a, int G, cudaStream_t st) {
+  CUtensorMap tkc, tvc, tkn, tvn;
+  const uint64_t es = 2;
+  const uint64_t dc[4] = {(uint64_t)D, (uint64_t)kPage, (uint64_t)a->Hkv,
+                          (uint64_t)a->num_pages};
+  const uint64_t sc[3] = {D * es, (uint64_t)kPage * D * es,
+                          (uint64_t)a->Hkv * kPage * D * es};
+  const uint32_t bc[4] = {64, (uint32_t)kPage, 1, 1};
+  const uint64_t dn[4] = {(uint64_t)D, (uint64_t)a->Hkv, (uint64_t)a->K,
+                          (uint64_t)a->B};
+  const uint64_t sn[3] = {D * es, (uint64_t)a->Hkv * D * es,
+                          (uint64_t)a->K * a->Hkv * D * es};
+  const uint32_t bn[4] = {64, 1, (uint32_t)kPage, 1};
+  if (!encode_4d(&tkc, a->k_cache, dc, sc, bc) ||
+      !encode_4d(&tvc, a->v_cache, dc, sc, bc) ||
+      !encode_4d(&tkn, a->k_new, dn, sn, bn) ||
+      !encode_4d(&tvn, a->v_new, dn, sn, bn))
+    return ISD_ERR_CUDA;
+  AttnDev p;
+  p.B = a->B; p.Hq = a->Hq; p.Hkv = a->Hkv; p.K = a->K;
+  p.g = a->Hq / a->Hkv; p.M = a->K * p.g; p.P = a->num_pages;
+  p.stride = a->page_table_stride;
+  p.RG = p.M / (16 * MW); p.KS = kCWarps / p.RG;
+  p.scale_log2 = a->softmax_scale * kLog2e;
+  p.q = static_cast<const __nv_bfloat16*>(a->q);
+  p.out = static_cast<__nv_bfloat16*>(a->out);
+  p.lse = a->lse; p.page_table = a->page_table; p.seq_len = a->seq_len;
+  p.status = a->status;
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  p.ws_int = reinterpret_cast<int32_t*>(ws);
+  p.part = reinterpret_cast<float*>(
+      ws + (((size_t)(a->B + 2) * 4 + 255) & ~size_t(255)));
+  const size_t smem = attn_smem_bytes(D, MW, a->B);
+  static bool attr_set[2] = {false, false};
+  static size_t attr_val[2] = {0, 0};
+  auto kern = attn_bf16_kernel<D, MW>;
+  const int slot = 0;
+  if (!attr_set[slot] || attr_val[slot] < smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return ISD_ERR_CUDA;
+    attr_set[slot] = true;
+    attr_val[slot] = smem;
+  }
+  kern<<<G, kAttnThreads, smem, st>>>(tkc, tvc, tkn, tvn, p);
+  attn_combine_kernel<D><<<dim3(a->Hkv, a->B), 256, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ISD_OK : ISD_ERR_CUDA;
+}
+
+int launch_attn_bf16(const isd_attn_args* a, int G, cudaStream_t st) {
+  const int M = a->K * (a->Hq / a->Hkv);
+  const int MW = M == 16 ? 1 : 2;
+  if (a->d == 128) return MW == 1 ? launch_bf16<128, 1>(a, G, st)
+                                  : launch_bf16<128, 2>(a, G, st);
+  return MW == 1 ? launch_bf16<64, 1>(a, G, st) : launch_bf16<64, 2>(a, G, st);
+}
+
+int launch_attn_f32(const isd_attn_args* a, cudaStream_t st) {
+  const int rows = a->B * a->K * a->Hq;
+  const int blocks = (rows + 3) / 4;
+#define ISD_F32_CASE(DPL)                                                     \
+  attn_f32_kernel<DPL><<<blocks, 128, 0, st>>>(                               \
+      a->B, a->Hq, a->Hkv, a->K, a->page_table_stride, a->num_pages,          \
+      a->softmax_scale, (const float*)a->q, (const float*)a->k_new,           \
+      (const float*)a->v_new, (const float*)a->k_cache,                       \
+      (const float*)a->v_cache, a->page_table, a->seq_len, (float*)a->out,    \
+      a->lse, a->status)
+  switch (a->d / 32) {
+    case 1: ISD_F32_CASE(1); break;
+    case 2: ISD_F32_CASE(2); break;
+    case 3: ISD_F32_CASE(3); break;
+    case 4: ISD_F32_CASE(4); break;
+    default: return ISD_ERR_UNSUPPORTED;
+  }
+#undef ISD_F32_CASE
+  return cudaGetLastError() == cudaSuccess ? ISD_OK : ISD_ERR_CUDA;
+}
+
+}  // namespace isd

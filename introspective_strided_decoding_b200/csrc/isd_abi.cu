@@ -1,0 +1,182 @@
+// C ABI of libisd.so (declared in include/isd.h): host-side validation and
+// dispatch.  Nothing here allocates, frees or synchronises.
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace isd {
+size_t accept_workspace_bytes(int B, int N, int K, int V);
+int launch_accept(const isd_accept_args* a, cudaStream_t st);
+size_t commit_workspace_bytes(int B);
+int launch_commit(const isd_commit_args* a, cudaStream_t st);
+size_t attn_workspace_bytes_impl(int B, int M, int D, int G);
+size_t attn_smem_bytes(int D, int MW, int B);
+int launch_attn_bf16(const isd_attn_args* a, int G, cudaStream_t st);
+int launch_attn_f32(const isd_attn_args* a, cudaStream_t st);
+}  // namespace isd
+
+namespace {
+
+bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
+      cudaSuccess)
+    return 0;
+  return n;
+}
+
+int attn_ctas(const isd_attn_args* a) {
+  if (a->num_ctas > 0) return a->num_ctas;
+  return sm_count();
+}
+
+// Shape checks shared by the workspace query and the call.
+int attn_check(const isd_attn_args* a) {
+  if (!a) return ISD_ERR_INVALID_ARG;
+  if (a->B <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->d <= 0 || a->K <= 0 ||
+      a->num_pages <= 0 || a->page_table_stride <= 0 || a->num_ctas < 0)
+    return ISD_ERR_INVALID_ARG;
+  if (a->Hq % a->Hkv != 0) return ISD_ERR_INVALID_ARG;
+  if (!(a->softmax_scale > 0.0f)) return ISD_ERR_INVALID_ARG;
+  if (a->dtype == ISD_BF16) {
+    const int M = a->K * (a->Hq / a->Hkv);
+    if (a->d != 64 && a->d != 128) return ISD_ERR_UNSUPPORTED;
+    if (!(M == 16 || M == 32 || M == 64 || M == 128)) return ISD_ERR_UNSUPPORTED;
+    if (a->K > ISD_PAGE_SIZE) return ISD_ERR_UNSUPPORTED;
+    if (isd::attn_smem_bytes(a->d, M == 16 ? 1 : 2, a->B) > 227 * 1024)
+      return ISD_ERR_UNSUPPORTED;
+  } else if (a->dtype == ISD_F32) {
+    if (a->d % 32 != 0 || a->d > 128) return ISD_ERR_UNSUPPORTED;
+  } else {
+    return ISD_ERR_INVALID_ARG;
+  }
+  return ISD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int isd_abi_version(void) { return ISD_ABI_VERSION; }
+
+const char* isd_status_string(int code) {
+  switch (code) {
+    case ISD_OK: return "ok";
+    case ISD_ERR_INVALID_ARG: return "invalid argument";
+    case ISD_ERR_UNSUPPORTED: return "unsupported shape or type";
+    case ISD_ERR_CUDA: return "CUDA error";
+    case ISD_ERR_WORKSPACE: return "workspace missing or too small";
+    case ISD_ERR_POOL_EXHAUSTED: return "KV page pool exhausted";
+    case ISD_ERR_PAGE_TABLE_FULL: return "page-table row full";
+    case ISD_ERR_BAD_STATE: return "malformed decoding state";
+    case ISD_ERR_BAD_PAGE: return "page id out of range";
+    default: return "unknown status";
+  }
+}
+
+// ------------------------------------------------------------- attention
+size_t isd_attn_workspace_bytes(const isd_attn_args* a) {
+  if (attn_check(a) != ISD_OK) return 0;
+  if (a->dtype == ISD_F32) return 0;
+  const int G = attn_ctas(a);
+  if (G <= 0) return 0;
+  return isd::attn_workspace_bytes_impl(a->B, a->K * (a->Hq / a->Hkv), a->d, G);
+}
+
+int isd_attn_strided(const isd_attn_args* a, void* stream) {
+  const int rc = attn_check(a);
+  if (rc != ISD_OK) return rc;
+  if (!a->q || !a->k_new || !a->v_new || !a->k_cache || !a->v_cache ||
+      !a->page_table || !a->seq_len || !a->out)
+    return ISD_ERR_INVALID_ARG;
+  if (!aligned16(a->q) || !aligned16(a->k_new) || !aligned16(a->v_new) ||
+      !aligned16(a->k_cache) || !aligned16(a->v_cache) || !aligned16(a->out))
+    return ISD_ERR_INVALID_ARG;
+  if (a->out == a->q || a->out == a->k_new || a->out == a->v_new ||
+      a->out == a->k_cache || a->out == a->v_cache)
+    return ISD_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (a->dtype == ISD_F32) return isd::launch_attn_f32(a, st);
+  const int G = attn_ctas(a);
+  if (G <= 0) return ISD_ERR_CUDA;
+  const size_t need =
+      isd::attn_workspace_bytes_impl(a->B, a->K * (a->Hq / a->Hkv), a->d, G);
+  if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace))
+    return ISD_ERR_WORKSPACE;
+  return isd::launch_attn_bf16(a, G, st);
+}
+
+// ---------------------------------------------------------------- accept
+static int accept_check(const isd_accept_args* a) {
+  if (!a) return ISD_ERR_INVALID_ARG;
+  if (a->B <= 0 || a->N < 2 || a->V <= 0 || a->K != 2 * a->N)
+    return ISD_ERR_INVALID_ARG;
+  if (a->N > 16) return ISD_ERR_UNSUPPORTED;
+  if (a->dtype != ISD_BF16 && a->dtype != ISD_F32) return ISD_ERR_INVALID_ARG;
+  return ISD_OK;
+}
+
+size_t isd_accept_workspace_bytes(const isd_accept_args* a) {
+  if (accept_check(a) != ISD_OK) return 0;
+  return isd::accept_workspace_bytes(a->B, a->N, a->K, a->V);
+}
+
+int isd_accept_resample(const isd_accept_args* a, void* stream) {
+  const int rc = accept_check(a);
+  if (rc != ISD_OK) return rc;
+  if (!a->logits_cur || !a->logits_prev || !a->seq_len || !a->pending_in ||
+      !a->n_pending_in || !a->q_row_in || !a->q_stats_in || !a->pending_out ||
+      !a->n_pending_out || !a->q_row_out || !a->q_stats_out || !a->n_commit ||
+      !a->commit_tokens)
+    return ISD_ERR_INVALID_ARG;
+  if ((const void*)a->pending_out == (const void*)a->pending_in ||
+      (const void*)a->n_pending_out == (const void*)a->n_pending_in ||
+      (const void*)a->q_row_out == (const void*)a->q_row_in ||
+      (const void*)a->q_stats_out == (const void*)a->q_stats_in)
+    return ISD_ERR_INVALID_ARG;
+  if (!aligned16(a->logits_cur) || !aligned16(a->logits_prev))
+    return ISD_ERR_INVALID_ARG;
+  const size_t need = isd::accept_workspace_bytes(a->B, a->N, a->K, a->V);
+  if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace))
+    return ISD_ERR_WORKSPACE;
+  return isd::launch_accept(a, static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------- commit
+static int commit_check(const isd_commit_args* a) {
+  if (!a) return ISD_ERR_INVALID_ARG;
+  if (a->B <= 0 || a->K <= 0 || a->Hkv <= 0 || a->d <= 0 ||
+      a->num_pages <= 0 || a->page_table_stride <= 0)
+    return ISD_ERR_INVALID_ARG;
+  if (a->dtype != ISD_BF16 && a->dtype != ISD_F32) return ISD_ERR_INVALID_ARG;
+  const int es = a->dtype == ISD_BF16 ? 2 : 4;
+  if ((a->d * es) % 16 != 0) return ISD_ERR_UNSUPPORTED;
+  return ISD_OK;
+}
+
+size_t isd_commit_workspace_bytes(const isd_commit_args* a) {
+  if (commit_check(a) != ISD_OK) return 0;
+  return isd::commit_workspace_bytes(a->B);
+}
+
+int isd_kv_commit(const isd_commit_args* a, void* stream) {
+  const int rc = commit_check(a);
+  if (rc != ISD_OK) return rc;
+  if (!a->k_new || !a->v_new || !a->k_cache || !a->v_cache || !a->page_table ||
+      !a->seq_len || !a->n_commit || !a->free_stack || !a->free_top ||
+      !a->status)
+    return ISD_ERR_INVALID_ARG;
+  if (!aligned16(a->k_new) || !aligned16(a->v_new) || !aligned16(a->k_cache) ||
+      !aligned16(a->v_cache))
+    return ISD_ERR_INVALID_ARG;
+  const size_t need = isd::commit_workspace_bytes(a->B);
+  if (!a->workspace || a->workspace_bytes < need) return ISD_ERR_WORKSPACE;
+  return isd::launch_commit(a, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

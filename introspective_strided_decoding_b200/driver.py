@@ -1,0 +1,148 @@
+"""Stationary-batch ISD decode loop on one GPU.
+
+The pages' serving engine keeps batch membership fixed across steps
+("stationary-batch decode loop", hada.io summary, "Serving (SGLang)").
+``Decoder`` owns the per-step device buffers (logits ping-pong, decoding
+state ping-pong, attention output, workspaces) and runs one step as the
+three C-ABI calls on one stream:
+
+    isd_attn_strided -> (caller's LM head fills logits) -> isd_accept_resample
+    -> isd_kv_commit
+
+The argument structs are built once, so a step costs three ctypes calls on
+the host.  All memory is allocated here, through torch, never by the
+library.
+"""
+
+import ctypes
+import math
+
+import torch
+
+from . import isd
+
+
+class Decoder:
+    def __init__(self, w, cache, state0, device, seed, num_ctas=0,
+                 with_lse=False, record=False):
+        self.w = w
+        self.cache = cache
+        self.device = torch.device(device)
+        self.seed = int(seed)
+        B, K, N, V, Hq, d = w.B, w.K, w.N, w.V, w.Hq, w.d
+        dt = w.torch_dtype
+        dev = self.device
+        self.q = torch.zeros((B, K, Hq, d), dtype=dt, device=dev)
+        self.k_new = torch.zeros((B, K, w.Hkv, d), dtype=dt, device=dev)
+        self.v_new = torch.zeros((B, K, w.Hkv, d), dtype=dt, device=dev)
+        self.out = torch.empty((B, K, Hq, d), dtype=dt, device=dev)
+        self.lse = torch.empty((B, K, Hq), dtype=torch.float32, device=dev) \
+            if with_lse else None
+        self.logits = [torch.zeros((B, K, V), dtype=dt, device=dev)
+                       for _ in range(2)]
+        self.states = [isd.new_state(B, N, dev), isd.new_state(B, N, dev)]
+        for key in isd.STATE_KEYS:
+            self.states[0][key].copy_(state0[key])
+        self.n_commit = torch.zeros(B, dtype=torch.int32, device=dev)
+        self.commit_tokens = torch.zeros((B, N), dtype=torch.int32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        # Optional per-step diagnostics (row statistics, draft ratios).
+        self.row_stats = torch.full((B, K, 2), float("nan"),
+                                    dtype=torch.float32, device=dev) \
+            if record else None
+        self.ratio = torch.full((B, N), float("nan"), dtype=torch.float32,
+                                device=dev) if record else None
+        self.cur = 0
+        self.step_idx = 0
+        scale = 1.0 / math.sqrt(d)
+        self._attn = isd.attn_args(
+            self.q, self.k_new, self.v_new, cache["k_cache"],
+            cache["v_cache"], cache["page_table"], cache["seq_len"], self.out,
+            self.lse, self.status, scale, None, num_ctas)
+        self.ws_attn = torch.empty(max(isd.attn_workspace_bytes(self._attn),
+                                       16), dtype=torch.uint8, device=dev)
+        self._attn.workspace = ctypes.c_void_p(self.ws_attn.data_ptr())
+        self._attn.workspace_bytes = self.ws_attn.numel()
+        self._acc = []
+        for c in range(2):
+            a = isd.accept_args(self.logits[c], self.logits[1 - c],
+                                cache["seq_len"], self.states[c],
+                                self.states[1 - c], self.n_commit,
+                                self.commit_tokens, self.seed, 0,
+                                row_stats=self.row_stats, ratio=self.ratio,
+                                status=self.status)
+            self._acc.append(a)
+        self.ws_acc = torch.empty(isd.accept_workspace_bytes(self._acc[0]),
+                                  dtype=torch.uint8, device=dev)
+        for a in self._acc:
+            a.workspace = ctypes.c_void_p(self.ws_acc.data_ptr())
+            a.workspace_bytes = self.ws_acc.numel()
+        self._com = isd.commit_args(
+            self.k_new, self.v_new, cache["k_cache"], cache["v_cache"],
+            cache["page_table"], cache["seq_len"], self.n_commit,
+            cache["free_stack"], cache["free_top"], self.status)
+        self.ws_com = torch.empty(isd.commit_workspace_bytes(self._com),
+                                  dtype=torch.uint8, device=dev)
+        self._com.workspace = ctypes.c_void_p(self.ws_com.data_ptr())
+        self._com.workspace_bytes = self.ws_com.numel()
+        self._lib = isd.lib()
+
+    # The buffers the caller fills before a step.
+    @property
+    def logits_cur(self):
+        return self.logits[self.cur]
+
+    @property
+    def state(self):
+        """Decoding state entering the next step."""
+        return self.states[self.cur]
+
+    @property
+    def next_state(self):
+        """State written by the last step."""
+        return self.states[self.cur]
+
+    def attention(self, stream=None):
+        rc = self._lib.isd_attn_strided(ctypes.byref(self._attn),
+                                        isd._stream(stream))
+        if rc != isd.OK:
+            raise isd.IsdError(rc, "isd_attn_strided")
+
+    def accept(self, stream=None):
+        a = self._acc[self.cur]
+        a.step = self.step_idx & 0xFFFFFFFF
+        rc = self._lib.isd_accept_resample(ctypes.byref(a),
+                                           isd._stream(stream))
+        if rc != isd.OK:
+            raise isd.IsdError(rc, "isd_accept_resample")
+
+    def commit(self, stream=None):
+        rc = self._lib.isd_kv_commit(ctypes.byref(self._com),
+                                     isd._stream(stream))
+        if rc != isd.OK:
+            raise isd.IsdError(rc, "isd_kv_commit")
+
+    def advance(self):
+        self.cur ^= 1
+        self.step_idx += 1
+
+    def step(self, stream=None, events=None):
+        """Attention, accept/resample and commit; ``events`` (4 CUDA events)
+        are recorded around the three calls when given."""
+        s = stream if stream is not None else torch.cuda.current_stream()
+        if events:
+            events[0].record(s)
+        self.attention(s)
+        if events:
+            events[1].record(s)
+        self.accept(s)
+        if events:
+            events[2].record(s)
+        self.commit(s)
+        if events:
+            events[3].record(s)
+        self.advance()
+
+    # Kernel launches per step: attention + combine, four accept kernels,
+    # commit plan + copy.
+    LAUNCHES_PER_STEP = 8

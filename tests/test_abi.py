@@ -1,0 +1,123 @@
+"""The C ABI: libisd.so builds, loads and exports every symbol include/isd.h
+declares; host-side validation rejects bad arguments before any launch.
+These run without a GPU (no call here reaches a kernel or the device)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from introspective_strided_decoding_b200 import build, isd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "isd.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return isd.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w \*]*?\b(isd_\w+)\s*\(", text,
+                                 flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    fns = header_functions()
+    for name in ("isd_attn_strided", "isd_accept_resample", "isd_kv_commit",
+                 "isd_attn_workspace_bytes", "isd_accept_workspace_bytes",
+                 "isd_commit_workspace_bytes", "isd_abi_version",
+                 "isd_status_string"):
+        assert name in fns
+    assert set(fns) == set(isd.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", isd.lib_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (isd_\w+)", out))
+    for name in header_functions():
+        assert name in exported
+        assert getattr(lib, name) is not None
+
+
+def test_abi_version_and_status_strings(lib):
+    assert isd.abi_version() == 1
+    assert isd.status_string(isd.ERR_POOL_EXHAUSTED) == "KV page pool exhausted"
+    assert isd.status_string(12345) == "unknown status"
+
+
+def _attn_args(**kw):
+    base = dict(B=1, Hq=32, Hkv=8, d=128, K=8, num_pages=10,
+                page_table_stride=4, dtype=isd.BF16, softmax_scale=0.088,
+                num_ctas=0)
+    base.update(kw)
+    return isd.AttnArgs(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), isd.ERR_INVALID_ARG),
+    (dict(Hq=30), isd.ERR_INVALID_ARG),            # Hq % Hkv != 0
+    (dict(softmax_scale=0.0), isd.ERR_INVALID_ARG),
+    (dict(d=96), isd.ERR_UNSUPPORTED),              # bf16 path: d 64 or 128
+    (dict(K=6), isd.ERR_UNSUPPORTED),               # K*g = 24 rows
+    (dict(K=32, Hq=8), isd.ERR_UNSUPPORTED),        # K above a page
+    (dict(dtype=7), isd.ERR_INVALID_ARG),
+    (dict(dtype=isd.F32, d=48), isd.ERR_UNSUPPORTED),
+    (dict(), isd.ERR_INVALID_ARG),                  # null tensors
+])
+def test_attn_host_validation(lib, kw, code):
+    a = _attn_args(**kw)
+    assert lib.isd_attn_strided(ctypes.byref(a), None) == code
+
+
+def test_attn_workspace_query_rejects_bad_shapes(lib):
+    assert lib.isd_attn_workspace_bytes(ctypes.byref(_attn_args(d=96))) == 0
+    assert lib.isd_attn_workspace_bytes(None) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=1, K=2), isd.ERR_INVALID_ARG),
+    (dict(K=9), isd.ERR_INVALID_ARG),               # K must be 2N
+    (dict(N=17, K=34), isd.ERR_UNSUPPORTED),
+    (dict(V=0), isd.ERR_INVALID_ARG),
+    (dict(), isd.ERR_INVALID_ARG),                  # null tensors
+])
+def test_accept_host_validation(lib, kw, code):
+    base = dict(B=4, N=4, K=8, V=1024, dtype=isd.BF16, step=0, seed=0)
+    base.update(kw)
+    a = isd.AcceptArgs(**base)
+    assert lib.isd_accept_resample(ctypes.byref(a), None) == code
+
+
+def test_accept_rejects_in_place_state(lib):
+    fake = ctypes.c_void_p(0x10000)
+    a = isd.AcceptArgs(B=1, N=2, K=4, V=64, dtype=isd.F32, logits_cur=fake,
+                       logits_prev=fake, seq_len=fake, pending_in=fake,
+                       n_pending_in=fake, q_row_in=fake, q_stats_in=fake,
+                       pending_out=fake, n_pending_out=ctypes.c_void_p(0x20000),
+                       q_row_out=ctypes.c_void_p(0x30000),
+                       q_stats_out=ctypes.c_void_p(0x40000), n_commit=fake,
+                       commit_tokens=fake)
+    assert lib.isd_accept_resample(ctypes.byref(a), None) == isd.ERR_INVALID_ARG
+
+
+def test_commit_host_validation(lib):
+    a = isd.CommitArgs(B=2, K=8, Hkv=8, d=128, num_pages=4,
+                       page_table_stride=2, dtype=isd.BF16)
+    assert lib.isd_kv_commit(ctypes.byref(a), None) == isd.ERR_INVALID_ARG
+    a.d = 4                                          # 8-byte rows
+    assert lib.isd_kv_commit(ctypes.byref(a), None) == isd.ERR_UNSUPPORTED
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(isd, "_lib", None)
+    monkeypatch.setattr(isd, "_LIB_PATH", str(tmp_path / "libisd.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        isd.lib()
