@@ -71,8 +71,8 @@ CASES = [
     (synth.Workload("f32_v1000_scalar", B=8, Hq=32, Hkv=8, d=128, N=3,
                     L_lo=10, L_hi=90, V=1000, dtype="f32", sigma_p=2.0,
                     sigma_q=0.6), 8),
-    (synth.Workload("bf16_n8_p07", B=6, Hq=64, Hkv=8, d=128, N=8, L_lo=1000,
-                    L_hi=2000, V=151936, target_accept=0.7), 5),
+    (synth.Workload("bf16_n8_p07", B=32, Hq=64, Hkv=8, d=128, N=8, L_lo=1000,
+                    L_hi=2000, V=151936, target_accept=0.7), 6),
     (synth.C64.with_(steps=1), 3),
 ]
 
