@@ -187,6 +187,36 @@ size_t isd_accept_workspace_bytes(const isd_accept_args* a);
 int isd_accept_resample(const isd_accept_args* a, void* stream);
 
 /* ------------------------------------------------------------------------
+ * isd_accept_resample_static -- the same step as isd_accept_resample, for
+ * callers that cannot allocate device memory.  The paper's pages have no
+ * counterpart to this entry point: it exists for integration only.
+ *
+ * Some callers have no way to provide the workspace: a host program that
+ * links this C ABI directly and has no device allocator of its own (a
+ * cudaMalloc per call would synchronise the device and fragment memory), or
+ * a serving process whose framework has already reserved the device memory
+ * pool.  This entry point takes its scratch from a buffer of
+ * ISD_ACCEPT_STATIC_SCRATCH bytes compiled into the library; every GPU that
+ * loads the library holds that buffer until the process exits.  It calls no
+ * allocating routine.
+ *
+ * - `workspace` and `workspace_bytes` in *a are ignored; every other field
+ *   means what it means for isd_accept_resample, with the same results.
+ * - Problems whose isd_accept_workspace_bytes(a) exceeds
+ *   ISD_ACCEPT_STATIC_SCRATCH are rejected with ISD_ERR_WORKSPACE before any
+ *   launch (at N = 4 and V = 151 936 the limit admits about 3 300 sequences).
+ * - The first call on each device looks up the buffer's device address
+ *   (with that device current) and keeps it; make that first call before
+ *   any stream capture begins.
+ * - All calls on a device share the one buffer, which keeps the previous
+ *   call's contents (nothing needs clearing: each call writes every scratch
+ *   word before reading it).  Calls whose work may overlap on the GPU, such
+ *   as calls on two unordered streams, race on it: order them.
+ * ---------------------------------------------------------------------- */
+#define ISD_ACCEPT_STATIC_SCRATCH (4u << 20)
+int isd_accept_resample_static(const isd_accept_args* a, void* stream);
+
+/* ------------------------------------------------------------------------
  * isd_kv_commit -- copy the staged K/V of rows 0 .. n_commit[b]-1 to cache
  * positions L_b .. L_b + n_commit[b] - 1 and grow seq_len[b] by n_commit[b].
  * Rows >= n_commit[b] (rejected drafts, MASK rows) are never written: that

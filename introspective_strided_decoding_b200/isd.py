@@ -77,6 +77,8 @@ SIGNATURES = {
     "isd_accept_workspace_bytes": (ctypes.c_size_t,
                                    [ctypes.POINTER(AcceptArgs)]),
     "isd_accept_resample": (ctypes.c_int, [ctypes.POINTER(AcceptArgs), _VP]),
+    "isd_accept_resample_static": (ctypes.c_int,
+                                   [ctypes.POINTER(AcceptArgs), _VP]),
     "isd_commit_workspace_bytes": (ctypes.c_size_t,
                                    [ctypes.POINTER(CommitArgs)]),
     "isd_kv_commit": (ctypes.c_int, [ctypes.POINTER(CommitArgs), _VP]),
@@ -289,6 +291,24 @@ def accept_resample(logits_cur, logits_prev, seq_len, state_in, state_out,
         a.workspace_bytes = workspace.numel()
     _raise(lib().isd_accept_resample(ctypes.byref(a), _stream(stream)),
            "isd_accept_resample")
+
+
+ACCEPT_STATIC_SCRATCH = 4 << 20
+
+
+def accept_resample_static(logits_cur, logits_prev, seq_len, state_in,
+                           state_out, n_commit, commit_tokens, seed, step,
+                           row_stats=None, ratio=None, status=None,
+                           stream=None):
+    """isd_accept_resample_static: the accept step without a caller
+    workspace, for callers that cannot allocate device memory (its scratch
+    is a fixed buffer inside the library; see include/isd.h)."""
+    a = accept_args(logits_cur, logits_prev, seq_len, state_in, state_out,
+                    n_commit, commit_tokens, seed, step, None, row_stats,
+                    ratio, status)
+    _raise(lib().isd_accept_resample_static(ctypes.byref(a),
+                                            _stream(stream)),
+           "isd_accept_resample_static")
 
 
 # ------------------------------------------------------------------ commit
