@@ -259,6 +259,10 @@ def run_isd(args, world, rank, local):
         kv_bytes.append(kv)
         logit_rows.append(rows)
         n_in = dec.state["n_pending"].clone()
+        # A short device-side sleep ahead of the first event: the host
+        # queues the whole step while it runs, so the timed window holds
+        # the step's kernels and not the host's launch latency.
+        torch.cuda._sleep(100_000)
         dec.step(stream, ev[s])
         tok_dev += dec.n_commit.sum()
         # Drafts tested: the accepted ones plus the first rejected one.

@@ -181,6 +181,9 @@ typedef struct {
   int32_t* status;             /* optional                                */
   void* workspace;
   size_t workspace_bytes;
+  const uint32_t* step_dev;    /* optional: read the step index from device
+                                  memory instead of `step` (lets one
+                                  captured CUDA graph serve every step)    */
 } isd_accept_args;
 
 size_t isd_accept_workspace_bytes(const isd_accept_args* a);
@@ -204,7 +207,7 @@ int isd_accept_resample(const isd_accept_args* a, void* stream);
  *   means what it means for isd_accept_resample, with the same results.
  * - Problems whose isd_accept_workspace_bytes(a) exceeds
  *   ISD_ACCEPT_STATIC_SCRATCH are rejected with ISD_ERR_WORKSPACE before any
- *   launch (at N = 4 and V = 151 936 the limit admits about 3 300 sequences).
+ *   launch (at N = 4 and V = 151 936 the limit admits about 2 200 sequences).
  * - The first call on each device looks up the buffer's device address
  *   (with that device current) and keeps it; make that first call before
  *   any stream capture begins.

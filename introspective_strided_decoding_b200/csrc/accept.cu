@@ -17,8 +17,11 @@
 //             max(0, p - q)                                       [HBM bound]
 //   sample    grid (N, B): chunk located from the chunk masses, then a
 //             block-wide ordered scan inside the chunk
-// Fixed chunking and fixed reduction trees make every run bitwise
-// reproducible.
+// Element masses are fp32 (MUFU exp2 of exactly formed differences); every
+// sum that places a sampling boundary or normalises a probability is
+// accumulated in fp64 in a fixed order, so draws agree with an fp64
+// reference except within a few 1e-8 of a boundary, and every run is
+// bitwise reproducible.
 #include "common.cuh"
 
 namespace isd {
@@ -32,6 +35,7 @@ template <typename T>
 struct AcceptDev {
   int B, N, K, V, C, RU;
   uint32_t step;
+  const uint32_t* step_dev;  // when set, the step index is read from here
   uint64_t seed;
   const T* lc;
   const T* lp;
@@ -50,10 +54,12 @@ struct AcceptDev {
   float* ratio_out;
   int32_t* status;
   // workspace
-  float* chunk_stats;  // [B][RU][C][2]
-  float* rstats;       // [B][K][2]
+  double* csum;        // [B][RU][C] chunk sum of exp(l - chunk max)
+  double* rsum;        // [B][K] row normaliser s
+  double* resid;       // [B][C] residual chunk mass
+  float* cmax;         // [B][RU][C] chunk max
+  float* rmax;         // [B][K] row max m
   int32_t* decision;   // [B][4]: valid, rejected, a, n
-  float* resid;        // [B][C]
 };
 
 // Loads elements [idx, idx+8) of a row; out-of-range ones read as -inf.
@@ -69,6 +75,11 @@ ISD_DEV void load_row8(const T* row, int idx, int hi, float (&v)[8]) {
 }
 
 template <typename T>
+ISD_DEV uint32_t step_of(const AcceptDev<T>& p) {
+  return p.step_dev ? *p.step_dev : p.step;
+}
+
+template <typename T>
 ISD_DEV bool state_ok(const AcceptDev<T>& p, int b) {
   const int n = p.n_in[b];
   return (n == 1 || n == p.N) && p.seq_len[b] >= 0;
@@ -79,6 +90,7 @@ template <typename T, bool kVec>
 __global__ void __launch_bounds__(kAThreads)
     accept_stats_kernel(AcceptDev<T> p) {
   __shared__ float red[32];
+  __shared__ double redd[32];
   const int c = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
   if (!state_ok(p, b)) return;
   if (j >= p.n_in[b] + p.N - 1) return;
@@ -94,16 +106,19 @@ __global__ void __launch_bounds__(kAThreads)
 #pragma unroll
     for (int k = 0; k < 8; ++k) m = fmaxf(m, v[r][k]);
   m = block_reduce<true>(m, red);
-  float s = 0.0f;
+  double s = 0.0;
 #pragma unroll
-  for (int r = 0; r < kRounds; ++r)
+  for (int r = 0; r < kRounds; ++r) {
+    float t = 0.0f;  // 8 terms in fp32, then fp64 across groups
 #pragma unroll
-    for (int k = 0; k < 8; ++k) s += ex2((v[r][k] - m) * kLog2e);
-  s = block_reduce<false>(s, red);
+    for (int k = 0; k < 8; ++k) t += ex2((v[r][k] - m) * kLog2e);
+    s += (double)t;
+  }
+  s = block_sum(s, redd);
   if (threadIdx.x == 0) {
-    float* o = p.chunk_stats + (((size_t)b * p.RU + j) * p.C + c) * 2;
-    o[0] = m;
-    o[1] = s;
+    const size_t o = ((size_t)b * p.RU + j) * p.C + c;
+    p.cmax[o] = m;
+    p.csum[o] = s;
   }
 }
 
@@ -144,37 +159,40 @@ __global__ void __launch_bounds__(128) accept_decide_kernel(AcceptDev<T> p) {
   }
   // Row statistics: lane l merges the chunks of row l in a fixed order.
   const int rows_used = n + N - 1;
-  float m = 0.0f, s = 1.0f;
+  float m = 0.0f;
+  double s = 1.0;
   if (lane < rows_used) {
-    const float* cs = p.chunk_stats + ((size_t)b * p.RU + lane) * p.C * 2;
+    const size_t o = ((size_t)b * p.RU + lane) * p.C;
     m = -INFINITY;
-    for (int c = 0; c < p.C; ++c) m = fmaxf(m, cs[2 * c]);
-    s = 0.0f;
-    for (int c = 0; c < p.C; ++c) s += cs[2 * c + 1] * expf(cs[2 * c] - m);
-    p.rstats[(b * K + lane) * 2] = m;
-    p.rstats[(b * K + lane) * 2 + 1] = s;
+    for (int c = 0; c < p.C; ++c) m = fmaxf(m, p.cmax[o + c]);
+    s = 0.0;
+    for (int c = 0; c < p.C; ++c)
+      s += p.csum[o + c] * exp((double)(p.cmax[o + c] - m));
+    p.rmax[b * K + lane] = m;
+    p.rsum[b * K + lane] = s;
     if (p.row_stats_out) {
       p.row_stats_out[(b * K + lane) * 2] = m;
-      p.row_stats_out[(b * K + lane) * 2 + 1] = s;
+      p.row_stats_out[(b * K + lane) * 2 + 1] = (float)s;
     }
   }
   // Ratio test of drafts 1..n-1: lane i verifies draft i with row i-1.
+  // l - m is exact in fp32 (both are logits); p, q and the ratio in fp64.
   const float m_prev = __shfl_up_sync(0xffffffffu, m, 1);
-  const float s_prev = __shfl_up_sync(0xffffffffu, s, 1);
+  const double s_prev = __shfl_up_sync(0xffffffffu, s, 1);
   bool acc = true;
   if (lane >= 1 && lane < n) {
     const float lx = to_f(p.lc[((size_t)b * K + lane - 1) * p.V + tok]);
-    const float px = expf(lx - m_prev) / s_prev;
+    const double px = exp((double)(lx - m_prev)) / s_prev;
     const int qr = p.q_row_in[b * N + lane];
     const float mq = p.q_stats_in[(b * N + lane) * 2];
     const float sq = p.q_stats_in[(b * N + lane) * 2 + 1];
     const float lqx = to_f(p.lp[((size_t)b * K + qr) * p.V + tok]);
-    const float qx = expf(lqx - mq) / sq;
-    const float r = qx > 0.0f ? px / qx : INFINITY;
-    const float u = uniform(p.seed, (uint32_t)b, p.step, (uint32_t)(L + lane),
-                            ISD_STREAM_ACCEPT);
-    acc = u < r;
-    if (p.ratio_out) p.ratio_out[b * N + lane] = r;
+    const double qx = exp((double)(lqx - mq)) / (double)sq;
+    const double r = qx > 0.0 ? px / qx : INFINITY;
+    const float u = uniform(p.seed, (uint32_t)b, step_of(p),
+                            (uint32_t)(L + lane), ISD_STREAM_ACCEPT);
+    acc = (double)u < r;
+    if (p.ratio_out) p.ratio_out[b * N + lane] = (float)r;
   }
   const uint32_t mask = __ballot_sync(0xffffffffu, acc);
   const uint32_t drafts = ((n >= 32) ? 0xffffffffu : ((1u << n) - 1u)) & ~1u;
@@ -185,12 +203,12 @@ __global__ void __launch_bounds__(128) accept_decide_kernel(AcceptDev<T> p) {
   // Next drafts' q rows and their statistics (lane j reads row n + j - 1).
   const int src = min(n + lane - 1, 31);
   const float mq_next = __shfl_sync(0xffffffffu, m, src);
-  const float sq_next = __shfl_sync(0xffffffffu, s, src);
+  const double sq_next = __shfl_sync(0xffffffffu, s, src);
   if (lane < N) {
     const bool has = !rejected && lane >= 1;
     p.q_row_out[b * N + lane] = has ? n + lane - 1 : -1;
     p.q_stats_out[(b * N + lane) * 2] = has ? mq_next : 0.0f;
-    p.q_stats_out[(b * N + lane) * 2 + 1] = has ? sq_next : 0.0f;
+    p.q_stats_out[(b * N + lane) * 2 + 1] = has ? (float)sq_next : 0.0f;
   }
   if (lane == 0) {
     p.n_commit[b] = a + 1;
@@ -218,8 +236,8 @@ ISD_DEV ResidRows resid_rows(const AcceptDev<T>& p, int b, int a,
   prow = p.lc + ((size_t)b * K + a) * p.V;
   qrow = p.lp + ((size_t)b * K + qr) * p.V;
   ResidRows r;
-  r.mp = p.rstats[(b * K + a) * 2];
-  r.inv_sp = 1.0f / p.rstats[(b * K + a) * 2 + 1];
+  r.mp = p.rmax[b * K + a];
+  r.inv_sp = (float)(1.0 / p.rsum[b * K + a]);
   r.mq = p.q_stats_in[(b * N + a + 1) * 2];
   r.inv_sq = 1.0f / p.q_stats_in[(b * N + a + 1) * 2 + 1];
   return r;
@@ -228,24 +246,26 @@ ISD_DEV ResidRows resid_rows(const AcceptDev<T>& p, int b, int a,
 template <typename T, bool kVec>
 __global__ void __launch_bounds__(kAThreads)
     accept_residual_kernel(AcceptDev<T> p) {
-  __shared__ float red[32];
+  __shared__ double redd[32];
   const int c = blockIdx.x, b = blockIdx.y;
   const int32_t* dec = p.decision + b * 4;
   if (dec[0] == 0 || dec[1] == 0) return;
   const T *prow, *qrow;
   const ResidRows rr = resid_rows(p, b, dec[2], prow, qrow);
   const int lo = c * kChunk, hi = min(p.V, lo + kChunk);
-  float s = 0.0f;
+  double s = 0.0;
 #pragma unroll
   for (int r = 0; r < kRounds; ++r) {
     const int idx = lo + (r * kAThreads + threadIdx.x) * 8;
     float vp[8], vq[8];
     load_row8<T, kVec>(prow, idx, hi, vp);
     load_row8<T, kVec>(qrow, idx, hi, vq);
+    float t = 0.0f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) s += resid_w(rr, vp[k], vq[k]);
+    for (int k = 0; k < 8; ++k) t += resid_w(rr, vp[k], vq[k]);
+    s += (double)t;
   }
-  s = block_reduce<false>(s, red);
+  s = block_sum(s, redd);
   if (threadIdx.x == 0) p.resid[(size_t)b * p.C + c] = s;
 }
 
@@ -253,9 +273,9 @@ __global__ void __launch_bounds__(kAThreads)
 template <typename T, bool kVec>
 __global__ void __launch_bounds__(kAThreads)
     accept_sample_kernel(AcceptDev<T> p) {
-  __shared__ float sh[32];
+  __shared__ double sh[32];
   __shared__ int s_chunk, s_found, s_last;
-  __shared__ float s_target;
+  __shared__ double s_target;
   const int t = blockIdx.x, b = blockIdx.y;
   const int N = p.N, K = p.K;
   const int32_t* dec = p.decision + b * 4;
@@ -279,11 +299,11 @@ __global__ void __launch_bounds__(kAThreads)
   }
   const int C = p.C;
   if (mode == 0) {  // zero residual mass: draw from p instead
-    float W = 0.0f;
+    double W = 0.0;
     for (int c = 0; c < C; ++c) W += p.resid[(size_t)b * C + c];
-    if (!(W > 0.0f)) mode = 1;
+    if (!(W > 0.0)) mode = 1;
   }
-  const float u = uniform(p.seed, (uint32_t)b, p.step, pos, stream);
+  const float u = uniform(p.seed, (uint32_t)b, step_of(p), pos, stream);
   const T* prow = p.lc + ((size_t)b * K + row) * p.V;
   const T* qrow = nullptr;
   ResidRows rr{};
@@ -291,23 +311,24 @@ __global__ void __launch_bounds__(kAThreads)
   if (mode == 0) {
     rr = resid_rows(p, b, a, prow, qrow);
   } else {
-    m_row = p.rstats[(b * K + row) * 2];
+    m_row = p.rmax[b * K + row];
   }
-  // Locate the chunk (one thread, fixed order).
+  // Locate the chunk (one thread, fixed order, fp64).  Chunk masses are in
+  // units of exp(l - m_row) for p/q rows, probability units for residuals.
   if (threadIdx.x == 0) {
-    const float* cs = p.chunk_stats + ((size_t)b * p.RU + row) * C * 2;
-    float total = 0.0f;
-    for (int c = 0; c < C; ++c)
-      total += mode == 0 ? p.resid[(size_t)b * C + c]
-                         : cs[2 * c + 1] * expf(cs[2 * c] - m_row);
-    const float target = u * total;
-    float cum = 0.0f;
+    const size_t o = ((size_t)b * p.RU + row) * C;
+    auto mass = [&](int c) -> double {
+      return mode == 0 ? p.resid[(size_t)b * C + c]
+                       : p.csum[o + c] * exp((double)(p.cmax[o + c] - m_row));
+    };
+    double total = 0.0;
+    for (int c = 0; c < C; ++c) total += mass(c);
+    const double target = (double)u * total;
+    double cum = 0.0, rem = 0.0;
     int chosen = -1, last_pos = 0;
-    float rem = 0.0f;
     for (int c = 0; c < C; ++c) {
-      const float mc = mode == 0 ? p.resid[(size_t)b * C + c]
-                                 : cs[2 * c + 1] * expf(cs[2 * c] - m_row);
-      if (mc > 0.0f) last_pos = c;
+      const double mc = mass(c);
+      if (mc > 0.0) last_pos = c;
       if (chosen < 0 && cum + mc > target) { chosen = c; rem = target - cum; }
       cum += mc;
     }
@@ -319,38 +340,48 @@ __global__ void __launch_bounds__(kAThreads)
   }
   __syncthreads();
   const int c = s_chunk;
-  float rem = s_target;
+  double rem = s_target;
   const int lo = c * kChunk, hi = min(p.V, lo + kChunk);
+  // All four rounds' loads are issued before the scans.
+  float w[kRounds][8];
+#pragma unroll
+  for (int r = 0; r < kRounds; ++r)
+    load_row8<T, kVec>(prow, lo + (r * kAThreads + threadIdx.x) * 8, hi, w[r]);
+  if (mode == 0) {
+#pragma unroll
+    for (int r = 0; r < kRounds; ++r) {
+      float vq[8];
+      load_row8<T, kVec>(qrow, lo + (r * kAThreads + threadIdx.x) * 8, hi, vq);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w[r][k] = resid_w(rr, w[r][k], vq[k]);
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < kRounds; ++r)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w[r][k] = ex2((w[r][k] - m_row) * kLog2e);
+  }
   int my_last = -1;
+#pragma unroll
   for (int r = 0; r < kRounds; ++r) {
     const int idx = lo + (r * kAThreads + threadIdx.x) * 8;
-    float w[8];
-    load_row8<T, kVec>(prow, idx, hi, w);
-    if (mode == 0) {
-      float vq[8];
-      load_row8<T, kVec>(qrow, idx, hi, vq);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) w[k] = resid_w(rr, w[k], vq[k]);
-    } else {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) w[k] = ex2((w[k] - m_row) * kLog2e);
-    }
-    float own = 0.0f;
+    float own32 = 0.0f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      own += w[k];
-      if (w[k] > 0.0f) my_last = idx + k;
+      own32 += w[r][k];
+      if (w[r][k] > 0.0f) my_last = idx + k;
     }
-    float total, excl;
-    const float incl = block_inclusive_scan(own, sh, excl, total);
+    double total, excl;
+    const double incl = block_inclusive_scan<double>((double)own32, sh, excl,
+                                                     total);
     if (rem < total) {
       if (incl > rem && excl <= rem) {
-        float run = excl;
+        double run = excl;
         int pick = -1, lastp = -1;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          run += w[k];
-          if (w[k] > 0.0f) lastp = idx + k;
+          run += (double)w[r][k];
+          if (w[r][k] > 0.0f) lastp = idx + k;
           if (pick < 0 && run > rem) pick = idx + k;
         }
         atomicMax(&s_found, pick >= 0 ? pick : lastp);
@@ -372,14 +403,37 @@ __global__ void __launch_bounds__(kAThreads)
 // ---------------------------------------------------------------------------
 // Host-side launcher (called from the C ABI after validation).
 
+struct AcceptLayout {
+  size_t csum, rsum, resid, cmax, rmax, decision, total;
+};
+
+static AcceptLayout accept_layout(int B, int N, int K, int V) {
+  const size_t C = (V + kChunk - 1) / kChunk;
+  const size_t RU = 2 * N - 1;
+  AcceptLayout l;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = (off + bytes + 255) & ~size_t(255);
+    return at;
+  };
+  l.csum = take((size_t)B * RU * C * 8);
+  l.rsum = take((size_t)B * K * 8);
+  l.resid = take((size_t)B * C * 8);
+  l.cmax = take((size_t)B * RU * C * 4);
+  l.rmax = take((size_t)B * K * 4);
+  l.decision = take((size_t)B * 4 * 4);
+  l.total = off;
+  return l;
+}
+
 template <typename T>
-static int launch_accept_t(const isd_accept_args* a, float* ws_f,
-                           cudaStream_t st) {
+static int launch_accept_t(const isd_accept_args* a, cudaStream_t st) {
   AcceptDev<T> p;
   p.B = a->B; p.N = a->N; p.K = a->K; p.V = a->V;
   p.C = (a->V + kChunk - 1) / kChunk;
   p.RU = 2 * a->N - 1;
-  p.step = a->step; p.seed = a->seed;
+  p.step = a->step; p.step_dev = a->step_dev; p.seed = a->seed;
   p.lc = static_cast<const T*>(a->logits_cur);
   p.lp = static_cast<const T*>(a->logits_prev);
   p.seq_len = a->seq_len; p.pending_in = a->pending_in; p.n_in = a->n_pending_in;
@@ -388,11 +442,14 @@ static int launch_accept_t(const isd_accept_args* a, float* ws_f,
   p.q_row_out = a->q_row_out; p.q_stats_out = a->q_stats_out;
   p.n_commit = a->n_commit; p.commit_tokens = a->commit_tokens;
   p.row_stats_out = a->row_stats; p.ratio_out = a->ratio; p.status = a->status;
-  size_t off = 0;
-  p.chunk_stats = ws_f + off; off += (size_t)p.B * p.RU * p.C * 2;
-  p.rstats = ws_f + off; off += (size_t)p.B * p.K * 2;
-  p.resid = ws_f + off; off += (size_t)p.B * p.C;
-  p.decision = reinterpret_cast<int32_t*>(ws_f + off);
+  const AcceptLayout l = accept_layout(a->B, a->N, a->K, a->V);
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  p.csum = reinterpret_cast<double*>(ws + l.csum);
+  p.rsum = reinterpret_cast<double*>(ws + l.rsum);
+  p.resid = reinterpret_cast<double*>(ws + l.resid);
+  p.cmax = reinterpret_cast<float*>(ws + l.cmax);
+  p.rmax = reinterpret_cast<float*>(ws + l.rmax);
+  p.decision = reinterpret_cast<int32_t*>(ws + l.decision);
   const bool vec = (a->V % 8) == 0;
   dim3 g_stats(p.C, p.RU, p.B), g_res(p.C, p.B), g_samp(p.N, p.B);
   if (vec) {
@@ -410,16 +467,12 @@ static int launch_accept_t(const isd_accept_args* a, float* ws_f,
 }
 
 size_t accept_workspace_bytes(int B, int N, int K, int V) {
-  const size_t C = (V + kChunk - 1) / kChunk;
-  const size_t RU = 2 * N - 1;
-  size_t f = (size_t)B * RU * C * 2 + (size_t)B * K * 2 + (size_t)B * C;
-  return f * 4 + (size_t)B * 4 * 4 + 256;
+  return accept_layout(B, N, K, V).total;
 }
 
 int launch_accept(const isd_accept_args* a, cudaStream_t st) {
-  float* ws = static_cast<float*>(a->workspace);
-  if (a->dtype == ISD_BF16) return launch_accept_t<__nv_bfloat16>(a, ws, st);
-  return launch_accept_t<float>(a, ws, st);
+  if (a->dtype == ISD_BF16) return launch_accept_t<__nv_bfloat16>(a, st);
+  return launch_accept_t<float>(a, st);
 }
 
 }  // namespace isd

@@ -12,11 +12,11 @@
 // (sequence b, KV head h), one unit per cached page plus one tail unit for
 // the stride's own rows.  Each persistent CTA takes an equal contiguous
 // range of that list (no per-sequence imbalance, whatever the lengths).
-// Inside a CTA one producer warp walks the range and issues TMA loads of
-// each unit's K and V tiles (16 tokens x d, 128-byte swizzle) into a ring
-// of mbarrier-guarded stages; four consumer warps compute S = Q K^T and
-// O += P V with mma.sync m16n8k16 (bf16 in, fp32 accumulate) and an online
-// softmax in base 2.  All K*g query rows of a KV head share every K/V tile,
+// Inside a CTA four loader warps walk the range and copy each unit's K and
+// V tiles (16 tokens x d, 128-byte-swizzled layout) into a ring of
+// mbarrier-guarded stages with 16-byte cp.async; consumer warps compute
+// S = Q K^T and O += P V with mma.sync m16n8k16 (bf16 in, fp32 accumulate)
+// and an online softmax in base 2.  All K*g query rows of a KV head share every K/V tile,
 // which is read from HBM exactly once.  Consumer warps split the rows into
 // groups of 16*MW and, when rows are few, split the units of a segment
 // round-robin and merge through shared memory at the segment's end.  A
@@ -28,21 +28,23 @@
 
 namespace isd {
 
-constexpr int kCWarps = 4;                      // consumer warps
-constexpr int kAttnThreads = (kCWarps + 1) * 32;
-constexpr int kStages = 12;
+constexpr int kStages = 16;                     // power of two
 constexpr uint64_t kWaitCycles = 4000000000ull; // ~2 s at boost clock
 
 struct AttnDev {
   int B, Hq, Hkv, K, g, M, P, stride, RG, KS;
-  float scale_log2;
+  float scale_log2;   // softmax scale * log2(e)
   const __nv_bfloat16* q;
+  const __nv_bfloat16* kc;   // [P][Hkv][16][D]
+  const __nv_bfloat16* vc;
+  const __nv_bfloat16* kn;   // [B][K][Hkv][D]
+  const __nv_bfloat16* vn;
   __nv_bfloat16* out;
   float* lse;
   const int32_t* page_table;
   const int32_t* seq_len;
   int32_t* status;
-  float* part;        // [G][2][M][D + 2]
+  float* part;        // [G][2][M][D + 2]: unnormalised O, raw max, sum
   int32_t* ws_int;    // [B + 1] unit prefix, then G
 };
 
@@ -63,7 +65,7 @@ ISD_DEV int pages_of(const AttnDev& p, int b, bool* bad) {
   return n;
 }
 
-// Position of unit u: sequence b (prefix[b] <= u < prefix[b+1]).
+// Sequence b of unit u (prefix[b] <= u < prefix[b+1]).
 ISD_DEV int find_seq(const int* prefix, int B, int u) {
   int lo = 0, hi = B - 1;
   while (lo < hi) {
@@ -73,31 +75,25 @@ ISD_DEV int find_seq(const int* prefix, int B, int u) {
   return lo;
 }
 
-template <int D>
-ISD_DEV uint32_t swz(uint32_t base, int key, int chunk) {
-  // 128-byte swizzle of a [16 rows][64 cols] bf16 box; boxes of the d
-  // dimension are 2048 bytes apart.
-  return base + (chunk >> 3) * 2048 + key * 128 + (((chunk & 7) ^ (key & 7)) << 4);
-}
+// Threads per CTA: NW consumer warps + NL loader warps.
+template <int NW, int NL> constexpr int attn_threads() { return (NW + NL) * 32; }
 
-template <int D, int MW>
-__global__ void __launch_bounds__(kAttnThreads, 1)
-    attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_kc,
-                     const __grid_constant__ CUtensorMap tm_vc,
-                     const __grid_constant__ CUtensorMap tm_kn,
-                     const __grid_constant__ CUtensorMap tm_vn, AttnDev p) {
+template <int D, int MW, int NW, int NL>
+__global__ void __launch_bounds__(attn_threads<NW, NL>(), 1)
+    attn_bf16_kernel(AttnDev p) {
   constexpr int kTile = 16 * D * 2;            // one K or V tile, bytes
   constexpr int kStage = 2 * kTile;
   constexpr int RW = 16 * MW;                  // rows per consumer warp
-  constexpr int kRedRow = D + 4;
+  constexpr int kRedRow = D + 8;               // conflict-free float2 rows
   constexpr int kRedWarp = RW * kRedRow + 2 * RW;
+  constexpr int KK = D / 16;                   // k-steps of Q K^T
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages * kStage);
   uint64_t* empty = full + kStages;
   float* red = reinterpret_cast<float*>(empty + kStages);
-  int* prefix = reinterpret_cast<int*>(red + kCWarps * kRedWarp);
+  int* prefix = reinterpret_cast<int*>(red + NW * kRedWarp);
   __shared__ int scan_sh[33];
   __shared__ int s_bad;
 
@@ -120,7 +116,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int u1 = (int)(((long long)(c + 1) * T) / G);
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], NL * 32);
       mbar_init(&empty[s], p.RG);
     }
     fence_barrier_init();
@@ -135,32 +131,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   if (u0 >= u1) return;
 
-  // ------------------------------------------------------------- producer
-  // The whole warp resolves 32 units at a time (sequence, head, page id:
-  // one coalesced page-table load), prefetching the next 32 while lane 0
-  // issues the current ones, so no TMA waits on a dependent global load.
-  if (warp == kCWarps) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_kc);
-      tma_prefetch_desc(&tm_vc);
-      tma_prefetch_desc(&tm_kn);
-      tma_prefetch_desc(&tm_vn);
+  // --------------------------------------------------------------- loaders
+  // NL loader warps copy every unit's K and V tiles into the stage with
+  // 16-byte cp.async (many independent requests per SM: a 4 KB gather
+  // streams at HBM rate only with this much memory-level parallelism),
+  // writing the 128-byte-swizzled layout the consumers' ldmatrix expects.
+  // Each loader thread arrives on the stage's full barrier when its own
+  // copies land.  Units are resolved 32 at a time per warp (sequence,
+  // head, page id from one coalesced page-table load), one batch ahead.
+  if (warp >= NW) {
+    constexpr int kLT = NL * 32;
+    constexpr int kCPR = D / 8;                  // 16-byte chunks per row
+    constexpr int kCPT = 16 * kCPR;              // chunks per tile
+    constexpr int kPer = 2 * kCPT / kLT;         // chunks per thread per unit
+    static_assert((2 * kCPT) % kLT == 0, "loader split");
+    const int lt = tid - NW * 32;
+    uint32_t soff[kPer];
+    int srow[kPer], scol[kPer], sten[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int q = lt + i * kLT;
+      sten[i] = q / kCPT;
+      const int w = q - sten[i] * kCPT;
+      srow[i] = w / kCPR;
+      scol[i] = w - srow[i] * kCPR;
+      soff[i] = sten[i] * kTile + (scol[i] >> 3) * 2048 + srow[i] * 128 +
+                (((scol[i] & 7) ^ (srow[i] & 7)) << 4);
     }
     auto resolve = [&](int u, int& bb, int& hh, int& page) {
-      // page >= 0: cached page id; page == -1 - b marks the tail unit.
-      if (u >= u1) { bb = 0; hh = 0; page = 0; return; }
+      // page >= 0: cached page id; -1: the tail unit; -2: bad page id.
+      if (u >= u1) { bb = 0; hh = 0; page = -2; return; }
       bb = find_seq(prefix, B, u);
       const int units = (prefix[bb + 1] - prefix[bb]) / Hkv;
       const int rel = u - prefix[bb];
       hh = rel / units;
-      const int idx = rel % units;
+      const int idx = rel - hh * units;
       if (idx == units - 1) {
         page = -1;
       } else {
         page = p.page_table[(size_t)bb * p.stride + idx];
         if (page < 0 || page >= p.P) {
           if (p.status) *p.status = ISD_ERR_BAD_PAGE;
-          page = p.P;  // out of range: TMA fills zeros, no fault
+          page = -2;  // read as zeros
         }
       }
     };
@@ -174,34 +186,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int b = __shfl_sync(0xffffffffu, cb, j);
         const int h = __shfl_sync(0xffffffffu, ch, j);
         const int page = __shfl_sync(0xffffffffu, cp, j);
-        if (lane == 0) {
-          const int it = base - u0 + j;
-          const int s = it % kStages;
-          if (!failed && !wait_bounded(&empty[s], ((it / kStages) & 1) ^ 1)) {
-            failed = true;
-            if (p.status) *p.status = ISD_ERR_CUDA;
-          }
-          uint8_t* kdst = ring + s * kStage;
-          uint8_t* vdst = kdst + kTile;
-          mbar_arrive_expect_tx(&full[s], kStage);
-          if (page < 0) {  // tail: the stride's own rows (TMA zero-fills
-                           // rows >= K)
-#pragma unroll
-            for (int bi = 0; bi < D / 64; ++bi) {
-              tma_load_4d(kdst + bi * 2048, &tm_kn, &full[s], bi * 64, h, 0, b);
-              tma_load_4d(vdst + bi * 2048, &tm_vn, &full[s], bi * 64, h, 0, b);
-            }
-          } else {
-#pragma unroll
-            for (int bi = 0; bi < D / 64; ++bi) {
-              tma_load_4d(kdst + bi * 2048, &tm_kc, &full[s], bi * 64, 0, h,
-                          page);
-              tma_load_4d(vdst + bi * 2048, &tm_vc, &full[s], bi * 64, 0, h,
-                          page);
-            }
-          }
+        const int it = base - u0 + j;
+        const int s = it & (kStages - 1);
+        if (!failed && !wait_bounded(&empty[s], ((it / kStages) & 1) ^ 1)) {
+          failed = true;
+          if (p.status) *p.status = ISD_ERR_CUDA;
         }
-        __syncwarp();
+        const uint32_t stage = smem_u32(ring + s * kStage);
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+          const __nv_bfloat16* src;
+          uint32_t bytes = 16;
+          if (page >= 0) {
+            src = (sten[i] ? p.vc : p.kc) +
+                  (((size_t)page * Hkv + h) * kPage + srow[i]) * D + scol[i] * 8;
+          } else if (page == -1 && srow[i] < p.K) {
+            src = (sten[i] ? p.vn : p.kn) +
+                  (((size_t)b * p.K + srow[i]) * Hkv + h) * D + scol[i] * 8;
+          } else {
+            src = p.kc;  // tail rows >= K, bad page: zero-fill, nothing read
+            bytes = 0;
+          }
+          cp_async_16(stage + soff[i], src, bytes);
+        }
+        cp_async_arrive(&full[s]);
       }
       cb = nb; ch = nh; cp = np;
     }
@@ -210,16 +218,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   // ------------------------------------------------------------ consumers
   const int KS = p.KS;
-  const int rg = warp / KS, ks = warp % KS;
+  const int rg = warp / KS, ks = warp - (warp / KS) * KS;
   const int g = p.g, K = p.K, Hq = p.Hq;
+  const float c2 = p.scale_log2;
   float* my_red = red + warp * kRedWarp;
+  // Per-lane ldmatrix offsets inside a 16 x D tile (128-byte swizzle:
+  // 16-byte chunk index XOR row % 8; 64-column boxes 2048 bytes apart).
+  // K (non-transposed, B operand of Q K^T): matrices (keys 0-7 | 8-15) x
+  // (chunk 2kk | 2kk+1).  V (transposed, B operand of P V): matrices
+  // (keys 0-7 | 8-15) x (chunk 2np | 2np+1).
+  const int k_key = ((lane >> 4) << 3) + (lane & 7);
+  const int k_c0 = (lane >> 3) & 1;
+  const int v_key = (((lane >> 3) & 1) << 3) + (lane & 7);
+  const int v_c0 = lane >> 4;
+  const uint32_t k_row = k_key * 128, v_row = v_key * 128;
+  const int k_x = (k_key & 7), v_x = (v_key & 7);
   bool failed = false;
   int u = u0, it = 0;
   while (u < u1) {
     const int b = find_seq(prefix, B, u);
     const int units = (prefix[b + 1] - prefix[b]) / Hkv;
     const int rel = u - prefix[b];
-    const int h = rel / units, idx0 = rel % units;
+    const int h = rel / units, idx0 = rel - h * units;
     const int bh_end = prefix[b] + (h + 1) * units;
     const int seg_end = min(u1, bh_end);
     const int nseg = seg_end - u;
@@ -227,24 +247,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int npg = units - 1;
     const int L = p.seq_len[b];
 
-    // Q fragments of this warp's rows.
-    uint32_t qa[MW][D / 16][4];
+    // Q fragments of this warp's rows (A operand, row-major m16 x k16).
+    uint32_t qa[MW][KK][4];
     int rrow[MW][2];
 #pragma unroll
     for (int mt = 0; mt < MW; ++mt) {
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int m = rg * RW + mt * 16 + (lane >> 2) + hf * 8;
-        rrow[mt][hf] = m / g;
-      }
       const int m0 = rg * RW + mt * 16 + (lane >> 2);
       const int m1 = m0 + 8;
+      rrow[mt][0] = m0 / g;
+      rrow[mt][1] = m1 / g;
       const __nv_bfloat16* q0 =
           p.q + (((size_t)b * K + m0 / g) * Hq + h * g + m0 % g) * D;
       const __nv_bfloat16* q1 =
           p.q + (((size_t)b * K + m1 / g) * Hq + h * g + m1 % g) * D;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
+      for (int kk = 0; kk < KK; ++kk) {
         const int col = kk * 16 + 2 * (lane & 3);
         qa[mt][kk][0] = *reinterpret_cast<const uint32_t*>(q0 + col);
         qa[mt][kk][1] = *reinterpret_cast<const uint32_t*>(q1 + col);
@@ -264,10 +281,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       lrow[mt][0] = lrow[mt][1] = 0.0f;
     }
 
-    for (int k = 0; k < nseg; ++k) {
+    // This warp's units: k = first, first + KS, ... (unit it + k is owned
+    // by key split (it + k) % KS).
+    int first = (ks - it) % KS;
+    if (first < 0) first += KS;
+    for (int k = first; k < nseg; k += KS) {
       const int itk = it + k;
-      if (itk % KS != ks) continue;
-      const int s = itk % kStages;
+      const int s = itk & (kStages - 1);
       if (!failed && !wait_bounded(&full[s], (itk / kStages) & 1)) {
         failed = true;
         if (p.status) *p.status = ISD_ERR_CUDA;
@@ -275,87 +295,126 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int uidx = idx0 + k;
       const bool tail = uidx == npg;
       const int valid = tail ? K : min(kPage, L - uidx * kPage);
+      const bool masked = tail || valid < kPage;
       const uint32_t kb = smem_u32(ring + s * kStage);
       const uint32_t vb = kb + kTile;
 
-      // S = Q K^T over this tile's 16 keys.
-      float sc[MW][2][4];
+      // S = Q K^T for this tile's 16 keys; with 16-row warps the even and
+      // odd k-steps accumulate separately to halve the dependent-mma chains.
+      float sc[MW][2][4], sd[MW][2][4];
 #pragma unroll
       for (int mt = 0; mt < MW; ++mt)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sc[mt][nt][e] = 0.0f;
+          for (int e = 0; e < 4; ++e) sc[mt][nt][e] = sd[mt][nt][e] = 0.0f;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const int key = ((lane >> 4) << 3) + (lane & 7);
-        const int chunk = 2 * kk + ((lane >> 3) & 1);
+      for (int kk = 0; kk < KK; ++kk) {
+        const int chunk = 2 * kk + k_c0;
+        const uint32_t addr = kb + (chunk >> 3) * 2048 + k_row +
+                              (((chunk & 7) ^ k_x) << 4);
         uint32_t b0, b1, b2, b3;
-        ldmatrix_x4(swz<D>(kb, key, chunk), b0, b1, b2, b3);
+        ldmatrix_x4(addr, b0, b1, b2, b3);
 #pragma unroll
         for (int mt = 0; mt < MW; ++mt) {
-          mma_bf16_16816(sc[mt][0], qa[mt][kk], b0, b1);
-          mma_bf16_16816(sc[mt][1], qa[mt][kk], b2, b3);
+          if (MW == 1 && (kk & 1)) {
+            mma_bf16_16816(sd[mt][0], qa[mt][kk], b0, b1);
+            mma_bf16_16816(sd[mt][1], qa[mt][kk], b2, b3);
+          } else {
+            mma_bf16_16816(sc[mt][0], qa[mt][kk], b0, b1);
+            mma_bf16_16816(sc[mt][1], qa[mt][kk], b2, b3);
+          }
         }
       }
-      // Mask, online softmax (base 2), P as bf16 A fragments.
+      if (MW == 1) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[0][nt][e] += sd[0][nt][e];
+      }
+      if (masked) {
+        // Tail: row r sees stride rows 0..r; partial page: slots < valid.
+#pragma unroll
+        for (int mt = 0; mt < MW; ++mt)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int lim = tail ? min(valid - 1, rrow[mt][hf]) : valid - 1;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+              for (int e = 0; e < 2; ++e)
+                if (nt * 8 + 2 * (lane & 3) + e > lim)
+                  sc[mt][nt][hf * 2 + e] = -INFINITY;
+          }
+      }
+      // Online softmax in base 2 on raw scores: p = 2^(s*c - m*c).
+      bool grew = false;
+      float mnew[MW][2];
+#pragma unroll
+      for (int mt = 0; mt < MW; ++mt)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float mx = fmaxf(fmaxf(sc[mt][0][hf * 2], sc[mt][0][hf * 2 + 1]),
+                           fmaxf(sc[mt][1][hf * 2], sc[mt][1][hf * 2 + 1]));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          mnew[mt][hf] = fmaxf(mrow[mt][hf], mx);
+          grew |= mnew[mt][hf] > mrow[mt][hf];
+        }
+      if (__any_sync(0xffffffffu, grew)) {
+#pragma unroll
+        for (int mt = 0; mt < MW; ++mt)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const float alpha = ex2((mrow[mt][hf] - mnew[mt][hf]) * c2);
+            lrow[mt][hf] *= alpha;
+#pragma unroll
+            for (int nt = 0; nt < D / 8; ++nt) {
+              acc[mt][nt][hf * 2] *= alpha;
+              acc[mt][nt][hf * 2 + 1] *= alpha;
+            }
+            mrow[mt][hf] = mnew[mt][hf];
+          }
+      }
       uint32_t pa[MW][4];
 #pragma unroll
       for (int mt = 0; mt < MW; ++mt) {
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-          const int r = rrow[mt][hf];
-          float mx = -INFINITY;
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int key = nt * 8 + 2 * (lane & 3) + e;
-              const bool ok = key < valid && (!tail || key <= r);
-              float& x = sc[mt][nt][hf * 2 + e];
-              x = ok ? x * p.scale_log2 : -INFINITY;
-              mx = fmaxf(mx, x);
-            }
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-          const float mnew = fmaxf(mrow[mt][hf], mx);
-          const float alpha = ex2(mrow[mt][hf] - mnew);
-          mrow[mt][hf] = mnew;
+          const float off = mrow[mt][hf] * c2;
           float ls = 0.0f;
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               float& x = sc[mt][nt][hf * 2 + e];
-              x = ex2(x - mnew);
+              x = ex2(fmaf(x, c2, -off));
               ls += x;
             }
-          lrow[mt][hf] = lrow[mt][hf] * alpha + ls;
-#pragma unroll
-          for (int nt = 0; nt < D / 8; ++nt) {
-            acc[mt][nt][hf * 2] *= alpha;
-            acc[mt][nt][hf * 2 + 1] *= alpha;
-          }
+          lrow[mt][hf] += ls;
         }
         pa[mt][0] = pack_bf16(sc[mt][0][0], sc[mt][0][1]);
         pa[mt][1] = pack_bf16(sc[mt][0][2], sc[mt][0][3]);
         pa[mt][2] = pack_bf16(sc[mt][1][0], sc[mt][1][1]);
         pa[mt][3] = pack_bf16(sc[mt][1][2], sc[mt][1][3]);
       }
-      // Invalid V rows (unwritten slots of a partial page) may hold any
+      // O += P V.  V rows of unwritten slots (a partial page) may hold any
       // bits; zero them in the fragments so 0 * NaN cannot reach O.
-      const int k0 = 2 * (lane & 3);
-      const uint32_t mlo = (k0 < valid ? 0x0000FFFFu : 0u) |
-                           (k0 + 1 < valid ? 0xFFFF0000u : 0u);
-      const uint32_t mhi = (k0 + 8 < valid ? 0x0000FFFFu : 0u) |
-                           (k0 + 9 < valid ? 0xFFFF0000u : 0u);
-      // O += P V.
+      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+      if (masked) {
+        const int k0 = 2 * (lane & 3);
+        mlo = (k0 < valid ? 0x0000FFFFu : 0u) |
+              (k0 + 1 < valid ? 0xFFFF0000u : 0u);
+        mhi = (k0 + 8 < valid ? 0x0000FFFFu : 0u) |
+              (k0 + 9 < valid ? 0xFFFF0000u : 0u);
+      }
 #pragma unroll
       for (int np = 0; np < D / 16; ++np) {
-        const int key = (((lane >> 3) & 1) << 3) + (lane & 7);
-        const int chunk = 2 * np + (lane >> 4);
+        const int chunk = 2 * np + v_c0;
+        const uint32_t addr = vb + (chunk >> 3) * 2048 + v_row +
+                              (((chunk & 7) ^ v_x) << 4);
         uint32_t b0, b1, b2, b3;
-        ldmatrix_x4_trans(swz<D>(vb, key, chunk), b0, b1, b2, b3);
+        ldmatrix_x4_trans(addr, b0, b1, b2, b3);
         b0 &= mlo; b1 &= mhi; b2 &= mlo; b3 &= mhi;
 #pragma unroll
         for (int mt = 0; mt < MW; ++mt) {
@@ -401,7 +460,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             if (p.lse && (lane & 3) == 0)
               p.lse[((size_t)b * K + r) * Hq + h * g + j] =
-                  (mr + log2f(l)) * kLn2;
+                  (mr * c2 + log2f(l)) * kLn2;
           } else {
 #pragma unroll
             for (int nt = 0; nt < D / 8; ++nt) {
@@ -433,10 +492,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             my_red[RW * kRedRow + RW + rl] = lrow[mt][hf];
           }
         }
-      asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32));
+      asm volatile("bar.sync 1, %0;" ::"r"(NW * 32));
       const int cols = D / KS;
       for (int e = lane; e < RW * cols; e += 32) {
-        const int rl = e / cols, col = ks * cols + e % cols;
+        const int rl = e / cols, col = ks * cols + (e - rl * cols);
         float mstar = -INFINITY;
         for (int q2 = 0; q2 < KS; ++q2) {
           const float* rw = red + (rg * KS + q2) * kRedWarp;
@@ -446,7 +505,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int q2 = 0; q2 < KS; ++q2) {
           const float* rw = red + (rg * KS + q2) * kRedWarp;
           const float mq = rw[RW * kRedRow + rl];
-          const float wgt = mq == -INFINITY ? 0.0f : ex2(mq - mstar);
+          const float wgt = mq == -INFINITY ? 0.0f : ex2((mq - mstar) * c2);
           o += rw[rl * kRedRow + col] * wgt;
           l += rw[RW * kRedRow + RW + rl] * wgt;
         }
@@ -457,7 +516,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               __float2bfloat16_rn(o / l);
           if (p.lse && col == 0)
             p.lse[((size_t)b * K + r) * Hq + h * g + j] =
-                (mstar + log2f(l)) * kLn2;
+                (mstar * c2 + log2f(l)) * kLn2;
         } else {
           part[(size_t)m * D + col] = o;
           if (col == ks * cols) {
@@ -466,16 +525,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
       }
-      asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32));
+      asm volatile("bar.sync 1, %0;" ::"r"(NW * 32));
     }
     it += nseg;
     u = seg_end;
   }
 }
 
-// Merge the partials of every (b, h) whose units straddled CTAs.
+// Merge the partials of every (b, h) whose units straddled CTAs, in CTA
+// order.  The CTAs and slots holding them are listed once per block.
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(AttnDev p) {
+  extern __shared__ int s_part[];   // partial offsets (in floats)
+  __shared__ int s_n;
   const int h = blockIdx.x, b = blockIdx.y;
   const int B = p.B;
   const int* prefix = p.ws_int;
@@ -484,36 +546,42 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(AttnDev p) {
   const int units = (prefix[b + 1] - prefix[b]) / p.Hkv;
   const long long s = prefix[b] + (long long)h * units;
   const long long e = s + units;
-  auto cta_of = [&](long long uu) { return (int)(((uu + 1) * G - 1) / T); };
-  const int cf = cta_of(s), cl = cta_of(e - 1);
+  const int cf = (int)(((s + 1) * G - 1) / T);
+  const int cl = (int)(((e) * G - 1) / T);
   if (cf == cl) return;
   const int M = p.M, g = p.g, K = p.K, Hq = p.Hq;
-  for (int i = threadIdx.x; i < M * D; i += blockDim.x) {
-    const int m = i / D, col = i % D;
-    float mstar = -INFINITY;
+  if (threadIdx.x == 0) {
+    int n = 0;
     for (int cc = cf; cc <= cl; ++cc) {
       const long long u0 = ((long long)cc * T) / G;
       if (u0 == ((long long)(cc + 1) * T) / G) continue;  // empty range
       const int slot = (cc == cf && u0 != s) ? 1 : 0;
-      const float* part = p.part + ((size_t)(cc * 2 + slot)) * M * (D + 2);
-      mstar = fmaxf(mstar, part[(size_t)M * D + m]);
+      s_part[n++] = (cc * 2 + slot) * M * (D + 2);
     }
+    s_n = n;
+  }
+  __syncthreads();
+  const int n = s_n;
+  const float c2 = p.scale_log2;
+  for (int i = threadIdx.x; i < M * D; i += blockDim.x) {
+    const int m = i / D, col = i - m * D;
+    float mstar = -INFINITY;
+    for (int k = 0; k < n; ++k)
+      mstar = fmaxf(mstar, p.part[s_part[k] + M * D + m]);
     float o = 0.0f, l = 0.0f;
-    for (int cc = cf; cc <= cl; ++cc) {
-      const long long u0 = ((long long)cc * T) / G;
-      if (u0 == ((long long)(cc + 1) * T) / G) continue;  // empty range
-      const int slot = (cc == cf && u0 != s) ? 1 : 0;
-      const float* part = p.part + ((size_t)(cc * 2 + slot)) * M * (D + 2);
-      const float mq = part[(size_t)M * D + m];
-      const float w = mq == -INFINITY ? 0.0f : ex2(mq - mstar);
+    for (int k = 0; k < n; ++k) {
+      const float* part = p.part + s_part[k];
+      const float mq = part[M * D + m];
+      const float w = mq == -INFINITY ? 0.0f : ex2((mq - mstar) * c2);
       o += part[(size_t)m * D + col] * w;
-      l += part[(size_t)M * D + M + m] * w;
+      l += part[M * D + M + m] * w;
     }
     const int r = m / g, j = m % g;
     p.out[(((size_t)b * K + r) * Hq + h * g + j) * D + col] =
         __float2bfloat16_rn(o / l);
     if (p.lse && col == 0)
-      p.lse[((size_t)b * K + r) * Hq + h * g + j] = (mstar + log2f(l)) * kLn2;
+      p.lse[((size_t)b * K + r) * Hq + h * g + j] =
+          (mstar * c2 + log2f(l)) * kLn2;
   }
 }
 
@@ -581,9 +649,15 @@ __global__ void __launch_bounds__(128)
 // ---------------------------------------------------------------------------
 // Host side.
 
+// Consumer warps of each instantiation: 16-row warps (MW = 1) run eight
+// consumers (two per SM sub-partition); 32-row warps (MW = 2) run four.
+// Every instantiation adds kLoaderWarps loader warps.
+constexpr int nw_of(int MW) { return MW == 1 ? 8 : 4; }
+constexpr int kLoaderWarps = 4;
+
 size_t attn_smem_bytes(int D, int MW, int B) {
   const int RW = 16 * MW;
-  const size_t red = (size_t)kCWarps * (RW * (D + 4) + 2 * RW) * 4;
+  const size_t red = (size_t)nw_of(MW) * (RW * (D + 8) + 2 * RW) * 4;
   return 1024 + (size_t)kStages * 2 * (16 * D * 2) + 2 * kStages * 8 + red +
          (size_t)(B + 1) * 4;
 }
@@ -593,68 +667,22 @@ size_t attn_workspace_bytes_impl(int B, int M, int D, int G) {
   return ints + (size_t)G * 2 * M * (D + 2) * 4;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
-                                  void*, const cuuint64_t*, const cuuint64_t*,
-                                  const cuuint32_t*, const cuuint32_t*,
-                                  CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr,
-                                cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-static bool encode_4d(CUtensorMap* m, const void* base, const uint64_t dims[4],
-                      const uint64_t strides_bytes[3], const uint32_t box[4]) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (!fn) return false;
-  cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
-  cuuint64_t gs[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
-  cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
-  cuuint32_t es[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), gd,
-            gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int MW>
 static int launch_bf16(const isd_attn_args* a, int G, cudaStream_t st) {
-  CUtensorMap tkc, tvc, tkn, tvn;
-  const uint64_t es = 2;
-  const uint64_t dc[4] = {(uint64_t)D, (uint64_t)kPage, (uint64_t)a->Hkv,
-                          (uint64_t)a->num_pages};
-  const uint64_t sc[3] = {D * es, (uint64_t)kPage * D * es,
-                          (uint64_t)a->Hkv * kPage * D * es};
-  const uint32_t bc[4] = {64, (uint32_t)kPage, 1, 1};
-  const uint64_t dn[4] = {(uint64_t)D, (uint64_t)a->Hkv, (uint64_t)a->K,
-                          (uint64_t)a->B};
-  const uint64_t sn[3] = {D * es, (uint64_t)a->Hkv * D * es,
-                          (uint64_t)a->K * a->Hkv * D * es};
-  const uint32_t bn[4] = {64, 1, (uint32_t)kPage, 1};
-  if (!encode_4d(&tkc, a->k_cache, dc, sc, bc) ||
-      !encode_4d(&tvc, a->v_cache, dc, sc, bc) ||
-      !encode_4d(&tkn, a->k_new, dn, sn, bn) ||
-      !encode_4d(&tvn, a->v_new, dn, sn, bn))
-    return ISD_ERR_CUDA;
+  constexpr int NW = nw_of(MW);
+  constexpr int NL = kLoaderWarps;
   AttnDev p;
   p.B = a->B; p.Hq = a->Hq; p.Hkv = a->Hkv; p.K = a->K;
   p.g = a->Hq / a->Hkv; p.M = a->K * p.g; p.P = a->num_pages;
   p.stride = a->page_table_stride;
-  p.RG = p.M / (16 * MW); p.KS = kCWarps / p.RG;
+  p.RG = p.M / (16 * MW); p.KS = NW / p.RG;
+  if (p.KS < 1 || p.RG * p.KS != NW) return ISD_ERR_UNSUPPORTED;
   p.scale_log2 = a->softmax_scale * kLog2e;
   p.q = static_cast<const __nv_bfloat16*>(a->q);
+  p.kc = static_cast<const __nv_bfloat16*>(a->k_cache);
+  p.vc = static_cast<const __nv_bfloat16*>(a->v_cache);
+  p.kn = static_cast<const __nv_bfloat16*>(a->k_new);
+  p.vn = static_cast<const __nv_bfloat16*>(a->v_new);
   p.out = static_cast<__nv_bfloat16*>(a->out);
   p.lse = a->lse; p.page_table = a->page_table; p.seq_len = a->seq_len;
   p.status = a->status;
@@ -663,25 +691,20 @@ static int launch_bf16(const isd_attn_args* a, int G, cudaStream_t st) {
   p.part = reinterpret_cast<float*>(
       ws + (((size_t)(a->B + 2) * 4 + 255) & ~size_t(255)));
   const size_t smem = attn_smem_bytes(D, MW, a->B);
-  static bool attr_set[2] = {false, false};
-  static size_t attr_val[2] = {0, 0};
-  auto kern = attn_bf16_kernel<D, MW>;
-  const int slot = 0;
-  if (!attr_set[slot] || attr_val[slot] < smem) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return ISD_ERR_CUDA;
-    attr_set[slot] = true;
-    attr_val[slot] = smem;
-  }
-  kern<<<G, kAttnThreads, smem, st>>>(tkc, tvc, tkn, tvn, p);
-  attn_combine_kernel<D><<<dim3(a->Hkv, a->B), 256, 0, st>>>(p);
+  auto kern = attn_bf16_kernel<D, MW, NW, NL>;
+  // The shared-memory opt-in is per device; it is set on every call (a
+  // host-side attribute, no device work).
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return ISD_ERR_CUDA;
+  kern<<<G, attn_threads<NW, NL>(), smem, st>>>(p);
+  attn_combine_kernel<D><<<dim3(a->Hkv, a->B), 256, (size_t)G * 4, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? ISD_OK : ISD_ERR_CUDA;
 }
 
 int launch_attn_bf16(const isd_attn_args* a, int G, cudaStream_t st) {
   const int M = a->K * (a->Hq / a->Hkv);
-  const int MW = M == 16 ? 1 : 2;
+  const int MW = M <= 32 ? 1 : 2;
   if (a->d == 128) return MW == 1 ? launch_bf16<128, 1>(a, G, st)
                                   : launch_bf16<128, 2>(a, G, st);
   return MW == 1 ? launch_bf16<64, 1>(a, G, st) : launch_bf16<64, 2>(a, G, st);

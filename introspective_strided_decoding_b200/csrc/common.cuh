@@ -108,7 +108,7 @@ ISD_DEV float warp_sum(float v) {
   return v;
 }
 
-// Block-wide reduction; `red` holds >= 32 floats; all threads get the result.
+// Block-wide reduction; `red` holds >= 32 values; all threads get the result.
 template <bool kMax>
 ISD_DEV float block_reduce(float v, float* red) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -122,20 +122,34 @@ ISD_DEV float block_reduce(float v, float* red) {
   return r;
 }
 
-// Inclusive scan over the block of one float per thread (fixed order).
-// Returns the inclusive prefix; `excl` gets exactly the previous thread's
-// inclusive prefix (0 for thread 0) and `total` the block sum.  `sh` >= 32.
-ISD_DEV float block_inclusive_scan(float v, float* sh, float& excl,
-                                   float& total) {
+ISD_DEV double block_sum(double v, double* red) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int nw = (blockDim.x + 31) >> 5;
-  float x = v;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  double r = lane < nw ? red[lane] : 0.0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+  return r;
+}
+
+// Inclusive scan over the block of one value per thread (fixed order).
+// Returns the inclusive prefix; `excl` gets exactly the previous thread's
+// inclusive prefix (0 for thread 0) and `total` the block sum.  `sh` >= 32.
+template <typename T>
+ISD_DEV T block_inclusive_scan(T v, T* sh, T& excl, T& total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int nw = (blockDim.x + 31) >> 5;
+  T x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const float y = __shfl_up_sync(0xffffffffu, x, o);
+    const T y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  float prev = __shfl_up_sync(0xffffffffu, x, 1);
+  T prev = __shfl_up_sync(0xffffffffu, x, 1);
   __syncthreads();
   if (lane == 31) sh[wid] = x;
   __syncthreads();
@@ -145,8 +159,8 @@ ISD_DEV float block_inclusive_scan(float v, float* sh, float& excl,
     for (int w = 1; w < nw; ++w) sh[w] = sh[w - 1] + sh[w];
   __syncthreads();
   total = sh[nw - 1];
-  const float base = wid > 0 ? sh[wid - 1] : 0.0f;
-  if (lane == 0) prev = 0.0f;
+  const T base = wid > 0 ? sh[wid - 1] : T(0);
+  if (lane == 0) prev = T(0);
   // Apply the warp offset to both prefixes with the same single addition,
   // so thread i's excl equals thread i-1's result bit for bit.
   excl = (lane == 0) ? base : (wid > 0 ? base + prev : prev);
@@ -251,6 +265,21 @@ ISD_DEV void tma_load_4d(void* dst, const CUtensorMap* m, uint64_t* bar,
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1),
       "r"(c2), "r"(c3)
       : "memory");
+}
+
+// 16-byte asynchronous global -> shared copy (L2 only); `src_bytes` < 16
+// zero-fills the rest (0 reads nothing).
+ISD_DEV void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far completes
+// (counts as one of the barrier's expected arrivals).
+ISD_DEV void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
 }
 
 ISD_DEV void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,

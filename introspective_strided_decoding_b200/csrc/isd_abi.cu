@@ -48,7 +48,7 @@ int attn_check(const isd_attn_args* a) {
     if (a->d != 64 && a->d != 128) return ISD_ERR_UNSUPPORTED;
     if (!(M == 16 || M == 32 || M == 64 || M == 128)) return ISD_ERR_UNSUPPORTED;
     if (a->K > ISD_PAGE_SIZE) return ISD_ERR_UNSUPPORTED;
-    if (isd::attn_smem_bytes(a->d, M == 16 ? 1 : 2, a->B) > 227 * 1024)
+    if (isd::attn_smem_bytes(a->d, M <= 32 ? 1 : 2, a->B) > 227 * 1024)
       return ISD_ERR_UNSUPPORTED;
   } else if (a->dtype == ISD_F32) {
     if (a->d % 32 != 0 || a->d > 128) return ISD_ERR_UNSUPPORTED;

@@ -110,7 +110,7 @@ class Decoder:
 
     def accept(self, stream=None):
         a = self._acc[self.cur]
-        a.step = self.step_idx & 0xFFFFFFFF
+        a.step = self.step_idx & 0xFFFFFFFF  # unused once step_dev is set
         rc = self._lib.isd_accept_resample(ctypes.byref(a),
                                            isd._stream(stream))
         if rc != isd.OK:
@@ -141,6 +141,37 @@ class Decoder:
         self.commit(s)
         if events:
             events[3].record(s)
+        self.advance()
+
+    # ------------------------------------------------------ CUDA graphs
+    def capture(self, stream=None):
+        """Capture the step into two CUDA graphs, one per ping-pong parity
+        (the pages' serving stack replays a captured decode step; "Serving
+        (SGLang)" credits CUDA-graph capture with the largest gain).  The
+        accept call then reads the step index from a device counter that
+        the graph itself advances, so the same graph serves every step."""
+        dev = self.device
+        self.step_dev = torch.full((1,), self.step_idx, dtype=torch.int32,
+                                   device=dev)
+        for a in self._acc:
+            a.step_dev = ctypes.c_void_p(self.step_dev.data_ptr())
+        cur0 = self.cur
+        s = stream if stream is not None else torch.cuda.Stream(dev)
+        self.graphs = []
+        for parity in (0, 1):
+            self.cur = parity
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                self.attention()
+                self.accept()
+                self.commit()
+                self.step_dev.add_(1)
+            self.graphs.append(g)
+        self.cur = cur0
+
+    def replay(self):
+        """One step from the captured graph of the current parity."""
+        self.graphs[self.cur].replay()
         self.advance()
 
     # Kernel launches per step: attention + combine, four accept kernels,

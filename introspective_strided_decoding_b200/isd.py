@@ -56,7 +56,8 @@ class AcceptArgs(ctypes.Structure):
                 ("q_row_out", _VP), ("q_stats_out", _VP),
                 ("n_commit", _VP), ("commit_tokens", _VP),
                 ("row_stats", _VP), ("ratio", _VP), ("status", _VP),
-                ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t),
+                ("step_dev", _VP)]
 
 
 class CommitArgs(ctypes.Structure):
@@ -235,7 +236,7 @@ def new_state(B, N, device):
 
 def accept_args(logits_cur, logits_prev, seq_len, state_in, state_out,
                 n_commit, commit_tokens, seed, step, workspace=None,
-                row_stats=None, ratio=None, status=None):
+                row_stats=None, ratio=None, status=None, step_dev=None):
     B, K, V = logits_cur.shape
     N = K // 2
     dev, dt = logits_cur.device, logits_cur.dtype
@@ -255,6 +256,8 @@ def accept_args(logits_cur, logits_prev, seq_len, state_in, state_out,
         _check(ratio, "ratio", (B, N), torch.float32, dev)
     if status is not None:
         _check(status, "status", (1,), torch.int32, dev)
+    if step_dev is not None:
+        _check(step_dev, "step_dev", (1,), torch.int32, dev)
     return AcceptArgs(
         B=B, N=N, K=K, V=V, dtype=_dtype_code(logits_cur),
         step=int(step) & 0xFFFFFFFF, seed=int(seed) & 0xFFFFFFFFFFFFFFFF,
@@ -270,7 +273,8 @@ def accept_args(logits_cur, logits_prev, seq_len, state_in, state_out,
         row_stats=_ptr(row_stats), ratio=_ptr(ratio), status=_ptr(status),
         workspace=_ptr(workspace),
         workspace_bytes=0 if workspace is None else
-        workspace.numel() * workspace.element_size())
+        workspace.numel() * workspace.element_size(),
+        step_dev=_ptr(step_dev))
 
 
 def accept_workspace_bytes(args):
