@@ -702,7 +702,31 @@ static int launch_bf16(const isd_attn_args* a, int G, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? ISD_OK : ISD_ERR_CUDA;
 }
 
+// Merges the split-KV partials any attention kernel left in the workspace
+// (same partial layout for the mma.sync and the tcgen05 kernels).
+int launch_attn_combine(const isd_attn_args* a, int G, cudaStream_t st) {
+  AttnDev p{};
+  p.B = a->B; p.Hq = a->Hq; p.Hkv = a->Hkv; p.K = a->K;
+  p.g = a->Hq / a->Hkv; p.M = a->K * p.g;
+  p.scale_log2 = a->softmax_scale * kLog2e;
+  p.out = static_cast<__nv_bfloat16*>(a->out);
+  p.lse = a->lse;
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  p.ws_int = reinterpret_cast<int32_t*>(ws);
+  p.part = reinterpret_cast<float*>(
+      ws + (((size_t)(a->B + 2) * 4 + 255) & ~size_t(255)));
+  if (a->d == 128)
+    attn_combine_kernel<128><<<dim3(a->Hkv, a->B), 256, (size_t)G * 4, st>>>(p);
+  else
+    attn_combine_kernel<64><<<dim3(a->Hkv, a->B), 256, (size_t)G * 4, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ISD_OK : ISD_ERR_CUDA;
+}
+
+bool attn_tc_supported(const isd_attn_args* a);
+int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st);
+
 int launch_attn_bf16(const isd_attn_args* a, int G, cudaStream_t st) {
+  if (attn_tc_supported(a)) return launch_attn_tc(a, G, st);
   const int M = a->K * (a->Hq / a->Hkv);
   const int MW = M <= 32 ? 1 : 2;
   if (a->d == 128) return MW == 1 ? launch_bf16<128, 1>(a, G, st)
