@@ -91,9 +91,10 @@ enum { ISD_STREAM_ACCEPT = 0, ISD_STREAM_RESAMPLE = 1, ISD_STREAM_DRAFT = 2 };
  * Layouts: q, out [B][K][Hq][d]; k_new, v_new [B][K][Hkv][d];
  * k_cache, v_cache [num_pages][Hkv][16][d]; page_table int32
  * [B][page_table_stride]; seq_len int32 [B]; lse f32 [B][K][Hq] or NULL.
- * dtype ISD_BF16 (tensor-core path; d = 128 or 64, K * g a multiple of 16
- * and at most 128) or ISD_F32 (exact-fp32 SIMT path; d a multiple of 32,
- * at most 128).  `out` may not alias any input.
+ * dtype ISD_BF16 (tensor cores; K <= 16 and K * g <= 128; d = 128 runs on
+ * tcgen05 with any K * g, d = 64 on mma.sync with K * g one of 16, 32, 64,
+ * 128) or ISD_F32 (exact-fp32 SIMT path; d a multiple of 32, at most 128).
+ * `out` may not alias any input.
  * Workspace: isd_attn_workspace_bytes(args) bytes (split-KV partials);
  * its contents need no initialisation.  `status` (optional) receives
  * ISD_ERR_BAD_PAGE / ISD_ERR_PAGE_TABLE_FULL for malformed page tables;
@@ -148,6 +149,7 @@ int isd_attn_strided(const isd_attn_args* a, void* stream);
  *  of Philox4x32-10(key = (seed lo, seed hi), counter = (b, step, pos,
  *  stream)) (Salmon et al., SC'11).
  *
+ * Sizes: N <= 16, V <= 262 144 (otherwise ISD_ERR_UNSUPPORTED).
  * Layouts: logits_cur, logits_prev [B][K][V] (dtype); pending_*, q_row_*
  * int32 [B][N]; n_pending_* int32 [B]; q_stats_* f32 [B][N][2] (entry 0
  * unused); n_commit int32 [B]; commit_tokens int32 [B][N]; row_stats f32

@@ -313,30 +313,40 @@ __global__ void __launch_bounds__(kAThreads)
   } else {
     m_row = p.rmax[b * K + row];
   }
-  // Locate the chunk (one thread, fixed order, fp64).  Chunk masses are in
-  // units of exp(l - m_row) for p/q rows, probability units for residuals.
-  if (threadIdx.x == 0) {
+  // Locate the chunk: warp 0, one lane per chunk (C <= 32 is checked on
+  // the host), an inclusive fp64 scan in a fixed shuffle tree, so the
+  // choice is deterministic.  Chunk masses are in units of exp(l - m_row)
+  // for p/q rows, probability units for residuals.
+  if (threadIdx.x < 32) {
+    const int ln = threadIdx.x;
     const size_t o = ((size_t)b * p.RU + row) * C;
-    auto mass = [&](int c) -> double {
-      return mode == 0 ? p.resid[(size_t)b * C + c]
-                       : p.csum[o + c] * exp((double)(p.cmax[o + c] - m_row));
-    };
-    double total = 0.0;
-    for (int c = 0; c < C; ++c) total += mass(c);
-    const double target = (double)u * total;
-    double cum = 0.0, rem = 0.0;
-    int chosen = -1, last_pos = 0;
-    for (int c = 0; c < C; ++c) {
-      const double mc = mass(c);
-      if (mc > 0.0) last_pos = c;
-      if (chosen < 0 && cum + mc > target) { chosen = c; rem = target - cum; }
-      cum += mc;
+    double mc = 0.0;
+    if (ln < C)
+      mc = mode == 0 ? p.resid[(size_t)b * C + ln]
+                     : p.csum[o + ln] * exp((double)(p.cmax[o + ln] - m_row));
+    double incl = mc;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (ln >= off) incl += y;
     }
-    if (chosen < 0) { chosen = last_pos; rem = INFINITY; }
-    s_chunk = chosen;
-    s_target = rem;
-    s_found = -1;
-    s_last = -1;
+    const double total = __shfl_sync(0xffffffffu, incl, 31);
+    const double target = (double)u * total;
+    // Exclusive prefix = the previous lane's inclusive value, bit for bit.
+    double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (ln == 0) excl = 0.0;
+    // First chunk whose inclusive sum exceeds the target (rounding past
+    // the end: the last chunk with positive mass, scanned to its end).
+    const uint32_t hit = __ballot_sync(0xffffffffu, ln < C && incl > target);
+    const uint32_t pos = __ballot_sync(0xffffffffu, ln < C && mc > 0.0);
+    const int chosen = hit ? (__ffs(hit) - 1) : (pos ? 31 - __clz(pos) : 0);
+    const double ex_ch = __shfl_sync(0xffffffffu, excl, chosen);
+    if (ln == 0) {
+      s_chunk = chosen;
+      s_target = hit ? target - ex_ch : INFINITY;
+      s_found = -1;
+      s_last = -1;
+    }
   }
   __syncthreads();
   const int c = s_chunk;

@@ -12,11 +12,14 @@
 // per persistent CTA.  Inside a CTA the units of each (b, h) segment are
 // taken in blocks of up to kNB pages (16 * kNB keys).  Warp roles:
 //
-//   loaders (kLoadWarps)  16-byte cp.async of each block's K and V pages
-//                         into a stage, laid out as 128-byte-swizzled
-//                         K-major tiles (pages stacked along the key axis),
-//                         and of each segment's Q rows; every loader thread
-//                         arrives on the stage barrier when its copies land
+//   loaders (kLoadWarps)  each block's K pages through the TMA engine (one
+//                         thread, 64-column boxes) and its V pages with
+//                         16-byte cp.async from every loader thread, both
+//                         into 128-byte-swizzled tiles with the pages
+//                         stacked along the key axis; two copy engines run
+//                         in parallel.  Also each segment's Q rows.  The
+//                         stage barrier counts every loader thread's
+//                         cp.async arrival plus the TMA transaction bytes
 //   MMA warp              one thread issues S = Q K^T (M = 128 padded rows,
 //                         N = keys of the block, 8 k-steps) into a double-
 //                         buffered S in TMEM, and O += P V (one k-step per
@@ -227,7 +230,20 @@ struct BlockWalk {
   }
 };
 
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
+// R: replicas of the query rows in the 128-row tile (4 for up to 32 rows,
+// 2 for up to 64, 1 for 128).  With R > 1 every TMEM lane quarter holds a
+// copy of the rows, so all four softmax warps work on every block: warp w
+// takes 4/R pages of it for its 32 rows, the warps sharing rows exchange
+// row maxima, and P and O come out replicated, the output columns split
+// between the replicas.
+template <int R>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kc,
+                   const __grid_constant__ CUtensorMap tm_kn, Params p) {
+  constexpr int Mq = 128 / R;            // rows per replica (padded)
+  constexpr int QPR = Mq / 32;           // lane quarters per replica
+  constexpr int UPW = kNB / R;           // pages per softmax warp and block
+  constexpr int OPW = D / R;             // output columns per softmax warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -250,10 +266,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
   int* prefix = reinterpret_cast<int*>(tmem_slot + 4);
   __shared__ int scan_sh[33];
   __shared__ int s_bad;
+  __shared__ float x_max[2][kSmWarps][32];   // row-max exchange, per S buffer
+  __shared__ float x_sum[kSmWarps][32];      // row-sum exchange (epilogue)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int B = p.B, Hkv = p.Hkv, M = p.M;
-  const int active_sm = (M + 31) / 32;                 // softmax warps in use
+  const int active_sm = kSmWarps;                      // all take part
   if (tid == 0) s_bad = 0;
   __syncthreads();
   const int T = block_exclusive_scan_int(
@@ -274,7 +292,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
   const int u1 = (int)(((long long)(c + 1) * T) / G);
   if (tid == 0) {
     for (int s = 0; s < kStagesTc; ++s) {
-      mbar_init(&kv_full[s], kLoadThreads);
+      // Loader threads' cp.async arrivals (V) + one expect_tx arrival
+      // covering the TMA bytes (K).
+      mbar_init(&kv_full[s], kLoadThreads + 1);
       mbar_init(&kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -290,9 +310,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
     mbar_init(fin, 1);
     fence_barrier_init();
   }
-  // Q rows >= M stay zero for the whole kernel.
-  for (int i = tid; i < (128 - M) * 16; i += blockDim.x) {
-    const int row = M + i / 16, ch = i % 16;
+  // Padding rows of every replica (index within the replica >= M) stay
+  // zero for the whole kernel.
+  for (int i = tid; i < 128 * 16; i += blockDim.x) {
+    const int row = i / 16, ch = i % 16;
+    if (row % Mq < M) continue;
     *reinterpret_cast<uint4*>(qs + (ch >> 3) * kQHalf + row * 128 +
                               (((ch & 7) ^ (row & 7)) << 4)) =
         make_uint4(0, 0, 0, 0);
@@ -329,13 +351,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
       if (w.first()) {
         // Q rows of (b, h): row m = r * g + j holds q[b][r][h*g + j][:].
         wait_or_fail(q_empty, (nseg_done & 1) ^ 1, failed, p.status);
-        for (int q = lt; q < M * 16; q += kLoadThreads) {
-          const int m = q >> 4, ch = q & 15;
+        for (int q = lt; q < R * M * 16; q += kLoadThreads) {
+          const int rep = q / (M * 16), rem = q - rep * M * 16;
+          const int m = rem >> 4, ch = rem & 15;
           const int r = m / p.g, j = m - r * p.g;
+          const int row = rep * Mq + m;
           const __nv_bfloat16* src =
               p.q + (((size_t)w.b * p.K + r) * p.Hq + w.h * p.g + j) * D + ch * 8;
-          cp_async_16(q_s + (ch >> 3) * kQHalf + m * 128 +
-                          (((ch & 7) ^ (m & 7)) << 4),
+          cp_async_16(q_s + (ch >> 3) * kQHalf + row * 128 +
+                          (((ch & 7) ^ (row & 7)) << 4),
                       src, 16);
         }
         cp_async_arrive(q_full);
@@ -345,32 +369,54 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
       wait_or_fail(&kv_empty[st], ((i / kStagesTc) & 1) ^ 1, failed, p.status);
       const int nu = w.nu();
       const uint32_t sb = kv_s + st * kStageBytes;
+      uint8_t* sbp = kv + st * kStageBytes;
       const int Lb = p.seq_len[w.b];
-      for (int q = lt; q < nu * 512; q += kLoadThreads) {
-        const int k = q >> 9, ww = q & 511;
-        const int ten = ww >> 8, row = (ww >> 4) & 15, ch = ww & 15;
+      // K tiles through the TMA engine (one thread): two 64-column boxes per
+      // page, landing in the block's 128-byte-swizzled K-major halves.
+      // Rows past K of the tail lie outside the staging tensor and read as
+      // zeros, as does a page id out of range.
+      if (lt == 0) {
+        mbar_arrive_expect_tx(&kv_full[st], nu * 2 * 2048);
+        for (int k = 0; k < nu; ++k) {
+          const int uidx = w.idx0 + w.k + k;
+          if (uidx == w.units - 1) {
+            for (int hb = 0; hb < 2; ++hb)
+              tma_load_4d(sbp + hb * kHalf + k * 2048, &tm_kn, &kv_full[st],
+                          hb * 64, w.h, 0, w.b);
+          } else {
+            int page = p.page_table[(size_t)w.b * p.stride + uidx];
+            if (page < 0 || page >= p.P) {
+              if (p.status) *p.status = ISD_ERR_BAD_PAGE;
+              page = p.P;
+            }
+            for (int hb = 0; hb < 2; ++hb)
+              tma_load_4d(sbp + hb * kHalf + k * 2048, &tm_kc, &kv_full[st],
+                          hb * 64, 0, w.h, page);
+          }
+        }
+      }
+      // V tiles with cp.async from every loader thread.  Slots past L_b (a
+      // partial last page) are zero-filled, never copied: they may hold any
+      // bits, and 0 * NaN would reach O through P V.
+      for (int q = lt; q < nu * 256; q += kLoadThreads) {
+        const int k = q >> 8, ww = q & 255;
+        const int row = ww >> 4, ch = ww & 15;
         const int uidx = w.idx0 + w.k + k;
         const int key = k * 16 + row;
-        const uint32_t dst = sb + ten * 2 * kHalf + (ch >> 3) * kHalf +
-                             key * 128 + (((ch & 7) ^ (key & 7)) << 4);
-        const __nv_bfloat16* src = p.kc;
+        const uint32_t dst = sb + 2 * kHalf + (ch >> 3) * kHalf + key * 128 +
+                             (((ch & 7) ^ (key & 7)) << 4);
+        const __nv_bfloat16* src = p.vc;
         uint32_t bytes = 0;
         if (uidx == w.units - 1) {          // tail: the stride's own rows
           if (row < p.K) {
-            src = (ten ? p.vn : p.kn) +
-                  (((size_t)w.b * p.K + row) * Hkv + w.h) * D + ch * 8;
+            src = p.vn + (((size_t)w.b * p.K + row) * Hkv + w.h) * D + ch * 8;
             bytes = 16;
           }
         } else if (row < Lb - uidx * kPage) {
-          // Slots past L_b (a partial last page) are never copied: they
-          // may hold any bits, and 0 * NaN would reach O through P V.
           const int page = p.page_table[(size_t)w.b * p.stride + uidx];
           if (page >= 0 && page < p.P) {
-            src = (ten ? p.vc : p.kc) +
-                  (((size_t)page * Hkv + w.h) * kPage + row) * D + ch * 8;
+            src = p.vc + (((size_t)page * Hkv + w.h) * kPage + row) * D + ch * 8;
             bytes = 16;
-          } else if (p.status && row == 0 && ch == 0 && ten == 0) {
-            *p.status = ISD_ERR_BAD_PAGE;   // read as zeros
           }
         }
         cp_async_16(dst, src, bytes);
@@ -414,6 +460,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
       }
       wait_or_fail(&kv_full[st], (i / kStagesTc) & 1, failed, p.status);
       wait_or_fail(&s_free[sbuf], ((i >> 1) & 1) ^ 1, failed, p.status);
+      // Q and V arrived through cp.async (generic proxy); the tensor core
+      // reads them through the async proxy.
+      proxy_fence();
       tc_fence_after();
       const int nu = w.nu();
       if (lane == 0) {
@@ -449,17 +498,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
     __syncwarp();
     bool fin_failed = false;
     wait_or_fail(fin, 0, fin_failed, p.status);
-  } else if (warp < active_sm) {
+  } else if (warp < kSmWarps) {
     // ---------------------------------------------------------- softmax
-    const int row = warp * 32 + lane;                  // query row m
+    const int rep = warp / QPR;                        // replica of this warp
+    const int rbase = (warp % QPR) * 32;
+    const int row = rbase + lane;                      // query row m
     const bool real = row < M;
     const int rq = real ? row / p.g : 0, jq = real ? row - rq * p.g : 0;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const float c2 = p.scale_log2;
     BlockWalk w;
     w.init(prefix, B, Hkv, u0, u1);
-    int i = 0, nseg = 0;
-    float m_ref = -INFINITY, l = 0.0f;
+    int i = 0;
+    float m_ref = -INFINITY, l = 0.0f;                 // l: this warp's pages
     while (!w.done()) {
       const int sbuf = i & 1;
       const bool first = w.first();
@@ -468,12 +519,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
       const int L = p.seq_len[w.b];
       wait_or_fail(&s_full[sbuf], (i >> 1) & 1, failed, p.status);
       tc_fence_after();
-      float s[kBlockKeys];
+      float s[UPW * 16];
 #pragma unroll
-      for (int k = 0; k < kNB; ++k) {
-        if (k < nu) {
+      for (int k = 0; k < UPW; ++k) {
+        const int ku = rep * UPW + k;                  // page within block
+        if (ku < nu) {
           float v[16];
-          tmem_ld16(tmem + lane_base + 128 + sbuf * kBlockKeys + k * 16, v);
+          tmem_ld16(tmem + lane_base + 128 + sbuf * kBlockKeys + ku * 16, v);
 #pragma unroll
           for (int e = 0; e < 16; ++e) s[k * 16 + e] = v[e];
         } else {
@@ -488,9 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
       // unit stride rows after this row's own (causal inside the stride).
       float mx = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < kNB; ++k) {
-        if (k < nu) {
-          const int uidx = w.idx0 + w.k + k;
+      for (int k = 0; k < UPW; ++k) {
+        const int ku = rep * UPW + k;
+        if (ku < nu) {
+          const int uidx = w.idx0 + w.k + ku;
           const bool tail = uidx == w.units - 1;
           const int valid = tail ? min(p.K, rq + 1)
                                  : min(kPage, L - uidx * kPage);
@@ -502,17 +555,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
           }
         }
       }
+      if (R > 1) {
+        // Row max over the block: combine the R warps holding these rows.
+        x_max[sbuf][warp][lane] = mx;
+        asm volatile("bar.sync 1, %0;" ::"r"(kSmWarps * 32));
+#pragma unroll
+        for (int o = 0; o < R; ++o)
+          mx = fmaxf(mx, x_max[sbuf][(warp % QPR) + o * QPR][lane]);
+      }
       // Lazy rescale: move the reference max only when it grew by more
-      // than 2^kRescaleLog2 (or on the segment's first block).
+      // than 2^kRescaleLog2 (or on the segment's first block).  The warps
+      // sharing rows take the same decision (same maxima).
       bool need = (mx - m_ref) * c2 > kRescaleLog2;
       if (first) need = false;
       if (__any_sync(0xffffffffu, need)) {
-        // O must hold every earlier block's P V before it is scaled.
+        // O must hold every earlier block's P V before it is scaled; each
+        // warp scales the output columns it owns in its own lane quarter.
         wait_or_fail(o_done, (i - 1) & 1, failed, p.status);
         tc_fence_after();
         const float alpha = need ? ex2((m_ref - mx) * c2) : 1.0f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 16) {
+        for (int c0 = rep * OPW; c0 < (rep + 1) * OPW; c0 += 16) {
           float v[16];
           tmem_ld16(tmem + lane_base + c0, v);
 #pragma unroll
@@ -524,23 +587,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
         if (need) m_ref = mx;
       }
       if (first) m_ref = mx;
-      // P = 2^((s - m_ref) c) in bf16, one 128-byte row per thread.
+      // P = 2^((s - m_ref) c) in bf16 for this warp's pages, written into
+      // every replica of these rows.
       wait_or_fail(&p_empty[sbuf], ((i >> 1) & 1) ^ 1, failed, p.status);
       const float off = m_ref * c2;
-      uint8_t* prow = ps + sbuf * kPBytes + row * 128;
       float ls = 0.0f;
 #pragma unroll
-      for (int ch = 0; ch < kBlockKeys / 8; ++ch) {
-        uint32_t pk[4];
+      for (int k = 0; k < UPW; ++k) {
+        uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = ex2(fmaf(s[ch * 8 + 2 * e], c2, -off));
-          const float b2 = ex2(fmaf(s[ch * 8 + 2 * e + 1], c2, -off));
+        for (int e = 0; e < 8; ++e) {
+          const float a = ex2(fmaf(s[k * 16 + 2 * e], c2, -off));
+          const float b2 = ex2(fmaf(s[k * 16 + 2 * e + 1], c2, -off));
           ls += a + b2;
           pk[e] = pack_bf16(a, b2);
         }
-        *reinterpret_cast<uint4*>(prow + (((ch & 7) ^ (row & 7)) << 4)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        const int ch0 = (rep * UPW + k) * 2;           // 16-byte chunk
+#pragma unroll
+        for (int o = 0; o < R; ++o) {
+          const int trow = o * Mq + row;
+          uint8_t* prow = ps + sbuf * kPBytes + trow * 128;
+          *reinterpret_cast<uint4*>(prow + (((ch0 & 7) ^ (trow & 7)) << 4)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(
+              prow + ((((ch0 + 1) & 7) ^ (trow & 7)) << 4)) =
+              make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
       }
       l += ls;
       proxy_fence();
@@ -549,13 +621,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
       if (lane == 0) mbar_arrive(&p_full[sbuf]);
       if (w.last()) {
         // Epilogue: O of this segment is complete once its last P V lands.
+        float lt = l;
+        if (R > 1) {
+          x_sum[warp][lane] = l;
+          asm volatile("bar.sync 1, %0;" ::"r"(kSmWarps * 32));
+          lt = 0.0f;
+#pragma unroll
+          for (int o = 0; o < R; ++o) lt += x_sum[(warp % QPR) + o * QPR][lane];
+          asm volatile("bar.sync 1, %0;" ::"r"(kSmWarps * 32));
+        }
         wait_or_fail(o_done, i & 1, failed, p.status);
         tc_fence_after();
         const int slot = (w.seg_begin_u == u0) ? 0 : 1;
         float* part = p.part + ((size_t)(c * 2 + slot)) * M * (D + 2);
-        const float inv = 1.0f / l;
+        const float inv = 1.0f / lt;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 16) {
+        for (int c0 = rep * OPW; c0 < (rep + 1) * OPW; c0 += 16) {
           float v[16];
           tmem_ld16(tmem + lane_base + c0, v);
           if (real) {
@@ -578,20 +659,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
             }
           }
         }
-        if (real) {
+        if (real && rep == 0) {
           if (w.complete) {
             if (p.lse)
               p.lse[((size_t)w.b * p.K + rq) * p.Hq + w.h * p.g + jq] =
-                  (m_ref * c2 + log2f(l)) * kLn2;
+                  (m_ref * c2 + log2f(lt)) * kLn2;
           } else {
             part[(size_t)M * D + row] = m_ref;
-            part[(size_t)M * D + M + row] = l;
+            part[(size_t)M * D + M + row] = lt;
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(o_free);
-        ++nseg;
       }
       w.next();
       ++i;
@@ -610,6 +690,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Params p) {
 
 }  // namespace tc
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
+                                  void*, const cuuint64_t*, const cuuint64_t*,
+                                  const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr,
+                                cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+static bool encode_tiled_4d(CUtensorMap* m, const void* base,
+                            const uint64_t dims[4], const uint64_t strides[3],
+                            const uint32_t box[4]) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
+  cuuint64_t gs[3] = {strides[0], strides[1], strides[2]};
+  cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
+            gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 size_t attn_tc_smem_bytes(int B) {
   return 1024 + (size_t)tc::kStagesTc * tc::kStageBytes + tc::kQBytes +
          2 * tc::kPBytes + 32 * 8 + 16 + (size_t)(B + 1) * 4;
@@ -617,7 +736,7 @@ size_t attn_tc_smem_bytes(int B) {
 
 bool attn_tc_supported(const isd_attn_args* a) {
   const int M = a->K * (a->Hq / a->Hkv);
-  return a->dtype == ISD_BF16 && a->d == 128 && M % 16 == 0 && M <= 128 &&
+  return a->dtype == ISD_BF16 && a->d == 128 && M >= 1 && M <= 128 &&
          a->K <= kPage && attn_tc_smem_bytes(a->B) <= 227 * 1024;
 }
 
@@ -639,12 +758,30 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
   p.ws_int = reinterpret_cast<int32_t*>(ws);
   p.part = reinterpret_cast<float*>(
       ws + (((size_t)(a->B + 2) * 4 + 255) & ~size_t(255)));
+  // K tensor maps: the cache [P][Hkv][16][128] and the stride's staged
+  // rows [B][K][Hkv][128], 64-column boxes with the 128-byte swizzle.
+  CUtensorMap tkc, tkn;
+  const uint64_t dc[4] = {128, (uint64_t)kPage, (uint64_t)a->Hkv,
+                          (uint64_t)a->num_pages};
+  const uint64_t sc[3] = {256, (uint64_t)kPage * 256,
+                          (uint64_t)a->Hkv * kPage * 256};
+  const uint32_t bc[4] = {64, (uint32_t)kPage, 1, 1};
+  const uint64_t dn[4] = {128, (uint64_t)a->Hkv, (uint64_t)a->K,
+                          (uint64_t)a->B};
+  const uint64_t sn[3] = {256, (uint64_t)a->Hkv * 256,
+                          (uint64_t)a->K * a->Hkv * 256};
+  const uint32_t bn[4] = {64, 1, (uint32_t)kPage, 1};
+  if (!encode_tiled_4d(&tkc, a->k_cache, dc, sc, bc) ||
+      !encode_tiled_4d(&tkn, a->k_new, dn, sn, bn))
+    return ISD_ERR_CUDA;
   const size_t smem = attn_tc_smem_bytes(a->B);
-  if (cudaFuncSetAttribute(tc::attn_tc_kernel,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = p.M <= 32 ? tc::attn_tc_kernel<4>
+                        : (p.M <= 64 ? tc::attn_tc_kernel<2>
+                                     : tc::attn_tc_kernel<1>);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return ISD_ERR_CUDA;
-  tc::attn_tc_kernel<<<G, tc::kThreads, smem, st>>>(p);
+  kern<<<G, tc::kThreads, smem, st>>>(tkc, tkn, p);
   if (cudaGetLastError() != cudaSuccess) return ISD_ERR_CUDA;
   return launch_attn_combine(a, G, st);
 }

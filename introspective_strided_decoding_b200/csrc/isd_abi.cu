@@ -11,6 +11,7 @@ size_t commit_workspace_bytes(int B);
 int launch_commit(const isd_commit_args* a, cudaStream_t st);
 size_t attn_workspace_bytes_impl(int B, int M, int D, int G);
 size_t attn_smem_bytes(int D, int MW, int B);
+size_t attn_tc_smem_bytes(int B);
 int launch_attn_bf16(const isd_attn_args* a, int G, cudaStream_t st);
 int launch_attn_f32(const isd_attn_args* a, cudaStream_t st);
 }  // namespace isd
@@ -45,11 +46,18 @@ int attn_check(const isd_attn_args* a) {
   if (!(a->softmax_scale > 0.0f)) return ISD_ERR_INVALID_ARG;
   if (a->dtype == ISD_BF16) {
     const int M = a->K * (a->Hq / a->Hkv);
-    if (a->d != 64 && a->d != 128) return ISD_ERR_UNSUPPORTED;
-    if (!(M == 16 || M == 32 || M == 64 || M == 128)) return ISD_ERR_UNSUPPORTED;
-    if (a->K > ISD_PAGE_SIZE) return ISD_ERR_UNSUPPORTED;
-    if (isd::attn_smem_bytes(a->d, M <= 32 ? 1 : 2, a->B) > 227 * 1024)
+    if (a->K > ISD_PAGE_SIZE || M > 128) return ISD_ERR_UNSUPPORTED;
+    if (a->d == 128) {
+      // tcgen05 path: any row count up to 128 (rows padded to 128).
+      if (isd::attn_tc_smem_bytes(a->B) > 227 * 1024) return ISD_ERR_UNSUPPORTED;
+    } else if (a->d == 64) {
+      // mma.sync path: rows in warps of 16 or 32.
+      if (!(M == 16 || M == 32 || M == 64 || M == 128)) return ISD_ERR_UNSUPPORTED;
+      if (isd::attn_smem_bytes(a->d, M <= 32 ? 1 : 2, a->B) > 227 * 1024)
+        return ISD_ERR_UNSUPPORTED;
+    } else {
       return ISD_ERR_UNSUPPORTED;
+    }
   } else if (a->dtype == ISD_F32) {
     if (a->d % 32 != 0 || a->d > 128) return ISD_ERR_UNSUPPORTED;
   } else {
@@ -117,6 +125,7 @@ static int accept_check(const isd_accept_args* a) {
   if (a->B <= 0 || a->N < 2 || a->V <= 0 || a->K != 2 * a->N)
     return ISD_ERR_INVALID_ARG;
   if (a->N > 16) return ISD_ERR_UNSUPPORTED;
+  if (a->V > 32 * 8192) return ISD_ERR_UNSUPPORTED;  // at most 32 chunks
   if (a->dtype != ISD_BF16 && a->dtype != ISD_F32) return ISD_ERR_INVALID_ARG;
   return ISD_OK;
 }

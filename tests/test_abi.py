@@ -66,7 +66,8 @@ def _attn_args(**kw):
     (dict(Hq=30), isd.ERR_INVALID_ARG),            # Hq % Hkv != 0
     (dict(softmax_scale=0.0), isd.ERR_INVALID_ARG),
     (dict(d=96), isd.ERR_UNSUPPORTED),              # bf16 path: d 64 or 128
-    (dict(K=6), isd.ERR_UNSUPPORTED),               # K*g = 24 rows
+    (dict(K=6, d=64), isd.ERR_UNSUPPORTED),         # d 64: K*g = 24 rows
+    (dict(K=16, Hq=96, Hkv=8), isd.ERR_UNSUPPORTED),  # K*g = 192 rows
     (dict(K=32, Hq=8), isd.ERR_UNSUPPORTED),        # K above a page
     (dict(dtype=7), isd.ERR_INVALID_ARG),
     (dict(dtype=isd.F32, d=48), isd.ERR_UNSUPPORTED),

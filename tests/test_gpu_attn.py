@@ -39,6 +39,9 @@ SMALL = [
     _bf(name="bf16_m64", B=2, Hq=16, Hkv=2, L_lo=17, L_hi=260),
     _bf(name="bf16_m128", B=2, Hq=16, Hkv=2, N=8, L_lo=1, L_hi=300),
     _bf(name="bf16_m128_g4", B=2, Hq=8, Hkv=2, N=8, L_lo=30, L_hi=40),
+    _bf(name="bf16_m24", B=3, Hq=6, Hkv=2, N=4, L_lo=3, L_hi=140),
+    _bf(name="bf16_m48", B=2, Hq=12, Hkv=2, N=4, L_lo=40, L_hi=150),
+    _bf(name="bf16_m96", B=2, Hq=12, Hkv=2, N=8, L_lo=20, L_hi=90),
 ]
 
 
