@@ -10,37 +10,44 @@
 // Work split: the flat list of (sequence, KV head, page) units plus one
 // tail unit per (sequence, head) is cut into equal contiguous ranges, one
 // per persistent CTA.  Inside a CTA the units of each (b, h) segment are
-// taken in blocks of up to kNB pages (16 * kNB keys).  Warp roles:
+// taken in blocks of up to kNB = 8 pages: 128 keys.
 //
-//   loaders (kLoadWarps)  each block's K pages through the TMA engine (one
-//                         thread, 64-column boxes) and its V pages with
-//                         16-byte cp.async from every loader thread, both
-//                         into 128-byte-swizzled tiles with the pages
-//                         stacked along the key axis; two copy engines run
-//                         in parallel.  Also each segment's Q rows.  The
-//                         stage barrier counts every loader thread's
-//                         cp.async arrival plus the TMA transaction bytes
-//   MMA warp              one thread issues S = Q K^T (M = 128 padded rows,
-//                         N = keys of the block, 8 k-steps) into a double-
-//                         buffered S in TMEM, and O += P V (one k-step per
-//                         page) into O in TMEM; completion is committed to
-//                         mbarriers.  QK of block i+1 is issued before PV of
-//                         block i so the softmax of a block overlaps the
-//                         tensor core.  It also allocates and frees TMEM.
-//   softmax (4 warps)     one query row per thread: reads its S row from
-//                         TMEM, masks the tail / partial page, keeps the
-//                         running max and sum in registers, writes P (bf16)
-//                         to shared memory; O is rescaled in TMEM only when
-//                         a row's max grows by more than 2^8 (base 2), so
-//                         most blocks need no correction.  At a segment's
-//                         end it reads O, normalises and stores it (or a
-//                         partial for the combine kernel when the (b, h)
-//                         straddles CTAs).
+// Transposed products.  A decoding stride has few query rows per KV head
+// (M = K * g, often 32) and many keys, so the keys take the MMA's 128-row
+// side and the rows its N side (N = M rounded up to 32):
+//   S^T[key][row]  = K Q^T        (A = K tile, B = Q, both K-major)
+//   O^T[d][row]   += V^T P^T      (A = V tile read MN-major, B = P^T)
+// with S^T, O^T and the per-key partial row sums in TMEM.  No MMA row is
+// padding, and each block costs 16 MMAs whatever M is.
 //
-// Shared operands use the tensor cores' canonical 128-byte-swizzle layouts:
-// Q and K and P K-major (reduction dimension contiguous), V MN-major (head
-// dimension contiguous).  Every mbarrier wait is bounded; after one timeout
-// a thread records ISD_ERR_CUDA and stops waiting, so the kernel ends.
+// Warp roles:
+//   loaders (4 warps)   warp k copies pages k and k + 4 of every block: its
+//                       lane 0 issues the K and V pages through the TMA
+//                       engine (64-column boxes, 128-byte swizzle).  Four
+//                       issuing threads keep enough copies in flight to
+//                       saturate HBM; one does not.  A partial last page
+//                       takes V by cp.async so that its unused slots are
+//                       zero-filled.
+//                       Page ids are read one block ahead.  Also each
+//                       segment's Q rows (cp.async).
+//   MMA warp            one thread issues S^T of block i into a double-
+//                       buffered S in TMEM, then O^T += V^T P^T of block
+//                       i-1, and commits completion to mbarriers.  It also
+//                       allocates and frees TMEM.
+//   softmax (4 warps)   thread t owns key t of the block (TMEM lane t): it
+//                       masks its scores, writes P = 2^(s c - m_row c) in
+//                       bf16 into P^T, and adds P to its per-row partial
+//                       sums (TMEM).  The reference max m_row moves only
+//                       when some score of the block exceeds it by more
+//                       than 2^8 (a vote over the 128 threads); then the
+//                       exact block max is reduced across the threads and
+//                       O^T and the sums are rescaled.  At a segment's end
+//                       the sums are reduced over the keys and O^T / l is
+//                       stored (or a partial for the combine kernel when
+//                       the (b, h) straddles CTAs).
+//
+// Every mbarrier wait is bounded; after one timeout a thread records
+// ISD_ERR_CUDA and stops waiting, so the kernel ends.
 #include "common.cuh"
 
 namespace isd {
@@ -51,31 +58,27 @@ int launch_attn_combine(const isd_attn_args* a, int G, cudaStream_t st);
 namespace tc {
 
 constexpr int D = 128;
-constexpr int kNB = 4;                       // pages per block
-constexpr int kBlockKeys = 16 * kNB;         // 64
-constexpr int kStagesTc = 4;
-constexpr int kHalf = kBlockKeys * 128;      // one 64-column half, bytes
-constexpr int kStageBytes = 4 * kHalf;       // K0 K1 V0 V1 = 32 KB
-constexpr int kQHalf = 128 * 128;            // 128 rows x 128 B
-constexpr int kQBytes = 2 * kQHalf;          // 32 KB
-constexpr int kPBytes = 128 * 128;           // 128 rows x 64 keys bf16
+constexpr int kNB = 8;                       // pages per block
+constexpr int kKeys = kNB * kPage;           // 128 keys = TMEM lanes
+constexpr int kKH = kKeys * 128;             // one 64-column half of K or V
+constexpr int kStageBytes = 4 * kKH;         // K0 K1 V0 V1 = 64 KB
 constexpr int kSmWarps = 4;
 constexpr int kMmaWarp = 4;
-constexpr int kLoadWarps = 11;
-constexpr int kThreads = (kSmWarps + 1 + kLoadWarps) * 32;   // 512
+constexpr int kLoadWarps = 4;
+constexpr int kPagesPerLoader = kNB / kLoadWarps;
+constexpr int kThreads = (kSmWarps + 1 + kLoadWarps) * 32;   // 288
 constexpr int kLoadThreads = kLoadWarps * 32;
-constexpr uint32_t kTmemCols = 256;          // O: 0..127, S: 128..255
+constexpr int kMaxStages = 3;
+constexpr int kBarBytes = 32 * 8;            // mbarriers (2 * stages + 13)
+constexpr int kStaticSmem = 2048;            // __shared__ arrays, rounded up
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint64_t kWaitCycles = 400000000ull;   // ~0.2 s
 
 struct Params {
-  int B, Hq, Hkv, K, g, M, P, stride;
+  int B, Hq, Hkv, K, g, M, P, stride, stages;
   float scale_log2;
   const __nv_bfloat16* q;
-  const __nv_bfloat16* kc;
   const __nv_bfloat16* vc;
-  const __nv_bfloat16* kn;
-  const __nv_bfloat16* vn;
   __nv_bfloat16* out;
   float* lse;
   const int32_t* page_table;
@@ -94,11 +97,12 @@ ISD_DEV uint64_t sdesc(uint32_t start, uint32_t lbo, uint32_t sbo) {
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
          (2ull << 61);
 }
-ISD_DEV uint32_t idesc_bf16(int M, int N, int b_mn_major) {
-  // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B,
-  // A K-major, B K-major (0) or MN-major (1), N >> 3, M >> 4.
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+ISD_DEV uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
+  // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, each
+  // K-major (0) or MN-major (1), N >> 3, M >> 4.
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) |
+         ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
 }
 ISD_DEV void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id,
                   uint32_t accumulate) {
@@ -124,33 +128,43 @@ ISD_DEV void tc_fence_after() {
 ISD_DEV void proxy_fence() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// TMEM -> registers, 16 columns of this thread's lane.  The wait is tied
-// to the destination registers ("+r"), so no use can be scheduled before
-// the load has landed.
-ISD_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
+// TMEM -> registers, 32 columns of this thread's lane.  The wait is tied
+// to the destination registers so no use is scheduled before it.
+ISD_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,"
-      "%10,%11,%12,%13,%14,%15}, [%16];"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,"
+      "%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,"
+      "%27,%28,%29,%30,%31}, [%32];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
         "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
         "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15])
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;"
                : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]),
                  "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]),
                  "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-                 "+r"(r[14]), "+r"(r[15])
+                 "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+                 "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
                :
                : "memory");
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-ISD_DEV void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+// Registers -> TMEM, 32 columns of this thread's lane; waits until the
+// store has completed.
+ISD_DEV void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,"
-      "%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,"
+      "%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,"
+      "%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
       "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
       "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
       "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
@@ -158,11 +172,85 @@ ISD_DEV void tmem_st16(uint32_t taddr, const float (&v)[16]) {
       "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])),
       "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
       "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
+      "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])),
+      "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
+      "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
+      "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
-}
-ISD_DEV void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Scales 32 TMEM columns of this thread's lane by f[0..31] (shared
+// memory), 16 at a time.
+ISD_DEV void tmem_scale32(uint32_t taddr, const float* f) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,"
+        "%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
+          "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
+          "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15])
+        : "r"(taddr + h * 16));
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]),
+                   "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]),
+                   "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      r[e] = __float_as_uint(__uint_as_float(r[e]) * f[h * 16 + e]);
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,"
+        "%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr + h * 16),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]),
+        "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+  }
+}
+
+// Named barrier 1 joins the four softmax warps.
+ISD_DEV void sm_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// OR of `v` over the four softmax warps (also a barrier among them).
+ISD_DEV bool sm_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+      " bar.red.or.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+// v[c] of every lane combined over the warp; afterwards lane c holds the
+// result for column c in v[0].  Recursive halving: at distance o each lane
+// keeps the half of its columns selected by its bit o and trades the other
+// half with lane ^ o (31 shuffles in all).
+template <bool kMax>
+ISD_DEV void warp_transpose_reduce(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < o; ++j) {
+      const float send = upper ? v[j] : v[j + o];
+      const float keep = upper ? v[j + o] : v[j];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+      v[j] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
 }
 
 // Bounded wait; after the first timeout (`failed` set) waits are skipped.
@@ -230,48 +318,57 @@ struct BlockWalk {
   }
 };
 
-// R: replicas of the query rows in the 128-row tile (4 for up to 32 rows,
-// 2 for up to 64, 1 for 128).  With R > 1 every TMEM lane quarter holds a
-// copy of the rows, so all four softmax warps work on every block: warp w
-// takes 4/R pages of it for its 32 rows, the warps sharing rows exchange
-// row maxima, and P and O come out replicated, the output columns split
-// between the replicas.
-template <int R>
+// Byte offset of bf16 element (row, col) in a K-major tile of 64-column
+// halves (128-byte rows, 128-byte swizzle); `half` = bytes of one half.
+ISD_DEV uint32_t sw128_off(int row, int col, int half) {
+  return (uint32_t)((col >> 6) * half + row * 128 +
+                    ((((col >> 3) & 7) ^ (row & 7)) << 4) + (col & 7) * 2);
+}
+
+// NCH: 32-column chunks of the padded query rows (N = 32 * NCH).
+template <int NCH>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kc,
-                   const __grid_constant__ CUtensorMap tm_kn, Params p) {
-  constexpr int Mq = 128 / R;            // rows per replica (padded)
-  constexpr int QPR = Mq / 32;           // lane quarters per replica
-  constexpr int UPW = kNB / R;           // pages per softmax warp and block
-  constexpr int OPW = D / R;             // output columns per softmax warp
+                   const __grid_constant__ CUtensorMap tm_vc,
+                   const __grid_constant__ CUtensorMap tm_kn,
+                   const __grid_constant__ CUtensorMap tm_vn, Params p) {
+  constexpr int N = 32 * NCH;
+  constexpr int QH = N * 128;              // one 64-column half of Q
+  constexpr int PH = N * 128;              // one 64-key half of P^T
+  constexpr int PB = 2 * PH;               // one P^T buffer
+  constexpr int NPB = NCH == 4 ? 1 : 2;    // P^T buffers (one at N = 128)
+  constexpr uint32_t kO = 0, kS = N, kL = 3 * N;       // TMEM columns
+  constexpr uint32_t kCols = 4 * N <= 128 ? 128 : (4 * N <= 256 ? 256 : 512);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* kv = base;                                  // stages
-  uint8_t* qs = kv + kStagesTc * kStageBytes;          // Q tile
-  uint8_t* ps = qs + kQBytes;                          // 2 P tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + 2 * kPBytes);
-  uint64_t* kv_full = bars;                            // [kStagesTc]
-  uint64_t* kv_empty = kv_full + kStagesTc;            // [kStagesTc]
-  uint64_t* s_full = kv_empty + kStagesTc;             // [2]
+  const int S = p.stages;
+  uint8_t* kv = base;                                  // S stages
+  uint8_t* qs = kv + S * kStageBytes;                  // Q tile [N][128]
+  uint8_t* ps = qs + 2 * QH;                           // NPB P^T tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + NPB * PB);
+  uint64_t* kv_full = bars;                            // [S]
+  uint64_t* kv_empty = kv_full + S;                    // [S]
+  uint64_t* s_full = kv_empty + S;                     // [2]
   uint64_t* s_free = s_full + 2;                       // [2]
-  uint64_t* p_full = s_free + 2;                       // [2]
-  uint64_t* p_empty = p_full + 2;                      // [2]
+  uint64_t* p_full = s_free + 2;                       // [NPB]
+  uint64_t* p_empty = p_full + 2;                      // [NPB]
   uint64_t* q_full = p_empty + 2;
   uint64_t* q_empty = q_full + 1;
   uint64_t* o_done = q_empty + 1;
   uint64_t* o_free = o_done + 1;
   uint64_t* fin = o_free + 1;                          // all MMAs done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBarBytes / 8);
   int* prefix = reinterpret_cast<int*>(tmem_slot + 4);
   __shared__ int scan_sh[33];
   __shared__ int s_bad;
-  __shared__ float x_max[2][kSmWarps][32];   // row-max exchange, per S buffer
-  __shared__ float x_sum[kSmWarps][32];      // row-sum exchange (epilogue)
+  __shared__ __align__(16) float m_raw[N];    // reference max per row (raw)
+  __shared__ __align__(16) float m_sc[N];     // the same times c (-inf kept)
+  __shared__ float x_red[kSmWarps][32];       // cross-warp reduction
+  __shared__ __align__(16) float r_val[32];   // per-row factor of a chunk
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int B = p.B, Hkv = p.Hkv, M = p.M;
-  const int active_sm = kSmWarps;                      // all take part
   if (tid == 0) s_bad = 0;
   __syncthreads();
   const int T = block_exclusive_scan_int(
@@ -291,31 +388,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int u0 = (int)(((long long)c * T) / G);
   const int u1 = (int)(((long long)(c + 1) * T) / G);
   if (tid == 0) {
-    for (int s = 0; s < kStagesTc; ++s) {
-      // Loader threads' cp.async arrivals (V) + one expect_tx arrival
-      // covering the TMA bytes (K).
-      mbar_init(&kv_full[s], kLoadThreads + 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&kv_full[s], kLoadWarps);   // one arrival per loader warp
       mbar_init(&kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], active_sm);
-      mbar_init(&p_full[s], active_sm);
+      mbar_init(&s_free[s], kSmWarps);
+      mbar_init(&p_full[s], kSmWarps);
       mbar_init(&p_empty[s], 1);
     }
     mbar_init(q_full, kLoadThreads);
     mbar_init(q_empty, 1);
     mbar_init(o_done, 1);
-    mbar_init(o_free, active_sm);
+    mbar_init(o_free, kSmWarps);
     mbar_init(fin, 1);
     fence_barrier_init();
   }
-  // Padding rows of every replica (index within the replica >= M) stay
-  // zero for the whole kernel.
-  for (int i = tid; i < 128 * 16; i += blockDim.x) {
-    const int row = i / 16, ch = i % 16;
-    if (row % Mq < M) continue;
-    *reinterpret_cast<uint4*>(qs + (ch >> 3) * kQHalf + row * 128 +
+  // Padding rows of Q (M..N-1) stay zero for the whole kernel.
+  for (int i = tid; i < N * 16; i += blockDim.x) {
+    const int row = i >> 4, ch = i & 15;
+    if (row < M) continue;
+    *reinterpret_cast<uint4*>(qs + (ch >> 3) * QH + row * 128 +
                               (((ch & 7) ^ (row & 7)) << 4)) =
         make_uint4(0, 0, 0, 0);
   }
@@ -324,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile(
         "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::
             "r"(smem_u32(tmem_slot)),
-        "r"(kTmemCols));
+        "r"(kCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
@@ -343,86 +437,117 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp > kMmaWarp) {
     // ------------------------------------------------------------ loaders
+    // Loader warp lw copies pages lw and lw + 4 of every block; its lane 0
+    // issues their TMA boxes, so four threads keep copies in flight (one
+    // cannot saturate HBM).  Each warp registers its TMA bytes and then
+    // arrives once per stage on kv_full.
     const int lt = tid - (kMmaWarp + 1) * 32;
+    const int lw = lt >> 5;
     BlockWalk w;
     w.init(prefix, B, Hkv, u0, u1);
+    // Page ids of this warp's pages in the next block (-1: none or the
+    // tail) and its sequence length, read one block ahead: a copy must not
+    // wait on a page-table load issued just before it.
+    static_assert(kPagesPerLoader == 2, "two pages per loader warp");
+    int pid0 = -1, pid1 = -1, Lb = 0;
+    auto page_id = [&](int k) {
+      const int uidx = w.idx0 + w.k + k;
+      return (k < w.nu() && uidx != w.units - 1)
+                 ? __ldg(p.page_table + (size_t)w.b * p.stride + uidx)
+                 : -1;
+    };
+    auto load_ids = [&]() {
+      pid0 = page_id(lw);
+      pid1 = page_id(lw + kLoadWarps);
+      Lb = __ldg(p.seq_len + w.b);
+    };
+    if (!w.done()) load_ids();
     int i = 0, nseg_done = 0;
     while (!w.done()) {
       if (w.first()) {
         // Q rows of (b, h): row m = r * g + j holds q[b][r][h*g + j][:].
         wait_or_fail(q_empty, (nseg_done & 1) ^ 1, failed, p.status);
-        for (int q = lt; q < R * M * 16; q += kLoadThreads) {
-          const int rep = q / (M * 16), rem = q - rep * M * 16;
-          const int m = rem >> 4, ch = rem & 15;
+        for (int q = lt; q < M * 16; q += kLoadThreads) {
+          const int m = q >> 4, ch = q & 15;
           const int r = m / p.g, j = m - r * p.g;
-          const int row = rep * Mq + m;
           const __nv_bfloat16* src =
               p.q + (((size_t)w.b * p.K + r) * p.Hq + w.h * p.g + j) * D + ch * 8;
-          cp_async_16(q_s + (ch >> 3) * kQHalf + row * 128 +
-                          (((ch & 7) ^ (row & 7)) << 4),
+          cp_async_16(q_s + (ch >> 3) * QH + m * 128 +
+                          (((ch & 7) ^ (m & 7)) << 4),
                       src, 16);
         }
         cp_async_arrive(q_full);
         ++nseg_done;
       }
-      const int st = i % kStagesTc;
-      wait_or_fail(&kv_empty[st], ((i / kStagesTc) & 1) ^ 1, failed, p.status);
-      const int nu = w.nu();
-      const uint32_t sb = kv_s + st * kStageBytes;
-      uint8_t* sbp = kv + st * kStageBytes;
-      const int Lb = p.seq_len[w.b];
-      // K tiles through the TMA engine (one thread): two 64-column boxes per
-      // page, landing in the block's 128-byte-swizzled K-major halves.
-      // Rows past K of the tail lie outside the staging tensor and read as
-      // zeros, as does a page id out of range.
-      if (lt == 0) {
-        mbar_arrive_expect_tx(&kv_full[st], nu * 2 * 2048);
-        for (int k = 0; k < nu; ++k) {
-          const int uidx = w.idx0 + w.k + k;
-          if (uidx == w.units - 1) {
-            for (int hb = 0; hb < 2; ++hb)
-              tma_load_4d(sbp + hb * kHalf + k * 2048, &tm_kn, &kv_full[st],
-                          hb * 64, w.h, 0, w.b);
-          } else {
-            int page = p.page_table[(size_t)w.b * p.stride + uidx];
-            if (page < 0 || page >= p.P) {
-              if (p.status) *p.status = ISD_ERR_BAD_PAGE;
-              page = p.P;
-            }
-            for (int hb = 0; hb < 2; ++hb)
-              tma_load_4d(sbp + hb * kHalf + k * 2048, &tm_kc, &kv_full[st],
-                          hb * 64, 0, w.h, page);
-          }
-        }
-      }
-      // V tiles with cp.async from every loader thread.  Slots past L_b (a
-      // partial last page) are zero-filled, never copied: they may hold any
-      // bits, and 0 * NaN would reach O through P V.
-      for (int q = lt; q < nu * 256; q += kLoadThreads) {
-        const int k = q >> 8, ww = q & 255;
-        const int row = ww >> 4, ch = ww & 15;
+      const int st = i % S;
+      wait_or_fail(&kv_empty[st], ((i / S) & 1) ^ 1, failed, p.status);
+      uint64_t* bar = &kv_full[st];
+      bool partial_v = false;    // some page's V goes by cp.async
+#pragma unroll
+      for (int q = 0; q < kPagesPerLoader; ++q) {
+        const int k = lw + q * kLoadWarps;
+        if (k >= w.nu()) continue;
+        uint8_t* kd = kv + st * kStageBytes + k * 2048;   // K half 0, page k
+        uint8_t* vd = kd + 2 * kKH;                       // V half 0, page k
         const int uidx = w.idx0 + w.k + k;
-        const int key = k * 16 + row;
-        const uint32_t dst = sb + 2 * kHalf + (ch >> 3) * kHalf + key * 128 +
-                             (((ch & 7) ^ (key & 7)) << 4);
-        const __nv_bfloat16* src = p.vc;
-        uint32_t bytes = 0;
-        if (uidx == w.units - 1) {          // tail: the stride's own rows
-          if (row < p.K) {
-            src = p.vn + (((size_t)w.b * p.K + row) * Hkv + w.h) * D + ch * 8;
-            bytes = 16;
+        if (uidx == w.units - 1) {
+          // Tail: the stride's own K and V rows; rows past K lie outside
+          // the staging tensors and read as zeros.
+          if (lane == 0) {
+            mbar_expect_tx(bar, 4 * 2048);
+            for (int hb = 0; hb < 2; ++hb) {
+              tma_load_4d(kd + hb * kKH, &tm_kn, bar, hb * 64, w.h, 0, w.b);
+              tma_load_4d(vd + hb * kKH, &tm_vn, bar, hb * 64, w.h, 0, w.b);
+            }
           }
-        } else if (row < Lb - uidx * kPage) {
-          const int page = p.page_table[(size_t)w.b * p.stride + uidx];
-          if (page >= 0 && page < p.P) {
-            src = p.vc + (((size_t)page * Hkv + w.h) * kPage + row) * D + ch * 8;
-            bytes = 16;
+          continue;
+        }
+        int page = q == 0 ? pid0 : pid1;
+        const bool bad = page < 0 || page >= p.P;
+        if (bad) {
+          // Out of range: record it and read zeros (coordinate P lies
+          // outside the cache tensors).
+          if (lane == 0 && p.status) *p.status = ISD_ERR_BAD_PAGE;
+          page = p.P;
+        }
+        const int valid = Lb - uidx * kPage;   // >= 1 for a cached unit
+        const bool part = valid < kPage && !bad;
+        if (lane == 0) {
+          mbar_expect_tx(bar, (part ? 2 : 4) * 2048);
+          for (int hb = 0; hb < 2; ++hb) {
+            tma_load_4d(kd + hb * kKH, &tm_kc, bar, hb * 64, 0, w.h, page);
+            if (!part)
+              tma_load_4d(vd + hb * kKH, &tm_vc, bar, hb * 64, 0, w.h, page);
           }
         }
-        cp_async_16(dst, src, bytes);
+        if (part) {
+          // Partial last page: V slots past L_b are zero-filled, never
+          // copied (they may hold any bits, and 0 * NaN would reach O
+          // through P V).  K there is harmless: those scores are masked.
+          partial_v = true;
+          for (int e = lane; e < kPage * 16; e += 32) {
+            const int row = e >> 4, ch = e & 15;
+            const int key = k * kPage + row;
+            const uint32_t dst = kv_s + st * kStageBytes + 2 * kKH +
+                                 (ch >> 3) * kKH + key * 128 +
+                                 (((ch & 7) ^ (key & 7)) << 4);
+            const bool in = row < valid;
+            const __nv_bfloat16* src =
+                in ? p.vc + (((size_t)page * Hkv + w.h) * kPage + row) * D +
+                         ch * 8
+                   : p.vc;
+            cp_async_16(dst, src, in ? 16u : 0u);
+          }
+        }
       }
-      cp_async_arrive(&kv_full[st]);
+      if (partial_v) {
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        proxy_fence();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
       w.next();
+      if (!w.done()) load_ids();
       ++i;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
@@ -433,17 +558,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     int i = 0, nseg = 0;
     int prev_nu = 0, prev_st = 0, prev_pb = 0;
     bool prev_first = false, have_prev = false;
-    const uint32_t id_pv = idesc_bf16(128, D, 1);
+    const uint32_t id_qk = idesc_bf16(128, N, 0, 0);
+    const uint32_t id_pv = idesc_bf16(128, N, 1, 0);
     auto issue_pv = [&](int j_blk) {
-      // O += P V for block j_blk (its P buffer, stage and page count).
-      wait_or_fail(&p_full[prev_pb], (j_blk >> 1) & 1, failed, p.status);
+      // O^T += V^T P^T for block j_blk: one k-step of 16 keys per page.
+      wait_or_fail(&p_full[prev_pb], (j_blk / NPB) & 1, failed, p.status);
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t pa = p_s + prev_pb * kPBytes;
-        const uint32_t vb = kv_s + prev_st * kStageBytes + 2 * kHalf;
+        const uint32_t pa = p_s + prev_pb * PB;
+        const uint32_t vb = kv_s + prev_st * kStageBytes + 2 * kKH;
         for (int j = 0; j < prev_nu; ++j)
-          umma(tmem, sdesc(pa + j * 32, 16, 1024),
-               sdesc(vb + j * 2048, kHalf, 1024), id_pv,
+          umma(tmem + kO, sdesc(vb + j * 2048, kKH, 1024),
+               sdesc(pa + (j >> 2) * PH + (j & 3) * 32, 16, 1024), id_pv,
                (prev_first && j == 0) ? 0u : 1u);
         umma_commit(&kv_empty[prev_st]);
         umma_commit(&p_empty[prev_pb]);
@@ -453,25 +579,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     int seg_pv = 0;  // segments whose first PV has been issued
     while (!w.done()) {
-      const int st = i % kStagesTc, sbuf = i & 1;
+      const int st = i % S, sbuf = i & 1;
       if (w.first()) {
         wait_or_fail(q_full, nseg & 1, failed, p.status);
+        // Q arrived through cp.async (generic proxy); the tensor core
+        // reads it through the async proxy.  K and V came by TMA, or, for
+        // a partial page's V, by cp.async that its loader warp fenced.
+        proxy_fence();
         ++nseg;
       }
-      wait_or_fail(&kv_full[st], (i / kStagesTc) & 1, failed, p.status);
+      wait_or_fail(&kv_full[st], (i / S) & 1, failed, p.status);
       wait_or_fail(&s_free[sbuf], ((i >> 1) & 1) ^ 1, failed, p.status);
-      // Q and V arrived through cp.async (generic proxy); the tensor core
-      // reads them through the async proxy.
-      proxy_fence();
       tc_fence_after();
-      const int nu = w.nu();
       if (lane == 0) {
-        const uint32_t id_qk = idesc_bf16(128, 16 * nu, 0);
+        // S^T = K Q^T over the 128 keys of the stage (rows of pages past
+        // the block's end hold stale data; their scores are masked).
         const uint32_t kb = kv_s + st * kStageBytes;
         for (int kk = 0; kk < 8; ++kk)
-          umma(tmem + 128 + sbuf * kBlockKeys,
-               sdesc(q_s + (kk >> 2) * kQHalf + (kk & 3) * 32, 16, 1024),
-               sdesc(kb + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024), id_qk,
+          umma(tmem + kS + sbuf * N,
+               sdesc(kb + (kk >> 2) * kKH + (kk & 3) * 32, 16, 1024),
+               sdesc(q_s + (kk >> 2) * QH + (kk & 3) * 32, 16, 1024), id_qk,
                kk > 0 ? 1u : 0u);
         umma_commit(&s_full[sbuf]);
         if (w.last()) umma_commit(q_empty);
@@ -484,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_pv(i - 1);
       }
       have_prev = true;
-      prev_nu = nu; prev_st = st; prev_pb = sbuf; prev_first = w.first();
+      prev_nu = w.nu(); prev_st = st; prev_pb = i % NPB; prev_first = w.first();
       w.next();
       ++i;
     }
@@ -498,175 +625,175 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     bool fin_failed = false;
     wait_or_fail(fin, 0, fin_failed, p.status);
-  } else if (warp < kSmWarps) {
+  } else {
     // ---------------------------------------------------------- softmax
-    const int rep = warp / QPR;                        // replica of this warp
-    const int rbase = (warp % QPR) * 32;
-    const int row = rbase + lane;                      // query row m
-    const bool real = row < M;
-    const int rq = real ? row / p.g : 0, jq = real ? row - rq * p.g : 0;
+    const int kl = tid;                       // key of the block = TMEM lane
+    const int kp = kl >> 4, rr = kl & 15;     // its page and slot
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const float c2 = p.scale_log2;
     BlockWalk w;
     w.init(prefix, B, Hkv, u0, u1);
-    int i = 0;
-    float m_ref = -INFINITY, l = 0.0f;                 // l: this warp's pages
+    int i = 0, L = 0;
     while (!w.done()) {
       const int sbuf = i & 1;
       const bool first = w.first();
-      if (first) { m_ref = -INFINITY; l = 0.0f; }
-      const int nu = w.nu();
-      const int L = p.seq_len[w.b];
+      if (first) L = __ldg(p.seq_len + w.b);
+      // Which rows may see this thread's key: every row for a cached slot
+      // inside the prefix; rows at stride position >= rr for stride row rr
+      // of the tail (columns col >= rr * g); none past the block's end.
+      const int uidx = w.idx0 + w.k + kp;
+      const bool in_blk = kp < w.nu();
+      const bool tail = in_blk && uidx == w.units - 1;
+      const bool key_all = in_blk && !tail && rr < L - uidx * kPage;
+      const int col_min =
+          (tail && rr < p.K) ? rr * p.g : (key_all ? 0 : (1 << 30));
       wait_or_fail(&s_full[sbuf], (i >> 1) & 1, failed, p.status);
       tc_fence_after();
-      float s[UPW * 16];
-#pragma unroll
-      for (int k = 0; k < UPW; ++k) {
-        const int ku = rep * UPW + k;                  // page within block
-        if (ku < nu) {
-          float v[16];
-          tmem_ld16(tmem + lane_base + 128 + sbuf * kBlockKeys + ku * 16, v);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) s[k * 16 + e] = v[e];
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) s[k * 16 + e] = -INFINITY;
+      const int pbi = i % NPB;
+      wait_or_fail(&p_empty[pbi], ((i / NPB) & 1) ^ 1, failed, p.status);
+      bool o_ready = false;
+      uint8_t* pt = ps + pbi * PB;
+#pragma unroll 1
+      for (int ch = 0; ch < NCH; ++ch) {
+        float s[32];
+        tmem_ld32(tmem + lane_base + kS + sbuf * N + ch * 32, s);
+        if (ch == NCH - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_free[sbuf]);
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sbuf]);
-      // Mask: keys past the valid slots of a partial page, and for the tail
-      // unit stride rows after this row's own (causal inside the stride).
-      float mx = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < UPW; ++k) {
-        const int ku = rep * UPW + k;
-        if (ku < nu) {
-          const int uidx = w.idx0 + w.k + ku;
-          const bool tail = uidx == w.units - 1;
-          const int valid = tail ? min(p.K, rq + 1)
-                                 : min(kPage, L - uidx * kPage);
+        for (int e = 0; e < 32; ++e)
+          s[e] = (ch * 32 + e >= col_min) ? s[e] : -INFINITY;
+        // Vote: does any score exceed its row's reference by 2^8?  (A row
+        // with reference -inf votes yes on any unmasked score.)
+        bool need = first;
+        if (!first) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float& x = s[k * 16 + e];
-            x = e < valid ? x : -INFINITY;
-            mx = fmaxf(mx, x);
+          for (int e = 0; e < 32; e += 4) {
+            const float4 m4 =
+                *reinterpret_cast<const float4*>(&m_sc[ch * 32 + e]);
+            const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              need |= s[e + u] != -INFINITY &&
+                      fmaf(s[e + u], c2, -mm[u]) > kRescaleLog2;
           }
         }
-      }
-      if (R > 1) {
-        // Row max over the block: combine the R warps holding these rows.
-        x_max[sbuf][warp][lane] = mx;
-        asm volatile("bar.sync 1, %0;" ::"r"(kSmWarps * 32));
+        if (sm_any(need)) {
+          // Exact block max per row, then move the references.
+          float v[32];
 #pragma unroll
-        for (int o = 0; o < R; ++o)
-          mx = fmaxf(mx, x_max[sbuf][(warp % QPR) + o * QPR][lane]);
-      }
-      // Lazy rescale: move the reference max only when it grew by more
-      // than 2^kRescaleLog2 (or on the segment's first block).  The warps
-      // sharing rows take the same decision (same maxima).
-      bool need = (mx - m_ref) * c2 > kRescaleLog2;
-      if (first) need = false;
-      if (__any_sync(0xffffffffu, need)) {
-        // O must hold every earlier block's P V before it is scaled; each
-        // warp scales the output columns it owns in its own lane quarter.
-        wait_or_fail(o_done, (i - 1) & 1, failed, p.status);
-        tc_fence_after();
-        const float alpha = need ? ex2((m_ref - mx) * c2) : 1.0f;
-#pragma unroll 1
-        for (int c0 = rep * OPW; c0 < (rep + 1) * OPW; c0 += 16) {
-          float v[16];
-          tmem_ld16(tmem + lane_base + c0, v);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] *= alpha;
-          tmem_st16(tmem + lane_base + c0, v);
-          tmem_st_wait();
+          for (int e = 0; e < 32; ++e) v[e] = s[e];
+          warp_transpose_reduce<true>(v, lane);
+          x_red[warp][lane] = v[0];
+          sm_sync();
+          if (warp == 0) {
+            const int col = ch * 32 + lane;
+            const float bm = fmaxf(fmaxf(x_red[0][lane], x_red[1][lane]),
+                                   fmaxf(x_red[2][lane], x_red[3][lane]));
+            const float m_old = first ? -INFINITY : m_raw[col];
+            const float m_new = fmaxf(m_old, bm);
+            r_val[lane] =
+                m_old == -INFINITY ? 0.0f : ex2((m_old - m_new) * c2);
+            m_raw[col] = m_new;
+            m_sc[col] = m_new * c2;
+          }
+          sm_sync();
+          if (!first) {
+            // O^T must hold every earlier block's P V before it is scaled.
+            if (!o_ready) {
+              wait_or_fail(o_done, (i - 1) & 1, failed, p.status);
+              tc_fence_after();
+              o_ready = true;
+            }
+            tmem_scale32(tmem + lane_base + kO + ch * 32, r_val);
+            tmem_scale32(tmem + lane_base + kL + ch * 32, r_val);
+          }
         }
-        l *= alpha;
-        if (need) m_ref = mx;
-      }
-      if (first) m_ref = mx;
-      // P = 2^((s - m_ref) c) in bf16 for this warp's pages, written into
-      // every replica of these rows.
-      wait_or_fail(&p_empty[sbuf], ((i >> 1) & 1) ^ 1, failed, p.status);
-      const float off = m_ref * c2;
-      float ls = 0.0f;
+        // P = 2^(s c - m c) (0 where masked; a row whose reference is still
+        // -inf has only masked scores), added to this key's row sums and
+        // written into column kl of P^T.
+        float l[32];
+        if (first) {
 #pragma unroll
-      for (int k = 0; k < UPW; ++k) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float a = ex2(fmaf(s[k * 16 + 2 * e], c2, -off));
-          const float b2 = ex2(fmaf(s[k * 16 + 2 * e + 1], c2, -off));
-          ls += a + b2;
-          pk[e] = pack_bf16(a, b2);
+          for (int e = 0; e < 32; ++e) l[e] = 0.0f;
+        } else {
+          tmem_ld32(tmem + lane_base + kL + ch * 32, l);
         }
-        const int ch0 = (rep * UPW + k) * 2;           // 16-byte chunk
 #pragma unroll
-        for (int o = 0; o < R; ++o) {
-          const int trow = o * Mq + row;
-          uint8_t* prow = ps + sbuf * kPBytes + trow * 128;
-          *reinterpret_cast<uint4*>(prow + (((ch0 & 7) ^ (trow & 7)) << 4)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(
-              prow + ((((ch0 + 1) & 7) ^ (trow & 7)) << 4)) =
-              make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        for (int e = 0; e < 32; e += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(&m_sc[ch * 32 + e]);
+          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float off = mm[u] == -INFINITY ? 0.0f : mm[u];
+            const float pv = ex2(fmaf(s[e + u], c2, -off));
+            l[e + u] += pv;
+            *reinterpret_cast<__nv_bfloat16*>(
+                pt + sw128_off(ch * 32 + e + u, kl, PH)) = __float2bfloat16_rn(pv);
+          }
         }
+        tmem_st32(tmem + lane_base + kL + ch * 32, l);
       }
-      l += ls;
       proxy_fence();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sbuf]);
+      if (lane == 0) mbar_arrive(&p_full[pbi]);
       if (w.last()) {
-        // Epilogue: O of this segment is complete once its last P V lands.
-        float lt = l;
-        if (R > 1) {
-          x_sum[warp][lane] = l;
-          asm volatile("bar.sync 1, %0;" ::"r"(kSmWarps * 32));
-          lt = 0.0f;
-#pragma unroll
-          for (int o = 0; o < R; ++o) lt += x_sum[(warp % QPR) + o * QPR][lane];
-          asm volatile("bar.sync 1, %0;" ::"r"(kSmWarps * 32));
-        }
+        // Epilogue: O^T of this segment is complete once its last P V
+        // lands; the row sums are reduced over the 128 keys.
         wait_or_fail(o_done, i & 1, failed, p.status);
         tc_fence_after();
         const int slot = (w.seg_begin_u == u0) ? 0 : 1;
         float* part = p.part + ((size_t)(c * 2 + slot)) * M * (D + 2);
-        const float inv = 1.0f / lt;
 #pragma unroll 1
-        for (int c0 = rep * OPW; c0 < (rep + 1) * OPW; c0 += 16) {
-          float v[16];
-          tmem_ld16(tmem + lane_base + c0, v);
-          if (real) {
-            if (w.complete) {
-              __nv_bfloat16* o = p.out +
-                  (((size_t)w.b * p.K + rq) * p.Hq + w.h * p.g + jq) * D + c0;
-              uint32_t pk[8];
+        for (int ch = 0; ch < NCH; ++ch) {
+          float v[32];
+          tmem_ld32(tmem + lane_base + kL + ch * 32, v);
+          warp_transpose_reduce<false>(v, lane);
+          x_red[warp][lane] = v[0];
+          sm_sync();
+          if (warp == 0)
+            r_val[lane] = (x_red[0][lane] + x_red[1][lane]) +
+                          (x_red[2][lane] + x_red[3][lane]);
+          sm_sync();
+          float lsum[32], o[32];
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                pk[e] = pack_bf16(v[2 * e] * inv, v[2 * e + 1] * inv);
-              *reinterpret_cast<uint4*>(o) =
-                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              *reinterpret_cast<uint4*>(o + 8) =
-                  make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            } else {
+          for (int e = 0; e < 32; e += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(&r_val[e]);
+            lsum[e] = l4.x; lsum[e + 1] = l4.y;
+            lsum[e + 2] = l4.z; lsum[e + 3] = l4.w;
+          }
+          tmem_ld32(tmem + lane_base + kO + ch * 32, o);   // lane = d = kl
 #pragma unroll
-              for (int e = 0; e < 16; e += 4)
-                *reinterpret_cast<float4*>(part + (size_t)row * D + c0 + e) =
-                    make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          for (int e = 0; e < 32; ++e) {
+            const int col = ch * 32 + e;
+            if (col < M) {
+              if (w.complete) {
+                const int rq = col / p.g, jq = col - rq * p.g;
+                p.out[(((size_t)w.b * p.K + rq) * p.Hq + w.h * p.g + jq) * D +
+                      kl] = __float2bfloat16_rn(o[e] / lsum[e]);
+              } else {
+                part[(size_t)col * D + kl] = o[e];
+              }
             }
           }
-        }
-        if (real && rep == 0) {
-          if (w.complete) {
-            if (p.lse)
-              p.lse[((size_t)w.b * p.K + rq) * p.Hq + w.h * p.g + jq] =
-                  (m_ref * c2 + log2f(lt)) * kLn2;
-          } else {
-            part[(size_t)M * D + row] = m_ref;
-            part[(size_t)M * D + M + row] = lt;
+          if (warp == 0) {
+            const int col = ch * 32 + lane;
+            if (col < M) {
+              const float lt = r_val[lane], mr = m_raw[col];
+              if (w.complete) {
+                if (p.lse) {
+                  const int rq = col / p.g, jq = col - rq * p.g;
+                  p.lse[((size_t)w.b * p.K + rq) * p.Hq + w.h * p.g + jq] =
+                      (mr * c2 + log2f(lt)) * kLn2;
+                }
+              } else {
+                part[(size_t)M * D + col] = mr;
+                part[(size_t)M * D + M + col] = lt;
+              }
+            }
           }
         }
         tc_fence_before();
@@ -684,7 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(
                      tmem),
-                 "r"(kTmemCols));
+                 "r"(kCols));
   }
 }
 
@@ -729,15 +856,34 @@ static bool encode_tiled_4d(CUtensorMap* m, const void* base,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t attn_tc_smem_bytes(int B) {
-  return 1024 + (size_t)tc::kStagesTc * tc::kStageBytes + tc::kQBytes +
-         2 * tc::kPBytes + 32 * 8 + 16 + (size_t)(B + 1) * 4;
+constexpr size_t kSmemLimit = 227 * 1024;
+
+// Dynamic shared memory of the kernel for N = 32 * nch rows and `stages`
+// (one P^T buffer at N = 128, two below).
+static size_t tc_smem(int B, int nch, int stages) {
+  const size_t N = 32 * (size_t)nch;
+  const size_t npb = nch == 4 ? 1 : 2;
+  return 1024 + (size_t)stages * tc::kStageBytes + 2 * N * 128 +
+         npb * 2 * N * 128 + tc::kBarBytes + 16 + (size_t)(B + 1) * 4;
+}
+
+// Stages for M query rows (3 when they fit, else 2; 0 if neither does).
+static int tc_stages(int B, int M) {
+  const int nch = (M + 31) / 32;
+  for (int s = tc::kMaxStages; s >= 2; --s)
+    if (tc_smem(B, nch, s) + tc::kStaticSmem <= kSmemLimit) return s;
+  return 0;
+}
+
+size_t attn_tc_smem_bytes(int B, int M) {
+  const int s = tc_stages(B, M);
+  return s ? tc_smem(B, (M + 31) / 32, s) : (size_t)-1;
 }
 
 bool attn_tc_supported(const isd_attn_args* a) {
   const int M = a->K * (a->Hq / a->Hkv);
   return a->dtype == ISD_BF16 && a->d == 128 && M >= 1 && M <= 128 &&
-         a->K <= kPage && attn_tc_smem_bytes(a->B) <= 227 * 1024;
+         a->K <= kPage && tc_stages(a->B, M) > 0;
 }
 
 int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
@@ -745,12 +891,11 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
   p.B = a->B; p.Hq = a->Hq; p.Hkv = a->Hkv; p.K = a->K;
   p.g = a->Hq / a->Hkv; p.M = a->K * p.g; p.P = a->num_pages;
   p.stride = a->page_table_stride;
+  p.stages = tc_stages(a->B, p.M);
+  if (p.stages == 0) return ISD_ERR_UNSUPPORTED;
   p.scale_log2 = a->softmax_scale * kLog2e;
   p.q = static_cast<const __nv_bfloat16*>(a->q);
-  p.kc = static_cast<const __nv_bfloat16*>(a->k_cache);
   p.vc = static_cast<const __nv_bfloat16*>(a->v_cache);
-  p.kn = static_cast<const __nv_bfloat16*>(a->k_new);
-  p.vn = static_cast<const __nv_bfloat16*>(a->v_new);
   p.out = static_cast<__nv_bfloat16*>(a->out);
   p.lse = a->lse; p.page_table = a->page_table; p.seq_len = a->seq_len;
   p.status = a->status;
@@ -758,9 +903,9 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
   p.ws_int = reinterpret_cast<int32_t*>(ws);
   p.part = reinterpret_cast<float*>(
       ws + (((size_t)(a->B + 2) * 4 + 255) & ~size_t(255)));
-  // K tensor maps: the cache [P][Hkv][16][128] and the stride's staged
-  // rows [B][K][Hkv][128], 64-column boxes with the 128-byte swizzle.
-  CUtensorMap tkc, tkn;
+  // K and V tensor maps: the caches [P][Hkv][16][128] and the stride's
+  // staged rows [B][K][Hkv][128], 64-column boxes with the 128-byte swizzle.
+  CUtensorMap tkc, tvc, tkn, tvn;
   const uint64_t dc[4] = {128, (uint64_t)kPage, (uint64_t)a->Hkv,
                           (uint64_t)a->num_pages};
   const uint64_t sc[3] = {256, (uint64_t)kPage * 256,
@@ -772,16 +917,20 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
                           (uint64_t)a->K * a->Hkv * 256};
   const uint32_t bn[4] = {64, 1, (uint32_t)kPage, 1};
   if (!encode_tiled_4d(&tkc, a->k_cache, dc, sc, bc) ||
-      !encode_tiled_4d(&tkn, a->k_new, dn, sn, bn))
+      !encode_tiled_4d(&tvc, a->v_cache, dc, sc, bc) ||
+      !encode_tiled_4d(&tkn, a->k_new, dn, sn, bn) ||
+      !encode_tiled_4d(&tvn, a->v_new, dn, sn, bn))
     return ISD_ERR_CUDA;
-  const size_t smem = attn_tc_smem_bytes(a->B);
-  auto kern = p.M <= 32 ? tc::attn_tc_kernel<4>
-                        : (p.M <= 64 ? tc::attn_tc_kernel<2>
-                                     : tc::attn_tc_kernel<1>);
+  const int nch = (p.M + 31) / 32;
+  const size_t smem = tc_smem(a->B, nch, p.stages);
+  auto kern = nch == 1 ? tc::attn_tc_kernel<1>
+            : nch == 2 ? tc::attn_tc_kernel<2>
+            : nch == 3 ? tc::attn_tc_kernel<3>
+                       : tc::attn_tc_kernel<4>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return ISD_ERR_CUDA;
-  kern<<<G, tc::kThreads, smem, st>>>(tkc, tkn, p);
+  kern<<<G, tc::kThreads, smem, st>>>(tkc, tvc, tkn, tvn, p);
   if (cudaGetLastError() != cudaSuccess) return ISD_ERR_CUDA;
   return launch_attn_combine(a, G, st);
 }

@@ -223,6 +223,14 @@ ISD_DEV void mbar_arrive(uint64_t* bar) {
                    smem_u32(bar))
                : "memory");
 }
+// Adds `bytes` to the transaction count the current phase waits for,
+// without arriving.
+ISD_DEV void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
 ISD_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile(
       "mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(

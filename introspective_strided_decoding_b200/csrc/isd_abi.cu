@@ -11,7 +11,7 @@ size_t commit_workspace_bytes(int B);
 int launch_commit(const isd_commit_args* a, cudaStream_t st);
 size_t attn_workspace_bytes_impl(int B, int M, int D, int G);
 size_t attn_smem_bytes(int D, int MW, int B);
-size_t attn_tc_smem_bytes(int B);
+size_t attn_tc_smem_bytes(int B, int M);
 int launch_attn_bf16(const isd_attn_args* a, int G, cudaStream_t st);
 int launch_attn_f32(const isd_attn_args* a, cudaStream_t st);
 }  // namespace isd
@@ -48,8 +48,10 @@ int attn_check(const isd_attn_args* a) {
     const int M = a->K * (a->Hq / a->Hkv);
     if (a->K > ISD_PAGE_SIZE || M > 128) return ISD_ERR_UNSUPPORTED;
     if (a->d == 128) {
-      // tcgen05 path: any row count up to 128 (rows padded to 128).
-      if (isd::attn_tc_smem_bytes(a->B) > 227 * 1024) return ISD_ERR_UNSUPPORTED;
+      // tcgen05 path: any row count up to 128 (rows padded to a multiple
+      // of 32); the stage ring must fit next to Q, P and the unit prefix.
+      if (isd::attn_tc_smem_bytes(a->B, M) == (size_t)-1)
+        return ISD_ERR_UNSUPPORTED;
     } else if (a->d == 64) {
       // mma.sync path: rows in warps of 16 or 32.
       if (!(M == 16 || M == 32 || M == 64 || M == 128)) return ISD_ERR_UNSUPPORTED;
