@@ -16,7 +16,8 @@
 // (M = K * g, often 32) and many keys, so the keys take the MMA's 128-row
 // side and the rows its N side (N = M rounded up to 32):
 //   S^T[key][row]  = K Q^T        (A = K tile, B = Q, both K-major)
-//   O^T[d][row]   += V^T P^T      (A = V tile read MN-major, B = P^T)
+//   O^T[d][row]   += V^T P^T      (A = V tile read MN-major, B = P^T read
+//                                  MN-major from a [key][row] tile)
 // with S^T, O^T and the per-key partial row sums in TMEM.  No MMA row is
 // padding, and each block costs 16 MMAs whatever M is.
 //
@@ -61,21 +62,22 @@ constexpr int D = 128;
 constexpr int kNB = 8;                       // pages per block
 constexpr int kKeys = kNB * kPage;           // 128 keys = TMEM lanes
 constexpr int kKH = kKeys * 128;             // one 64-column half of K or V
-constexpr int kStageBytes = 4 * kKH;         // K0 K1 V0 V1 = 64 KB
+constexpr int kTile = 2 * kKH;               // a K or V tile: 32 KB
 constexpr int kSmWarps = 4;
 constexpr int kMmaWarp = 4;
 constexpr int kLoadWarps = 4;
 constexpr int kPagesPerLoader = kNB / kLoadWarps;
 constexpr int kThreads = (kSmWarps + 1 + kLoadWarps) * 32;   // 288
 constexpr int kLoadThreads = kLoadWarps * 32;
-constexpr int kMaxStages = 3;
-constexpr int kBarBytes = 32 * 8;            // mbarriers (2 * stages + 13)
+constexpr int kKStages = 2;                  // K ring
+constexpr int kMaxVStages = 4;               // V ring (fewer if Q, P are big)
+constexpr int kBarBytes = 32 * 8;            // mbarriers (2 (SK + SV) + 12)
 constexpr int kStaticSmem = 2048;            // __shared__ arrays, rounded up
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint64_t kWaitCycles = 400000000ull;   // ~0.2 s
 
 struct Params {
-  int B, Hq, Hkv, K, g, M, P, stride, stages;
+  int B, Hq, Hkv, K, g, M, P, stride, sv;
   float scale_log2;
   const __nv_bfloat16* q;
   const __nv_bfloat16* vc;
@@ -89,13 +91,15 @@ struct Params {
 };
 
 // ------------------------------------------------------------------ PTX
-ISD_DEV uint64_t sdesc(uint32_t start, uint32_t lbo, uint32_t sbo) {
-  // Shared-memory matrix descriptor (sm_100): start, leading / stride byte
-  // offsets (16-byte units), descriptor version 1, 128-byte swizzle.
+// Shared-memory matrix descriptor (sm_100): start, leading / stride byte
+// offsets (16-byte units), descriptor version 1, swizzle mode (2: 128-byte,
+// 4: 64-byte).
+ISD_DEV uint64_t sdesc(uint32_t start, uint32_t lbo, uint32_t sbo,
+                       uint32_t swz = 2) {
   return (uint64_t)((start >> 4) & 0x3FFFu) |
          ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
-         (2ull << 61);
+         ((uint64_t)swz << 61);
 }
 ISD_DEV uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
   // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, each
@@ -318,13 +322,6 @@ struct BlockWalk {
   }
 };
 
-// Byte offset of bf16 element (row, col) in a K-major tile of 64-column
-// halves (128-byte rows, 128-byte swizzle); `half` = bytes of one half.
-ISD_DEV uint32_t sw128_off(int row, int col, int half) {
-  return (uint32_t)((col >> 6) * half + row * 128 +
-                    ((((col >> 3) & 7) ^ (row & 7)) << 4) + (col & 7) * 2);
-}
-
 // NCH: 32-column chunks of the padded query rows (N = 32 * NCH).
 template <int NCH>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -334,29 +331,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tm_vn, Params p) {
   constexpr int N = 32 * NCH;
   constexpr int QH = N * 128;              // one 64-column half of Q
-  constexpr int PH = N * 128;              // one 64-key half of P^T
-  constexpr int PB = 2 * PH;               // one P^T buffer
+  // P tile [128 keys][N rows]: 32-row atoms of 128 keys x 64 B (64-byte
+  // swizzle), atom a holding rows 32a..32a+31.
+  constexpr int PA = kKeys * 64;           // one 32-row atom (8 KB)
+  constexpr int PB = NCH * PA;             // one P buffer
   constexpr int NPB = NCH == 4 ? 1 : 2;    // P^T buffers (one at N = 128)
   constexpr uint32_t kO = 0, kS = N, kL = 3 * N;       // TMEM columns
   constexpr uint32_t kCols = 4 * N <= 128 ? 128 : (4 * N <= 256 ? 256 : 512);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int S = p.stages;
-  uint8_t* kv = base;                                  // S stages
-  uint8_t* qs = kv + S * kStageBytes;                  // Q tile [N][128]
+  // K and V rings: a K tile is consumed by the QK MMAs of its block and
+  // freed right after them; a V tile waits for the block's softmax and its
+  // P V, so the V ring is deeper.
+  constexpr int SK = kKStages;
+  const int SV = p.sv;
+  uint8_t* kr = base;                                  // SK K tiles
+  uint8_t* vr = kr + SK * kTile;                       // SV V tiles
+  uint8_t* qs = vr + SV * kTile;                       // Q tile [N][128]
   uint8_t* ps = qs + 2 * QH;                           // NPB P^T tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(ps + NPB * PB);
-  uint64_t* kv_full = bars;                            // [S]
-  uint64_t* kv_empty = kv_full + S;                    // [S]
-  uint64_t* s_full = kv_empty + S;                     // [2]
+  uint64_t* k_full = bars;                             // [SK]
+  uint64_t* k_empty = k_full + SK;                     // [SK]
+  uint64_t* v_full = k_empty + SK;                     // [SV]
+  uint64_t* v_empty = v_full + SV;                     // [SV]
+  uint64_t* s_full = v_empty + SV;                     // [2]
   uint64_t* s_free = s_full + 2;                       // [2]
   uint64_t* p_full = s_free + 2;                       // [NPB]
   uint64_t* p_empty = p_full + 2;                      // [NPB]
   uint64_t* q_full = p_empty + 2;
   uint64_t* q_empty = q_full + 1;
-  uint64_t* o_done = q_empty + 1;
-  uint64_t* o_free = o_done + 1;
+  uint64_t* o_free = q_empty + 1;
   uint64_t* fin = o_free + 1;                          // all MMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBarBytes / 8);
   int* prefix = reinterpret_cast<int*>(tmem_slot + 4);
@@ -388,9 +393,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int u0 = (int)(((long long)c * T) / G);
   const int u1 = (int)(((long long)(c + 1) * T) / G);
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&kv_full[s], kLoadWarps);   // one arrival per loader warp
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < SK; ++s) {
+      mbar_init(&k_full[s], kLoadWarps);    // one arrival per loader warp
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < SV; ++s) {
+      mbar_init(&v_full[s], kLoadWarps);
+      mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
@@ -400,7 +409,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(q_full, kLoadThreads);
     mbar_init(q_empty, 1);
-    mbar_init(o_done, 1);
     mbar_init(o_free, kSmWarps);
     mbar_init(fin, 1);
     fence_barrier_init();
@@ -432,7 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (s_bad && p.status) *p.status = ISD_ERR_PAGE_TABLE_FULL;
     }
   }
-  const uint32_t kv_s = smem_u32(kv), q_s = smem_u32(qs), p_s = smem_u32(ps);
+  const uint32_t kr_s = smem_u32(kr), vr_s = smem_u32(vr);
+  const uint32_t q_s = smem_u32(qs), p_s = smem_u32(ps);
   bool failed = false;
 
   if (warp > kMmaWarp) {
@@ -440,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Loader warp lw copies pages lw and lw + 4 of every block; its lane 0
     // issues their TMA boxes, so four threads keep copies in flight (one
     // cannot saturate HBM).  Each warp registers its TMA bytes and then
-    // arrives once per stage on kv_full.
+    // arrives once per block on k_full and on v_full.
     const int lt = tid - (kMmaWarp + 1) * 32;
     const int lw = lt >> 5;
     BlockWalk w;
@@ -479,65 +488,85 @@ __global__ void __launch_bounds__(kThreads, 1)
         cp_async_arrive(q_full);
         ++nseg_done;
       }
-      const int st = i % S;
-      wait_or_fail(&kv_empty[st], ((i / S) & 1) ^ 1, failed, p.status);
-      uint64_t* bar = &kv_full[st];
-      bool partial_v = false;    // some page's V goes by cp.async
+      // This warp's pages of the block: page id (out of range: recorded,
+      // then read as zeros from coordinate P, outside the cache tensors),
+      // tail or cached, partial or full.
+      bool use[kPagesPerLoader], tail[kPagesPerLoader], part[kPagesPerLoader];
+      int page[kPagesPerLoader], valid[kPagesPerLoader];
 #pragma unroll
       for (int q = 0; q < kPagesPerLoader; ++q) {
         const int k = lw + q * kLoadWarps;
-        if (k >= w.nu()) continue;
-        uint8_t* kd = kv + st * kStageBytes + k * 2048;   // K half 0, page k
-        uint8_t* vd = kd + 2 * kKH;                       // V half 0, page k
         const int uidx = w.idx0 + w.k + k;
-        if (uidx == w.units - 1) {
-          // Tail: the stride's own K and V rows; rows past K lie outside
-          // the staging tensors and read as zeros.
+        use[q] = k < w.nu();
+        tail[q] = use[q] && uidx == w.units - 1;
+        int pg = q == 0 ? pid0 : pid1;
+        const bool bad = use[q] && !tail[q] && (pg < 0 || pg >= p.P);
+        if (bad) {
+          if (lane == 0 && p.status) *p.status = ISD_ERR_BAD_PAGE;
+          pg = p.P;
+        }
+        page[q] = pg;
+        valid[q] = Lb - uidx * kPage;          // >= 1 for a cached unit
+        part[q] = use[q] && !tail[q] && !bad && valid[q] < kPage;
+      }
+      // K tiles.  Rows past K of the tail lie outside the staging tensor
+      // and read as zeros.
+      const int ks = i % SK;
+      wait_or_fail(&k_empty[ks], ((i / SK) & 1) ^ 1, failed, p.status);
+      if (lane == 0) {
+#pragma unroll
+        for (int q = 0; q < kPagesPerLoader; ++q) {
+          if (!use[q]) continue;
+          uint8_t* kd = kr + ks * kTile + (lw + q * kLoadWarps) * 2048;
+          mbar_expect_tx(&k_full[ks], 2 * 2048);
+          for (int hb = 0; hb < 2; ++hb) {
+            if (tail[q])
+              tma_load_4d(kd + hb * kKH, &tm_kn, &k_full[ks], hb * 64, w.h, 0, w.b);
+            else
+              tma_load_4d(kd + hb * kKH, &tm_kc, &k_full[ks], hb * 64, 0, w.h,
+                          page[q]);
+          }
+        }
+        mbar_arrive(&k_full[ks]);
+      }
+      // V tiles.  A partial last page's V takes cp.async: slots past L_b
+      // are zero-filled, never copied (they may hold any bits, and 0 * NaN
+      // would reach O through P V).  K there is harmless: those scores are
+      // masked.
+      const int vs = i % SV;
+      wait_or_fail(&v_empty[vs], ((i / SV) & 1) ^ 1, failed, p.status);
+      bool partial_v = false;
+#pragma unroll
+      for (int q = 0; q < kPagesPerLoader; ++q) {
+        if (!use[q]) continue;
+        const int k = lw + q * kLoadWarps;
+        uint8_t* vd = vr + vs * kTile + k * 2048;
+        if (!part[q]) {
           if (lane == 0) {
-            mbar_expect_tx(bar, 4 * 2048);
+            mbar_expect_tx(&v_full[vs], 2 * 2048);
             for (int hb = 0; hb < 2; ++hb) {
-              tma_load_4d(kd + hb * kKH, &tm_kn, bar, hb * 64, w.h, 0, w.b);
-              tma_load_4d(vd + hb * kKH, &tm_vn, bar, hb * 64, w.h, 0, w.b);
+              if (tail[q])
+                tma_load_4d(vd + hb * kKH, &tm_vn, &v_full[vs], hb * 64, w.h, 0,
+                            w.b);
+              else
+                tma_load_4d(vd + hb * kKH, &tm_vc, &v_full[vs], hb * 64, 0, w.h,
+                            page[q]);
             }
           }
           continue;
         }
-        int page = q == 0 ? pid0 : pid1;
-        const bool bad = page < 0 || page >= p.P;
-        if (bad) {
-          // Out of range: record it and read zeros (coordinate P lies
-          // outside the cache tensors).
-          if (lane == 0 && p.status) *p.status = ISD_ERR_BAD_PAGE;
-          page = p.P;
-        }
-        const int valid = Lb - uidx * kPage;   // >= 1 for a cached unit
-        const bool part = valid < kPage && !bad;
-        if (lane == 0) {
-          mbar_expect_tx(bar, (part ? 2 : 4) * 2048);
-          for (int hb = 0; hb < 2; ++hb) {
-            tma_load_4d(kd + hb * kKH, &tm_kc, bar, hb * 64, 0, w.h, page);
-            if (!part)
-              tma_load_4d(vd + hb * kKH, &tm_vc, bar, hb * 64, 0, w.h, page);
-          }
-        }
-        if (part) {
-          // Partial last page: V slots past L_b are zero-filled, never
-          // copied (they may hold any bits, and 0 * NaN would reach O
-          // through P V).  K there is harmless: those scores are masked.
-          partial_v = true;
-          for (int e = lane; e < kPage * 16; e += 32) {
-            const int row = e >> 4, ch = e & 15;
-            const int key = k * kPage + row;
-            const uint32_t dst = kv_s + st * kStageBytes + 2 * kKH +
-                                 (ch >> 3) * kKH + key * 128 +
-                                 (((ch & 7) ^ (key & 7)) << 4);
-            const bool in = row < valid;
-            const __nv_bfloat16* src =
-                in ? p.vc + (((size_t)page * Hkv + w.h) * kPage + row) * D +
-                         ch * 8
-                   : p.vc;
-            cp_async_16(dst, src, in ? 16u : 0u);
-          }
+        partial_v = true;
+        for (int e = lane; e < kPage * 16; e += 32) {
+          const int row = e >> 4, ch = e & 15;
+          const int key = k * kPage + row;
+          const uint32_t dst = vr_s + vs * kTile + (ch >> 3) * kKH + key * 128 +
+                               (((ch & 7) ^ (key & 7)) << 4);
+          const bool in = row < valid[q];
+          const __nv_bfloat16* src =
+              in ? p.vc + (((size_t)page[q] * Hkv + w.h) * kPage + row) * D +
+                       ch * 8
+                 : p.vc;
+          cp_async_16(dst, src, in ? 16u : 0u);
         }
       }
       if (partial_v) {
@@ -545,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         proxy_fence();
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar);
+      if (lane == 0) mbar_arrive(&v_full[vs]);
       w.next();
       if (!w.done()) load_ids();
       ++i;
@@ -556,30 +585,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     BlockWalk w;
     w.init(prefix, B, Hkv, u0, u1);
     int i = 0, nseg = 0;
-    int prev_nu = 0, prev_st = 0, prev_pb = 0;
+    int prev_nu = 0, prev_pb = 0;
     bool prev_first = false, have_prev = false;
     const uint32_t id_qk = idesc_bf16(128, N, 0, 0);
-    const uint32_t id_pv = idesc_bf16(128, N, 1, 0);
+    const uint32_t id_pv = idesc_bf16(128, N, 1, 1);
     auto issue_pv = [&](int j_blk) {
       // O^T += V^T P^T for block j_blk: one k-step of 16 keys per page.
+      const int vs = j_blk % SV;
       wait_or_fail(&p_full[prev_pb], (j_blk / NPB) & 1, failed, p.status);
+      wait_or_fail(&v_full[vs], (j_blk / SV) & 1, failed, p.status);
       tc_fence_after();
       if (lane == 0) {
         const uint32_t pa = p_s + prev_pb * PB;
-        const uint32_t vb = kv_s + prev_st * kStageBytes + 2 * kKH;
+        const uint32_t vb = vr_s + vs * kTile;
         for (int j = 0; j < prev_nu; ++j)
           umma(tmem + kO, sdesc(vb + j * 2048, kKH, 1024),
-               sdesc(pa + (j >> 2) * PH + (j & 3) * 32, 16, 1024), id_pv,
+               sdesc(pa + j * 1024, PA, 512, 4), id_pv,
                (prev_first && j == 0) ? 0u : 1u);
-        umma_commit(&kv_empty[prev_st]);
+        umma_commit(&v_empty[vs]);
         umma_commit(&p_empty[prev_pb]);
-        umma_commit(o_done);
       }
       __syncwarp();
     };
     int seg_pv = 0;  // segments whose first PV has been issued
     while (!w.done()) {
-      const int st = i % S, sbuf = i & 1;
+      const int ks = i % SK, sbuf = i & 1;
       if (w.first()) {
         wait_or_fail(q_full, nseg & 1, failed, p.status);
         // Q arrived through cp.async (generic proxy); the tensor core
@@ -588,19 +618,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         proxy_fence();
         ++nseg;
       }
-      wait_or_fail(&kv_full[st], (i / S) & 1, failed, p.status);
+      wait_or_fail(&k_full[ks], (i / SK) & 1, failed, p.status);
       wait_or_fail(&s_free[sbuf], ((i >> 1) & 1) ^ 1, failed, p.status);
       tc_fence_after();
       if (lane == 0) {
-        // S^T = K Q^T over the 128 keys of the stage (rows of pages past
+        // S^T = K Q^T over the 128 keys of the tile (rows of pages past
         // the block's end hold stale data; their scores are masked).
-        const uint32_t kb = kv_s + st * kStageBytes;
+        const uint32_t kb = kr_s + ks * kTile;
         for (int kk = 0; kk < 8; ++kk)
           umma(tmem + kS + sbuf * N,
                sdesc(kb + (kk >> 2) * kKH + (kk & 3) * 32, 16, 1024),
                sdesc(q_s + (kk >> 2) * QH + (kk & 3) * 32, 16, 1024), id_qk,
                kk > 0 ? 1u : 0u);
         umma_commit(&s_full[sbuf]);
+        umma_commit(&k_empty[ks]);
         if (w.last()) umma_commit(q_empty);
       }
       __syncwarp();
@@ -611,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_pv(i - 1);
       }
       have_prev = true;
-      prev_nu = w.nu(); prev_st = st; prev_pb = i % NPB; prev_first = w.first();
+      prev_nu = w.nu(); prev_pb = i % NPB; prev_first = w.first();
       w.next();
       ++i;
     }
@@ -653,6 +684,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_or_fail(&p_empty[pbi], ((i / NPB) & 1) ^ 1, failed, p.status);
       bool o_ready = false;
       uint8_t* pt = ps + pbi * PB;
+      uint8_t* prow = pt + kl * 64;               // this key's row of P
+      const int psw = (kl >> 1) & 3;              // its 64-byte swizzle
 #pragma unroll 1
       for (int ch = 0; ch < NCH; ++ch) {
         float s[32];
@@ -662,23 +695,54 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&s_free[sbuf]);
         }
+        if (col_min != 0) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          s[e] = (ch * 32 + e >= col_min) ? s[e] : -INFINITY;
-        // Vote: does any score exceed its row's reference by 2^8?  (A row
-        // with reference -inf votes yes on any unmasked score.)
+          for (int e = 0; e < 32; ++e)
+            s[e] = (ch * 32 + e >= col_min) ? s[e] : -INFINITY;
+        }
+        // P = 2^(s c - m c) against the current references (masked scores
+        // give 0), written as this key's 32 values of the chunk and added
+        // to its row sums.  Returns the largest exponent s c - m c.
+        float l[32];
+        auto p_pass = [&]() {
+          float xmax = -INFINITY;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float4 ma = *reinterpret_cast<const float4*>(&m_sc[ch * 32 + q * 8]);
+            const float4 mb = *reinterpret_cast<const float4*>(&m_sc[ch * 32 + q * 8 + 4]);
+            const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+            uint32_t pk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int e = q * 8 + 2 * u;
+              const float x0 = fmaf(s[e], c2, -mm[2 * u]);
+              const float x1 = fmaf(s[e + 1], c2, -mm[2 * u + 1]);
+              xmax = fmaxf(xmax, fmaxf(x0, x1));
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              l[e] += p0;
+              l[e + 1] += p1;
+              pk[u] = pack_bf16(p0, p1);
+            }
+            *reinterpret_cast<uint4*>(prow + ch * PA + ((q ^ psw) << 4)) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+          return xmax;
+        };
+        auto load_l = [&]() {
+          if (first) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) l[e] = 0.0f;
+          } else {
+            tmem_ld32(tmem + lane_base + kL + ch * 32, l);
+          }
+        };
+        // Optimistic pass; the vote asks whether any exponent exceeded 8
+        // (then the references move and the pass is redone).  The first
+        // block of a segment has no references yet.
         bool need = first;
         if (!first) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 m4 =
-                *reinterpret_cast<const float4*>(&m_sc[ch * 32 + e]);
-            const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              need |= s[e + u] != -INFINITY &&
-                      fmaf(s[e + u], c2, -mm[u]) > kRescaleLog2;
-          }
+          load_l();
+          need = p_pass() > kRescaleLog2;
         }
         if (sm_any(need)) {
           // Exact block max per row, then move the references.
@@ -697,42 +761,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             r_val[lane] =
                 m_old == -INFINITY ? 0.0f : ex2((m_old - m_new) * c2);
             m_raw[col] = m_new;
-            m_sc[col] = m_new * c2;
+            // Finite stand-in for a row with no key yet, so that masked
+            // scores still give 0 and an unmasked one votes.
+            m_sc[col] = fmaxf(m_new * c2, -3.0e38f);
           }
           sm_sync();
           if (!first) {
             // O^T must hold every earlier block's P V before it is scaled.
+            // P V of block j completes phase j / NPB of p_empty[j % NPB],
+            // a barrier this thread waits on every NPB blocks, so a parity
+            // wait names that phase unambiguously.
             if (!o_ready) {
-              wait_or_fail(o_done, (i - 1) & 1, failed, p.status);
+              wait_or_fail(&p_empty[(i - 1) % NPB], ((i - 1) / NPB) & 1, failed,
+                           p.status);
               tc_fence_after();
               o_ready = true;
             }
             tmem_scale32(tmem + lane_base + kO + ch * 32, r_val);
             tmem_scale32(tmem + lane_base + kL + ch * 32, r_val);
           }
-        }
-        // P = 2^(s c - m c) (0 where masked; a row whose reference is still
-        // -inf has only masked scores), added to this key's row sums and
-        // written into column kl of P^T.
-        float l[32];
-        if (first) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) l[e] = 0.0f;
-        } else {
-          tmem_ld32(tmem + lane_base + kL + ch * 32, l);
-        }
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 m4 = *reinterpret_cast<const float4*>(&m_sc[ch * 32 + e]);
-          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float off = mm[u] == -INFINITY ? 0.0f : mm[u];
-            const float pv = ex2(fmaf(s[e + u], c2, -off));
-            l[e + u] += pv;
-            *reinterpret_cast<__nv_bfloat16*>(
-                pt + sw128_off(ch * 32 + e + u, kl, PH)) = __float2bfloat16_rn(pv);
-          }
+          load_l();
+          p_pass();
         }
         tmem_st32(tmem + lane_base + kL + ch * 32, l);
       }
@@ -742,8 +791,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&p_full[pbi]);
       if (w.last()) {
         // Epilogue: O^T of this segment is complete once its last P V
-        // lands; the row sums are reduced over the 128 keys.
-        wait_or_fail(o_done, i & 1, failed, p.status);
+        // (block i) lands; the row sums are reduced over the 128 keys.
+        wait_or_fail(&p_empty[pbi], (i / NPB) & 1, failed, p.status);
         tc_fence_after();
         const int slot = (w.seg_begin_u == u0) ? 0 : 1;
         float* part = p.part + ((size_t)(c * 2 + slot)) * M * (D + 2);
@@ -858,32 +907,33 @@ static bool encode_tiled_4d(CUtensorMap* m, const void* base,
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
-// Dynamic shared memory of the kernel for N = 32 * nch rows and `stages`
-// (one P^T buffer at N = 128, two below).
-static size_t tc_smem(int B, int nch, int stages) {
+// Dynamic shared memory of the kernel for N = 32 * nch rows and a V ring
+// of `sv` tiles (one P buffer at N = 128, two below).
+static size_t tc_smem(int B, int nch, int sv) {
   const size_t N = 32 * (size_t)nch;
   const size_t npb = nch == 4 ? 1 : 2;
-  return 1024 + (size_t)stages * tc::kStageBytes + 2 * N * 128 +
+  return 1024 + (size_t)(tc::kKStages + sv) * tc::kTile + 2 * N * 128 +
          npb * 2 * N * 128 + tc::kBarBytes + 16 + (size_t)(B + 1) * 4;
 }
 
-// Stages for M query rows (3 when they fit, else 2; 0 if neither does).
-static int tc_stages(int B, int M) {
+// Deepest V ring (at most 4, at least 2 tiles) that fits for M query rows;
+// 0 if none does.
+static int tc_vstages(int B, int M) {
   const int nch = (M + 31) / 32;
-  for (int s = tc::kMaxStages; s >= 2; --s)
+  for (int s = tc::kMaxVStages; s >= 2; --s)
     if (tc_smem(B, nch, s) + tc::kStaticSmem <= kSmemLimit) return s;
   return 0;
 }
 
 size_t attn_tc_smem_bytes(int B, int M) {
-  const int s = tc_stages(B, M);
+  const int s = tc_vstages(B, M);
   return s ? tc_smem(B, (M + 31) / 32, s) : (size_t)-1;
 }
 
 bool attn_tc_supported(const isd_attn_args* a) {
   const int M = a->K * (a->Hq / a->Hkv);
   return a->dtype == ISD_BF16 && a->d == 128 && M >= 1 && M <= 128 &&
-         a->K <= kPage && tc_stages(a->B, M) > 0;
+         a->K <= kPage && tc_vstages(a->B, M) > 0;
 }
 
 int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
@@ -891,8 +941,8 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
   p.B = a->B; p.Hq = a->Hq; p.Hkv = a->Hkv; p.K = a->K;
   p.g = a->Hq / a->Hkv; p.M = a->K * p.g; p.P = a->num_pages;
   p.stride = a->page_table_stride;
-  p.stages = tc_stages(a->B, p.M);
-  if (p.stages == 0) return ISD_ERR_UNSUPPORTED;
+  p.sv = tc_vstages(a->B, p.M);
+  if (p.sv == 0) return ISD_ERR_UNSUPPORTED;
   p.scale_log2 = a->softmax_scale * kLog2e;
   p.q = static_cast<const __nv_bfloat16*>(a->q);
   p.vc = static_cast<const __nv_bfloat16*>(a->v_cache);
@@ -922,7 +972,7 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
       !encode_tiled_4d(&tvn, a->v_new, dn, sn, bn))
     return ISD_ERR_CUDA;
   const int nch = (p.M + 31) / 32;
-  const size_t smem = tc_smem(a->B, nch, p.stages);
+  const size_t smem = tc_smem(a->B, nch, p.sv);
   auto kern = nch == 1 ? tc::attn_tc_kernel<1>
             : nch == 2 ? tc::attn_tc_kernel<2>
             : nch == 3 ? tc::attn_tc_kernel<3>
