@@ -44,7 +44,8 @@ struct AttnDev {
   const int32_t* page_table;
   const int32_t* seq_len;
   int32_t* status;
-  float* part;        // [G][2][M][D + 2]: unnormalised O, raw max, sum
+  float* part_o;      // [G][2][M][D]: unnormalised O of split segments
+  float* part_ml;     // [G][2][2][M]: their raw row max, then row sum
   int32_t* ws_int;    // [B + 1] unit prefix, then G
 };
 
@@ -437,7 +438,8 @@ __global__ void __launch_bounds__(attn_threads<NW, NL>(), 1)
       }
 
     const int slot = (u == u0) ? 0 : 1;
-    float* part = p.part + ((size_t)(c * 2 + slot)) * p.M * (D + 2);
+    float* part = p.part_o + ((size_t)(c * 2 + slot)) * p.M * D;
+    float* pml = p.part_ml + ((size_t)(c * 2 + slot)) * 2 * p.M;
     if (KS == 1) {
       // Write this warp's rows straight from registers.
 #pragma unroll
@@ -469,8 +471,8 @@ __global__ void __launch_bounds__(attn_threads<NW, NL>(), 1)
                   make_float2(acc[mt][nt][hf * 2], acc[mt][nt][hf * 2 + 1]);
             }
             if ((lane & 3) == 0) {
-              part[(size_t)p.M * D + m] = mr;
-              part[(size_t)p.M * D + p.M + m] = l;
+              pml[m] = mr;
+              pml[p.M + m] = l;
             }
           }
         }
@@ -520,8 +522,8 @@ __global__ void __launch_bounds__(attn_threads<NW, NL>(), 1)
         } else {
           part[(size_t)m * D + col] = o;
           if (col == ks * cols) {
-            part[(size_t)p.M * D + m] = mstar;
-            part[(size_t)p.M * D + p.M + m] = l;
+            pml[m] = mstar;
+            pml[p.M + m] = l;
           }
         }
       }
@@ -536,7 +538,7 @@ __global__ void __launch_bounds__(attn_threads<NW, NL>(), 1)
 // order.  The CTAs and slots holding them are listed once per block.
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(AttnDev p) {
-  extern __shared__ int s_part[];   // partial offsets (in floats)
+  extern __shared__ int s_part[];   // partial indices (CTA * 2 + slot)
   __shared__ int s_n;
   const int h = blockIdx.x, b = blockIdx.y;
   const int B = p.B;
@@ -556,7 +558,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(AttnDev p) {
       const long long u0 = ((long long)cc * T) / G;
       if (u0 == ((long long)(cc + 1) * T) / G) continue;  // empty range
       const int slot = (cc == cf && u0 != s) ? 1 : 0;
-      s_part[n++] = (cc * 2 + slot) * M * (D + 2);
+      s_part[n++] = cc * 2 + slot;
     }
     s_n = n;
   }
@@ -567,14 +569,14 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(AttnDev p) {
     const int m = i / D, col = i - m * D;
     float mstar = -INFINITY;
     for (int k = 0; k < n; ++k)
-      mstar = fmaxf(mstar, p.part[s_part[k] + M * D + m]);
+      mstar = fmaxf(mstar, p.part_ml[(size_t)s_part[k] * 2 * M + m]);
     float o = 0.0f, l = 0.0f;
     for (int k = 0; k < n; ++k) {
-      const float* part = p.part + s_part[k];
-      const float mq = part[M * D + m];
+      const float* ml = p.part_ml + (size_t)s_part[k] * 2 * M;
+      const float mq = ml[m];
       const float w = mq == -INFINITY ? 0.0f : ex2((mq - mstar) * c2);
-      o += part[(size_t)m * D + col] * w;
-      l += part[M * D + M + m] * w;
+      o += p.part_o[((size_t)s_part[k] * M + m) * D + col] * w;
+      l += ml[M + m] * w;
     }
     const int r = m / g, j = m % g;
     p.out[(((size_t)b * K + r) * Hq + h * g + j) * D + col] =
@@ -662,9 +664,22 @@ size_t attn_smem_bytes(int D, int MW, int B) {
          (size_t)(B + 1) * 4;
 }
 
+// Workspace: the unit prefix (ints), then the split-segment partials
+// part_o [G][2][M][D] and part_ml [G][2][2][M] (fp32).
+static size_t ws_ints_bytes(int B) {
+  return ((size_t)(B + 2) * 4 + 255) & ~size_t(255);
+}
+
 size_t attn_workspace_bytes_impl(int B, int M, int D, int G) {
-  const size_t ints = ((size_t)(B + 2) * 4 + 255) & ~size_t(255);
-  return ints + (size_t)G * 2 * M * (D + 2) * 4;
+  return ws_ints_bytes(B) + (size_t)G * 2 * M * (D + 2) * 4;
+}
+
+void attn_partial_ptrs(const isd_attn_args* a, int G, float** part_o,
+                       float** part_ml) {
+  const int M = a->K * (a->Hq / a->Hkv);
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  *part_o = reinterpret_cast<float*>(ws + ws_ints_bytes(a->B));
+  *part_ml = *part_o + (size_t)G * 2 * M * a->d;
 }
 
 template <int D, int MW>
@@ -688,8 +703,7 @@ static int launch_bf16(const isd_attn_args* a, int G, cudaStream_t st) {
   p.status = a->status;
   uint8_t* ws = static_cast<uint8_t*>(a->workspace);
   p.ws_int = reinterpret_cast<int32_t*>(ws);
-  p.part = reinterpret_cast<float*>(
-      ws + (((size_t)(a->B + 2) * 4 + 255) & ~size_t(255)));
+  attn_partial_ptrs(a, G, &p.part_o, &p.part_ml);
   const size_t smem = attn_smem_bytes(D, MW, a->B);
   auto kern = attn_bf16_kernel<D, MW, NW, NL>;
   // The shared-memory opt-in is per device; it is set on every call (a
@@ -713,8 +727,7 @@ int launch_attn_combine(const isd_attn_args* a, int G, cudaStream_t st) {
   p.lse = a->lse;
   uint8_t* ws = static_cast<uint8_t*>(a->workspace);
   p.ws_int = reinterpret_cast<int32_t*>(ws);
-  p.part = reinterpret_cast<float*>(
-      ws + (((size_t)(a->B + 2) * 4 + 255) & ~size_t(255)));
+  attn_partial_ptrs(a, G, &p.part_o, &p.part_ml);
   if (a->d == 128)
     attn_combine_kernel<128><<<dim3(a->Hkv, a->B), 256, (size_t)G * 4, st>>>(p);
   else

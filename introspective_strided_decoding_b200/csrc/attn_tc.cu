@@ -55,6 +55,8 @@ namespace isd {
 
 // Shared with attn.cu: unit prefix, partial layout and combine kernel.
 int launch_attn_combine(const isd_attn_args* a, int G, cudaStream_t st);
+void attn_partial_ptrs(const isd_attn_args* a, int G, float** part_o,
+                       float** part_ml);
 
 namespace tc {
 
@@ -68,11 +70,10 @@ constexpr int kMmaWarp = 4;
 constexpr int kLoadWarps = 4;
 constexpr int kPagesPerLoader = kNB / kLoadWarps;
 constexpr int kThreads = (kSmWarps + 1 + kLoadWarps) * 32;   // 288
-constexpr int kLoadThreads = kLoadWarps * 32;
 constexpr int kKStages = 2;                  // K ring
 constexpr int kMaxVStages = 4;               // V ring (fewer if Q, P are big)
-constexpr int kBarBytes = 32 * 8;            // mbarriers (2 (SK + SV) + 12)
-constexpr int kStaticSmem = 2048;            // __shared__ arrays, rounded up
+constexpr int kBarBytes = 32 * 8;            // mbarriers (2 (SK + SV) + 17)
+constexpr int kStaticSmem = 3072;            // __shared__ arrays, rounded up
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint64_t kWaitCycles = 400000000ull;   // ~0.2 s
 
@@ -86,7 +87,10 @@ struct Params {
   const int32_t* page_table;
   const int32_t* seq_len;
   int32_t* status;
-  float* part;
+  float* part_o;      // [G][2][M][128]: unnormalised O of split segments
+  float* part_ml;     // [G][2][2][M]: raw row max, then row sum
+  int lse_tma;        // lse [B][K][Hq] written by TMA (else plain stores)
+  int ml_bulk;        // part_ml rows written by a bulk copy (else plain)
   int32_t* ws_int;
 };
 
@@ -224,6 +228,49 @@ ISD_DEV void tmem_scale32(uint32_t taddr, const float* f) {
   }
 }
 
+// TMA stores from shared memory (bulk async-group completion).
+ISD_DEV void tma_store_4d(const CUtensorMap* m, const void* src, int c0, int c1,
+                          int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, "
+      "%5}], [%1];" ::"l"(m),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+ISD_DEV void tma_store_2d(const CUtensorMap* m, const void* src, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], "
+      "[%1];" ::"l"(m),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1)
+      : "memory");
+}
+ISD_DEV void tma_store_3d(const CUtensorMap* m, const void* src, int c0, int c1,
+                          int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], "
+      "[%1];" ::"l"(m),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+// Plain bulk copy shared -> global (16-byte aligned, size a multiple of 16).
+ISD_DEV void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile(
+      "cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+      "r"(smem_u32(src)), "r"(bytes)
+      : "memory");
+}
+ISD_DEV void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Source shared memory of every committed store has been read.
+ISD_DEV void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Every committed store has completed.
+ISD_DEV void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // Named barrier 1 joins the four softmax warps.
 ISD_DEV void sm_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 // OR of `v` over the four softmax warps (also a barrier among them).
@@ -322,22 +369,185 @@ struct BlockWalk {
   }
 };
 
+// What the segment epilogue needs besides the finished segment itself.
+template <int NCH>
+struct EpiIn {
+  __nv_bfloat16* out;
+  float* part_o;
+  float* lse;
+  float* part_ml;
+  int32_t* status;
+  const CUtensorMap* tm_out;
+  const CUtensorMap* tm_part;
+  const CUtensorMap* tm_lse;
+  float* small;              // staged lse, or the partial's max and sum
+  int lse_tma, ml_bulk;
+  uint32_t tmem_lane;        // TMEM base + this warp's lane quarter
+  uint8_t* ps;               // P tiles (staging)
+  uint64_t* p_empty;
+  uint64_t* o_free;
+  const float* m_raw;        // [NOB][N]
+  float* x_red;              // [4][32]
+  float* r_val;              // [32]
+  int g, K, Hq, M, c;
+  float c2;
+};
+
+// Stores the finished segment `code` (packed b, h, O buffer, complete,
+// slot) whose last block is `blk`: reduces the per-key row sums over the
+// 128 keys, stages O / l (bf16) or the unnormalised O (fp32, 64 columns
+// at a time) in the P tile of block blk, and writes it with TMA stores
+// issued by thread 0; the lse or the partial's max and sum go directly.
+// Runs on the four softmax warps.  Not inlined: its registers would
+// otherwise add to those live across the block loop.  `stage_buf` is a
+// P tile an earlier store may still be reading.  Returns `failed`.
+template <int NCH>
+__device__ __noinline__ bool store_segment(const EpiIn<NCH>& in, int blk, int code,
+                                           int stage_buf, bool failed) {
+  constexpr int N = 32 * NCH;
+  constexpr int NPB = NCH >= 3 ? 1 : 2;
+  constexpr int NOB = NCH <= 2 ? 2 : 1;
+  constexpr int PB = NCH * kKeys * 64;
+  constexpr uint32_t kO = 0, kL = NOB * N + 2 * N;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, kl = tid;
+  const int b = code >> 12, h = (code >> 3) & 511, tb = (code >> 2) & 1;
+  const bool complete = (code >> 1) & 1;
+  const int slot = code & 1, M = in.M;
+  auto stage_sync = [&]() {    // the earlier store has read its tile
+    if (tid == 0) bulk_wait_read();
+    sm_sync();
+  };
+  // O^T of the segment is complete once the P V of its last block lands:
+  // phase blk / NPB of p_empty[blk % NPB], at most one phase past the last
+  // one these threads waited for there.
+  wait_or_fail(&in.p_empty[blk % NPB], (blk / NPB) & 1, failed, in.status);
+  tc_fence_after();
+  if (stage_buf >= 0) stage_sync();
+  const uint32_t eo = kO + tb * N, el = kL + tb * N;
+  const float* em = in.m_raw + tb * N;
+  uint8_t* stg = in.ps + (blk % NPB) * PB;          // N * 256 bytes
+  float* pml = in.part_ml + ((size_t)(in.c * 2 + slot)) * 2 * M;
+  const int prow = (in.c * 2 + slot) * M;           // first part_o row
+#pragma unroll 1
+  for (int hb = 0; hb < (complete ? 1 : 2); ++hb) {
+    // A complete segment stores bf16 rows [M][128] in one pass; a partial
+    // one fp32 rows, 64 columns per pass ([M][64] staged).
+    if (hb == 1) stage_sync();
+#pragma unroll 1
+    for (int ch = 0; ch < NCH; ++ch) {
+      float v[32];
+      tmem_ld32(in.tmem_lane + el + ch * 32, v);
+      warp_transpose_reduce<false>(v, lane);
+      in.x_red[warp * 32 + lane] = v[0];
+      sm_sync();
+      if (warp == 0)
+        in.r_val[lane] = (in.x_red[lane] + in.x_red[32 + lane]) +
+                         (in.x_red[64 + lane] + in.x_red[96 + lane]);
+      sm_sync();
+      float o[32];
+      tmem_ld32(in.tmem_lane + eo + ch * 32, o);   // lane = d = kl
+      if (complete) {
+#pragma unroll
+        for (int q = 0; q < 32; q += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(&in.r_val[q]);
+          const float inv[4] = {1.0f / l4.x, 1.0f / l4.y, 1.0f / l4.z,
+                                1.0f / l4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int col = ch * 32 + q + u;
+            if (col < M)
+              *reinterpret_cast<__nv_bfloat16*>(stg + col * 256 + kl * 2) =
+                  __float2bfloat16_rn(o[q + u] * inv[u]);
+          }
+        }
+      } else if ((kl >> 6) == hb) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const int col = ch * 32 + q;
+          if (col < M)
+            *reinterpret_cast<float*>(stg + col * 256 + (kl & 63) * 4) = o[q];
+        }
+      }
+      if (warp == 0 && hb == 0) {
+        // lse, or the partial's max and sum: staged for a TMA / bulk store
+        // when the layout allows one (plain stores stall behind the KV
+        // stream), else written directly.
+        const int col = ch * 32 + lane;
+        if (col < M) {
+          const float lt = in.r_val[lane], mr = em[col];
+          if (complete) {
+            if (in.lse) {
+              const float v = (mr * in.c2 + log2f(lt)) * kLn2;
+              if (in.lse_tma) {
+                in.small[col] = v;
+              } else {
+                const int rq = col / in.g, jq = col - rq * in.g;
+                in.lse[((size_t)b * in.K + rq) * in.Hq + h * in.g + jq] = v;
+              }
+            }
+          } else if (in.ml_bulk) {
+            in.small[col] = mr;
+            in.small[M + col] = lt;
+          } else {
+            pml[col] = mr;
+            pml[M + col] = lt;
+          }
+        }
+      }
+    }
+    // Staged rows -> global through the async proxy.
+    proxy_fence();
+    sm_sync();
+    if (tid == 0) {
+      if (complete) {
+        tma_store_4d(in.tm_out, stg, 0, h * in.g, 0, b);
+        if (in.lse && in.lse_tma) tma_store_3d(in.tm_lse, in.small, h * in.g, 0, b);
+      } else {
+        tma_store_2d(in.tm_part, stg, hb * 64, prow);
+        if (hb == 0 && in.ml_bulk) bulk_store(pml, in.small, 8 * M);
+      }
+      bulk_commit();
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&in.o_free[tb]);
+  return failed;
+}
+
 // NCH: 32-column chunks of the padded query rows (N = 32 * NCH).
 template <int NCH>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kc,
                    const __grid_constant__ CUtensorMap tm_vc,
                    const __grid_constant__ CUtensorMap tm_kn,
-                   const __grid_constant__ CUtensorMap tm_vn, Params p) {
+                   const __grid_constant__ CUtensorMap tm_vn,
+                   const __grid_constant__ CUtensorMap tm_out,
+                   const __grid_constant__ CUtensorMap tm_part,
+                   const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_lse, Params p) {
   constexpr int N = 32 * NCH;
   constexpr int QH = N * 128;              // one 64-column half of Q
   // P tile [128 keys][N rows]: 32-row atoms of 128 keys x 64 B (64-byte
   // swizzle), atom a holding rows 32a..32a+31.
   constexpr int PA = kKeys * 64;           // one 32-row atom (8 KB)
   constexpr int PB = NCH * PA;             // one P buffer
-  constexpr int NPB = NCH == 4 ? 1 : 2;    // P^T buffers (one at N = 128)
-  constexpr uint32_t kO = 0, kS = N, kL = 3 * N;       // TMEM columns
-  constexpr uint32_t kCols = 4 * N <= 128 ? 128 : (4 * N <= 256 ? 256 : 512);
+  // Buffers per segment-level resource: two let the next (b, h) segment
+  // start (its Q load, its first P V) while the previous one finishes;
+  // the largest row counts keep one where memory is short.
+  constexpr int NQB = NCH == 4 ? 1 : 2;    // Q tiles (shared memory)
+  constexpr int NPB = NCH >= 3 ? 1 : 2;    // P tiles (shared memory)
+  // O^T accumulators, row-sum partials (TMEM) and row maxima: with two, a
+  // segment's epilogue is deferred until the next segment's first block
+  // has been handed to the MMA warp, so the pipeline never waits on it.
+  constexpr int NOB = NCH <= 2 ? 2 : 1;
+  constexpr bool kDefer = NOB == 2;
+  constexpr int QB = 2 * QH;               // one Q tile
+  // TMEM columns: O^T buffers, two S^T buffers, the row-sum buffers.
+  constexpr uint32_t kO = 0, kS = NOB * N, kL = NOB * N + 2 * N;
+  constexpr uint32_t kColsUsed = kL + NOB * N;
+  constexpr uint32_t kCols = kColsUsed <= 128 ? 128 : (kColsUsed <= 256 ? 256 : 512);
+  static_assert(kColsUsed <= 512, "TMEM columns");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -349,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* kr = base;                                  // SK K tiles
   uint8_t* vr = kr + SK * kTile;                       // SV V tiles
   uint8_t* qs = vr + SV * kTile;                       // Q tile [N][128]
-  uint8_t* ps = qs + 2 * QH;                           // NPB P^T tiles
+  uint8_t* ps = qs + NQB * QB;                         // NPB P^T tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(ps + NPB * PB);
   uint64_t* k_full = bars;                             // [SK]
   uint64_t* k_empty = k_full + SK;                     // [SK]
@@ -359,18 +569,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_free = s_full + 2;                       // [2]
   uint64_t* p_full = s_free + 2;                       // [NPB]
   uint64_t* p_empty = p_full + 2;                      // [NPB]
-  uint64_t* q_full = p_empty + 2;
-  uint64_t* q_empty = q_full + 1;
-  uint64_t* o_free = q_empty + 1;
-  uint64_t* fin = o_free + 1;                          // all MMAs done
+  uint64_t* q_full = p_empty + 2;                      // [NQB]
+  uint64_t* q_empty = q_full + 2;                      // [NQB]
+  uint64_t* o_free = q_empty + 2;                      // [NOB]
+  uint64_t* fin = o_free + 2;                          // all MMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBarBytes / 8);
-  int* prefix = reinterpret_cast<int*>(tmem_slot + 4);
+  int* prefix = reinterpret_cast<int*>(tmem_slot + 4);  // [B + 1]
+  int* seqL = prefix + p.B + 1;                          // [B] clamped L_b
   __shared__ int scan_sh[33];
   __shared__ int s_bad;
-  __shared__ __align__(16) float m_raw[N];    // reference max per row (raw)
+  __shared__ __align__(16) float m_raw[NOB][N];  // reference max per row
   __shared__ __align__(16) float m_sc[N];     // the same times c (-inf kept)
   __shared__ float x_red[kSmWarps][32];       // cross-warp reduction
   __shared__ __align__(16) float r_val[32];   // per-row factor of a chunk
+  __shared__ __align__(128) float ep_small[2 * 128];  // staged lse / max, sum
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int B = p.B, Hkv = p.Hkv, M = p.M;
@@ -383,8 +595,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool bad = false;
         if (L < 0) { bad = true; L = 0; }
         int n = (L + kPage - 1) / kPage;
-        if (n > p.stride) { bad = true; n = p.stride; }
+        if (n > p.stride) { bad = true; n = p.stride; L = n * kPage; }
         if (bad) s_bad = 1;
+        seqL[b] = L;
         return Hkv * (n + 1);
       },
       prefix, scan_sh);
@@ -407,17 +620,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[s], kSmWarps);
       mbar_init(&p_empty[s], 1);
     }
-    mbar_init(q_full, kLoadThreads);
-    mbar_init(q_empty, 1);
-    mbar_init(o_free, kSmWarps);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);             // one expect_tx arrival (TMA)
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&o_free[s], kSmWarps);
+    }
     mbar_init(fin, 1);
     fence_barrier_init();
   }
   // Padding rows of Q (M..N-1) stay zero for the whole kernel.
-  for (int i = tid; i < N * 16; i += blockDim.x) {
-    const int row = i >> 4, ch = i & 15;
+  for (int i = tid; i < NQB * N * 16; i += blockDim.x) {
+    const int qb = i / (N * 16), row = (i >> 4) % N, ch = i & 15;
     if (row < M) continue;
-    *reinterpret_cast<uint4*>(qs + (ch >> 3) * QH + row * 128 +
+    *reinterpret_cast<uint4*>(qs + qb * QB + (ch >> 3) * QH + row * 128 +
                               (((ch & 7) ^ (row & 7)) << 4)) =
         make_uint4(0, 0, 0, 0);
   }
@@ -454,40 +669,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lw = lt >> 5;
     BlockWalk w;
     w.init(prefix, B, Hkv, u0, u1);
-    // Page ids of this warp's pages in the next block (-1: none or the
-    // tail) and its sequence length, read one block ahead: a copy must not
-    // wait on a page-table load issued just before it.
+    // Page ids of this warp's pages (-1: none or the tail), read two blocks
+    // ahead: a global load waits microseconds behind the KV stream, and a
+    // copy must not wait on one.
     static_assert(kPagesPerLoader == 2, "two pages per loader warp");
-    int pid0 = -1, pid1 = -1, Lb = 0;
-    auto page_id = [&](int k) {
-      const int uidx = w.idx0 + w.k + k;
-      return (k < w.nu() && uidx != w.units - 1)
-                 ? __ldg(p.page_table + (size_t)w.b * p.stride + uidx)
+    auto page_id = [&](const BlockWalk& x, int k) {
+      const int uidx = x.idx0 + x.k + k;
+      return (k < x.nu() && uidx != x.units - 1)
+                 ? __ldg(p.page_table + (size_t)x.b * p.stride + uidx)
                  : -1;
     };
-    auto load_ids = [&]() {
-      pid0 = page_id(lw);
-      pid1 = page_id(lw + kLoadWarps);
-      Lb = __ldg(p.seq_len + w.b);
-    };
-    if (!w.done()) load_ids();
-    int i = 0, nseg_done = 0;
+    BlockWalk wa = w;                 // two blocks ahead of w
+    int pa0 = -1, pa1 = -1, pb0 = -1, pb1 = -1;   // blocks i and i + 1
+    if (!wa.done()) {
+      pa0 = page_id(wa, lw); pa1 = page_id(wa, lw + kLoadWarps); wa.next();
+    }
+    if (!wa.done()) {
+      pb0 = page_id(wa, lw); pb1 = page_id(wa, lw + kLoadWarps); wa.next();
+    }
+    int i = 0, t = 0;    // block and segment of this CTA
     while (!w.done()) {
-      if (w.first()) {
-        // Q rows of (b, h): row m = r * g + j holds q[b][r][h*g + j][:].
-        wait_or_fail(q_empty, (nseg_done & 1) ^ 1, failed, p.status);
-        for (int q = lt; q < M * 16; q += kLoadThreads) {
-          const int m = q >> 4, ch = q & 15;
-          const int r = m / p.g, j = m - r * p.g;
-          const __nv_bfloat16* src =
-              p.q + (((size_t)w.b * p.K + r) * p.Hq + w.h * p.g + j) * D + ch * 8;
-          cp_async_16(q_s + (ch >> 3) * QH + m * 128 +
-                          (((ch & 7) ^ (m & 7)) << 4),
-                      src, 16);
-        }
-        cp_async_arrive(q_full);
-        ++nseg_done;
+      const int Lb = seqL[w.b];
+      const int pid0 = pa0, pid1 = pa1;
+      if (w.first() && lt == 0) {
+        // Q rows of (b, h) by TMA: row m = r * g + j holds q[b][r][h*g + j],
+        // the box {64, g, K} of the [B][K][Hq][128] tensor, per 64 columns.
+        const int qb = t % NQB;
+        wait_or_fail(&q_empty[qb], ((t / NQB) & 1) ^ 1, failed, p.status);
+        mbar_arrive_expect_tx(&q_full[qb], 2 * M * 128);
+        for (int hb = 0; hb < 2; ++hb)
+          tma_load_4d(qs + qb * QB + hb * QH, &tm_q, &q_full[qb], hb * 64,
+                      w.h * p.g, 0, w.b);
       }
+      if (w.first()) ++t;
       // This warp's pages of the block: page id (out of range: recorded,
       // then read as zeros from coordinate P, outside the cache tensors),
       // tail or cached, partial or full.
@@ -576,7 +790,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&v_full[vs]);
       w.next();
-      if (!w.done()) load_ids();
+      pa0 = pb0; pa1 = pb1;
+      pb0 = pb1 = -1;
+      if (!wa.done()) {
+        pb0 = page_id(wa, lw); pb1 = page_id(wa, lw + kLoadWarps); wa.next();
+      }
       ++i;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
@@ -584,8 +802,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------------------------- MMA
     BlockWalk w;
     w.init(prefix, B, Hkv, u0, u1);
-    int i = 0, nseg = 0;
-    int prev_nu = 0, prev_pb = 0;
+    int i = 0, t = -1;   // block and segment of this CTA
+    int prev_nu = 0, prev_pb = 0, prev_t = 0;
     bool prev_first = false, have_prev = false;
     const uint32_t id_qk = idesc_bf16(128, N, 0, 0);
     const uint32_t id_pv = idesc_bf16(128, N, 1, 1);
@@ -599,7 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t pa = p_s + prev_pb * PB;
         const uint32_t vb = vr_s + vs * kTile;
         for (int j = 0; j < prev_nu; ++j)
-          umma(tmem + kO, sdesc(vb + j * 2048, kKH, 1024),
+          umma(tmem + kO + (prev_t % NOB) * N, sdesc(vb + j * 2048, kKH, 1024),
                sdesc(pa + j * 1024, PA, 512, 4), id_pv,
                (prev_first && j == 0) ? 0u : 1u);
         umma_commit(&v_empty[vs]);
@@ -607,17 +825,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
-    int seg_pv = 0;  // segments whose first PV has been issued
     while (!w.done()) {
       const int ks = i % SK, sbuf = i & 1;
       if (w.first()) {
-        wait_or_fail(q_full, nseg & 1, failed, p.status);
-        // Q arrived through cp.async (generic proxy); the tensor core
-        // reads it through the async proxy.  K and V came by TMA, or, for
-        // a partial page's V, by cp.async that its loader warp fenced.
-        proxy_fence();
-        ++nseg;
+        ++t;
+        // Q, K and V arrive by TMA (a partial page's V by cp.async that its
+        // loader warp fences before arriving).
+        wait_or_fail(&q_full[t % NQB], (t / NQB) & 1, failed, p.status);
       }
+      const int qb = t % NQB;
       wait_or_fail(&k_full[ks], (i / SK) & 1, failed, p.status);
       wait_or_fail(&s_free[sbuf], ((i >> 1) & 1) ^ 1, failed, p.status);
       tc_fence_after();
@@ -628,27 +844,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < 8; ++kk)
           umma(tmem + kS + sbuf * N,
                sdesc(kb + (kk >> 2) * kKH + (kk & 3) * 32, 16, 1024),
-               sdesc(q_s + (kk >> 2) * QH + (kk & 3) * 32, 16, 1024), id_qk,
+               sdesc(q_s + qb * QB + (kk >> 2) * QH + (kk & 3) * 32, 16, 1024),
+               id_qk,
                kk > 0 ? 1u : 0u);
         umma_commit(&s_full[sbuf]);
         umma_commit(&k_empty[ks]);
-        if (w.last()) umma_commit(q_empty);
+        if (w.last()) umma_commit(&q_empty[qb]);
       }
       __syncwarp();
       if (have_prev) {
-        if (prev_first && seg_pv > 0)
-          wait_or_fail(o_free, (seg_pv - 1) & 1, failed, p.status);
-        if (prev_first) ++seg_pv;
+        // The first P V of segment t overwrites O^T buffer t % NOB: the
+        // epilogue of segment t - NOB must have read it.
+        if (prev_first && prev_t >= NOB)
+          wait_or_fail(&o_free[prev_t % NOB], ((prev_t / NOB) & 1) ^ 1, failed,
+                       p.status);
         issue_pv(i - 1);
       }
       have_prev = true;
-      prev_nu = w.nu(); prev_pb = i % NPB; prev_first = w.first();
+      prev_nu = w.nu(); prev_pb = i % NPB; prev_first = w.first(); prev_t = t;
       w.next();
       ++i;
     }
     if (have_prev) {
-      if (prev_first && seg_pv > 0)
-        wait_or_fail(o_free, (seg_pv - 1) & 1, failed, p.status);
+      if (prev_first && prev_t >= NOB)
+        wait_or_fail(&o_free[prev_t % NOB], ((prev_t / NOB) & 1) ^ 1, failed,
+                     p.status);
       issue_pv(i - 1);
     }
     // Every MMA this CTA issued has completed before TMEM is released.
@@ -664,11 +884,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c2 = p.scale_log2;
     BlockWalk w;
     w.init(prefix, B, Hkv, u0, u1);
-    int i = 0, L = 0;
+    // A finished segment whose O^T and row sums still have to be stored.
+    // Packed into two words (the pending state lives across the block loop):
+    // blk, then b << 12 | h << 3 | (t % NOB) << 2 | complete << 1 | slot.
+    struct Pending {
+      int blk, code;
+      ISD_DEV int b() const { return code >> 12; }
+      ISD_DEV int h() const { return (code >> 3) & 511; }
+      ISD_DEV int tb() const { return (code >> 2) & 1; }
+      ISD_DEV bool complete() const { return (code >> 1) & 1; }
+      ISD_DEV int slot() const { return code & 1; }
+    };
+    Pending ep{-1, 0};
+    // The epilogue stages each segment's output in the P tile of its last
+    // block (free once that block's P V has landed) and writes it with TMA
+    // stores issued by one thread: per-thread global stores queue behind
+    // the KV stream and stall the softmax warps for microseconds.
+    int stage_buf = -1;          // P tile a TMA store may still be reading
+    auto stage_sync = [&]() {    // wait for that read (all 128 threads)
+      if (tid == 0) bulk_wait_read();
+      sm_sync();
+      stage_buf = -1;
+    };
+    const EpiIn<NCH> ein{p.out, p.part_o, p.lse, p.part_ml, p.status, &tm_out,
+                         &tm_part, &tm_lse, ep_small, p.lse_tma, p.ml_bulk,
+                         tmem + lane_base, ps, p_empty, o_free, &m_raw[0][0],
+                         &x_red[0][0], r_val, p.g, p.K, p.Hq, M, c, c2};
+    auto epilogue = [&](const Pending& e) {
+      failed = store_segment<NCH>(ein, e.blk, e.code, stage_buf, failed);
+      stage_buf = e.blk % NPB;
+    };
+    int i = 0, t = -1, L = 0;    // block and segment of this CTA
     while (!w.done()) {
       const int sbuf = i & 1;
       const bool first = w.first();
-      if (first) L = __ldg(p.seq_len + w.b);
+      if (first) {
+        L = seqL[w.b];
+        ++t;
+      }
+      const uint32_t o_col = kO + (t % NOB) * N;   // this segment's O^T
+      const uint32_t l_col = kL + (t % NOB) * N;   // and row sums
+      float* m_row = m_raw[t % NOB];
       // Which rows may see this thread's key: every row for a cached slot
       // inside the prefix; rows at stride position >= rr for stride row rr
       // of the tail (columns col >= rr * g); none past the block's end.
@@ -682,6 +938,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int pbi = i % NPB;
       wait_or_fail(&p_empty[pbi], ((i / NPB) & 1) ^ 1, failed, p.status);
+      if (stage_buf == pbi) stage_sync();   // a TMA store still reads it
       bool o_ready = false;
       uint8_t* pt = ps + pbi * PB;
       uint8_t* prow = pt + kl * 64;               // this key's row of P
@@ -733,7 +990,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) l[e] = 0.0f;
           } else {
-            tmem_ld32(tmem + lane_base + kL + ch * 32, l);
+            tmem_ld32(tmem + lane_base + l_col + ch * 32, l);
           }
         };
         // Optimistic pass; the vote asks whether any exponent exceeded 8
@@ -756,11 +1013,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int col = ch * 32 + lane;
             const float bm = fmaxf(fmaxf(x_red[0][lane], x_red[1][lane]),
                                    fmaxf(x_red[2][lane], x_red[3][lane]));
-            const float m_old = first ? -INFINITY : m_raw[col];
+            const float m_old = first ? -INFINITY : m_row[col];
             const float m_new = fmaxf(m_old, bm);
             r_val[lane] =
                 m_old == -INFINITY ? 0.0f : ex2((m_old - m_new) * c2);
-            m_raw[col] = m_new;
+            m_row[col] = m_new;
             // Finite stand-in for a row with no key yet, so that masked
             // scores still give 0 and an unmasked one votes.
             m_sc[col] = fmaxf(m_new * c2, -3.0e38f);
@@ -777,81 +1034,33 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_after();
               o_ready = true;
             }
-            tmem_scale32(tmem + lane_base + kO + ch * 32, r_val);
-            tmem_scale32(tmem + lane_base + kL + ch * 32, r_val);
+            tmem_scale32(tmem + lane_base + o_col + ch * 32, r_val);
+            tmem_scale32(tmem + lane_base + l_col + ch * 32, r_val);
           }
           load_l();
           p_pass();
         }
-        tmem_st32(tmem + lane_base + kL + ch * 32, l);
+        tmem_st32(tmem + lane_base + l_col + ch * 32, l);
       }
       proxy_fence();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[pbi]);
+      if (kDefer) {
+        if (ep.blk >= 0) epilogue(ep);
+        ep.blk = -1;
+      }
       if (w.last()) {
-        // Epilogue: O^T of this segment is complete once its last P V
-        // (block i) lands; the row sums are reduced over the 128 keys.
-        wait_or_fail(&p_empty[pbi], (i / NPB) & 1, failed, p.status);
-        tc_fence_after();
-        const int slot = (w.seg_begin_u == u0) ? 0 : 1;
-        float* part = p.part + ((size_t)(c * 2 + slot)) * M * (D + 2);
-#pragma unroll 1
-        for (int ch = 0; ch < NCH; ++ch) {
-          float v[32];
-          tmem_ld32(tmem + lane_base + kL + ch * 32, v);
-          warp_transpose_reduce<false>(v, lane);
-          x_red[warp][lane] = v[0];
-          sm_sync();
-          if (warp == 0)
-            r_val[lane] = (x_red[0][lane] + x_red[1][lane]) +
-                          (x_red[2][lane] + x_red[3][lane]);
-          sm_sync();
-          float lsum[32], o[32];
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(&r_val[e]);
-            lsum[e] = l4.x; lsum[e + 1] = l4.y;
-            lsum[e + 2] = l4.z; lsum[e + 3] = l4.w;
-          }
-          tmem_ld32(tmem + lane_base + kO + ch * 32, o);   // lane = d = kl
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int col = ch * 32 + e;
-            if (col < M) {
-              if (w.complete) {
-                const int rq = col / p.g, jq = col - rq * p.g;
-                p.out[(((size_t)w.b * p.K + rq) * p.Hq + w.h * p.g + jq) * D +
-                      kl] = __float2bfloat16_rn(o[e] / lsum[e]);
-              } else {
-                part[(size_t)col * D + kl] = o[e];
-              }
-            }
-          }
-          if (warp == 0) {
-            const int col = ch * 32 + lane;
-            if (col < M) {
-              const float lt = r_val[lane], mr = m_raw[col];
-              if (w.complete) {
-                if (p.lse) {
-                  const int rq = col / p.g, jq = col - rq * p.g;
-                  p.lse[((size_t)w.b * p.K + rq) * p.Hq + w.h * p.g + jq] =
-                      (mr * c2 + log2f(lt)) * kLn2;
-                }
-              } else {
-                part[(size_t)M * D + col] = mr;
-                part[(size_t)M * D + M + col] = lt;
-              }
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(o_free);
+        const Pending cur{i, (w.b << 12) | (w.h << 3) | ((t % NOB) << 2) |
+                                 ((w.complete ? 1 : 0) << 1) |
+                                 (w.seg_begin_u == u0 ? 0 : 1)};
+        if (kDefer) ep = cur; else epilogue(cur);
       }
       w.next();
       ++i;
     }
+    if (kDefer && ep.blk >= 0) epilogue(ep);
+    if (tid == 0) bulk_wait_all();
   }
   // Everyone meets before TMEM is released.
   tc_fence_before();
@@ -890,30 +1099,44 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Tiled tensor map of `rank` <= 4 dimensions (innermost first; `strides`
+// in bytes for dimensions 1..rank-1).
+static bool encode_tiled(CUtensorMap* m, CUtensorMapDataType type, int rank,
+                         const void* base, const uint64_t* dims,
+                         const uint64_t* strides, const uint32_t* box,
+                         CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rank < 1 || rank > 4) return false;
+  cuuint64_t gd[4], gs[3];
+  cuuint32_t bx[4], es[4];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+    if (i > 0) gs[i - 1] = strides[i - 1];
+  }
+  return fn(m, type, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static bool encode_tiled_4d(CUtensorMap* m, const void* base,
                             const uint64_t dims[4], const uint64_t strides[3],
                             const uint32_t box[4]) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
-  cuuint64_t gs[3] = {strides[0], strides[1], strides[2]};
-  cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
-  cuuint32_t es[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
-            gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims,
+                      strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
 // Dynamic shared memory of the kernel for N = 32 * nch rows and a V ring
-// of `sv` tiles (one P buffer at N = 128, two below).
+// of `sv` tiles (Q and P buffer counts as in the kernel).
 static size_t tc_smem(int B, int nch, int sv) {
   const size_t N = 32 * (size_t)nch;
-  const size_t npb = nch == 4 ? 1 : 2;
-  return 1024 + (size_t)(tc::kKStages + sv) * tc::kTile + 2 * N * 128 +
-         npb * 2 * N * 128 + tc::kBarBytes + 16 + (size_t)(B + 1) * 4;
+  const size_t nqb = nch == 4 ? 1 : 2, npb = nch >= 3 ? 1 : 2;
+  return 1024 + (size_t)(tc::kKStages + sv) * tc::kTile + nqb * 2 * N * 128 +
+         npb * 2 * N * 128 + tc::kBarBytes + 16 + (size_t)(2 * B + 1) * 4;
 }
 
 // Deepest V ring (at most 4, at least 2 tiles) that fits for M query rows;
@@ -951,8 +1174,8 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
   p.status = a->status;
   uint8_t* ws = static_cast<uint8_t*>(a->workspace);
   p.ws_int = reinterpret_cast<int32_t*>(ws);
-  p.part = reinterpret_cast<float*>(
-      ws + (((size_t)(a->B + 2) * 4 + 255) & ~size_t(255)));
+  attn_partial_ptrs(a, G, &p.part_o, &p.part_ml);
+  float* part_o = p.part_o;
   // K and V tensor maps: the caches [P][Hkv][16][128] and the stride's
   // staged rows [B][K][Hkv][128], 64-column boxes with the 128-byte swizzle.
   CUtensorMap tkc, tvc, tkn, tvn;
@@ -971,6 +1194,45 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
       !encode_tiled_4d(&tkn, a->k_new, dn, sn, bn) ||
       !encode_tiled_4d(&tvn, a->v_new, dn, sn, bn))
     return ISD_ERR_CUDA;
+  // Store maps: out [B][K][Hq][128] bf16, one (b, h) block of g heads by K
+  // stride rows per box; part_o [G * 2 * M][128] fp32, 64-column boxes of
+  // M rows.  No swizzle (rows are staged plainly).
+  CUtensorMap tout, tpart;
+  const uint64_t dq[4] = {128, (uint64_t)a->Hq, (uint64_t)a->K,
+                          (uint64_t)a->B};
+  const uint64_t sq[3] = {256, (uint64_t)a->Hq * 256,
+                          (uint64_t)a->K * a->Hq * 256};
+  const uint32_t bq[4] = {128, (uint32_t)p.g, (uint32_t)a->K, 1};
+  const uint64_t dp[2] = {128, (uint64_t)G * 2 * p.M};
+  const uint64_t sp[1] = {512};
+  const uint32_t bp[2] = {64, (uint32_t)p.M};
+  if (!encode_tiled(&tout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a->out, dq, sq,
+                    bq, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tiled(&tpart, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, part_o, dp, sp,
+                    bp, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return ISD_ERR_CUDA;
+  // Q [B][K][Hq][128] bf16: a (b, h) tile is the box {64, g, K, 1}, landing
+  // as rows m = r * g + j of 128 bytes in the 128-byte swizzle.
+  CUtensorMap tq;
+  const uint32_t bqq[4] = {64, (uint32_t)p.g, (uint32_t)a->K, 1};
+  if (!encode_tiled(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a->q, dq, sq, bqq,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return ISD_ERR_CUDA;
+  // lse [B][K][Hq] fp32 by TMA when rows of g values are whole 16-byte
+  // units; part_ml rows (2M floats) by a bulk copy when M is even.
+  p.lse_tma = a->lse != nullptr &&
+              (reinterpret_cast<uintptr_t>(a->lse) & 15) == 0 &&
+              p.g % 4 == 0 && a->Hq % 4 == 0;
+  p.ml_bulk = p.M % 2 == 0;
+  CUtensorMap tlse = tpart;   // any valid map when lse is not stored by TMA
+  if (p.lse_tma) {
+    const uint64_t dl[3] = {(uint64_t)a->Hq, (uint64_t)a->K, (uint64_t)a->B};
+    const uint64_t sl[2] = {(uint64_t)a->Hq * 4, (uint64_t)a->K * a->Hq * 4};
+    const uint32_t bl[3] = {(uint32_t)p.g, (uint32_t)a->K, 1};
+    if (!encode_tiled(&tlse, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a->lse, dl, sl,
+                      bl, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return ISD_ERR_CUDA;
+  }
   const int nch = (p.M + 31) / 32;
   const size_t smem = tc_smem(a->B, nch, p.sv);
   auto kern = nch == 1 ? tc::attn_tc_kernel<1>
@@ -980,7 +1242,8 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return ISD_ERR_CUDA;
-  kern<<<G, tc::kThreads, smem, st>>>(tkc, tvc, tkn, tvn, p);
+  kern<<<G, tc::kThreads, smem, st>>>(tkc, tvc, tkn, tvn, tout, tpart, tq, tlse,
+                                      p);
   if (cudaGetLastError() != cudaSuccess) return ISD_ERR_CUDA;
   return launch_attn_combine(a, G, st);
 }
