@@ -105,7 +105,7 @@ typedef struct {
   int32_t num_pages, page_table_stride;
   int32_t dtype;
   float softmax_scale;
-  int32_t num_ctas;            /* 0: one CTA per SM                       */
+  int32_t num_ctas;            /* 0: one CTA per SM; else 1..1024 CTAs    */
   const void* q;
   const void* k_new;
   const void* v_new;

@@ -28,6 +28,8 @@
 
 namespace isd {
 
+int launch_attn_combine(const isd_attn_args* a, int G, cudaStream_t st);
+
 constexpr int kStages = 16;                     // power of two
 constexpr uint64_t kWaitCycles = 4000000000ull; // ~2 s at boost clock
 
@@ -113,8 +115,8 @@ __global__ void __launch_bounds__(attn_threads<NW, NL>(), 1)
       prefix, scan_sh);
   if (tid == 0) prefix[B] = T;
   const int G = gridDim.x, c = blockIdx.x;
-  const int u0 = (int)(((long long)c * T) / G);
-  const int u1 = (int)(((long long)(c + 1) * T) / G);
+  const int u0 = split_point(prefix, B, T, Hkv, c, G);
+  const int u1 = split_point(prefix, B, T, Hkv, c + 1, G);
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], NL * 32);
@@ -127,9 +129,11 @@ __global__ void __launch_bounds__(attn_threads<NW, NL>(), 1)
     for (int i = tid; i <= B; i += blockDim.x) p.ws_int[i] = prefix[i];
     if (tid == 0) {
       p.ws_int[B + 1] = G;
+      p.ws_int[B + 2 + G] = T;
       if (s_bad && p.status) *p.status = ISD_ERR_PAGE_TABLE_FULL;
     }
   }
+  if (tid == 0) p.ws_int[B + 2 + c] = u0;   // range starts, for the combine
   if (u0 >= u1) return;
 
   // --------------------------------------------------------------- loaders
@@ -534,56 +538,90 @@ __global__ void __launch_bounds__(attn_threads<NW, NL>(), 1)
   }
 }
 
-// Merge the partials of every (b, h) whose units straddled CTAs, in CTA
-// order.  The CTAs and slots holding them are listed once per block.
+// Merges the split-KV partials of each (b, h) segment that straddles CTAs:
+// O = sum_k w_k O_k / sum_k w_k l_k with w_k = 2^((m_k - m*) c) over the
+// CTAs k holding a part (m* = max_k m_k).  One block per (b, h); the CTA
+// ranges come from the starts the attention kernel recorded.  Per 32-row
+// chunk the normalised weights w_k / L are computed once into shared
+// memory, then each thread accumulates float4 columns with independent
+// loads (no dependent load chains per element).
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(AttnDev p) {
-  extern __shared__ int s_part[];   // partial indices (CTA * 2 + slot)
+  extern __shared__ int s_dyn[];     // [G] partial indices, [G][32] weights
   __shared__ int s_n;
-  const int h = blockIdx.x, b = blockIdx.y;
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int B = p.B;
   const int* prefix = p.ws_int;
-  const long long T = prefix[B];
-  const long long G = p.ws_int[B + 1];
+  const int G = p.ws_int[B + 1];
+  const int* starts = p.ws_int + B + 2;       // [G + 1] range starts
   const int units = (prefix[b + 1] - prefix[b]) / p.Hkv;
-  const long long s = prefix[b] + (long long)h * units;
-  const long long e = s + units;
-  const int cf = (int)(((s + 1) * G - 1) / T);
-  const int cl = (int)(((e) * G - 1) / T);
+  const int s = prefix[b] + h * units, e = s + units;
+  // CTAs whose range holds unit s and unit e - 1: the last c with
+  // starts[c] <= unit (empty ranges have equal neighbouring starts).
+  auto owner = [&](int u) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (starts[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
+  const int cf = owner(s), cl = owner(e - 1);
   if (cf == cl) return;
+  int* s_part = s_dyn;
+  float* s_w = reinterpret_cast<float*>(s_dyn + G);
   const int M = p.M, g = p.g, K = p.K, Hq = p.Hq;
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     int n = 0;
     for (int cc = cf; cc <= cl; ++cc) {
-      const long long u0 = ((long long)cc * T) / G;
-      if (u0 == ((long long)(cc + 1) * T) / G) continue;  // empty range
-      const int slot = (cc == cf && u0 != s) ? 1 : 0;
-      s_part[n++] = cc * 2 + slot;
+      if (starts[cc] == starts[cc + 1]) continue;   // empty range
+      // slot 0: the part that starts at the CTA's own first unit.
+      s_part[n++] = cc * 2 + (starts[cc] < s ? 1 : 0);
     }
     s_n = n;
   }
   __syncthreads();
   const int n = s_n;
   const float c2 = p.scale_log2;
-  for (int i = threadIdx.x; i < M * D; i += blockDim.x) {
-    const int m = i / D, col = i - m * D;
-    float mstar = -INFINITY;
-    for (int k = 0; k < n; ++k)
-      mstar = fmaxf(mstar, p.part_ml[(size_t)s_part[k] * 2 * M + m]);
-    float o = 0.0f, l = 0.0f;
-    for (int k = 0; k < n; ++k) {
-      const float* ml = p.part_ml + (size_t)s_part[k] * 2 * M;
-      const float mq = ml[m];
-      const float w = mq == -INFINITY ? 0.0f : ex2((mq - mstar) * c2);
-      o += p.part_o[((size_t)s_part[k] * M + m) * D + col] * w;
-      l += ml[M + m] * w;
+  for (int r0 = 0; r0 < M; r0 += 32) {
+    const int rows = min(32, M - r0);
+    if (tid < rows) {
+      const int m = r0 + tid;
+      float mstar = -INFINITY;
+      for (int k = 0; k < n; ++k)
+        mstar = fmaxf(mstar, p.part_ml[(size_t)s_part[k] * 2 * M + m]);
+      float l = 0.0f;
+      for (int k = 0; k < n; ++k) {
+        const float* ml = p.part_ml + (size_t)s_part[k] * 2 * M;
+        const float w = ml[m] == -INFINITY ? 0.0f : ex2((ml[m] - mstar) * c2);
+        s_w[k * 32 + tid] = w;
+        l += ml[M + m] * w;
+      }
+      const float inv = 1.0f / l;
+      for (int k = 0; k < n; ++k) s_w[k * 32 + tid] *= inv;
+      if (p.lse) {
+        const int r = m / g, j = m - r * g;
+        p.lse[((size_t)b * K + r) * Hq + h * g + j] =
+            (mstar * c2 + log2f(l)) * kLn2;
+      }
     }
-    const int r = m / g, j = m % g;
-    p.out[(((size_t)b * K + r) * Hq + h * g + j) * D + col] =
-        __float2bfloat16_rn(o / l);
-    if (p.lse && col == 0)
-      p.lse[((size_t)b * K + r) * Hq + h * g + j] =
-          (mstar * c2 + log2f(l)) * kLn2;
+    __syncthreads();
+    for (int q = tid; q < rows * (D / 4); q += blockDim.x) {
+      const int rl = q / (D / 4), col = (q - rl * (D / 4)) * 4;
+      const int m = r0 + rl;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int k = 0; k < n; ++k) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(
+            p.part_o + ((size_t)s_part[k] * M + m) * D + col));
+        const float w = s_w[k * 32 + rl];
+        acc.x += v.x * w; acc.y += v.y * w; acc.z += v.z * w; acc.w += v.w * w;
+      }
+      const int r = m / g, j = m - r * g;
+      __nv_bfloat16* o = p.out + (((size_t)b * K + r) * Hq + h * g + j) * D + col;
+      *reinterpret_cast<uint2*>(o) =
+          make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+    }
+    __syncthreads();
   }
 }
 
@@ -666,19 +704,20 @@ size_t attn_smem_bytes(int D, int MW, int B) {
 
 // Workspace: the unit prefix (ints), then the split-segment partials
 // part_o [G][2][M][D] and part_ml [G][2][2][M] (fp32).
-static size_t ws_ints_bytes(int B) {
-  return ((size_t)(B + 2) * 4 + 255) & ~size_t(255);
+// Integers: the unit prefix [B + 1], G, then the CTA range starts [G + 1].
+static size_t ws_ints_bytes(int B, int G) {
+  return ((size_t)(B + G + 3) * 4 + 255) & ~size_t(255);
 }
 
 size_t attn_workspace_bytes_impl(int B, int M, int D, int G) {
-  return ws_ints_bytes(B) + (size_t)G * 2 * M * (D + 2) * 4;
+  return ws_ints_bytes(B, G) + (size_t)G * 2 * M * (D + 2) * 4;
 }
 
 void attn_partial_ptrs(const isd_attn_args* a, int G, float** part_o,
                        float** part_ml) {
   const int M = a->K * (a->Hq / a->Hkv);
   uint8_t* ws = static_cast<uint8_t*>(a->workspace);
-  *part_o = reinterpret_cast<float*>(ws + ws_ints_bytes(a->B));
+  *part_o = reinterpret_cast<float*>(ws + ws_ints_bytes(a->B, G));
   *part_ml = *part_o + (size_t)G * 2 * M * a->d;
 }
 
@@ -712,8 +751,8 @@ static int launch_bf16(const isd_attn_args* a, int G, cudaStream_t st) {
                            (int)smem) != cudaSuccess)
     return ISD_ERR_CUDA;
   kern<<<G, attn_threads<NW, NL>(), smem, st>>>(p);
-  attn_combine_kernel<D><<<dim3(a->Hkv, a->B), 256, (size_t)G * 4, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? ISD_OK : ISD_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return ISD_ERR_CUDA;
+  return launch_attn_combine(a, G, st);
 }
 
 // Merges the split-KV partials any attention kernel left in the workspace
@@ -728,10 +767,14 @@ int launch_attn_combine(const isd_attn_args* a, int G, cudaStream_t st) {
   uint8_t* ws = static_cast<uint8_t*>(a->workspace);
   p.ws_int = reinterpret_cast<int32_t*>(ws);
   attn_partial_ptrs(a, G, &p.part_o, &p.part_ml);
-  if (a->d == 128)
-    attn_combine_kernel<128><<<dim3(a->Hkv, a->B), 256, (size_t)G * 4, st>>>(p);
-  else
-    attn_combine_kernel<64><<<dim3(a->Hkv, a->B), 256, (size_t)G * 4, st>>>(p);
+  // Shared memory: G partial indices and G x 32 weights.
+  const size_t smem = (size_t)G * 132;
+  auto kern = a->d == 128 ? attn_combine_kernel<128> : attn_combine_kernel<64>;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return ISD_ERR_CUDA;
+  kern<<<dim3(a->Hkv, a->B), 256, smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? ISD_OK : ISD_ERR_CUDA;
 }
 

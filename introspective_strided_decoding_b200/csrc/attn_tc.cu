@@ -603,8 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefix, scan_sh);
   if (tid == 0) prefix[B] = T;
   const int G = gridDim.x, c = blockIdx.x;
-  const int u0 = (int)(((long long)c * T) / G);
-  const int u1 = (int)(((long long)(c + 1) * T) / G);
+  const int u0 = split_point(prefix, B, T, Hkv, c, G);
+  const int u1 = split_point(prefix, B, T, Hkv, c + 1, G);
   if (tid == 0) {
     for (int s = 0; s < SK; ++s) {
       mbar_init(&k_full[s], kLoadWarps);    // one arrival per loader warp
@@ -652,9 +652,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = tid; i <= B; i += blockDim.x) p.ws_int[i] = prefix[i];
     if (tid == 0) {
       p.ws_int[B + 1] = G;
+      p.ws_int[B + 2 + G] = T;
       if (s_bad && p.status) *p.status = ISD_ERR_PAGE_TABLE_FULL;
     }
   }
+  if (tid == 0) p.ws_int[B + 2 + c] = u0;   // range starts, for the combine
   const uint32_t kr_s = smem_u32(kr), vr_s = smem_u32(vr);
   const uint32_t q_s = smem_u32(qs), p_s = smem_u32(ps);
   bool failed = false;

@@ -205,6 +205,40 @@ ISD_DEV int block_exclusive_scan_int(int n, F in, int* out, int* sh) {
 }
 
 // ---------------------------------------------------------------------------
+// Work split of the attention kernels.  The flat unit list (per sequence b,
+// per KV head h: its cached pages, then one tail unit) is cut into G
+// contiguous ranges of equal cost, a unit costing 1 and each (b, h) segment
+// kSegCost more for its fixed work (Q load, first-block max, epilogue), so
+// CTAs that meet many short sequences get fewer pages.
+
+constexpr int kSegCost = 16;
+
+// First unit of CTA c (c = G gives T).  prefix[b] = first unit of sequence
+// b for b < B; T = total units; every segment of b has the same length.
+// Nondecreasing in c.
+ISD_DEV int split_point(const int* prefix, int B, int T, int Hkv, int c,
+                        int G) {
+  const long long seg = (long long)kSegCost * Hkv;
+  const long long ctot = (long long)T + seg * B;
+  const long long x = (long long)c * ctot / G;
+  if (x >= ctot) return T;
+  int lo = 0, hi = B - 1;   // last b whose cost prefix is <= x
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((long long)prefix[mid] + seg * mid <= x) lo = mid; else hi = mid - 1;
+  }
+  const int b = lo;
+  const int end_b = b + 1 < B ? prefix[b + 1] : T;
+  const long long ub = (end_b - prefix[b]) / Hkv;   // units per segment
+  const long long rem = x - ((long long)prefix[b] + seg * b);
+  const long long h = rem / (ub + kSegCost);
+  if (h >= Hkv) return end_b;
+  const long long r = rem - h * (ub + kSegCost);
+  const long long off = r <= kSegCost ? 0 : min(r - kSegCost, ub);
+  return (int)(prefix[b] + h * ub + off);
+}
+
+// ---------------------------------------------------------------------------
 // mbarrier / TMA / ldmatrix / mma wrappers (inline PTX, sm_90+ forms).
 
 ISD_DEV uint32_t smem_u32(const void* p) {

@@ -40,7 +40,8 @@ int attn_ctas(const isd_attn_args* a) {
 int attn_check(const isd_attn_args* a) {
   if (!a) return ISD_ERR_INVALID_ARG;
   if (a->B <= 0 || a->Hq <= 0 || a->Hkv <= 0 || a->d <= 0 || a->K <= 0 ||
-      a->num_pages <= 0 || a->page_table_stride <= 0 || a->num_ctas < 0)
+      a->num_pages <= 0 || a->page_table_stride <= 0 || a->num_ctas < 0 ||
+      a->num_ctas > 1024)
     return ISD_ERR_INVALID_ARG;
   if (a->Hq % a->Hkv != 0) return ISD_ERR_INVALID_ARG;
   if (!(a->softmax_scale > 0.0f)) return ISD_ERR_INVALID_ARG;

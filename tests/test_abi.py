@@ -65,6 +65,8 @@ def _attn_args(**kw):
     (dict(B=0), isd.ERR_INVALID_ARG),
     (dict(Hq=30), isd.ERR_INVALID_ARG),            # Hq % Hkv != 0
     (dict(softmax_scale=0.0), isd.ERR_INVALID_ARG),
+    (dict(num_ctas=-1), isd.ERR_INVALID_ARG),
+    (dict(num_ctas=1025), isd.ERR_INVALID_ARG),     # at most 1024 CTAs
     (dict(d=96), isd.ERR_UNSUPPORTED),              # bf16 path: d 64 or 128
     (dict(K=6, d=64), isd.ERR_UNSUPPORTED),         # d 64: K*g = 24 rows
     (dict(K=16, Hq=96, Hkv=8), isd.ERR_UNSUPPORTED),  # K*g = 192 rows

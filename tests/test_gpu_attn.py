@@ -46,7 +46,7 @@ SMALL = [
 
 
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
-@pytest.mark.parametrize("num_ctas", [0, 1, 3, 7])
+@pytest.mark.parametrize("num_ctas", [0, 1, 3, 7, 300])
 @pytest.mark.parametrize("sharp", [False, True])
 def test_small_cases_every_output(w, num_ctas, sharp):
     cache = synth.make_cache(w, 11, DEV)
