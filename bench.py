@@ -18,6 +18,7 @@ the data path).
 """
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -52,6 +53,30 @@ def parse():
     ap.add_argument("--cpu-sample-seqs", type=int, default=4)
     ap.add_argument("--cpu-sample-steps", type=int, default=8)
     return ap.parse_args()
+
+
+# DRAM traffic of the attention kernel per algorithmic byte, from one ncu
+# capture of this workload at B = 16 (dram__bytes_read.sum +
+# dram__bytes_write.sum over the launch's algorithmic bytes; see
+# profiles/attn_tc_kernel_c64_b16_full.md).  Traffic tracks the algorithmic
+# bytes, so a full launch's traffic is this ratio times its bytes.  Valid only
+# for the kernel source the capture was taken on.
+TRAFFIC_PER_ALGO_BYTE = 340.05 / 332.02
+TRAFFIC_KERNEL_SHA256 = (
+    "71a076003bf7b68d3f9c2c4d7b2713ea6921847880a94e1e7c662821352cd6d0")
+
+
+def attention_traffic(bytes_per_launch):
+    path = os.path.join(ROOT, "introspective_strided_decoding_b200", "csrc",
+                        "attn_tc.cu")
+    try:
+        with open(path, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    if TRAFFIC_PER_ALGO_BYTE is None or sha != TRAFFIC_KERNEL_SHA256:
+        return None
+    return TRAFFIC_PER_ALGO_BYTE * bytes_per_launch
 
 
 def peaks():
@@ -366,10 +391,10 @@ def run_isd(args, world, rank, local):
                       "logits/Q/K/V generation between steps untimed",
             "parallelism": f"replicas x{world}"},
         "roofline": {
-            "kernel": "attn_bf16_kernel (+combine)", "bound": "hbm",
+            "kernel": "attn_tc_kernel (+combine)", "bound": "hbm",
             "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "peak_kind": peak_kind,
-            "traffic": None,
+            "traffic": attention_traffic(sum(attn_bytes) / len(attn_bytes)),
             "bytes_per_launch": sum(attn_bytes) / len(attn_bytes)},
         "e2e": e2e,
         "gpu_launches": Decoder.LAUNCHES_PER_STEP * args.steps,
