@@ -547,15 +547,20 @@ __global__ void __launch_bounds__(attn_threads<NW, NL>(), 1)
 // loads (no dependent load chains per element).
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(AttnDev p) {
-  extern __shared__ int s_dyn[];     // [G] partial indices, [G][32] weights
+  // Shared: [G] partial indices, [G][32] weights, [G + 1] range starts.
+  extern __shared__ int s_dyn[];
   __shared__ int s_n;
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int B = p.B;
   const int* prefix = p.ws_int;
   const int G = p.ws_int[B + 1];
-  const int* starts = p.ws_int + B + 2;       // [G + 1] range starts
   const int units = (prefix[b + 1] - prefix[b]) / p.Hkv;
   const int s = prefix[b] + h * units, e = s + units;
+  // The range starts are searched in shared memory: a binary search over
+  // global memory would chain ~log2(G) dependent loads.
+  int* starts = s_dyn + G * 33;
+  for (int i = tid; i <= G; i += blockDim.x) starts[i] = p.ws_int[B + 2 + i];
+  __syncthreads();
   // CTAs whose range holds unit s and unit e - 1: the last c with
   // starts[c] <= unit (empty ranges have equal neighbouring starts).
   auto owner = [&](int u) {
@@ -767,8 +772,8 @@ int launch_attn_combine(const isd_attn_args* a, int G, cudaStream_t st) {
   uint8_t* ws = static_cast<uint8_t*>(a->workspace);
   p.ws_int = reinterpret_cast<int32_t*>(ws);
   attn_partial_ptrs(a, G, &p.part_o, &p.part_ml);
-  // Shared memory: G partial indices and G x 32 weights.
-  const size_t smem = (size_t)G * 132;
+  // Shared memory: G partial indices, G x 32 weights, G + 1 range starts.
+  const size_t smem = (size_t)G * 136 + 4;
   auto kern = a->d == 128 ? attn_combine_kernel<128> : attn_combine_kernel<64>;
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
