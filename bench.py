@@ -174,6 +174,27 @@ def barrier(world):
         torch.distributed.barrier()
 
 
+def rank_seed(seed, rank):
+    """Each replica decodes its own seeded batch."""
+    return seed + 1000 * rank
+
+
+def job_figures(total_ms, tokens, e2e_ms, e2e_tokens, world, device):
+    """Whole-job figures over the replicas: the slowest rank's device time,
+    every rank's committed tokens (max and sum all-reductions; no-ops on
+    one rank)."""
+    mx = torch.distributed.ReduceOp.MAX if world > 1 else None
+    sm = torch.distributed.ReduceOp.SUM if world > 1 else None
+    total_ms_max = allreduce(total_ms, mx, world, device)
+    tokens_all = allreduce(tokens, sm, world, device)
+    e2e_ms_max = allreduce(e2e_ms, mx, world, device)
+    e2e_tokens_all = allreduce(e2e_tokens, sm, world, device)
+    return {"total_ms_max": total_ms_max, "tokens": tokens_all,
+            "value": tokens_all / (total_ms_max / 1e3),
+            "e2e_ms_max": e2e_ms_max, "e2e_tokens": e2e_tokens_all,
+            "e2e_value": e2e_tokens_all / (e2e_ms_max / 1e3)}
+
+
 # --------------------------------------------------------- oracle sample
 def oracle_sample(w, seed, n_seqs, steps=1, skip=0):
     """Time the fp64 oracle on a bounded sample of the workload: the first
@@ -239,7 +260,7 @@ def run_isd(args, world, rank, local):
     w = synth.C64.with_(steps=args.steps + args.warmup + args.e2e_steps + 2)
     if args.batch != w.B:
         w = w.with_(B=args.batch, name=f"{w.name}_b{args.batch}")
-    seed = args.seed + 1000 * rank
+    seed = rank_seed(args.seed, rank)
     cache = synth.make_cache(w, seed, dev)
     st0 = synth.initial_state(w, seed, dev)
     dec = Decoder(w, cache, st0, dev, seed)
@@ -306,11 +327,7 @@ def run_isd(args, world, rank, local):
     status = int(dec.status.item())
     if status != isd.OK:
         raise RuntimeError(f"device status {isd.status_string(status)}")
-    total_ms_max = allreduce(total_ms, torch.distributed.ReduceOp.MAX
-                             if world > 1 else None, world, dev)
-    tokens_all = allreduce(tokens, torch.distributed.ReduceOp.SUM
-                           if world > 1 else None, world, dev)
-    value = tokens_all / (total_ms_max / 1e3)
+
     attn_bytes = [kv + qo_bytes for kv in kv_bytes]
     achieved = sum(attn_bytes) / (sum(t_attn) / 1e3) / 1e9
     step_bytes = [kv + qo_bytes + r * row_bytes for kv, r in
@@ -367,11 +384,9 @@ def run_isd(args, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
-    e2e_ms = allreduce(e2e_ms, torch.distributed.ReduceOp.MAX
-                       if world > 1 else None, world, dev)
-    e2e_tok = allreduce(e2e_tokens, torch.distributed.ReduceOp.SUM
-                        if world > 1 else None, world, dev)
-    e2e = {"value": e2e_tok / (e2e_ms / 1e3), "unit": "tokens/s",
+    job = job_figures(total_ms, tokens, e2e_ms, e2e_tokens, world, dev)
+    total_ms_max, value = job["total_ms_max"], job["value"]
+    e2e = {"value": job["e2e_value"], "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "steps": n_e2e}
 
