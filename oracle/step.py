@@ -47,6 +47,14 @@ token, and the next drafts at L_b + n_b + j (j = 1 .. N - 1) are drawn
 from q of rows n_b + j - 1 (stream DRAFT).  Their q rows (this step's
 logits buffer, the next step's "previous" buffer) are remembered.
 
+Argmax proposals (the pages' serving option of proposing the most likely
+token at each MASK position).  Drafts are x = argmax q (lowest index among
+exact ties) instead of draws from q: the proposal is a point mass at x, so
+q(x) = 1 and the ratio test accepts x with probability min(1, p(x)) =
+p(x); the speculative-sampling residual max(0, p - delta_x) is p with x
+removed (renormalised).  The verified token is still distributed as p.
+The bonus and the replacement are drawn as before.
+
 KV commit and rollback.  The pending rows 0 .. a_b (the exact token and
 the accepted drafts) are committed: n_commit_b = 1 + a_b.  Their staged
 K/V rows are copied to cache positions L_b .. L_b + n_commit_b - 1 and
@@ -67,7 +75,8 @@ STATUS_PAGE_TABLE_FULL = "page_table_full"
 
 
 def accept_resample(logits_cur, logits_prev, pending, n_pending, q_row,
-                    seq_len, seed, step, N, tie_band=TIE_BAND):
+                    seq_len, seed, step, N, tie_band=TIE_BAND,
+                    proposal="sample"):
     """One accept / resample / bonus / draft step for every sequence.
 
     logits_cur  [B][K][V]  this forward pass's logits (fp64 copy)
@@ -76,10 +85,14 @@ def accept_resample(logits_cur, logits_prev, pending, n_pending, q_row,
     n_pending   int [B]    1 or N
     q_row       int [B][N] row of logits_prev that drafted pending[b][i]
     seq_len     int [B]    committed length L_b
+    proposal    "sample" (drafts drawn from q) or "argmax" (x = argmax q)
 
     Returns a dict of numpy arrays (padding -1 / NaN) and ``ties``, a list
     of (b, kind, index) naming every near-tie decision.
     """
+    if proposal not in ("sample", "argmax"):
+        raise ValueError(proposal)
+    argmax = proposal == "argmax"
     B, K, V = logits_cur.shape
     out = {
         "accepted": np.zeros(B, dtype=np.int64),
@@ -106,9 +119,12 @@ def accept_resample(logits_cur, logits_prev, pending, n_pending, q_row,
             x = int(pending[b][i])
             m_p, s_p = row_stats(lc[i - 1])
             p_x = prob_of(lc[i - 1], x, m_p, s_p)
-            q_src = logits_prev[b][int(q_row[b][i])]
-            m_q, s_q = row_stats(q_src)
-            q_x = prob_of(q_src, x, m_q, s_q)
+            if argmax:
+                q_x = 1.0          # the proposal is a point mass at x
+            else:
+                q_src = logits_prev[b][int(q_row[b][i])]
+                m_q, s_q = row_stats(q_src)
+                q_x = prob_of(q_src, x, m_q, s_q)
             r = p_x / q_x
             u = philox.uniform(seed, b, step, L + i, philox.STREAM_ACCEPT)
             out["ratio"][b, i] = r
@@ -126,7 +142,11 @@ def accept_resample(logits_cur, logits_prev, pending, n_pending, q_row,
         out["commit_tokens"][b, 0:1 + a] = pending[b][0:1 + a]
         if rejected:
             p = probs(lc[a])
-            q = probs(logits_prev[b][int(q_row[b][a + 1])])
+            if argmax:
+                q = np.zeros(V)
+                q[int(pending[b][a + 1])] = 1.0
+            else:
+                q = probs(logits_prev[b][int(q_row[b][a + 1])])
             w = np.maximum(0.0, p - q)
             if not np.sum(w) > 0.0:
                 w = p
@@ -147,11 +167,14 @@ def accept_resample(logits_cur, logits_prev, pending, n_pending, q_row,
             out["exact_token"][b] = tok
             for j in range(1, N):
                 row = n + j - 1
-                u = philox.uniform(seed, b, step, L + n + j,
-                                   philox.STREAM_DRAFT)
-                xj, near = inverse_cdf(probs(lc[row]), u, tie_band)
-                if near:
-                    ties.append((b, "draft", j))
+                if argmax:
+                    xj = int(np.argmax(lc[row]))   # first maximal index
+                else:
+                    u = philox.uniform(seed, b, step, L + n + j,
+                                       philox.STREAM_DRAFT)
+                    xj, near = inverse_cdf(probs(lc[row]), u, tie_band)
+                    if near:
+                        ties.append((b, "draft", j))
                 out["next_pending"][b, j] = xj
                 out["next_q_row"][b, j] = row
                 out["next_q_stats"][b, j] = row_stats(lc[row])
