@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--batch", type=int, default=64,
                     help="sequences per GPU (64 = the benchmark workload; "
                          "smaller only for profiling captures)")
+    ap.add_argument("--proposal", default="sample", choices=["sample", "argmax"],
+                    help="drafts drawn from q (default) or x = argmax q")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seqs", type=int, default=4)
@@ -263,7 +265,9 @@ def run_isd(args, world, rank, local):
     seed = rank_seed(args.seed, rank)
     cache = synth.make_cache(w, seed, dev)
     st0 = synth.initial_state(w, seed, dev)
-    dec = Decoder(w, cache, st0, dev, seed)
+    dec = Decoder(w, cache, st0, dev, seed,
+                  proposal=isd.PROPOSAL_ARGMAX if args.proposal == "argmax"
+                  else isd.PROPOSAL_SAMPLE)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     hbm_peak, peak_kind = peaks()
@@ -400,7 +404,7 @@ def run_isd(args, world, rank, local):
             "workload": w.name, "B": w.B, "N": w.N, "K": w.K, "Hq": w.Hq,
             "Hkv": w.Hkv, "d": w.d, "V": w.V, "page_size": 16,
             "prefix": [w.L_lo, w.L_hi], "pages": "shuffled",
-            "target_accept": w.target_accept,
+            "target_accept": w.target_accept, "proposal": args.proposal,
             "l2": "flushed (256 MB write) before every timed step",
             "timing": "CUDA events around attention+accept+commit per step; "
                       "logits/Q/K/V generation between steps untimed",

@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define ISD_ABI_VERSION 1
+#define ISD_ABI_VERSION 2
 #define ISD_PAGE_SIZE 16
 
 /* Return / status codes. */
@@ -149,6 +149,14 @@ int isd_attn_strided(const isd_attn_args* a, void* stream);
  *  of Philox4x32-10(key = (seed lo, seed hi), counter = (b, step, pos,
  *  stream)) (Salmon et al., SC'11).
  *
+ * Argmax proposals (proposal = ISD_PROPOSAL_ARGMAX): the pages' serving
+ *  option of proposing the most likely token at each MASK position
+ *  (summary, "Serving (SGLang)").  Drafts are x = argmax q (the first
+ *  maximal index) instead of draws, so the proposal is a point mass: a
+ *  draft is accepted iff u < p(x), and at a rejection the replacement is
+ *  drawn from p without x (max(0, p - delta_x)); stream DRAFT is unused.
+ *  The pending drafts must have been proposed the same way.
+ *
  * Sizes: N <= 16, V <= 262 144 (otherwise ISD_ERR_UNSUPPORTED).
  * Layouts: logits_cur, logits_prev [B][K][V] (dtype); pending_*, q_row_*
  * int32 [B][N]; n_pending_* int32 [B]; q_stats_* f32 [B][N][2] (entry 0
@@ -186,7 +194,11 @@ typedef struct {
   const uint32_t* step_dev;    /* optional: read the step index from device
                                   memory instead of `step` (lets one
                                   captured CUDA graph serve every step)    */
+  int32_t proposal;            /* ISD_PROPOSAL_SAMPLE or _ARGMAX          */
 } isd_accept_args;
+
+#define ISD_PROPOSAL_SAMPLE 0  /* drafts drawn from q (default)           */
+#define ISD_PROPOSAL_ARGMAX 1  /* drafts x = argmax q                      */
 
 size_t isd_accept_workspace_bytes(const isd_accept_args* a);
 int isd_accept_resample(const isd_accept_args* a, void* stream);
@@ -209,7 +221,7 @@ int isd_accept_resample(const isd_accept_args* a, void* stream);
  *   means what it means for isd_accept_resample, with the same results.
  * - Problems whose isd_accept_workspace_bytes(a) exceeds
  *   ISD_ACCEPT_STATIC_SCRATCH are rejected with ISD_ERR_WORKSPACE before any
- *   launch (at N = 4 and V = 151 936 the limit admits about 2 200 sequences).
+ *   launch (at N = 4 and V = 151 936 the limit admits about 1 750 sequences).
  * - The first call on each device looks up the buffer's device address
  *   (with that device current) and keeps it; make that first call before
  *   any stream capture begins.

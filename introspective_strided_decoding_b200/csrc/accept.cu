@@ -60,6 +60,8 @@ struct AcceptDev {
   float* cmax;         // [B][RU][C] chunk max
   float* rmax;         // [B][K] row max m
   int32_t* decision;   // [B][4]: valid, rejected, a, n
+  int32_t* cidx;       // [B][RU][C] first index of the chunk max (argmax)
+  int argmax;          // drafts are argmax q (point-mass proposals)
 };
 
 // Loads elements [idx, idx+8) of a row; out-of-range ones read as -inf.
@@ -115,8 +117,19 @@ __global__ void __launch_bounds__(kAThreads)
     s += (double)t;
   }
   s = block_sum(s, redd);
+  const size_t o = ((size_t)b * p.RU + j) * p.C + c;
+  if (p.argmax) {
+    // First index of the chunk max (exact compare of the same values).
+    int first = INT_MAX;
+#pragma unroll
+    for (int r = kRounds - 1; r >= 0; --r)
+#pragma unroll
+      for (int k = 7; k >= 0; --k)
+        if (v[r][k] == m) first = lo + (r * kAThreads + threadIdx.x) * 8 + k;
+    first = block_min_int(first, reinterpret_cast<int*>(red));
+    if (threadIdx.x == 0) p.cidx[o] = first;
+  }
   if (threadIdx.x == 0) {
-    const size_t o = ((size_t)b * p.RU + j) * p.C + c;
     p.cmax[o] = m;
     p.csum[o] = s;
   }
@@ -183,11 +196,14 @@ __global__ void __launch_bounds__(128) accept_decide_kernel(AcceptDev<T> p) {
   if (lane >= 1 && lane < n) {
     const float lx = to_f(p.lc[((size_t)b * K + lane - 1) * p.V + tok]);
     const double px = exp((double)(lx - m_prev)) / s_prev;
-    const int qr = p.q_row_in[b * N + lane];
-    const float mq = p.q_stats_in[(b * N + lane) * 2];
-    const float sq = p.q_stats_in[(b * N + lane) * 2 + 1];
-    const float lqx = to_f(p.lp[((size_t)b * K + qr) * p.V + tok]);
-    const double qx = exp((double)(lqx - mq)) / (double)sq;
+    double qx = 1.0;      // argmax drafts: the proposal is a point mass
+    if (!p.argmax) {
+      const int qr = p.q_row_in[b * N + lane];
+      const float mq = p.q_stats_in[(b * N + lane) * 2];
+      const float sq = p.q_stats_in[(b * N + lane) * 2 + 1];
+      const float lqx = to_f(p.lp[((size_t)b * K + qr) * p.V + tok]);
+      qx = exp((double)(lqx - mq)) / (double)sq;
+    }
     const double r = qx > 0.0 ? px / qx : INFINITY;
     const float u = uniform(p.seed, (uint32_t)b, step_of(p),
                             (uint32_t)(L + lane), ISD_STREAM_ACCEPT);
@@ -220,10 +236,14 @@ __global__ void __launch_bounds__(128) accept_decide_kernel(AcceptDev<T> p) {
 // ---------------------------------------------------------------------------
 // Residual element weight max(0, p - q), shared by the chunk sums and the
 // in-chunk scan so both see the same per-element values.
+// With argmax drafts q is a point mass at the rejected draft x, so the
+// residual is p without x.
 struct ResidRows {
   float mp, inv_sp, mq, inv_sq;
+  int x;          // rejected draft (argmax proposals), else -1
 };
-ISD_DEV float resid_w(const ResidRows& r, float lpv, float lqv) {
+ISD_DEV float resid_w(const ResidRows& r, float lpv, float lqv, int v) {
+  if (r.x >= 0) return v == r.x ? 0.0f : ex2((lpv - r.mp) * kLog2e) * r.inv_sp;
   return fmaxf(0.0f, ex2((lpv - r.mp) * kLog2e) * r.inv_sp -
                          ex2((lqv - r.mq) * kLog2e) * r.inv_sq);
 }
@@ -232,14 +252,21 @@ template <typename T>
 ISD_DEV ResidRows resid_rows(const AcceptDev<T>& p, int b, int a,
                              const T*& prow, const T*& qrow) {
   const int N = p.N, K = p.K;
-  const int qr = p.q_row_in[b * N + a + 1];
   prow = p.lc + ((size_t)b * K + a) * p.V;
-  qrow = p.lp + ((size_t)b * K + qr) * p.V;
   ResidRows r;
   r.mp = p.rmax[b * K + a];
   r.inv_sp = (float)(1.0 / p.rsum[b * K + a]);
-  r.mq = p.q_stats_in[(b * N + a + 1) * 2];
-  r.inv_sq = 1.0f / p.q_stats_in[(b * N + a + 1) * 2 + 1];
+  if (p.argmax) {
+    qrow = prow;                       // not read
+    r.mq = 0.0f; r.inv_sq = 0.0f;
+    r.x = p.pending_in[b * N + a + 1];
+  } else {
+    const int qr = p.q_row_in[b * N + a + 1];
+    qrow = p.lp + ((size_t)b * K + qr) * p.V;
+    r.mq = p.q_stats_in[(b * N + a + 1) * 2];
+    r.inv_sq = 1.0f / p.q_stats_in[(b * N + a + 1) * 2 + 1];
+    r.x = -1;
+  }
   return r;
 }
 
@@ -259,10 +286,10 @@ __global__ void __launch_bounds__(kAThreads)
     const int idx = lo + (r * kAThreads + threadIdx.x) * 8;
     float vp[8], vq[8];
     load_row8<T, kVec>(prow, idx, hi, vp);
-    load_row8<T, kVec>(qrow, idx, hi, vq);
+    if (rr.x < 0) load_row8<T, kVec>(qrow, idx, hi, vq);
     float t = 0.0f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) t += resid_w(rr, vp[k], vq[k]);
+    for (int k = 0; k < 8; ++k) t += resid_w(rr, vp[k], vq[k], idx + k);
     s += (double)t;
   }
   s = block_sum(s, redd);
@@ -298,6 +325,19 @@ __global__ void __launch_bounds__(kAThreads)
     mode = 1; row = n + t - 1; pos = L + n + t; stream = ISD_STREAM_DRAFT;
   }
   const int C = p.C;
+  if (p.argmax && t >= 1) {
+    // Argmax draft: the first chunk whose max is the row max holds the
+    // first maximal index (exact compares of the same values).
+    if (threadIdx.x == 0) {
+      const size_t o = ((size_t)b * p.RU + row) * C;
+      const float m = p.rmax[b * K + row];
+      int tok = -1;
+      for (int cc = 0; cc < C && tok < 0; ++cc)
+        if (p.cmax[o + cc] == m) tok = p.cidx[o + cc];
+      p.pending_out[b * N + t] = tok;
+    }
+    return;
+  }
   if (mode == 0) {  // zero residual mass: draw from p instead
     double W = 0.0;
     for (int c = 0; c < C; ++c) W += p.resid[(size_t)b * C + c];
@@ -360,10 +400,11 @@ __global__ void __launch_bounds__(kAThreads)
   if (mode == 0) {
 #pragma unroll
     for (int r = 0; r < kRounds; ++r) {
+      const int idx = lo + (r * kAThreads + threadIdx.x) * 8;
       float vq[8];
-      load_row8<T, kVec>(qrow, lo + (r * kAThreads + threadIdx.x) * 8, hi, vq);
+      if (rr.x < 0) load_row8<T, kVec>(qrow, idx, hi, vq);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) w[r][k] = resid_w(rr, w[r][k], vq[k]);
+      for (int k = 0; k < 8; ++k) w[r][k] = resid_w(rr, w[r][k], vq[k], idx + k);
     }
   } else {
 #pragma unroll
@@ -414,7 +455,7 @@ __global__ void __launch_bounds__(kAThreads)
 // Host-side launcher (called from the C ABI after validation).
 
 struct AcceptLayout {
-  size_t csum, rsum, resid, cmax, rmax, decision, total;
+  size_t csum, rsum, resid, cmax, rmax, decision, cidx, total;
 };
 
 static AcceptLayout accept_layout(int B, int N, int K, int V) {
@@ -433,6 +474,7 @@ static AcceptLayout accept_layout(int B, int N, int K, int V) {
   l.cmax = take((size_t)B * RU * C * 4);
   l.rmax = take((size_t)B * K * 4);
   l.decision = take((size_t)B * 4 * 4);
+  l.cidx = take((size_t)B * RU * C * 4);
   l.total = off;
   return l;
 }
@@ -460,6 +502,8 @@ static int launch_accept_t(const isd_accept_args* a, cudaStream_t st) {
   p.cmax = reinterpret_cast<float*>(ws + l.cmax);
   p.rmax = reinterpret_cast<float*>(ws + l.rmax);
   p.decision = reinterpret_cast<int32_t*>(ws + l.decision);
+  p.cidx = reinterpret_cast<int32_t*>(ws + l.cidx);
+  p.argmax = a->proposal == ISD_PROPOSAL_ARGMAX;
   const bool vec = (a->V % 8) == 0;
   dim3 g_stats(p.C, p.RU, p.B), g_res(p.C, p.B), g_samp(p.N, p.B);
   if (vec) {

@@ -1,6 +1,7 @@
 // Device helpers shared by the ISD kernels (sm_100a).
 #pragma once
 
+#include <climits>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -119,6 +120,21 @@ ISD_DEV float block_reduce(float v, float* red) {
   __syncthreads();
   float r = lane < nw ? red[lane] : (kMax ? -INFINITY : 0.0f);
   r = kMax ? warp_max(r) : warp_sum(r);
+  return r;
+}
+
+// Block-wide minimum of ints; `red` holds >= 32 ints; all threads get it.
+ISD_DEV int block_min_int(int v, int* red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  int r = lane < nw ? red[lane] : INT_MAX;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) r = min(r, __shfl_xor_sync(0xffffffffu, r, o));
   return r;
 }
 

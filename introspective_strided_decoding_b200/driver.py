@@ -24,7 +24,7 @@ from . import isd
 
 class Decoder:
     def __init__(self, w, cache, state0, device, seed, num_ctas=0,
-                 with_lse=False, record=False):
+                 with_lse=False, record=False, proposal=None):
         self.w = w
         self.cache = cache
         self.device = torch.device(device)
@@ -70,7 +70,7 @@ class Decoder:
                                 self.states[1 - c], self.n_commit,
                                 self.commit_tokens, self.seed, 0,
                                 row_stats=self.row_stats, ratio=self.ratio,
-                                status=self.status)
+                                status=self.status, proposal=proposal)
             self._acc.append(a)
         self.ws_acc = torch.empty(isd.accept_workspace_bytes(self._acc[0]),
                                   dtype=torch.uint8, device=dev)

@@ -26,6 +26,8 @@ ERR_PAGE_TABLE_FULL = 17
 ERR_BAD_STATE = 18
 ERR_BAD_PAGE = 19
 
+PROPOSAL_SAMPLE = 0   # drafts drawn from q
+PROPOSAL_ARGMAX = 1   # drafts x = argmax q
 BF16 = 0
 F32 = 1
 PAGE_SIZE = 16
@@ -57,7 +59,7 @@ class AcceptArgs(ctypes.Structure):
                 ("n_commit", _VP), ("commit_tokens", _VP),
                 ("row_stats", _VP), ("ratio", _VP), ("status", _VP),
                 ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t),
-                ("step_dev", _VP)]
+                ("step_dev", _VP), ("proposal", _I32)]
 
 
 class CommitArgs(ctypes.Structure):
@@ -236,7 +238,8 @@ def new_state(B, N, device):
 
 def accept_args(logits_cur, logits_prev, seq_len, state_in, state_out,
                 n_commit, commit_tokens, seed, step, workspace=None,
-                row_stats=None, ratio=None, status=None, step_dev=None):
+                row_stats=None, ratio=None, status=None, step_dev=None,
+                proposal=None):
     B, K, V = logits_cur.shape
     N = K // 2
     dev, dt = logits_cur.device, logits_cur.dtype
@@ -274,7 +277,8 @@ def accept_args(logits_cur, logits_prev, seq_len, state_in, state_out,
         workspace=_ptr(workspace),
         workspace_bytes=0 if workspace is None else
         workspace.numel() * workspace.element_size(),
-        step_dev=_ptr(step_dev))
+        step_dev=_ptr(step_dev),
+        proposal=PROPOSAL_SAMPLE if proposal is None else int(proposal))
 
 
 def accept_workspace_bytes(args):
@@ -283,11 +287,13 @@ def accept_workspace_bytes(args):
 
 def accept_resample(logits_cur, logits_prev, seq_len, state_in, state_out,
                     n_commit, commit_tokens, seed, step, workspace=None,
-                    row_stats=None, ratio=None, status=None, stream=None):
-    """isd_accept_resample on torch tensors (state dicts from new_state)."""
+                    row_stats=None, ratio=None, status=None, stream=None,
+                    proposal=None):
+    """isd_accept_resample on torch tensors (state dicts from new_state).
+    ``proposal``: PROPOSAL_SAMPLE (default) or PROPOSAL_ARGMAX."""
     a = accept_args(logits_cur, logits_prev, seq_len, state_in, state_out,
                     n_commit, commit_tokens, seed, step, workspace, row_stats,
-                    ratio, status)
+                    ratio, status, proposal=proposal)
     if workspace is None:
         workspace = torch.empty(accept_workspace_bytes(a), dtype=torch.uint8,
                                 device=logits_cur.device)
@@ -303,13 +309,13 @@ ACCEPT_STATIC_SCRATCH = 4 << 20
 def accept_resample_static(logits_cur, logits_prev, seq_len, state_in,
                            state_out, n_commit, commit_tokens, seed, step,
                            row_stats=None, ratio=None, status=None,
-                           stream=None):
+                           stream=None, proposal=None):
     """isd_accept_resample_static: the accept step without a caller
     workspace, for callers that cannot allocate device memory (its scratch
     is a fixed buffer inside the library; see include/isd.h)."""
     a = accept_args(logits_cur, logits_prev, seq_len, state_in, state_out,
                     n_commit, commit_tokens, seed, step, None, row_stats,
-                    ratio, status)
+                    ratio, status, proposal=proposal)
     _raise(lib().isd_accept_resample_static(ctypes.byref(a),
                                             _stream(stream)),
            "isd_accept_resample_static")

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert isd.abi_version() == 1
+    assert isd.abi_version() == 2
     assert isd.status_string(isd.ERR_POOL_EXHAUSTED) == "KV page pool exhausted"
     assert isd.status_string(12345) == "unknown status"
 
@@ -90,6 +90,7 @@ def test_attn_workspace_query_rejects_bad_shapes(lib):
     (dict(K=9), isd.ERR_INVALID_ARG),               # K must be 2N
     (dict(N=17, K=34), isd.ERR_UNSUPPORTED),
     (dict(V=0), isd.ERR_INVALID_ARG),
+    (dict(proposal=2), isd.ERR_INVALID_ARG),        # sample (0) or argmax (1)
     (dict(), isd.ERR_INVALID_ARG),                  # null tensors
 ])
 def test_accept_host_validation(lib, kw, code):
