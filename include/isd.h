@@ -221,7 +221,7 @@ int isd_accept_resample(const isd_accept_args* a, void* stream);
  *   means what it means for isd_accept_resample, with the same results.
  * - Problems whose isd_accept_workspace_bytes(a) exceeds
  *   ISD_ACCEPT_STATIC_SCRATCH are rejected with ISD_ERR_WORKSPACE before any
- *   launch (at N = 4 and V = 151 936 the limit admits about 1 750 sequences).
+ *   launch (at N = 4 and V = 151 936 the limit admits 1 840 sequences).
  * - The first call on each device looks up the buffer's device address
  *   (with that device current) and keeps it; make that first call before
  *   any stream capture begins.
@@ -230,7 +230,7 @@ int isd_accept_resample(const isd_accept_args* a, void* stream);
  *   word before reading it).  Calls whose work may overlap on the GPU, such
  *   as calls on two unordered streams, race on it: order them.
  * ---------------------------------------------------------------------- */
-#define ISD_ACCEPT_STATIC_SCRATCH (4u << 20)
+#define ISD_ACCEPT_STATIC_SCRATCH (16u << 20)
 int isd_accept_resample_static(const isd_accept_args* a, void* stream);
 
 /* ------------------------------------------------------------------------

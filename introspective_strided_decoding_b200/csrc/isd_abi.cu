@@ -128,7 +128,7 @@ static int accept_check(const isd_accept_args* a) {
   if (a->B <= 0 || a->N < 2 || a->V <= 0 || a->K != 2 * a->N)
     return ISD_ERR_INVALID_ARG;
   if (a->N > 16) return ISD_ERR_UNSUPPORTED;
-  if (a->V > 32 * 8192) return ISD_ERR_UNSUPPORTED;  // at most 32 chunks
+  if (a->V > 128 * 2048) return ISD_ERR_UNSUPPORTED;  // <= 128 sub-chunks
   if (a->dtype != ISD_BF16 && a->dtype != ISD_F32) return ISD_ERR_INVALID_ARG;
   if (a->proposal != ISD_PROPOSAL_SAMPLE && a->proposal != ISD_PROPOSAL_ARGMAX)
     return ISD_ERR_INVALID_ARG;

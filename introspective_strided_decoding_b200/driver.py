@@ -174,6 +174,6 @@ class Decoder:
         self.graphs[self.cur].replay()
         self.advance()
 
-    # Kernel launches per step: attention + combine, four accept kernels,
-    # commit plan + copy.
-    LAUNCHES_PER_STEP = 8
+    # Kernel launches per step: attention + combine, three accept kernels
+    # (stats, decide, draw), commit plan + copy.
+    LAUNCHES_PER_STEP = 7

@@ -303,7 +303,7 @@ def accept_resample(logits_cur, logits_prev, seq_len, state_in, state_out,
            "isd_accept_resample")
 
 
-ACCEPT_STATIC_SCRATCH = 4 << 20
+ACCEPT_STATIC_SCRATCH = 16 << 20
 
 
 def accept_resample_static(logits_cur, logits_prev, seq_len, state_in,

@@ -76,6 +76,18 @@ CASES = [
     (synth.Workload("bf16_n8_p07", B=32, Hq=64, Hkv=8, d=128, N=8, L_lo=1000,
                     L_hi=2000, V=151936, target_accept=0.7), 6),
     (synth.C64.with_(steps=1), 3),
+    # Rows whose byte length is not a multiple of 16: plain-load statistics
+    # and element-wise draws (V = 1001: one ragged sub-chunk; V = 2050: two,
+    # the second of two elements).
+    (synth.Workload("bf16_v1001_unaligned", B=8, Hq=32, Hkv=8, d=128, N=3,
+                    L_lo=10, L_hi=90, V=1001, sigma_p=2.0, sigma_q=0.6), 8),
+    (synth.Workload("f32_v2050_unaligned", B=8, Hq=32, Hkv=8, d=128, N=3,
+                    L_lo=10, L_hi=90, V=2050, dtype="f32", sigma_p=2.0,
+                    sigma_q=0.6), 8),
+    # The largest vocabulary accepted: 128 sub-chunks, every lane's share of
+    # the sub-chunk scan full.
+    (synth.Workload("bf16_v262144_max", B=4, Hq=32, Hkv=8, d=128, N=2,
+                    L_lo=10, L_hi=90, V=262144, sigma_p=3.0, sigma_q=0.5), 6),
 ]
 
 
@@ -99,6 +111,8 @@ ARGMAX_CASES = [
     (synth.Workload("f32_v1000_scalar", B=8, Hq=32, Hkv=8, d=128, N=3,
                     L_lo=10, L_hi=90, V=1000, dtype="f32", sigma_p=2.0,
                     sigma_q=0.6), 8),
+    (synth.Workload("bf16_v1001_unaligned", B=8, Hq=32, Hkv=8, d=128, N=3,
+                    L_lo=10, L_hi=90, V=1001, sigma_p=2.0, sigma_q=0.6), 8),
     (synth.SHAPE_8B, 8),
     (synth.Workload("bf16_n8_p07", B=32, Hq=64, Hkv=8, d=128, N=8, L_lo=1000,
                     L_hi=2000, V=151936, target_accept=0.7), 4),
