@@ -8,7 +8,8 @@
 // ("Introspective Strided Decoding").  Row r of sequence b (position
 // L_b + r) attends to cached positions [0, L_b) and stride rows 0..r.
 //
-// bf16 path (tensor cores).  Work is a flat list of "units": for every
+// bf16 path for head dim 64 (mma.sync tensor cores; head dim 128 runs on
+// the tcgen05 kernel of attn_tc.cu).  Work is a flat list of "units": for every
 // (sequence b, KV head h), one unit per cached page plus one tail unit for
 // the stride's own rows.  Each persistent CTA takes an equal contiguous
 // range of that list (no per-sequence imbalance, whatever the lengths).
@@ -786,13 +787,13 @@ int launch_attn_combine(const isd_attn_args* a, int G, cudaStream_t st) {
 bool attn_tc_supported(const isd_attn_args* a);
 int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st);
 
+// Head dim 128 runs on the tcgen05 kernel (every shape the host check
+// admits), head dim 64 on the mma.sync kernel.
 int launch_attn_bf16(const isd_attn_args* a, int G, cudaStream_t st) {
   if (attn_tc_supported(a)) return launch_attn_tc(a, G, st);
+  if (a->d != 64) return ISD_ERR_UNSUPPORTED;
   const int M = a->K * (a->Hq / a->Hkv);
-  const int MW = M <= 32 ? 1 : 2;
-  if (a->d == 128) return MW == 1 ? launch_bf16<128, 1>(a, G, st)
-                                  : launch_bf16<128, 2>(a, G, st);
-  return MW == 1 ? launch_bf16<64, 1>(a, G, st) : launch_bf16<64, 2>(a, G, st);
+  return M <= 32 ? launch_bf16<64, 1>(a, G, st) : launch_bf16<64, 2>(a, G, st);
 }
 
 int launch_attn_f32(const isd_attn_args* a, cudaStream_t st) {
