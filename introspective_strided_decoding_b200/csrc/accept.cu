@@ -11,11 +11,12 @@
 // The vocabulary is cut into sub-chunks of 2048 elements, one warp's work
 // (64 elements a lane), so no step needs a block-wide barrier.  Three
 // kernels, one stream, no inter-CTA waiting:
-//   stats   one CTA per SM.  A producer thread streams the used rows'
-//           sub-chunks into a shared-memory ring with bulk asynchronous
-//           copies (TMA engine, completion counted on mbarriers); 16
-//           consumer warps reduce one sub-chunk each at a time to its max,
-//           the first index of that max and the sum of exp(l - max).
+//   stats   one CTA per SM.  Six producer lanes stream the used rows into
+//           a 12-slot shared-memory ring in 16 KB bulk asynchronous copies
+//           (TMA engine, completion counted on mbarriers); six groups of
+//           four consumer warps take the copies in turn, each warp reducing
+//           one sub-chunk to its max, the first index of that max and the
+//           sum of exp(l - max), in two passes over shared memory.
 //           Rows whose byte length is not a multiple of 16 cannot be bulk
 //           copied and go through a plain-load variant with the same
 //           element order and arithmetic.                         [HBM bound]
