@@ -18,6 +18,7 @@ more arrivals than it expects, and that everything terminates.  A negative
 control (one warp per production, slots not owned) must be caught.
 """
 
+import math
 import os
 import random
 import re
@@ -36,7 +37,7 @@ def _constants():
     for n in names:
         m = re.search(r"constexpr int %s = ([0-9 *]+);" % n, text)
         assert m, n
-        out[n] = eval(m.group(1))  # plain integer products only
+        out[n] = math.prod(int(f) for f in m.group(1).split("*"))
     return out
 
 
