@@ -1,20 +1,24 @@
 """Benchmark of one ISD step (attention + accept/resample + KV commit).
 
-Workload: the C=64 stationary batch (64 sequences, 32 query / 8 KV heads,
-head dim 128, prefixes uniform in [1024, 8192] on a shuffled paged cache,
-N=4 so K=8 query rows, vocabulary 151 936, draft noise tuned for mean
+Default workload: the C=64 stationary batch (64 sequences, 32 query / 8 KV
+heads, head dim 128, prefixes uniform in [1024, 8192] on a shuffled paged
+cache, N=4 so K=8 query rows, vocabulary 151 936, draft noise tuned for mean
 acceptance 0.9), run for consecutive steps with KV commit and rollback.
 Inputs are seeded synthetic tensors; the logits of each step (the LM head's
 output, not part of the timed path) are generated between steps, and L2 is
 flushed before every timed step.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl isd|reference]
+                  [--workload c64_stationary|8b_b1|32b_b32|sweep|all]
+                  [--eager]
 
-Prints one JSON line (rank 0).  ``value`` is accepted (committed) tokens
-per second over all ranks, device-timed with CUDA events around the three
-library calls of every step, max over ranks.  With N > 1 every rank runs
-its own 64-sequence replica (the path shards by sequence; no collective on
-the data path).
+Prints one JSON line (rank 0) per workload (the default: one).  ``value`` is
+accepted (committed) tokens per second over all ranks: every step runs as
+one replay of the captured CUDA graph of the three library calls (the
+serving path), device-timed with CUDA events around it, max over ranks.
+``--eager`` times the three calls launched one by one instead.  With N > 1
+every rank runs its own replica (the path shards by sequence; no
+collective on the data path).
 """
 
 import argparse
@@ -36,6 +40,8 @@ sys.path.insert(0, ROOT)
 METRIC = ("ISD accepted tokens/s at B=64,N=4; achieved HBM GB/s as fraction "
           "of B200 peak")
 FALLBACK_HBM_GBS = 6650.0
+SWEEP = [(B, N, p) for B in (1, 8, 32, 64) for N in (2, 4, 8)
+         for p in (0.5, 0.9)]
 
 
 def parse():
@@ -44,28 +50,36 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="isd", choices=["isd", "reference"])
+    ap.add_argument("--workload", default="c64_stationary",
+                    choices=["c64_stationary", "8b_b1", "32b_b32", "sweep",
+                             "all"])
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--batch", type=int, default=64,
-                    help="sequences per GPU (64 = the benchmark workload; "
-                         "smaller only for profiling captures)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's sequences per GPU (only "
+                         "for profiling captures of a smaller case)")
     ap.add_argument("--proposal", default="sample", choices=["sample", "argmax"],
                     help="drafts drawn from q (default) or x = argmax q")
+    ap.add_argument("--eager", action="store_true",
+                    help="time eager launches instead of graph replays")
+    ap.add_argument("--phase-steps", type=int, default=5,
+                    help="eager steps timed per phase for the split")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-seqs", type=int, default=4)
-    ap.add_argument("--cpu-sample-steps", type=int, default=8)
+    ap.add_argument("--cpu-sample-steps", type=int, default=4)
+    ap.add_argument("--cpu-sample-seqs", type=int, default=0,
+                    help="oracle worker processes (0: one per host core, "
+                         "at most one per sequence)")
     return ap.parse_args()
 
 
 # DRAM traffic of the attention kernel per algorithmic byte, from one ncu
-# capture of this workload at B = 16 (dram__bytes_read.sum +
-# dram__bytes_write.sum over the launch's algorithmic bytes; see
-# profiles/attn_tc_kernel_c64_b16_full.md).  Traffic tracks the algorithmic
-# bytes, so a full launch's traffic is this ratio times its bytes.  Valid only
-# for the kernel source the capture was taken on.
-TRAFFIC_PER_ALGO_BYTE = 340.05 / 332.02
-TRAFFIC_KERNEL_SHA256 = (
-    "71a076003bf7b68d3f9c2c4d7b2713ea6921847880a94e1e7c662821352cd6d0")
+# capture of the C=64 workload at B = 16 (dram__bytes_read.sum +
+# dram__bytes_write.sum over the launch's algorithmic bytes).  Traffic tracks
+# the algorithmic bytes, so a full launch's traffic is this ratio times its
+# bytes.  Valid only for the kernel source the capture was taken on (None:
+# no capture of the current source).
+TRAFFIC_PER_ALGO_BYTE = None
+TRAFFIC_KERNEL_SHA256 = None
 
 
 def attention_traffic(bytes_per_launch):
@@ -89,6 +103,13 @@ def peaks():
         return float(j["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tpf_closed_form(p, N):
+    """The pages' memory-bound tokens-per-forward formula (hada.io summary,
+    "Speedup Factor Explorer"), for reporting beside the measured TPF."""
+    num = 2.0 + sum(p ** k for k in range(1, N - 1))
+    return num / (2.0 - p ** (N - 1))
 
 
 # ------------------------------------------------------------------ clocks
@@ -198,23 +219,26 @@ def job_figures(total_ms, tokens, e2e_ms, e2e_tokens, world, device):
 
 
 # --------------------------------------------------------- oracle sample
-def oracle_sample(w, seed, n_seqs, steps=1, skip=0):
-    """Time the fp64 oracle on a bounded sample of the workload: the first
-    ``n_seqs`` sequences, full step (attention for all their KV heads,
-    accept/resample, commit), ``skip + steps`` consecutive steps from the
-    start state, the first ``skip`` untimed.  Returns (tokens decided,
-    seconds, sample description) over the timed steps."""
-    from oracle import attention as oattn
-    from oracle import step as ostep
-    from introspective_strided_decoding_b200 import synth
+def _oracle_one_sequence(job):
+    """One worker of the CPU baseline: the fp64 oracle's full step
+    (attention over every KV head, accept/resample, commit) for one
+    sequence of the workload, ``skip + steps`` consecutive steps from the
+    start state, the first ``skip`` untimed.  Returns (tokens, seconds)."""
+    w, seed, b, steps, skip, proposal = job
     try:
         from threadpoolctl import threadpool_limits
-        limiter = threadpool_limits(limits=1)
+        threadpool_limits(limits=1)
     except Exception:
-        limiter = None
-    ws = w.with_(B=n_seqs)
-    cache = synth.make_cache(ws, seed, "cpu")
-    st = synth.initial_state(ws, seed, "cpu")
+        pass
+    torch.set_num_threads(1)
+    from introspective_strided_decoding_b200 import synth
+    from oracle import attention as oattn
+    from oracle import step as ostep
+    # Sequence b of the workload: its own prefix length, pages and state.
+    L_all = synth.prefix_lengths(w, seed)
+    ws = w.with_(B=1, L_lo=int(L_all[b]), L_hi=int(L_all[b]))
+    cache = synth.make_cache(ws, seed + 7919 * b, "cpu")
+    st = synth.initial_state(ws, seed + 7919 * b, "cpu")
     kc = cache["k_cache"].float().numpy()
     vc = cache["v_cache"].float().numpy()
     pt = cache["page_table"].long().numpy()
@@ -224,18 +248,19 @@ def oracle_sample(w, seed, n_seqs, steps=1, skip=0):
     pend = st["pending"].long().numpy()
     n = st["n_pending"].long().numpy()
     qrow = st["q_row"].long().numpy()
-    prev = np.zeros((ws.B, ws.K, ws.V), dtype=np.float32)
+    prev = np.zeros((1, ws.K, ws.V), dtype=np.float32)
     tokens, secs = 0, 0.0
     for s in range(skip + steps):
-        lc = synth.step_logits(ws, seed, torch.from_numpy(L),
+        lc = synth.step_logits(ws, seed + b, torch.from_numpy(L),
                                torch.from_numpy(n), s, "cpu").float().numpy()
-        q, k, v = (t.float().numpy() for t in synth.make_stride(ws, seed, s,
-                                                                "cpu"))
+        q, k, v = (t.float().numpy() for t in
+                   synth.make_stride(ws, seed + b, s, "cpu"))
         t0 = time.perf_counter()
         oattn.attn_strided(q.astype(np.float64), k.astype(np.float64),
                            v.astype(np.float64), kc, vc, pt, L,
                            1.0 / np.sqrt(ws.d))
-        o = ostep.accept_resample(lc, prev, pend, n, qrow, L, seed, s, ws.N)
+        o = ostep.accept_resample(lc, prev, pend, n, qrow, L, seed, s, ws.N,
+                                  proposal=proposal)
         kc, vc, pt, L2, top, _ = ostep.kv_commit(k, v, kc, vc, pt, L,
                                                  o["n_commit"], fs, top)
         if s >= skip:
@@ -244,23 +269,64 @@ def oracle_sample(w, seed, n_seqs, steps=1, skip=0):
         L = L2
         pend, n, qrow, prev = (o["next_pending"], o["next_n"],
                                o["next_q_row"], lc)
-    if limiter is not None:
-        limiter.restore_original_limits()
-    desc = (f"fp64 numpy oracle, first {n_seqs} of {w.B} sequences, steps "
-            f"{skip}..{skip + steps - 1} of the chain: attention (all KV "
-            f"heads), accept/resample, commit; 1 BLAS thread")
-    return tokens, secs, desc
+    return tokens, secs
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, seed, steps, skip=1, proposal="sample", seqs=0):
+    """Time the fp64 oracle on the host cores, on a bounded sample of the
+    workload: one sequence per core (the first min(cores, B) sequences),
+    ``steps`` timed steps each after ``skip`` untimed ones, one process per
+    sequence in a spawn pool (the CUDA context of this process is not
+    forked).  Throughput = tokens decided / the slowest worker's compute
+    time (the workers run concurrently).  Returns (tokens/s, cores,
+    description)."""
+    import multiprocessing as mp
+    cores = host_cores()
+    nseq = min(cores, w.B, seqs if seqs > 0 else cores)
+    jobs = [(w, seed, b, steps, skip, proposal) for b in range(nseq)]
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(nseq) as pool:
+        res = pool.map(_oracle_one_sequence, jobs)
+    tokens = sum(r[0] for r in res)
+    secs = max(r[1] for r in res)
+    desc = (f"fp64 numpy oracle, {nseq} of the {w.B} sequences (one per "
+            f"host core, spawn pool, 1 BLAS thread each), steps "
+            f"{skip}..{skip + steps - 1} of each chain: attention over every "
+            f"KV head, accept/resample, commit; tokens / slowest worker's "
+            f"compute time")
+    return tokens / secs, nseq, desc
 
 
 # --------------------------------------------------------------- isd arm
-def run_isd(args, world, rank, local):
+def workload_list(args):
+    from introspective_strided_decoding_b200 import synth
+    named = {"c64_stationary": synth.C64, "8b_b1": synth.SHAPE_8B,
+             "32b_b32": synth.SHAPE_32B}
+    if args.workload in named:
+        return [named[args.workload]]
+    sweep = [synth.sweep_workload(B, N, p) for B, N, p in SWEEP]
+    if args.workload == "sweep":
+        return sweep
+    return list(named.values()) + sweep
+
+
+def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
     from introspective_strided_decoding_b200 import build, isd, synth
     from introspective_strided_decoding_b200.driver import Decoder
     build.build()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = synth.C64.with_(steps=args.steps + args.warmup + args.e2e_steps + 2)
-    if args.batch != w.B:
+    phase_steps = max(1, args.phase_steps)
+    n_e2e = max(1, args.e2e_steps)
+    w = w.with_(steps=steps + warmup + phase_steps + 2 * n_e2e + 2)
+    if args.batch is not None and args.batch != w.B:
         w = w.with_(B=args.batch, name=f"{w.name}_b{args.batch}")
     seed = rank_seed(args.seed, rank)
     cache = synth.make_cache(w, seed, dev)
@@ -269,9 +335,12 @@ def run_isd(args, world, rank, local):
                   proposal=isd.PROPOSAL_ARGMAX if args.proposal == "argmax"
                   else isd.PROPOSAL_SAMPLE)
     stream = torch.cuda.current_stream(dev)
+    use_graph = not args.eager
+    if use_graph:
+        dec.capture()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     hbm_peak, peak_kind = peaks()
-    es = 2  # bf16
+    es = 2 if w.dtype == "bf16" else 4
     kv_row = w.Hkv * w.d * es * 2           # K and V of one token
     qo_bytes = 2 * w.B * w.K * w.Hq * w.d * es + 2 * w.B * w.K * w.Hkv * w.d * es
     row_bytes = w.V * es
@@ -291,20 +360,33 @@ def run_isd(args, world, rank, local):
         flush.fill_(step & 0xFF)            # evict L2 (256 MB > 126 MB)
         return kv, used_rows
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
-          for _ in range(args.steps)]
-    tok_dev = torch.zeros(1, dtype=torch.int64, device=dev)
-    tested = accepted = 0
-    for s in range(args.warmup):
+    def run_step(events=None):
+        if use_graph:
+            if events:
+                events[0].record(stream)
+            dec.replay()
+            if events:
+                events[-1].record(stream)
+        else:
+            dec.step(stream, events)
+
+    for _ in range(warmup):
         prepare(dec.step_idx)
-        dec.step(stream)
+        run_step()
     torch.cuda.synchronize(dev)
+
+    # ------------------------------------------------------- timed steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
+          for _ in range(steps)]
+    tok_dev = torch.zeros(1, dtype=torch.int64, device=dev)
+    tested_dev = torch.zeros(1, dtype=torch.int64, device=dev)
+    accepted_dev = torch.zeros(1, dtype=torch.int64, device=dev)
     kv_bytes, logit_rows = [], []
     clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize(dev)
     clocks.start()
-    for s in range(args.steps):
+    for s in range(steps):
         kv, rows = prepare(dec.step_idx)
         kv_bytes.append(kv)
         logit_rows.append(rows)
@@ -313,38 +395,52 @@ def run_isd(args, world, rank, local):
         # queues the whole step while it runs, so the timed window holds
         # the step's kernels and not the host's launch latency.
         torch.cuda._sleep(100_000)
-        dec.step(stream, ev[s])
+        run_step(ev[s])
         tok_dev += dec.n_commit.sum()
         # Drafts tested: the accepted ones plus the first rejected one.
         acc = (dec.n_commit - 1).clamp(min=0)
-        tested += int(acc.sum() + (dec.n_commit < n_in).sum())
-        accepted += int(acc.sum())
+        accepted_dev += acc.sum()
+        tested_dev += acc.sum() + (dec.n_commit < n_in).sum()
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
     barrier(world)
-    t_attn = [e[0].elapsed_time(e[1]) for e in ev]
-    t_acc = [e[1].elapsed_time(e[2]) for e in ev]
-    t_com = [e[2].elapsed_time(e[3]) for e in ev]
-    t_step = [e[0].elapsed_time(e[3]) for e in ev]
+    t_step = [e[0].elapsed_time(e[-1]) for e in ev]
     total_ms = sum(t_step)
     tokens = int(tok_dev.item())
+    tested, accepted = int(tested_dev.item()), int(accepted_dev.item())
     status = int(dec.status.item())
     if status != isd.OK:
         raise RuntimeError(f"device status {isd.status_string(status)}")
-
-    attn_bytes = [kv + qo_bytes for kv in kv_bytes]
-    achieved = sum(attn_bytes) / (sum(t_attn) / 1e3) / 1e9
     step_bytes = [kv + qo_bytes + r * row_bytes for kv, r in
                   zip(kv_bytes, logit_rows)]
     step_gbs = sum(step_bytes) / (total_ms / 1e3) / 1e9
 
+    # --------------------------------------- per-phase split (eager calls)
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
+           for _ in range(phase_steps)]
+    p_kv, p_rows = [], []
+    for s in range(phase_steps):
+        kv, rows = prepare(dec.step_idx)
+        p_kv.append(kv)
+        p_rows.append(rows)
+        torch.cuda._sleep(100_000)
+        dec.step(stream, pev[s])
+    torch.cuda.synchronize(dev)
+    t_attn = [e[0].elapsed_time(e[1]) for e in pev]
+    t_acc = [e[1].elapsed_time(e[2]) for e in pev]
+    t_com = [e[2].elapsed_time(e[3]) for e in pev]
+    attn_bytes = [kv + qo_bytes for kv in p_kv]
+    achieved = sum(attn_bytes) / (sum(t_attn) / 1e3) / 1e9
+    acc_bytes = sum(r * row_bytes for r in p_rows)
+    aa_gbs = (sum(attn_bytes) + acc_bytes) / \
+        ((sum(t_attn) + sum(t_acc)) / 1e3) / 1e9
+
     # ---------------------------------------------------------------- e2e
-    # Host-resident inputs (pinned), H2D copy + the three calls + D2H of
-    # the step's result, all inside the timed region.
-    n_e2e = max(1, args.e2e_steps)
-    # Each step's inputs depend on the state the previous steps left, so
-    # generate them by running the steps once, keep host copies, then
-    # rewind every piece of state for the timed replay.
+    # Host-resident inputs (pinned), H2D copy + the step through the public
+    # API + D2H of the step's result, all inside the timed region.  Each
+    # step's inputs depend on the state the previous steps left, so they
+    # are generated by running the steps once, kept on the host, and every
+    # piece of state is rewound for the timed replay.
     snap = {k: v.clone() for k, v in cache.items()}
     snap_state = {k: v.clone() for k, v in dec.state.items()}
     snap_prev = dec.logits[1 - dec.cur].clone()
@@ -354,14 +450,14 @@ def run_isd(args, world, rank, local):
         prepare(dec.step_idx)
         host_in.append(tuple(t.to("cpu").pin_memory() for t in
                              (dec.logits_cur, dec.q, dec.k_new, dec.v_new)))
-        dec.step(stream)
+        run_step()
     torch.cuda.synchronize(dev)
     for k, v in snap.items():
         cache[k].copy_(v)
-    dec.cur, dec.step_idx = snap_cur, snap_idx
     for k, v in snap_state.items():
-        dec.state[k].copy_(v)
-    dec.logits[1 - dec.cur].copy_(snap_prev)
+        dec.states[snap_cur][k].copy_(v)
+    dec.logits[1 - snap_cur].copy_(snap_prev)
+    dec.set_step(snap_cur, snap_idx)
     del snap, snap_prev
     res_host = torch.empty((w.B * (1 + w.N),), dtype=torch.int32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_in[0])
@@ -379,26 +475,31 @@ def run_isd(args, world, rank, local):
         dec.q.copy_(q, non_blocking=True)
         dec.k_new.copy_(k, non_blocking=True)
         dec.v_new.copy_(v, non_blocking=True)
-        dec.step(stream)
+        run_step()
         res_host[:w.B].copy_(dec.n_commit, non_blocking=True)
-        res_host[w.B:].copy_(dec.next_state["pending"].reshape(-1),
+        res_host[w.B:].copy_(dec.state["pending"].reshape(-1),
                              non_blocking=True)
         stream.synchronize()
         e2e_tokens += int(res_host[:w.B].sum())
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
+    if int(dec.status.item()) != isd.OK:
+        raise RuntimeError("device status after the e2e steps: "
+                           f"{isd.status_string(int(dec.status.item()))}")
+    dec.release_graphs()
     job = job_figures(total_ms, tokens, e2e_ms, e2e_tokens, world, dev)
     total_ms_max, value = job["total_ms_max"], job["value"]
     e2e = {"value": job["e2e_value"], "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "steps": n_e2e}
-
+    alpha = accepted / max(tested, 1)
+    tpf = tokens / (w.B * steps)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "n_gpus": world, "steps": steps, "warmup": warmup,
+        "ms_per_step": total_ms_max / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded; no weights or datasets)",
         "config": {
             "workload": w.name, "B": w.B, "N": w.N, "K": w.K, "Hq": w.Hq,
@@ -406,8 +507,11 @@ def run_isd(args, world, rank, local):
             "prefix": [w.L_lo, w.L_hi], "pages": "shuffled",
             "target_accept": w.target_accept, "proposal": args.proposal,
             "l2": "flushed (256 MB write) before every timed step",
-            "timing": "CUDA events around attention+accept+commit per step; "
-                      "logits/Q/K/V generation between steps untimed",
+            "timing": ("CUDA events around one CUDA-graph replay of "
+                       "attention+accept+commit per step" if use_graph else
+                       "CUDA events around the eager attention+accept+commit "
+                       "calls per step") +
+                      "; logits/Q/K/V generation between steps untimed",
             "parallelism": f"replicas x{world}"},
         "roofline": {
             "kernel": "attn_tc_kernel (+combine)", "bound": "hbm",
@@ -416,25 +520,45 @@ def run_isd(args, world, rank, local):
             "traffic": attention_traffic(sum(attn_bytes) / len(attn_bytes)),
             "bytes_per_launch": sum(attn_bytes) / len(attn_bytes)},
         "e2e": e2e,
-        "gpu_launches": Decoder.LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": dec.launches_per_step * steps,
         "clocks": clk,
         "detail": {
-            "attention_ms": sum(t_attn) / args.steps,
-            "accept_ms": sum(t_acc) / args.steps,
-            "commit_ms": sum(t_com) / args.steps,
-            "steps_per_s": args.steps / (total_ms / 1e3),
+            "graph": use_graph,
+            "attention_ms": sum(t_attn) / phase_steps,
+            "accept_ms": sum(t_acc) / phase_steps,
+            "commit_ms": sum(t_com) / phase_steps,
+            "phase_split": f"eager calls, {phase_steps} further steps",
+            "steps_per_s": steps / (total_ms / 1e3),
             "step_gbs": step_gbs, "step_frac": step_gbs / hbm_peak,
-            "tpf": tokens / (w.B * args.steps),
-            "accept_rate": accepted / max(tested, 1),
+            "attn_accept_gbs": aa_gbs,
+            "attn_accept_frac": aa_gbs / hbm_peak,
+            "tpf": tpf, "accept_rate": alpha,
+            "tpf_closed_form_at_rate": tpf_closed_form(alpha, w.N),
             "tokens": tokens},
     }
-    if rank == 0 and not args.no_cpu_baseline:
-        tok, secs, desc = oracle_sample(w, args.seed, args.cpu_sample_seqs,
-                                        steps=args.cpu_sample_steps, skip=2)
-        line["cpu_baseline"] = {"value": tok / secs, "unit": "tokens/s",
-                                "cores": 1, "kind": "oracle", "sample": desc}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    if rank == 0 and with_cpu:
+        v, cores, desc = oracle_sample(w, args.seed, args.cpu_sample_steps,
+                                       proposal=args.proposal,
+                                       seqs=args.cpu_sample_seqs)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s",
+                                "cores": cores, "kind": "oracle",
+                                "sample": desc}
+    del dec, cache, flush
+    torch.cuda.empty_cache()
+    return line
+
+
+def run_isd(args, world, rank, local):
+    wl = workload_list(args)
+    for i, w in enumerate(wl):
+        many = len(wl) > 1
+        steps = min(args.steps, 20) if many and w.name.startswith("sweep") \
+            else args.steps
+        warmup = max(3, min(args.warmup, 5)) if many else args.warmup
+        line = run_workload(w, args, world, rank, local, steps, warmup,
+                            with_cpu=(i == 0 and not args.no_cpu_baseline))
+        if rank == 0:
+            print(json.dumps(line), flush=True)
 
 
 # --------------------------------------------------------- reference arm
@@ -442,22 +566,27 @@ def run_reference(args, world, rank):
     """The oracle, as it stands, on the host cores, on the same config."""
     if rank != 0:
         return
-    from introspective_strided_decoding_b200 import synth
-    w = synth.C64
-    tokens, secs, desc = oracle_sample(w, args.seed, args.cpu_sample_seqs,
-                                       steps=args.steps, skip=args.warmup)
-    value = tokens / secs
+    w = workload_list(args)[0]
+    steps = max(1, args.steps)
+    value, cores, desc = oracle_sample(w, args.seed, steps,
+                                       skip=max(0, args.warmup),
+                                       proposal=args.proposal,
+                                       seqs=args.cpu_sample_seqs)
     line = {
         "impl": "reference", "metric": METRIC, "value": value,
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f64", "data": "synthetic (seeded; no weights or datasets)",
+        "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; no weights or datasets)",
         "config": {"workload": w.name, "B": w.B, "N": w.N, "K": w.K,
                    "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "V": w.V,
-                   "prefix": [w.L_lo, w.L_hi], "pages": "shuffled",
-                   "target_accept": w.target_accept},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1,
+                   "page_size": 16, "prefix": [w.L_lo, w.L_hi],
+                   "pages": "shuffled", "target_accept": w.target_accept,
+                   "proposal": args.proposal,
+                   "l2": "host memory (no device cache)",
+                   "parallelism": f"one process per host core, rank 0 of "
+                                  f"{world}"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},

@@ -37,9 +37,15 @@
  *   rejected on the host before anything is launched (ISD_ERR_INVALID_ARG,
  *   ISD_ERR_UNSUPPORTED, ISD_ERR_WORKSPACE).  A failed launch returns
  *   ISD_ERR_CUDA.  Conditions only the device can see (pool exhausted,
- *   page-table row full, malformed state, page id out of range) are written
- *   as an ISD_ERR_* code to the caller's `status` word, and the affected
- *   work is skipped; no kernel traps and no kernel waits on another.
+ *   page-table row full, malformed state, page id out of range, a bounded
+ *   wait that ran out) are written as an ISD_ERR_* code to the caller's
+ *   `status` word, and the affected work is skipped; no kernel traps and no
+ *   kernel waits on another.
+ * - The status word keeps the FIRST error written to it: kernels never
+ *   clear it and never replace an error already there (atomic
+ *   compare-and-swap from ISD_OK).  The caller zeroes it before use; one
+ *   word may serve all three calls of a step, and after the step it holds
+ *   the earliest failure.
  * - The calls are asynchronous and capture into CUDA graphs: they read no
  *   device memory on the host and launch a fixed set of kernels.
  */
@@ -53,7 +59,7 @@
 extern "C" {
 #endif
 
-#define ISD_ABI_VERSION 2
+#define ISD_ABI_VERSION 3
 #define ISD_PAGE_SIZE 16
 
 /* Return / status codes. */
@@ -91,9 +97,8 @@ enum { ISD_STREAM_ACCEPT = 0, ISD_STREAM_RESAMPLE = 1, ISD_STREAM_DRAFT = 2 };
  * Layouts: q, out [B][K][Hq][d]; k_new, v_new [B][K][Hkv][d];
  * k_cache, v_cache [num_pages][Hkv][16][d]; page_table int32
  * [B][page_table_stride]; seq_len int32 [B]; lse f32 [B][K][Hq] or NULL.
- * dtype ISD_BF16 (tensor cores; K <= 16 and K * g <= 128; d = 128 runs on
- * tcgen05 with any K * g, d = 64 on mma.sync with K * g one of 16, 32, 64,
- * 128) or ISD_F32 (exact-fp32 SIMT path; d a multiple of 32, at most 128).
+ * dtype ISD_BF16 (tcgen05 tensor cores: d = 128, K <= 16, K * g <= 128)
+ * or ISD_F32 (exact-fp32 SIMT path; d a multiple of 32, at most 128).
  * `out` may not alias any input.
  * Workspace: isd_attn_workspace_bytes(args) bytes (split-KV partials);
  * its contents need no initialisation.  `status` (optional) receives
@@ -131,8 +136,9 @@ int isd_attn_strided(const isd_attn_args* a, void* stream);
  *  1. Row statistics m = max_v l_v, s = sum_v exp(l_v - m) (fp32) of
  *     logits_cur rows 0 .. n + N - 2 (p rows 0..n-1, draft rows n..n+N-2).
  *  2. Drafts i = 1 .. n-1 in order: p_i(x) from row i-1 of logits_cur,
- *     q_i(x) from row q_row_in[b][i] of logits_prev with the stored
- *     (m, s) = q_stats_in[b][i]; u_i = U(seed, b, step, L + i, ACCEPT);
+ *     q_i(x) = exp(l_x - ln Z) from row q_row_in[b][i] of logits_prev and
+ *     its stored log-normaliser ln Z = q_stats_in[b][i][0] + [1];
+ *     u_i = U(seed, b, step, L + i, ACCEPT);
  *     accept iff u_i < p_i(x)/q_i(x).  a_b = drafts accepted before the
  *     first rejection; n_commit[b] = 1 + a_b; commit_tokens[b][0..a_b] =
  *     pending_in[b][0..a_b] (the rest -1).
@@ -141,8 +147,8 @@ int isd_attn_strided(const isd_attn_args* a, void* stream);
  *     mass is zero), stream RESAMPLE; next n = 1.
  *     All accepted: the exact token at L + n is drawn from p of row n-1
  *     (stream RESAMPLE), and drafts j = 1..N-1 at L + n + j from q of row
- *     n + j - 1 (stream DRAFT), whose (m, s) go to q_stats_out[b][j] and
- *     row index to q_row_out[b][j]; next n = N.
+ *     n + j - 1 (stream DRAFT), whose log-normaliser goes to
+ *     q_stats_out[b][j] and row index to q_row_out[b][j]; next n = N.
  *  A draw with uniform u from masses w returns the smallest index v whose
  *  running sum (ascending vocabulary order) exceeds u * sum(w).
  *  U(seed, b, step, pos, stream) = (x0 >> 8) * 2^-24 with x0 the first word
@@ -159,8 +165,11 @@ int isd_attn_strided(const isd_attn_args* a, void* stream);
  *
  * Sizes: N <= 16, V <= 262 144 (otherwise ISD_ERR_UNSUPPORTED).
  * Layouts: logits_cur, logits_prev [B][K][V] (dtype); pending_*, q_row_*
- * int32 [B][N]; n_pending_* int32 [B]; q_stats_* f32 [B][N][2] (entry 0
- * unused); n_commit int32 [B]; commit_tokens int32 [B][N]; row_stats f32
+ * int32 [B][N]; n_pending_* int32 [B]; q_stats_* f32 [B][N][2]: the
+ * natural-log normaliser ln sum_v exp(l_v) of each draft's q row as a float
+ * pair hi + lo (hi the value rounded to fp32, lo the remainder; fp32 alone
+ * would cost the residual of peaked rows its accuracy; entry 0 unused);
+ * n_commit int32 [B]; commit_tokens int32 [B][N]; row_stats f32
  * [B][K][2] or NULL (m, s of the rows used, others untouched); ratio f32
  * [B][N] or NULL (p/q of each verified draft, others untouched).
  * The *_out state arrays must not alias the *_in ones.  A sequence whose
@@ -219,12 +228,15 @@ int isd_accept_resample(const isd_accept_args* a, void* stream);
  *
  * - `workspace` and `workspace_bytes` in *a are ignored; every other field
  *   means what it means for isd_accept_resample, with the same results.
- * - Problems whose isd_accept_workspace_bytes(a) exceeds
- *   ISD_ACCEPT_STATIC_SCRATCH are rejected with ISD_ERR_WORKSPACE before any
- *   launch (at N = 4 and V = 151 936 the limit admits 1 840 sequences).
+ * - The arguments are checked exactly as isd_accept_resample checks them,
+ *   in the same order; then problems whose isd_accept_workspace_bytes(a)
+ *   exceeds ISD_ACCEPT_STATIC_SCRATCH are rejected with ISD_ERR_WORKSPACE
+ *   before any launch (at N = 4 and V = 151 936 the limit admits 1 840
+ *   sequences).
  * - The first call on each device looks up the buffer's device address
- *   (with that device current) and keeps it; make that first call before
- *   any stream capture begins.
+ *   (with that device current) and keeps it for the current CUDA context;
+ *   make that first call before any stream capture begins.  A call from a
+ *   different context on that device looks the address up again.
  * - All calls on a device share the one buffer, which keeps the previous
  *   call's contents (nothing needs clearing: each call writes every scratch
  *   word before reading it).  Calls whose work may overlap on the GPU, such
@@ -240,14 +252,21 @@ int isd_accept_resample_static(const isd_accept_args* a, void* stream);
  * is the rollback.  When a committed position enters a new page, pages are
  * popped from the free stack (entries [0, *free_top) are free, the top is
  * free_stack[*free_top - 1]), sequence 0 first, and recorded in the page
- * table; no page is freed.  All-or-nothing: if the pool or a page-table row
- * is too small, *status gets the code and nothing changes.
+ * table; no page is freed.  All-or-nothing: the whole commit is validated
+ * before anything is written, and if the pool or a page-table row is too
+ * small (ISD_ERR_POOL_EXHAUSTED, ISD_ERR_PAGE_TABLE_FULL), a length, count
+ * or free-stack top is out of range (ISD_ERR_BAD_STATE), or a page id the
+ * commit would write through or pop is outside [0, num_pages)
+ * (ISD_ERR_BAD_PAGE), *status gets the code (the lowest in that order when
+ * several hold) and no cache byte, page-table entry, length or top changes.
  *
  * Layouts: k_new, v_new [B][K][Hkv][d]; k_cache, v_cache
  * [num_pages][Hkv][16][d]; page_table int32 [B][page_table_stride];
  * seq_len, n_commit int32 [B] (0 <= n_commit <= K); free_stack int32
- * [num_pages]; free_top int32 [1]; status int32 [1] (required; set to
- * ISD_OK on success).  Workspace: isd_commit_workspace_bytes(args) bytes.
+ * [num_pages]; free_top int32 [1]; status int32 [1] (required; written
+ * only on error, see the conventions above).  B <= 32 768.
+ * Workspace: isd_commit_workspace_bytes(args) bytes (a counter), zeroed by
+ * the caller once before its first use; every call leaves it zeroed.
  * ---------------------------------------------------------------------- */
 typedef struct {
   int32_t B, K, Hkv, d;

@@ -298,6 +298,7 @@ __global__ void __launch_bounds__(kStatsThreads, 1)
     }
     fence_barrier_init();
   }
+  grid_dep_wait();
   __syncthreads();
 
   if (warp == kConsumers) {
@@ -359,7 +360,7 @@ __global__ void __launch_bounds__(kStatsThreads, 1)
       if (!failed) q0 += min(kIssuers, kGroups - m);
     }
     if (lane == 0) {
-      if (failed && p.status) *p.status = ISD_ERR_CUDA;
+      if (failed) report(p.status, ISD_ERR_CUDA);
       // Copies still in flight land before the CTA's shared memory goes
       // away (after a failure a slot may never fill: the wait is bounded).
       for (int k = max(0, q0 - kSlots); k < q0; ++k)
@@ -372,7 +373,7 @@ __global__ void __launch_bounds__(kStatsThreads, 1)
   for (int t = 0;; ++t) {
     const int q = g + t * kGroups, s = q % kSlots;
     if (!wait_bounded(&full[s], (q / kSlots) & 1)) {
-      if (lane == 0 && p.status) *p.status = ISD_ERR_CUDA;
+      if (lane == 0) report(p.status, ISD_ERR_CUDA);
       break;
     }
     const int it = item[s];
@@ -448,6 +449,7 @@ __global__ void __launch_bounds__(kStatsThreads, 1)
 template <typename T>
 __global__ void __launch_bounds__(256) accept_stats_plain_kernel(AcceptDev<T> p) {
   const int lane = threadIdx.x & 31;
+  grid_dep_wait();
   const int warps = gridDim.x * (blockDim.x >> 5);
   const int total = p.B * p.RU * p.C;
   for (int it = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -471,6 +473,7 @@ __global__ void __launch_bounds__(1024) accept_decide_kernel(AcceptDev<T> p) {
   __shared__ double s_s[32];
   const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = p.N, K = p.K;
+  grid_dep_wait();
   const int n = p.n_in[b];
   const int L = p.seq_len[b];
   const int tok = lane < N ? p.pending_in[b * N + lane] : 0;
@@ -486,7 +489,7 @@ __global__ void __launch_bounds__(1024) accept_decide_kernel(AcceptDev<T> p) {
   if (!ok) {
     if (warp != 0) return;
     if (lane == 0) {
-      if (p.status) *p.status = ISD_ERR_BAD_STATE;
+      report(p.status, ISD_ERR_BAD_STATE);
       p.n_commit[b] = 0;
       p.n_out[b] = n;
       p.count[b] = 0;
@@ -505,12 +508,12 @@ __global__ void __launch_bounds__(1024) accept_decide_kernel(AcceptDev<T> p) {
   // Warp 0 fetches the logits at the drafts first, so that their latency
   // overlaps the merge.
   const bool verifies = warp == 0 && lane >= 1 && lane < n;
-  float lx = 0.0f, lqx = 0.0f, mq = 0.0f, sq = 1.0f;
+  float lx = 0.0f, lqx = 0.0f, zhi = 0.0f, zlo = 0.0f;
   if (verifies) {
     lx = to_f(p.lc[((size_t)b * K + lane - 1) * p.V + tok]);
     if (!p.argmax) {
-      mq = p.q_stats_in[(b * N + lane) * 2];
-      sq = p.q_stats_in[(b * N + lane) * 2 + 1];
+      zhi = p.q_stats_in[(b * N + lane) * 2];
+      zlo = p.q_stats_in[(b * N + lane) * 2 + 1];
       lqx = to_f(p.lp[((size_t)b * K + qr) * p.V + tok]);
     }
   }
@@ -553,7 +556,7 @@ __global__ void __launch_bounds__(1024) accept_decide_kernel(AcceptDev<T> p) {
   if (verifies) {
     const double px = exp((double)(lx - s_m[lane - 1])) / s_s[lane - 1];
     double qx = 1.0;      // argmax drafts: the proposal is a point mass
-    if (!p.argmax) qx = exp((double)(lqx - mq)) / (double)sq;
+    if (!p.argmax) qx = exp(((double)lqx - (double)zhi) - (double)zlo);
     const double r = qx > 0.0 ? px / qx : INFINITY;
     const float u = uniform(p.seed, (uint32_t)b, step_of(p),
                             (uint32_t)(L + lane), ISD_STREAM_ACCEPT);
@@ -567,12 +570,15 @@ __global__ void __launch_bounds__(1024) accept_decide_kernel(AcceptDev<T> p) {
   const int a = rejected ? (__ffs(rej) - 2) : (n - 1);
   if (lane < N) {
     p.commit_tokens[b * N + lane] = lane <= a ? tok : -1;
-    // Next drafts' q rows and their statistics (lane j: row n + j - 1).
+    // Next drafts' q rows and the log-normaliser log sum_v exp(l_v) of
+    // each (lane j: row n + j - 1), stored as a float pair hi + lo.
     const bool has = !rejected && lane >= 1;
     const int src = n + lane - 1;
     p.q_row_out[b * N + lane] = has ? src : -1;
-    p.q_stats_out[(b * N + lane) * 2] = has ? s_m[src] : 0.0f;
-    p.q_stats_out[(b * N + lane) * 2 + 1] = has ? (float)s_s[src] : 0.0f;
+    const double lz = has ? (double)s_m[src] + log(s_s[src]) : 0.0;
+    const float lz_hi = (float)lz;
+    p.q_stats_out[(b * N + lane) * 2] = lz_hi;
+    p.q_stats_out[(b * N + lane) * 2 + 1] = (float)(lz - (double)lz_hi);
     // After a rejection only the replacement is pending.
     if (rejected && lane >= 1) p.pending_out[b * N + lane] = -1;
   }
@@ -589,14 +595,39 @@ __global__ void __launch_bounds__(1024) accept_decide_kernel(AcceptDev<T> p) {
 // the in-sub-chunk scan so both see the same per-element values.
 // With argmax drafts q is a point mass at the rejected draft x, so the
 // residual is p without x.
+//
+// Where p and q are close (peaked rows that agree on their top token) the
+// plain difference of two rounded masses cancels: its absolute error, a few
+// 1e-7 of q, can exceed the 1e-6 tie band of a small residual total.  Only
+// elements of large mass can do that (the error scales with the mass), so
+// for q > 2^-10 the weight is re-formed from delta = ln p - ln q =
+// (l_p - l_q) - C, with l_p - l_q exact and C = (m_p + ln s_p) - ln Z_q in
+// fp64 (a float pair): 0 for delta <= 0, q * expm1(delta) for
+// 0 < delta <= 1 (relative error a few ulp whatever the cancellation), and
+// the plain difference above 1 (p > e q: no cancellation).  That path is
+// rare and kept out of line, so the unrolled element loops stay compact.
 struct ResidRows {
-  float mp, inv_sp, mq, inv_sq;
-  int x;          // rejected draft (argmax proposals), else -1
+  float mp, inv_sp;       // p row: max and 1 / sum
+  float zq_hi, zq_lo;     // q row: log-normaliser ln Z_q as a float pair
+  float c_hi, c_lo;       // C as a float pair
+  int x;                  // rejected draft (argmax proposals), else -1
 };
+constexpr float kResidExactMass = 1.0f / 1024.0f;
+
+__device__ __noinline__ float resid_exact(float qv, float lpv, float lqv,
+                                          float c_hi, float c_lo, float w) {
+  const float delta = ((lpv - lqv) - c_hi) - c_lo;
+  if (!(delta > 0.0f)) return 0.0f;
+  return delta <= 1.0f ? qv * expm1f(delta) : w;
+}
+
 ISD_DEV float resid_w(const ResidRows& r, float lpv, float lqv, int v) {
-  if (r.x >= 0) return v == r.x ? 0.0f : ex2((lpv - r.mp) * kLog2e) * r.inv_sp;
-  return fmaxf(0.0f, ex2((lpv - r.mp) * kLog2e) * r.inv_sp -
-                         ex2((lqv - r.mq) * kLog2e) * r.inv_sq);
+  const float pv = ex2((lpv - r.mp) * kLog2e) * r.inv_sp;
+  if (r.x >= 0) return v == r.x ? 0.0f : pv;
+  const float qv = ex2(((lqv - r.zq_hi) - r.zq_lo) * kLog2e);
+  float w = pv - qv;
+  if (qv > kResidExactMass) w = resid_exact(qv, lpv, lqv, r.c_hi, r.c_lo, w);
+  return fmaxf(0.0f, w);
 }
 
 template <typename T>
@@ -606,16 +637,20 @@ ISD_DEV ResidRows resid_rows(const AcceptDev<T>& p, int b, int a,
   prow = p.lc + ((size_t)b * K + a) * p.V;
   ResidRows r;
   r.mp = p.rmax[b * K + a];
-  r.inv_sp = (float)(1.0 / p.rsum[b * K + a]);
+  const double sp = p.rsum[b * K + a];
+  r.inv_sp = (float)(1.0 / sp);
   if (p.argmax) {
     qrow = prow;                       // not read
-    r.mq = 0.0f; r.inv_sq = 0.0f;
+    r.zq_hi = r.zq_lo = r.c_hi = r.c_lo = 0.0f;
     r.x = p.pending_in[b * N + a + 1];
   } else {
     const int qr = p.q_row_in[b * N + a + 1];
     qrow = p.lp + ((size_t)b * K + qr) * p.V;
-    r.mq = p.q_stats_in[(b * N + a + 1) * 2];
-    r.inv_sq = 1.0f / p.q_stats_in[(b * N + a + 1) * 2 + 1];
+    r.zq_hi = p.q_stats_in[(b * N + a + 1) * 2];
+    r.zq_lo = p.q_stats_in[(b * N + a + 1) * 2 + 1];
+    const double c = ((double)r.mp + log(sp)) - ((double)r.zq_hi + (double)r.zq_lo);
+    r.c_hi = (float)c;
+    r.c_lo = (float)(c - (double)r.c_hi);
     r.x = -1;
   }
   return r;
@@ -757,6 +792,7 @@ __global__ void __launch_bounds__(kDrawWarps * 32,
   // (its draws, or its first residual sub-chunks) is scheduled first.
   const int b = blockIdx.x, lane = threadIdx.x & 31;
   const int wi = blockIdx.y * kDrawWarps + (threadIdx.x >> 5);
+  grid_dep_wait();
   const int32_t* dec = p.decision + b * 4;
   if (dec[0] == 0) return;  // malformed state: decide copied it through
   const bool rejected = dec[1] != 0;
@@ -924,18 +960,26 @@ static int launch_accept_t(const isd_accept_args* a, cudaStream_t st) {
     const int S = kCopyBytes / (kSub * (int)sizeof(T));
     const long long copies = (long long)p.B * p.RU * ((p.C + S - 1) / S);
     const int grid = (int)std::min<long long>(sms, copies);
-    kern<<<grid, kStatsThreads, kStatsSmem, st>>>(p);
+    if (launch_pdl(kern, dim3(grid), dim3(kStatsThreads), kStatsSmem, st, p) !=
+        cudaSuccess)
+      return ISD_ERR_CUDA;
   } else {
     const int grid = (int)std::min<long long>(8LL * sms, (items + 7) / 8);
-    accept_stats_plain_kernel<T><<<grid, 256, 0, st>>>(p);
+    if (launch_pdl(accept_stats_plain_kernel<T>, dim3(grid), dim3(256), 0, st,
+                   p) != cudaSuccess)
+      return ISD_ERR_CUDA;
   }
-  accept_decide_kernel<T><<<p.B, 32 * p.RU, 0, st>>>(p);
+  if (launch_pdl(accept_decide_kernel<T>, dim3(p.B), dim3(32 * p.RU), 0, st,
+                 p) != cudaSuccess)
+    return ISD_ERR_CUDA;
   const dim3 g_draw(p.B, (std::max(p.C, p.N) + kDrawWarps - 1) / kDrawWarps);
-  if ((a->V % 8) == 0)
-    accept_draw_kernel<T, true><<<g_draw, kDrawWarps * 32, 0, st>>>(p);
-  else
-    accept_draw_kernel<T, false><<<g_draw, kDrawWarps * 32, 0, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? ISD_OK : ISD_ERR_CUDA;
+  const cudaError_t e =
+      (a->V % 8) == 0
+          ? launch_pdl(accept_draw_kernel<T, true>, g_draw,
+                       dim3(kDrawWarps * 32), 0, st, p)
+          : launch_pdl(accept_draw_kernel<T, false>, g_draw,
+                       dim3(kDrawWarps * 32), 0, st, p);
+  return e == cudaSuccess ? ISD_OK : ISD_ERR_CUDA;
 }
 
 size_t accept_workspace_bytes(int B, int N, int K, int V) {

@@ -48,7 +48,8 @@
 //                       the (b, h) straddles CTAs).
 //
 // Every mbarrier wait is bounded; after one timeout a thread records
-// ISD_ERR_CUDA and stops waiting, so the kernel ends.
+// ISD_ERR_CUDA (unless an earlier error is already recorded) and stops
+// waiting, so the kernel ends.
 #include "common.cuh"
 
 namespace isd {
@@ -305,15 +306,16 @@ ISD_DEV void warp_transpose_reduce(float (&v)[32], int lane) {
 }
 
 // Bounded wait; after the first timeout (`failed` set) waits are skipped.
-ISD_DEV void wait_or_fail(uint64_t* bar, uint32_t parity, bool& failed,
-                          int32_t* status) {
+// The wait records nothing itself (a status write inside these loops slows
+// them): every thread that gave up reports ISD_ERR_CUDA once, at the end of
+// the kernel.
+ISD_DEV void wait_or_fail(uint64_t* bar, uint32_t parity, bool& failed) {
   if (failed) return;
   if (mbar_try_wait(bar, parity)) return;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if ((uint64_t)(clock64() - t0) > kWaitCycles) {
       failed = true;
-      if (status) *status = ISD_ERR_CUDA;
       return;
     }
   }
@@ -376,7 +378,6 @@ struct EpiIn {
   float* part_o;
   float* lse;
   float* part_ml;
-  int32_t* status;
   const CUtensorMap* tm_out;
   const CUtensorMap* tm_part;
   const CUtensorMap* tm_lse;
@@ -420,7 +421,7 @@ __device__ __noinline__ bool store_segment(const EpiIn<NCH>& in, int blk, int co
   // O^T of the segment is complete once the P V of its last block lands:
   // phase blk / NPB of p_empty[blk % NPB], at most one phase past the last
   // one these threads waited for there.
-  wait_or_fail(&in.p_empty[blk % NPB], (blk / NPB) & 1, failed, in.status);
+  wait_or_fail(&in.p_empty[blk % NPB], (blk / NPB) & 1, failed);
   tc_fence_after();
   if (stage_buf >= 0) stage_sync();
   const uint32_t eo = kO + tb * N, el = kL + tb * N;
@@ -586,26 +587,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int B = p.B, Hkv = p.Hkv, M = p.M;
-  if (tid == 0) s_bad = 0;
-  __syncthreads();
-  const int T = block_exclusive_scan_int(
-      B,
-      [&](int b) {
-        int L = p.seq_len[b];
-        bool bad = false;
-        if (L < 0) { bad = true; L = 0; }
-        int n = (L + kPage - 1) / kPage;
-        if (n > p.stride) { bad = true; n = p.stride; L = n * kPage; }
-        if (bad) s_bad = 1;
-        seqL[b] = L;
-        return Hkv * (n + 1);
-      },
-      prefix, scan_sh);
-  if (tid == 0) prefix[B] = T;
-  const int G = gridDim.x, c = blockIdx.x;
-  const int u0 = split_point(prefix, B, T, Hkv, c, G);
-  const int u1 = split_point(prefix, B, T, Hkv, c + 1, G);
   if (tid == 0) {
+    s_bad = 0;
     for (int s = 0; s < SK; ++s) {
       mbar_init(&k_full[s], kLoadWarps);    // one arrival per loader warp
       mbar_init(&k_empty[s], 1);
@@ -637,6 +620,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         make_uint4(0, 0, 0, 0);
   }
   proxy_fence();
+  // Everything above is independent of the kernel before this one.
+  grid_dep_wait();
+  __syncthreads();
+  const int T = block_exclusive_scan_int(
+      B,
+      [&](int b) {
+        int L = p.seq_len[b];
+        bool bad = false;
+        if (L < 0) { bad = true; L = 0; }
+        int n = (L + kPage - 1) / kPage;
+        if (n > p.stride) { bad = true; n = p.stride; L = n * kPage; }
+        if (bad) s_bad = 1;
+        seqL[b] = L;
+        return Hkv * (n + 1);
+      },
+      [&](int b, int v) { prefix[b] = v; }, scan_sh);
+  if (tid == 0) prefix[B] = T;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int u0 = split_point(prefix, B, T, Hkv, c, G);
+  const int u1 = split_point(prefix, B, T, Hkv, c + 1, G);
   if (warp == kMmaWarp) {
     asm volatile(
         "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::
@@ -653,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
       p.ws_int[B + 1] = G;
       p.ws_int[B + 2 + G] = T;
-      if (s_bad && p.status) *p.status = ISD_ERR_PAGE_TABLE_FULL;
+      if (s_bad) report(p.status, ISD_ERR_PAGE_TABLE_FULL);
     }
   }
   if (tid == 0) p.ws_int[B + 2 + c] = u0;   // range starts, for the combine
@@ -697,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Q rows of (b, h) by TMA: row m = r * g + j holds q[b][r][h*g + j],
         // the box {64, g, K} of the [B][K][Hq][128] tensor, per 64 columns.
         const int qb = t % NQB;
-        wait_or_fail(&q_empty[qb], ((t / NQB) & 1) ^ 1, failed, p.status);
+        wait_or_fail(&q_empty[qb], ((t / NQB) & 1) ^ 1, failed);
         mbar_arrive_expect_tx(&q_full[qb], 2 * M * 128);
         for (int hb = 0; hb < 2; ++hb)
           tma_load_4d(qs + qb * QB + hb * QH, &tm_q, &q_full[qb], hb * 64,
@@ -718,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int pg = q == 0 ? pid0 : pid1;
         const bool bad = use[q] && !tail[q] && (pg < 0 || pg >= p.P);
         if (bad) {
-          if (lane == 0 && p.status) *p.status = ISD_ERR_BAD_PAGE;
+          if (lane == 0) report(p.status, ISD_ERR_BAD_PAGE);
           pg = p.P;
         }
         page[q] = pg;
@@ -728,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // K tiles.  Rows past K of the tail lie outside the staging tensor
       // and read as zeros.
       const int ks = i % SK;
-      wait_or_fail(&k_empty[ks], ((i / SK) & 1) ^ 1, failed, p.status);
+      wait_or_fail(&k_empty[ks], ((i / SK) & 1) ^ 1, failed);
       if (lane == 0) {
 #pragma unroll
         for (int q = 0; q < kPagesPerLoader; ++q) {
@@ -750,7 +753,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // would reach O through P V).  K there is harmless: those scores are
       // masked.
       const int vs = i % SV;
-      wait_or_fail(&v_empty[vs], ((i / SV) & 1) ^ 1, failed, p.status);
+      wait_or_fail(&v_empty[vs], ((i / SV) & 1) ^ 1, failed);
       bool partial_v = false;
 #pragma unroll
       for (int q = 0; q < kPagesPerLoader; ++q) {
@@ -812,8 +815,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_pv = [&](int j_blk) {
       // O^T += V^T P^T for block j_blk: one k-step of 16 keys per page.
       const int vs = j_blk % SV;
-      wait_or_fail(&p_full[prev_pb], (j_blk / NPB) & 1, failed, p.status);
-      wait_or_fail(&v_full[vs], (j_blk / SV) & 1, failed, p.status);
+      wait_or_fail(&p_full[prev_pb], (j_blk / NPB) & 1, failed);
+      wait_or_fail(&v_full[vs], (j_blk / SV) & 1, failed);
       tc_fence_after();
       if (lane == 0) {
         const uint32_t pa = p_s + prev_pb * PB;
@@ -833,11 +836,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++t;
         // Q, K and V arrive by TMA (a partial page's V by cp.async that its
         // loader warp fences before arriving).
-        wait_or_fail(&q_full[t % NQB], (t / NQB) & 1, failed, p.status);
+        wait_or_fail(&q_full[t % NQB], (t / NQB) & 1, failed);
       }
       const int qb = t % NQB;
-      wait_or_fail(&k_full[ks], (i / SK) & 1, failed, p.status);
-      wait_or_fail(&s_free[sbuf], ((i >> 1) & 1) ^ 1, failed, p.status);
+      wait_or_fail(&k_full[ks], (i / SK) & 1, failed);
+      wait_or_fail(&s_free[sbuf], ((i >> 1) & 1) ^ 1, failed);
       tc_fence_after();
       if (lane == 0) {
         // S^T = K Q^T over the 128 keys of the tile (rows of pages past
@@ -858,8 +861,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The first P V of segment t overwrites O^T buffer t % NOB: the
         // epilogue of segment t - NOB must have read it.
         if (prev_first && prev_t >= NOB)
-          wait_or_fail(&o_free[prev_t % NOB], ((prev_t / NOB) & 1) ^ 1, failed,
-                       p.status);
+          wait_or_fail(&o_free[prev_t % NOB], ((prev_t / NOB) & 1) ^ 1, failed);
         issue_pv(i - 1);
       }
       have_prev = true;
@@ -869,15 +871,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (have_prev) {
       if (prev_first && prev_t >= NOB)
-        wait_or_fail(&o_free[prev_t % NOB], ((prev_t / NOB) & 1) ^ 1, failed,
-                     p.status);
+        wait_or_fail(&o_free[prev_t % NOB], ((prev_t / NOB) & 1) ^ 1, failed);
       issue_pv(i - 1);
     }
     // Every MMA this CTA issued has completed before TMEM is released.
     if (lane == 0) umma_commit(fin);
     __syncwarp();
     bool fin_failed = false;
-    wait_or_fail(fin, 0, fin_failed, p.status);
+    wait_or_fail(fin, 0, fin_failed);
+    failed = failed || fin_failed;
   } else {
     // ---------------------------------------------------------- softmax
     const int kl = tid;                       // key of the block = TMEM lane
@@ -908,7 +910,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       sm_sync();
       stage_buf = -1;
     };
-    const EpiIn<NCH> ein{p.out, p.part_o, p.lse, p.part_ml, p.status, &tm_out,
+    const EpiIn<NCH> ein{p.out, p.part_o, p.lse, p.part_ml, &tm_out,
                          &tm_part, &tm_lse, ep_small, p.lse_tma, p.ml_bulk,
                          tmem + lane_base, ps, p_empty, o_free, &m_raw[0][0],
                          &x_red[0][0], r_val, p.g, p.K, p.Hq, M, c, c2};
@@ -936,10 +938,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool key_all = in_blk && !tail && rr < L - uidx * kPage;
       const int col_min =
           (tail && rr < p.K) ? rr * p.g : (key_all ? 0 : (1 << 30));
-      wait_or_fail(&s_full[sbuf], (i >> 1) & 1, failed, p.status);
+      wait_or_fail(&s_full[sbuf], (i >> 1) & 1, failed);
       tc_fence_after();
       const int pbi = i % NPB;
-      wait_or_fail(&p_empty[pbi], ((i / NPB) & 1) ^ 1, failed, p.status);
+      wait_or_fail(&p_empty[pbi], ((i / NPB) & 1) ^ 1, failed);
       if (stage_buf == pbi) stage_sync();   // a TMA store still reads it
       bool o_ready = false;
       uint8_t* pt = ps + pbi * PB;
@@ -1031,8 +1033,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // a barrier this thread waits on every NPB blocks, so a parity
             // wait names that phase unambiguously.
             if (!o_ready) {
-              wait_or_fail(&p_empty[(i - 1) % NPB], ((i - 1) / NPB) & 1, failed,
-                           p.status);
+              wait_or_fail(&p_empty[(i - 1) % NPB], ((i - 1) / NPB) & 1, failed);
               tc_fence_after();
               o_ready = true;
             }
@@ -1064,6 +1065,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (kDefer && ep.blk >= 0) epilogue(ep);
     if (tid == 0) bulk_wait_all();
   }
+  if (failed) report(p.status, ISD_ERR_CUDA);   // a bounded wait ran out
   // Everyone meets before TMEM is released.
   tc_fence_before();
   __syncthreads();
@@ -1244,9 +1246,9 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return ISD_ERR_CUDA;
-  kern<<<G, tc::kThreads, smem, st>>>(tkc, tvc, tkn, tvn, tout, tpart, tq, tlse,
-                                      p);
-  if (cudaGetLastError() != cudaSuccess) return ISD_ERR_CUDA;
+  if (launch_pdl(kern, dim3(G), dim3(tc::kThreads), smem, st, tkc, tvc, tkn,
+                 tvn, tout, tpart, tq, tlse, p) != cudaSuccess)
+    return ISD_ERR_CUDA;
   return launch_attn_combine(a, G, st);
 }
 

@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "isd.h"
 
 #define ISD_DEV __device__ __forceinline__
@@ -43,6 +45,49 @@ ISD_DEV float uniform(uint64_t seed, uint32_t seq, uint32_t step, uint32_t pos,
   const U4 o = philox4x32_10(U4{seq, step, pos, stream}, (uint32_t)seed,
                              (uint32_t)(seed >> 32));
   return (float)(o.x >> 8) * (1.0f / 16777216.0f);
+}
+
+// ---------------------------------------------------------------------------
+// Device-side error reporting.  The caller's status word keeps the FIRST
+// error recorded in it: a kernel never clears it and never overwrites an
+// error that an earlier kernel (or call) left there, so a step's three calls
+// may share one word and the host reads the earliest failure after the step.
+
+// Kept out of line: it sits on the failure path of every bounded wait, and
+// an inlined atomic there slows the wait loops themselves (measured: the
+// attention kernel ran 2% slower).
+static __device__ __noinline__ void report(int32_t* status, int code) {
+  if (status) atomicCAS(reinterpret_cast<int*>(status), ISD_OK, code);
+}
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of a step is launched with
+// programmatic stream serialisation and waits (grid_dep_wait) for the
+// kernel before it on the stream to finish, its memory visible, before it
+// reads anything; work that does not depend on it (barrier set-up) comes
+// first.  No kernel triggers its dependents early: measured on the C=64
+// step, letting the next grid launch while the current one still runs put
+// waiting CTAs beside the running ones and cost more than it saved, while
+// the serialised form with these waits still shortens every boundary.
+// Without a programmatic predecessor the wait returns at once.
+
+ISD_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launches `kern` on `st` with programmatic stream serialisation.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block,
+                              size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // ---------------------------------------------------------------------------
@@ -109,84 +154,11 @@ ISD_DEV float warp_sum(float v) {
   return v;
 }
 
-// Block-wide reduction; `red` holds >= 32 values; all threads get the result.
-template <bool kMax>
-ISD_DEV float block_reduce(float v, float* red) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int nw = (blockDim.x + 31) >> 5;
-  v = kMax ? warp_max(v) : warp_sum(v);
-  __syncthreads();
-  if (lane == 0) red[wid] = v;
-  __syncthreads();
-  float r = lane < nw ? red[lane] : (kMax ? -INFINITY : 0.0f);
-  r = kMax ? warp_max(r) : warp_sum(r);
-  return r;
-}
-
-// Block-wide minimum of ints; `red` holds >= 32 ints; all threads get it.
-ISD_DEV int block_min_int(int v, int* red) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int nw = (blockDim.x + 31) >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
-  __syncthreads();
-  if (lane == 0) red[wid] = v;
-  __syncthreads();
-  int r = lane < nw ? red[lane] : INT_MAX;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) r = min(r, __shfl_xor_sync(0xffffffffu, r, o));
-  return r;
-}
-
-ISD_DEV double block_sum(double v, double* red) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int nw = (blockDim.x + 31) >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  __syncthreads();
-  if (lane == 0) red[wid] = v;
-  __syncthreads();
-  double r = lane < nw ? red[lane] : 0.0;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
-  return r;
-}
-
-// Inclusive scan over the block of one value per thread (fixed order).
-// Returns the inclusive prefix; `excl` gets exactly the previous thread's
-// inclusive prefix (0 for thread 0) and `total` the block sum.  `sh` >= 32.
-template <typename T>
-ISD_DEV T block_inclusive_scan(T v, T* sh, T& excl, T& total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int nw = (blockDim.x + 31) >> 5;
-  T x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const T y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  T prev = __shfl_up_sync(0xffffffffu, x, 1);
-  __syncthreads();
-  if (lane == 31) sh[wid] = x;
-  __syncthreads();
-  // Warp totals are scanned sequentially: sh[w] = sh[w-1] + total_w is then
-  // the very addition the last thread of warp w performs below.
-  if (threadIdx.x == 0)
-    for (int w = 1; w < nw; ++w) sh[w] = sh[w - 1] + sh[w];
-  __syncthreads();
-  total = sh[nw - 1];
-  const T base = wid > 0 ? sh[wid - 1] : T(0);
-  if (lane == 0) prev = T(0);
-  // Apply the warp offset to both prefixes with the same single addition,
-  // so thread i's excl equals thread i-1's result bit for bit.
-  excl = (lane == 0) ? base : (wid > 0 ? base + prev : prev);
-  return wid > 0 ? base + x : x;
-}
-
-// Exclusive scan of ints over the block (loops for n > blockDim).
-// out[i] = sum_{j<i} in(j), returns the total.  `sh` >= 33 ints.
-template <typename F>
-ISD_DEV int block_exclusive_scan_int(int n, F in, int* out, int* sh) {
+// Exclusive scan of ints over the block (loops for n > blockDim), in index
+// order: store(i, sum_{j<i} in(j)) for every i < n; returns the total.
+// Every thread of the block must call it.  `sh` >= 33 ints.
+template <typename F, typename S>
+ISD_DEV int block_exclusive_scan_int(int n, F in, S store, int* sh) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int nw = (blockDim.x + 31) >> 5;
   int carry = 0;
@@ -213,7 +185,7 @@ ISD_DEV int block_exclusive_scan_int(int n, F in, int* out, int* sh) {
     }
     __syncthreads();
     const int excl = x - v + (wid > 0 ? sh[wid - 1] : 0);
-    if (i < n) out[i] = carry + excl;
+    if (i < n) store(i, carry + excl);
     carry += sh[nw - 1];
     __syncthreads();
   }
@@ -255,7 +227,7 @@ ISD_DEV int split_point(const int* prefix, int B, int T, int Hkv, int c,
 }
 
 // ---------------------------------------------------------------------------
-// mbarrier / TMA / ldmatrix / mma wrappers (inline PTX, sm_90+ forms).
+// mbarrier / TMA wrappers (inline PTX, sm_90+ forms).
 
 ISD_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -300,20 +272,6 @@ ISD_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: gives up after `limit` polls and reports false.  Every
-// wait in this library is bounded so that a broken invariant ends the
-// kernel with an error status instead of hanging the device.
-ISD_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
-  for (uint32_t i = 0; i < limit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
-}
-
-ISD_DEV void tma_prefetch_desc(const CUtensorMap* m) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m))
-               : "memory");
-}
-
 // 4-D tiled TMA load into shared memory, completion on `bar` (tx bytes).
 ISD_DEV void tma_load_4d(void* dst, const CUtensorMap* m, uint64_t* bar,
                          int c0, int c1, int c2, int c3) {
@@ -332,39 +290,6 @@ ISD_DEV void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
                "l"(src), "r"(src_bytes)
                : "memory");
 }
-// Arrive on `bar` once every cp.async this thread issued so far completes
-// (counts as one of the barrier's expected arrivals).
-ISD_DEV void cp_async_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-ISD_DEV void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,
-                         uint32_t& r2, uint32_t& r3) {
-  asm volatile(
-      "ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-      : "r"(addr));
-}
-ISD_DEV void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
-                               uint32_t& r2, uint32_t& r3) {
-  asm volatile(
-      "ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-      : "r"(addr));
-}
-
-// D = A * B + D, m16n8k16, bf16 inputs, fp32 accumulators.
-ISD_DEV void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                            uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 ISD_DEV uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

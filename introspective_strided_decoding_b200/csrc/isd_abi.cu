@@ -8,9 +8,9 @@ namespace isd {
 size_t accept_workspace_bytes(int B, int N, int K, int V);
 int launch_accept(const isd_accept_args* a, cudaStream_t st);
 size_t commit_workspace_bytes(int B);
+int commit_max_batch();
 int launch_commit(const isd_commit_args* a, cudaStream_t st);
 size_t attn_workspace_bytes_impl(int B, int M, int D, int G);
-size_t attn_smem_bytes(int D, int MW, int B);
 size_t attn_tc_smem_bytes(int B, int M);
 int launch_attn_bf16(const isd_attn_args* a, int G, cudaStream_t st);
 int launch_attn_f32(const isd_attn_args* a, cudaStream_t st);
@@ -48,19 +48,12 @@ int attn_check(const isd_attn_args* a) {
   if (a->dtype == ISD_BF16) {
     const int M = a->K * (a->Hq / a->Hkv);
     if (a->K > ISD_PAGE_SIZE || M > 128) return ISD_ERR_UNSUPPORTED;
-    if (a->d == 128) {
-      // tcgen05 path: any row count up to 128 (rows padded to a multiple
-      // of 32); the stage ring must fit next to Q, P and the unit prefix.
-      if (isd::attn_tc_smem_bytes(a->B, M) == (size_t)-1)
-        return ISD_ERR_UNSUPPORTED;
-    } else if (a->d == 64) {
-      // mma.sync path: rows in warps of 16 or 32.
-      if (!(M == 16 || M == 32 || M == 64 || M == 128)) return ISD_ERR_UNSUPPORTED;
-      if (isd::attn_smem_bytes(a->d, M <= 32 ? 1 : 2, a->B) > 227 * 1024)
-        return ISD_ERR_UNSUPPORTED;
-    } else {
+    // tcgen05 path: head dim 128, any row count up to 128 (rows padded to
+    // a multiple of 32); the stage ring must fit next to Q, P and the unit
+    // prefix.
+    if (a->d != 128) return ISD_ERR_UNSUPPORTED;
+    if (isd::attn_tc_smem_bytes(a->B, M) == (size_t)-1)
       return ISD_ERR_UNSUPPORTED;
-    }
   } else if (a->dtype == ISD_F32) {
     if (a->d % 32 != 0 || a->d > 128) return ISD_ERR_UNSUPPORTED;
   } else {
@@ -70,6 +63,42 @@ int attn_check(const isd_attn_args* a) {
 }
 
 }  // namespace
+
+namespace isd {
+
+int accept_check(const isd_accept_args* a) {
+  if (!a) return ISD_ERR_INVALID_ARG;
+  if (a->B <= 0 || a->N < 2 || a->V <= 0 || a->K != 2 * a->N)
+    return ISD_ERR_INVALID_ARG;
+  if (a->N > 16) return ISD_ERR_UNSUPPORTED;
+  if (a->V > 128 * 2048) return ISD_ERR_UNSUPPORTED;  // <= 128 sub-chunks
+  if (a->dtype != ISD_BF16 && a->dtype != ISD_F32) return ISD_ERR_INVALID_ARG;
+  if (a->proposal != ISD_PROPOSAL_SAMPLE && a->proposal != ISD_PROPOSAL_ARGMAX)
+    return ISD_ERR_INVALID_ARG;
+  return ISD_OK;
+}
+
+// Every check of isd_accept_resample except the workspace's (shared with
+// the allocation-free entry point, so both report the same errors first).
+int accept_validate(const isd_accept_args* a) {
+  const int rc = accept_check(a);
+  if (rc != ISD_OK) return rc;
+  if (!a->logits_cur || !a->logits_prev || !a->seq_len || !a->pending_in ||
+      !a->n_pending_in || !a->q_row_in || !a->q_stats_in || !a->pending_out ||
+      !a->n_pending_out || !a->q_row_out || !a->q_stats_out || !a->n_commit ||
+      !a->commit_tokens)
+    return ISD_ERR_INVALID_ARG;
+  if ((const void*)a->pending_out == (const void*)a->pending_in ||
+      (const void*)a->n_pending_out == (const void*)a->n_pending_in ||
+      (const void*)a->q_row_out == (const void*)a->q_row_in ||
+      (const void*)a->q_stats_out == (const void*)a->q_stats_in)
+    return ISD_ERR_INVALID_ARG;
+  if (!aligned16(a->logits_cur) || !aligned16(a->logits_prev))
+    return ISD_ERR_INVALID_ARG;
+  return ISD_OK;
+}
+
+}  // namespace isd
 
 extern "C" {
 
@@ -123,38 +152,14 @@ int isd_attn_strided(const isd_attn_args* a, void* stream) {
 }
 
 // ---------------------------------------------------------------- accept
-static int accept_check(const isd_accept_args* a) {
-  if (!a) return ISD_ERR_INVALID_ARG;
-  if (a->B <= 0 || a->N < 2 || a->V <= 0 || a->K != 2 * a->N)
-    return ISD_ERR_INVALID_ARG;
-  if (a->N > 16) return ISD_ERR_UNSUPPORTED;
-  if (a->V > 128 * 2048) return ISD_ERR_UNSUPPORTED;  // <= 128 sub-chunks
-  if (a->dtype != ISD_BF16 && a->dtype != ISD_F32) return ISD_ERR_INVALID_ARG;
-  if (a->proposal != ISD_PROPOSAL_SAMPLE && a->proposal != ISD_PROPOSAL_ARGMAX)
-    return ISD_ERR_INVALID_ARG;
-  return ISD_OK;
-}
-
 size_t isd_accept_workspace_bytes(const isd_accept_args* a) {
-  if (accept_check(a) != ISD_OK) return 0;
+  if (isd::accept_check(a) != ISD_OK) return 0;
   return isd::accept_workspace_bytes(a->B, a->N, a->K, a->V);
 }
 
 int isd_accept_resample(const isd_accept_args* a, void* stream) {
-  const int rc = accept_check(a);
+  const int rc = isd::accept_validate(a);
   if (rc != ISD_OK) return rc;
-  if (!a->logits_cur || !a->logits_prev || !a->seq_len || !a->pending_in ||
-      !a->n_pending_in || !a->q_row_in || !a->q_stats_in || !a->pending_out ||
-      !a->n_pending_out || !a->q_row_out || !a->q_stats_out || !a->n_commit ||
-      !a->commit_tokens)
-    return ISD_ERR_INVALID_ARG;
-  if ((const void*)a->pending_out == (const void*)a->pending_in ||
-      (const void*)a->n_pending_out == (const void*)a->n_pending_in ||
-      (const void*)a->q_row_out == (const void*)a->q_row_in ||
-      (const void*)a->q_stats_out == (const void*)a->q_stats_in)
-    return ISD_ERR_INVALID_ARG;
-  if (!aligned16(a->logits_cur) || !aligned16(a->logits_prev))
-    return ISD_ERR_INVALID_ARG;
   const size_t need = isd::accept_workspace_bytes(a->B, a->N, a->K, a->V);
   if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace))
     return ISD_ERR_WORKSPACE;
@@ -170,6 +175,7 @@ static int commit_check(const isd_commit_args* a) {
   if (a->dtype != ISD_BF16 && a->dtype != ISD_F32) return ISD_ERR_INVALID_ARG;
   const int es = a->dtype == ISD_BF16 ? 2 : 4;
   if ((a->d * es) % 16 != 0) return ISD_ERR_UNSUPPORTED;
+  if (a->B > isd::commit_max_batch()) return ISD_ERR_UNSUPPORTED;
   return ISD_OK;
 }
 
@@ -189,7 +195,8 @@ int isd_kv_commit(const isd_commit_args* a, void* stream) {
       !aligned16(a->v_cache))
     return ISD_ERR_INVALID_ARG;
   const size_t need = isd::commit_workspace_bytes(a->B);
-  if (!a->workspace || a->workspace_bytes < need) return ISD_ERR_WORKSPACE;
+  if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace))
+    return ISD_ERR_WORKSPACE;
   return isd::launch_commit(a, static_cast<cudaStream_t>(stream));
 }
 

@@ -81,7 +81,7 @@ class Decoder:
             self.k_new, self.v_new, cache["k_cache"], cache["v_cache"],
             cache["page_table"], cache["seq_len"], self.n_commit,
             cache["free_stack"], cache["free_top"], self.status)
-        self.ws_com = torch.empty(isd.commit_workspace_bytes(self._com),
+        self.ws_com = torch.zeros(isd.commit_workspace_bytes(self._com),
                                   dtype=torch.uint8, device=dev)
         self._com.workspace = ctypes.c_void_p(self.ws_com.data_ptr())
         self._com.workspace_bytes = self.ws_com.numel()
@@ -94,12 +94,8 @@ class Decoder:
 
     @property
     def state(self):
-        """Decoding state entering the next step."""
-        return self.states[self.cur]
-
-    @property
-    def next_state(self):
-        """State written by the last step."""
+        """Decoding state the next step reads; after a step, the state that
+        step wrote (the ping-pong pair has already been swapped)."""
         return self.states[self.cur]
 
     def attention(self, stream=None):
@@ -174,6 +170,22 @@ class Decoder:
         self.graphs[self.cur].replay()
         self.advance()
 
-    # Kernel launches per step: attention + combine, three accept kernels
-    # (stats, decide, draw), commit plan + copy.
-    LAUNCHES_PER_STEP = 7
+    def set_step(self, cur, step_idx):
+        """Rewind (or move) the decoder to ping-pong parity ``cur`` and
+        step index ``step_idx``, the device step counter included."""
+        self.cur = int(cur)
+        self.step_idx = int(step_idx)
+        if getattr(self, "graphs", None):
+            self.step_dev.fill_(self.step_idx)
+
+    def release_graphs(self):
+        """Drop the captured graphs (before the buffers they use)."""
+        self.graphs = []
+
+    @property
+    def launches_per_step(self):
+        """This library's kernel launches per step: attention (bf16: the
+        tcgen05 kernel and the split-segment combine; fp32: one kernel),
+        the three accept kernels (statistics, decide, draws) and the
+        commit."""
+        return (2 if self.w.dtype == "bf16" else 1) + 3 + 1

@@ -359,7 +359,8 @@ def kv_commit(k_new, v_new, k_cache, v_cache, page_table, seq_len, n_commit,
     a = commit_args(k_new, v_new, k_cache, v_cache, page_table, seq_len,
                     n_commit, free_stack, free_top, status, workspace)
     if workspace is None:
-        workspace = torch.empty(commit_workspace_bytes(a), dtype=torch.uint8,
+        # The commit workspace is a counter that must start at zero.
+        workspace = torch.zeros(commit_workspace_bytes(a), dtype=torch.uint8,
                                 device=k_new.device)
         a.workspace = _ptr(workspace)
         a.workspace_bytes = workspace.numel()

@@ -17,6 +17,12 @@ t at step s carries the same row plus sigma_q * G'(seed, b, t, s).  The
 expected acceptance of a draft is then sum_v min(p_v, q_v); sigma_q is
 chosen per target acceptance from ``DRAFT_SIGMA_Q`` (values found by the
 calibration script ``tests/golden/calibrate_draft_noise.py``).
+
+Peaked rows.  A trained model's rows put most of their mass on a few
+tokens.  With ``peak`` > 0 every row of (b, t) adds ``peak`` to the logit
+of one keyed token, shared by the clean row and the MASK rows of that
+position, so p and q concentrate on the same token (peak = 18.6 gives that
+token about 0.9 of the mass at sigma_p = 3 and V = 151 936).
 """
 
 import math
@@ -60,6 +66,7 @@ class Workload:
     shuffle_pages: bool = True
     steps: int = 1
     spare_pages: int = 0         # extra free pages beyond growth over steps
+    peak: float = 0.0            # logit boost of one keyed token per row
     meta: dict = field(default_factory=dict, compare=False)
 
     @property
@@ -149,11 +156,18 @@ def keyed_normal(keys, V, device, chunk_rows=64):
     return out
 
 
-def logits_rows(seed, b, pos, mask_step, V, sigma_p, sigma_q, device):
+def peak_token(seed, b, pos, V):
+    """The keyed token a peaked row of (b, pos) boosts."""
+    return _row_keys(seed ^ 0x2545F491, b, pos, 7) % V
+
+
+def logits_rows(seed, b, pos, mask_step, V, sigma_p, sigma_q, device,
+                peak=0.0):
     """Logits rows for (sequence b, absolute position pos) pairs.
 
     ``mask_step`` is -1 for a clean (verify) row and the step index for a
-    MASK (draft) row.  Returns float32 [R][V].
+    MASK (draft) row.  ``peak`` is added to the logit of ``peak_token``.
+    Returns float32 [R][V].
     """
     b = torch.as_tensor(b, device=device).reshape(-1).to(torch.int64)
     pos = torch.as_tensor(pos, device=device).reshape(-1).to(torch.int64)
@@ -167,6 +181,9 @@ def logits_rows(seed, b, pos, mask_step, V, sigma_p, sigma_q, device):
             _row_keys(seed ^ 0x7F4A7C15, b[idx], pos[idx], ms[idx] + 1),
             V, device)
         base[idx] += sigma_q * noise
+    if peak != 0.0:
+        tok = peak_token(seed, b, pos, V)
+        base[torch.arange(base.shape[0], device=device), tok] += peak
     return base
 
 
@@ -186,7 +203,7 @@ def step_logits(w, seed, seq_len, n_pending, step, device, dtype=None):
     ms = torch.where(r[None, :] >= n[:, None],
                      torch.full_like(pos, int(step)), torch.full_like(pos, -1))
     rows = logits_rows(seed, bb.reshape(-1), pos.reshape(-1), ms.reshape(-1),
-                       V, w.sigma_p, draft_sigma(w), device)
+                       V, w.sigma_p, draft_sigma(w), device, peak=w.peak)
     return rows.reshape(B, K, V).to(dtype)
 
 

@@ -67,7 +67,8 @@ is freed.  The new exact token's KV is produced by the next step's row 0.
 import numpy as np
 
 from . import philox
-from .vocab import TIE_BAND, inverse_cdf, prob_of, probs, row_stats
+from .vocab import (TIE_BAND, inverse_cdf, log_normaliser, prob_of, probs,
+                    row_stats, tie_alternatives)
 
 STATUS_OK = "ok"
 STATUS_POOL_EXHAUSTED = "pool_exhausted"
@@ -76,7 +77,7 @@ STATUS_PAGE_TABLE_FULL = "page_table_full"
 
 def accept_resample(logits_cur, logits_prev, pending, n_pending, q_row,
                     seq_len, seed, step, N, tie_band=TIE_BAND,
-                    proposal="sample"):
+                    proposal="sample", flip=()):
     """One accept / resample / bonus / draft step for every sequence.
 
     logits_cur  [B][K][V]  this forward pass's logits (fp64 copy)
@@ -86,10 +87,18 @@ def accept_resample(logits_cur, logits_prev, pending, n_pending, q_row,
     q_row       int [B][N] row of logits_prev that drafted pending[b][i]
     seq_len     int [B]    committed length L_b
     proposal    "sample" (drafts drawn from q) or "argmax" (x = argmax q)
+    flip        (b, i) pairs whose ratio test is decided the other way: the
+                alternative branch of a near-tie ratio test, which a checker
+                may need because two roundings can legitimately decide it
+                either way
 
-    Returns a dict of numpy arrays (padding -1 / NaN) and ``ties``, a list
-    of (b, kind, index) naming every near-tie decision.
+    Returns a dict of numpy arrays (padding -1 / NaN), ``ties``, a list of
+    (b, kind, index) naming every near-tie decision, and ``tie_alts``,
+    mapping (b, slot of next_pending) of every near-tie draw to the sorted
+    tokens it may legitimately yield.  ``next_q_logz`` holds the natural-log
+    normaliser ln sum_v exp(l_v) of each next draft's q row.
     """
+    flip = set(flip)
     if proposal not in ("sample", "argmax"):
         raise ValueError(proposal)
     argmax = proposal == "argmax"
@@ -102,12 +111,13 @@ def accept_resample(logits_cur, logits_prev, pending, n_pending, q_row,
         "next_pending": np.full((B, N), -1, dtype=np.int64),
         "next_n": np.zeros(B, dtype=np.int64),
         "next_q_row": np.full((B, N), -1, dtype=np.int64),
-        "next_q_stats": np.full((B, N, 2), np.nan),
+        "next_q_logz": np.full((B, N), np.nan),
         "ratio": np.full((B, N), np.nan),
         "u_accept": np.full((B, N), np.nan),
         "exact_token": np.full(B, -1, dtype=np.int64),
     }
     ties = []
+    tie_alts = {}
     for b in range(B):
         n = int(n_pending[b])
         L = int(seq_len[b])
@@ -131,7 +141,7 @@ def accept_resample(logits_cur, logits_prev, pending, n_pending, q_row,
             out["u_accept"][b, i] = u
             if abs(u - r) < tie_band:
                 ties.append((b, "accept", i))
-            if u < r:
+            if (u < r) != ((b, i) in flip):
                 a += 1
             else:
                 rejected = True
@@ -155,6 +165,7 @@ def accept_resample(logits_cur, logits_prev, pending, n_pending, q_row,
             tok, near = inverse_cdf(w, u, tie_band)
             if near:
                 ties.append((b, "resample", 0))
+                tie_alts[(b, 0)] = tie_alternatives(w, u, tie_band)
             out["next_pending"][b, 0] = tok
             out["next_n"][b] = 1
             out["exact_token"][b] = tok
@@ -163,6 +174,8 @@ def accept_resample(logits_cur, logits_prev, pending, n_pending, q_row,
             tok, near = inverse_cdf(probs(lc[n - 1]), u, tie_band)
             if near:
                 ties.append((b, "bonus", 0))
+                tie_alts[(b, 0)] = tie_alternatives(probs(lc[n - 1]), u,
+                                                    tie_band)
             out["next_pending"][b, 0] = tok
             out["exact_token"][b] = tok
             for j in range(1, N):
@@ -175,11 +188,14 @@ def accept_resample(logits_cur, logits_prev, pending, n_pending, q_row,
                     xj, near = inverse_cdf(probs(lc[row]), u, tie_band)
                     if near:
                         ties.append((b, "draft", j))
+                        tie_alts[(b, j)] = tie_alternatives(probs(lc[row]),
+                                                            u, tie_band)
                 out["next_pending"][b, j] = xj
                 out["next_q_row"][b, j] = row
-                out["next_q_stats"][b, j] = row_stats(lc[row])
+                out["next_q_logz"][b, j] = log_normaliser(lc[row])
             out["next_n"][b] = N
     out["ties"] = ties
+    out["tie_alts"] = tie_alts
     return out
 
 

@@ -16,7 +16,9 @@ Readings for the sampler (the pages print no sampler):
   index with positive mass is returned;
 * a draw is a near-tie when u * sum(w) lies within ``tie_band * sum(w)``
   of either end of the chosen index's interval; fp32 and fp64 may then
-  legitimately choose neighbouring indices.
+  legitimately choose neighbouring indices: the positive-mass index on the
+  other side of each boundary the target is that close to
+  (``tie_alternatives``).
 """
 
 import numpy as np
@@ -65,3 +67,30 @@ def inverse_cdf(mass, u, tie_band=TIE_BAND):
     if v > 0:
         near = near or (t - float(c[v - 1])) < band
     return v, bool(near)
+
+
+def tie_alternatives(mass, u, tie_band=TIE_BAND):
+    """Every index a near-tie draw may legitimately return.
+
+    The target is t = u * sum(w); a draw whose running sums carry an error
+    below ``tie_band * sum(w)`` may land anywhere within that distance of
+    t.  Returned: every positive-mass index whose interval
+    [c[v - 1], c[v]) meets (t - band, t + band) -- the draw's own index and,
+    across each boundary that close, as many neighbours as lie in the band
+    (tiny masses can put several there).  Sorted.
+    """
+    w = np.asarray(mass, dtype=np.float64)
+    c = np.cumsum(w)
+    total = float(c[-1])
+    t = u * total
+    band = tie_band * total
+    v, _ = inverse_cdf(w, u, tie_band)
+    lo = np.concatenate([[0.0], c[:-1]])
+    hit = (w > 0) & (lo < t + band) & (c > t - band)
+    return sorted(set(np.nonzero(hit)[0].tolist()) | {v})
+
+
+def log_normaliser(logits):
+    """ln sum_v exp(l_v) = m + ln s (the log-partition function of a row)."""
+    m, s = row_stats(logits)
+    return m + float(np.log(s))

@@ -77,6 +77,14 @@ def oracle_attention_pairs(w, cache, q, k, v, pairs, page_table, seq_len):
 
 
 # ------------------------------------------------------------------ accept
+def q_pair(logz):
+    """The q_stats layout of a log-normaliser: fp32 hi and the fp32 rest."""
+    logz = np.nan_to_num(np.asarray(logz, dtype=np.float64))
+    hi = logz.astype(np.float32)
+    lo = (logz - hi.astype(np.float64)).astype(np.float32)
+    return np.stack([hi, lo], axis=-1)
+
+
 def gpu_state_from(ostate, device):
     return dict(
         pending=torch.as_tensor(ostate["pending"], dtype=torch.int32,
@@ -85,15 +93,20 @@ def gpu_state_from(ostate, device):
                                   device=device).contiguous(),
         q_row=torch.as_tensor(ostate["q_row"], dtype=torch.int32,
                               device=device).contiguous(),
-        q_stats=torch.as_tensor(np.nan_to_num(ostate["q_stats"]),
+        q_stats=torch.as_tensor(q_pair(ostate["q_logz"]),
                                 dtype=torch.float32, device=device)
         .contiguous())
 
 
 def oracle_initial_state(st):
+    B, N = st["pending"].shape
     return dict(pending=i64(st["pending"]), n_pending=i64(st["n_pending"]),
-                q_row=i64(st["q_row"]),
-                q_stats=st["q_stats"].detach().cpu().double().numpy())
+                q_row=i64(st["q_row"]), q_logz=np.full((B, N), np.nan))
+
+
+def next_oracle_state(ref):
+    return dict(pending=ref["next_pending"], n_pending=ref["next_n"],
+                q_row=ref["next_q_row"], q_logz=ref["next_q_logz"])
 
 
 class AcceptStep:
@@ -121,59 +134,123 @@ def gpu_accept(lc, lp, seq_len, state_in, seed, step, proposal=None):
     return o
 
 
-def compare_accept(o, ref, n_in, rows_cur_f64, tol_rel=1e-5):
-    """Compare GPU accept outputs with the oracle's.
+class _Host:
+    """Host copies of a GPU accept step's outputs."""
 
-    Near-ties (``ref["ties"]``) are handled per decision: a near-tie in a
-    ratio test leaves that sequence checked for validity only; a near-tie in
-    a draw leaves only that drawn token checked for validity.  Everything
-    else must match exactly (statistics and ratios within ``tol_rel``).
-    Returns counters: decisions compared exactly, near-ties, and near-ties
-    on which the GPU chose differently.
+    def __init__(self, o):
+        self.nc = i64(o.n_commit)
+        self.ct = i64(o.commit_tokens)
+        self.pend = i64(o.state_out["pending"])
+        self.n_out = i64(o.state_out["n_pending"])
+        self.qr = i64(o.state_out["q_row"])
+        qs = o.state_out["q_stats"].cpu().double().numpy()
+        self.logz = qs[..., 0] + qs[..., 1]
+        self.rs = o.row_stats.cpu().double().numpy()
+        self.ratio = o.ratio.cpu().double().numpy()
+
+
+def _branch_mismatch(g, r, b, N, tol_rel):
+    """Why sequence b of the GPU outputs ``g`` differs from oracle branch
+    ``r`` (None when it matches).  Draws that are near-ties in that branch
+    must land on one of their legitimate tokens; everything else is exact
+    (log-normalisers and ratios within ``tol_rel``)."""
+    if g.nc[b] != r["n_commit"][b]:
+        return f"n_commit {g.nc[b]} != {r['n_commit'][b]}"
+    if not np.array_equal(g.ct[b], r["commit_tokens"][b]):
+        return "commit_tokens"
+    if g.n_out[b] != r["next_n"][b]:
+        return "next n"
+    if not np.array_equal(g.qr[b], r["next_q_row"][b]):
+        return "next q rows"
+    for j in range(N):
+        alts = r["tie_alts"].get((b, j))
+        if alts is not None:
+            if g.pend[b, j] not in alts:
+                return f"tie draw slot {j}: {g.pend[b, j]} not in {alts}"
+        elif g.pend[b, j] != r["next_pending"][b, j]:
+            return f"pending slot {j}: {g.pend[b, j]} != " \
+                   f"{r['next_pending'][b, j]}"
+    for j in range(1, N):
+        if r["next_q_row"][b, j] >= 0:
+            if abs(g.logz[b, j] - r["next_q_logz"][b, j]) > tol_rel:
+                return f"q log-normaliser slot {j}"
+    for i in range(1, N):
+        if not np.isnan(r["ratio"][b, i]):
+            if abs(g.ratio[b, i] - r["ratio"][b, i]) > \
+                    tol_rel * r["ratio"][b, i]:
+                return f"ratio of draft {i}"
+    return None
+
+
+def compare_accept(o, ref, n_in, rows_cur_f64, rerun, pending_in,
+                   tol_rel=1e-5):
+    """Compare GPU accept outputs with the oracle's, decision by decision.
+
+    ``rerun(flip)`` re-runs the oracle on the same inputs with the ratio
+    tests named in ``flip`` decided the other way; ``pending_in`` is the
+    step's input pending tokens.
+
+    * A sequence without a ratio-test near-tie must match the oracle
+      exactly, except draws that are near-ties, whose token must be one of
+      the oracle's legitimate alternatives (the oracle's index or the
+      positive-mass index across the tied boundary).
+    * A sequence with a ratio-test near-tie must match exactly one branch
+      of the oracle (the tied tests decided either way, every combination),
+      with the same draw allowance; and the GPU's own decisions must agree
+      with the ratios it reports (accepted drafts have u <= ratio, a
+      rejected one u >= ratio).
+
+    Returns counters: sequence-steps compared exactly, near-ties, and
+    near-ties on which the GPU chose differently from the oracle's primary
+    branch.
     """
     B, N = ref["next_pending"].shape
-    accept_tie = {b for b, kind, _ in ref["ties"] if kind == "accept"}
-    slot_tie = {(b, 0 if kind in ("bonus", "resample") else j)
-                for b, kind, j in ref["ties"] if kind != "accept"}
-    nc = i64(o.n_commit)
-    ct = i64(o.commit_tokens)
-    pend = i64(o.state_out["pending"])
-    n_out = i64(o.state_out["n_pending"])
-    qr = i64(o.state_out["q_row"])
-    qs = o.state_out["q_stats"].cpu().double().numpy()
-    rs = o.row_stats.cpu().double().numpy()
-    ratio = o.ratio.cpu().double().numpy()
+    g = _Host(o)
+    accept_ties = {}
+    for b, kind, i in ref["ties"]:
+        if kind == "accept":
+            accept_ties.setdefault(b, []).append(i)
     out = dict(exact=0, ties=len(ref["ties"]), tie_differs=0)
+    branches = {}
     for b in range(B):
         n = int(n_in[b])
         for r in range(n + N - 1):
             m_ref, s_ref = row_stats(rows_cur_f64(b, r))
-            assert rs[b, r, 0] == m_ref, (b, r)
-            assert abs(rs[b, r, 1] - s_ref) <= tol_rel * s_ref, (b, r)
-        if b in accept_tie:
-            assert 1 <= nc[b] <= n
-            if nc[b] != ref["n_commit"][b]:
-                out["tie_differs"] += 1
-            continue
-        for i in range(1, n):
-            if not np.isnan(ref["ratio"][b, i]):
-                assert abs(ratio[b, i] - ref["ratio"][b, i]) <= \
-                    tol_rel * ref["ratio"][b, i], (b, i)
-        assert nc[b] == ref["n_commit"][b], b
-        assert np.array_equal(ct[b], ref["commit_tokens"][b]), b
-        assert n_out[b] == ref["next_n"][b], b
-        assert np.array_equal(qr[b], ref["next_q_row"][b]), b
-        for j in range(N):
-            if (b, j) in slot_tie:
-                assert ref["next_pending"][b, j] < 0 or pend[b, j] >= 0
-                if pend[b, j] != ref["next_pending"][b, j]:
+            assert g.rs[b, r, 0] == m_ref, (b, r)
+            assert abs(g.rs[b, r, 1] - s_ref) <= tol_rel * s_ref, (b, r)
+        # The committed tokens are the step's own pending prefix.
+        nc = int(g.nc[b])
+        assert 1 <= nc <= n, (b, nc)
+        assert np.array_equal(g.ct[b, :nc], pending_in[b, :nc]), b
+        assert (g.ct[b, nc:] == -1).all(), b
+        if b not in accept_ties:
+            why = _branch_mismatch(g, ref, b, N, tol_rel)
+            assert why is None, (b, why)
+            for j in range(N):
+                if (b, j) in ref["tie_alts"] and \
+                        g.pend[b, j] != ref["next_pending"][b, j]:
                     out["tie_differs"] += 1
-                continue
-            assert pend[b, j] == ref["next_pending"][b, j], (b, j)
-        for j in range(1, N):
-            if ref["next_q_row"][b, j] >= 0:
-                assert qs[b, j, 0] == ref["next_q_stats"][b, j, 0]
-                assert abs(qs[b, j, 1] - ref["next_q_stats"][b, j, 1]) <= \
-                    tol_rel * ref["next_q_stats"][b, j, 1]
-        out["exact"] += 1
+            out["exact"] += 1
+            continue
+        # Ratio-test near-tie: one of the oracle's branches.
+        tied = accept_ties[b]
+        matched = None
+        whys = []
+        for mask in range(1 << len(tied)):
+            flip = frozenset((b, tied[k]) for k in range(len(tied))
+                             if mask >> k & 1)
+            if flip not in branches:
+                branches[flip] = ref if not flip else rerun(flip)
+            why = _branch_mismatch(g, branches[flip], b, N, tol_rel)
+            if why is None:
+                matched = branches[flip]
+                break
+            whys.append(why)
+        assert matched is not None, (b, whys)
+        for i in range(1, nc):
+            assert matched["u_accept"][b, i] <= g.ratio[b, i], (b, i)
+        if nc < n:
+            assert matched["u_accept"][b, nc] >= g.ratio[b, nc], (b, nc)
+        if matched is not ref:
+            out["tie_differs"] += 1
     return out

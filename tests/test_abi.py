@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert isd.abi_version() == 2
+    assert isd.abi_version() == 3
     assert isd.status_string(isd.ERR_POOL_EXHAUSTED) == "KV page pool exhausted"
     assert isd.status_string(12345) == "unknown status"
 
@@ -67,8 +67,8 @@ def _attn_args(**kw):
     (dict(softmax_scale=0.0), isd.ERR_INVALID_ARG),
     (dict(num_ctas=-1), isd.ERR_INVALID_ARG),
     (dict(num_ctas=1025), isd.ERR_INVALID_ARG),     # at most 1024 CTAs
-    (dict(d=96), isd.ERR_UNSUPPORTED),              # bf16 path: d 64 or 128
-    (dict(K=6, d=64), isd.ERR_UNSUPPORTED),         # d 64: K*g = 24 rows
+    (dict(d=96), isd.ERR_UNSUPPORTED),              # bf16 path: d 128
+    (dict(d=64), isd.ERR_UNSUPPORTED),
     (dict(K=16, Hq=96, Hkv=8), isd.ERR_UNSUPPORTED),  # K*g = 192 rows
     (dict(K=32, Hq=8), isd.ERR_UNSUPPORTED),        # K above a page
     (dict(dtype=7), isd.ERR_INVALID_ARG),
@@ -118,6 +118,55 @@ def test_commit_host_validation(lib):
     assert lib.isd_kv_commit(ctypes.byref(a), None) == isd.ERR_INVALID_ARG
     a.d = 4                                          # 8-byte rows
     assert lib.isd_kv_commit(ctypes.byref(a), None) == isd.ERR_UNSUPPORTED
+    a.d = 128
+    a.B = 32769                                      # above 1024 CTAs x 32
+    assert lib.isd_kv_commit(ctypes.byref(a), None) == isd.ERR_UNSUPPORTED
+    assert lib.isd_commit_workspace_bytes(ctypes.byref(a)) == 0
+
+
+def _fake_accept_args(**kw):
+    """Accept arguments whose pointers are distinct, aligned and never
+    dereferenced (every call below is refused on the host)."""
+    ptr = iter(range(0x100000, 0x100000 + 0x10000 * 40, 0x10000))
+    fields = dict(logits_cur=None, logits_prev=None, seq_len=None,
+                  pending_in=None, n_pending_in=None, q_row_in=None,
+                  q_stats_in=None, pending_out=None, n_pending_out=None,
+                  q_row_out=None, q_stats_out=None, n_commit=None,
+                  commit_tokens=None)
+    for k in fields:
+        fields[k] = ctypes.c_void_p(next(ptr))
+    fields.update(kw)
+    return isd.AcceptArgs(**fields)
+
+
+def test_static_scratch_rejects_problems_above_its_limit(lib):
+    """The allocation-free accept entry point refuses, before any CUDA call,
+    a problem whose scratch would exceed its fixed buffer."""
+    a = _fake_accept_args(B=8192, N=16, K=32, V=151936, dtype=isd.BF16)
+    assert lib.isd_accept_workspace_bytes(ctypes.byref(a)) > \
+        isd.ACCEPT_STATIC_SCRATCH
+    assert lib.isd_accept_resample_static(ctypes.byref(a), None) == \
+        isd.ERR_WORKSPACE
+
+
+def test_static_scratch_checks_arguments_like_the_workspace_call(lib):
+    """Both accept entry points report the same error for the same bad
+    arguments, argument errors before the size limit."""
+    cases = [
+        dict(B=8192, N=16, K=32, V=151936, dtype=isd.BF16,
+             logits_cur=None),                       # null and oversized
+        dict(B=4, N=1, K=2, V=64, dtype=isd.BF16),   # N < 2
+        dict(B=4, N=4, K=8, V=64, dtype=isd.BF16, proposal=5),
+    ]
+    for kw in cases:
+        a = _fake_accept_args(**kw)
+        want = lib.isd_accept_resample(ctypes.byref(a), None)
+        assert want == isd.ERR_INVALID_ARG
+        assert lib.isd_accept_resample_static(ctypes.byref(a), None) == want
+    a = _fake_accept_args(B=8192, N=16, K=32, V=151936, dtype=isd.BF16)
+    a.q_stats_out = a.q_stats_in                     # in-place state
+    assert lib.isd_accept_resample_static(ctypes.byref(a), None) == \
+        isd.ERR_INVALID_ARG
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -73,7 +73,7 @@ def test_reference_arm_two_ranks():
            "--nproc-per-node", "2", "--master-addr", "127.0.0.1",
            "--master-port", str(port), os.path.join(ROOT, "bench.py"),
            "--impl", "reference", "--gpus", "2", "--steps", "1",
-           "--warmup", "0", "--cpu-sample-seqs", "1"]
+           "--warmup", "0", "--cpu-sample-seqs", "2"]
     r = subprocess.run(cmd, capture_output=True, text=True, timeout=600,
                        cwd=ROOT)
     assert r.returncode == 0, r.stderr[-2000:]

@@ -32,9 +32,7 @@ SMALL = [
     synth.TINY,                                              # fp32, d 64
     synth.TINY.with_(name="tiny_ragged", B=3, Hq=8, Hkv=2, L_lo=0, L_hi=70,
                      shuffle_pages=True),
-    _bf(name="bf16_m16_d64", Hq=8, Hkv=2, d=64, N=2, L_lo=1, L_hi=90),
     _bf(name="bf16_m32", L_lo=0, L_hi=100),
-    _bf(name="bf16_m32_d64", d=64, L_lo=5, L_hi=200),
     _bf(name="bf16_m16", N=2, L_lo=15, L_hi=130),
     _bf(name="bf16_m64", B=2, Hq=16, Hkv=2, L_lo=17, L_hi=260),
     _bf(name="bf16_m128", B=2, Hq=16, Hkv=2, N=8, L_lo=1, L_hi=300),

@@ -23,7 +23,7 @@ from oracle import attention as oattn
 from oracle import step as ostep
 from oracle import tpf
 from tests.gpu_util import (TOL, compare_accept, f32, f64, gpu_state_from, i64,
-                            oracle_initial_state)
+                            next_oracle_state, oracle_initial_state)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -107,11 +107,15 @@ def test_c64_stationary_lockstep_100_steps():
         dec.accept()
         torch.cuda.synchronize()
         lc_host = f32(lc)
-        ref = ostep.accept_resample(lc_host, lp_host, ostate["pending"],
-                                    ostate["n_pending"], ostate["q_row"], L,
-                                    seed, s, w.N)
+        def oracle(flip=(), lc_host=lc_host, lp_host=lp_host,
+                   ostate=ostate, L=L, s=s):
+            return ostep.accept_resample(lc_host, lp_host, ostate["pending"],
+                                         ostate["n_pending"], ostate["q_row"],
+                                         L, seed, s, w.N, flip=flip)
+        ref = oracle()
         c = compare_accept(_View(dec), ref, ostate["n_pending"],
-                           lambda b, r: lc_host[b, r].astype(np.float64))
+                           lambda b, r: lc_host[b, r].astype(np.float64),
+                           oracle, ostate["pending"])
         compared += c["exact"]
         ties += c["ties"]
         differs += c["tie_differs"]
@@ -146,8 +150,7 @@ def test_c64_stationary_lockstep_100_steps():
             logical[b][1] = np.concatenate([logical[b][1],
                                             vh_host[b, :nc[b]]])
         dec.advance()
-        ostate = dict(pending=ref["next_pending"], n_pending=ref["next_n"],
-                      q_row=ref["next_q_row"], q_stats=ref["next_q_stats"])
+        ostate = next_oracle_state(ref)
         L = L_new
         lp_host = lc_host
     print(f"lockstep: {compared} sequence-steps exact, {ties} near-ties, "

@@ -29,7 +29,7 @@ def _run(w, seed, steps, graphs):
             dec.replay()
         else:
             dec.step()
-        hist.append((dec.n_commit.clone(), dec.next_state["pending"].clone(),
+        hist.append((dec.n_commit.clone(), dec.state["pending"].clone(),
                      dec.out.clone()))
     torch.cuda.synchronize()
     assert int(dec.status.item()) == isd.OK

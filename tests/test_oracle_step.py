@@ -238,3 +238,66 @@ def test_commit_page_table_full():
     res = ostep.kv_commit(kn, vn, kc, vc, pt, L, nc, fs, top)
     assert res[5] == ostep.STATUS_PAGE_TABLE_FULL
     assert np.array_equal(res[3], L)
+
+
+def test_flip_takes_the_other_branch_of_a_ratio_test():
+    """flip decides one ratio test the other way and everything after it
+    follows that decision: flipping the first rejection accepts that draft
+    (and goes on testing), flipping an accepted draft rejects there."""
+    rng = np.random.default_rng(11)
+    V, B, N = 12, 400, 4
+    K = 2 * N
+    lc0 = rng.normal(0.0, 1.0, (B, K, V))
+    pending = np.full((B, N), -1)
+    pending[:, 0] = rng.integers(0, V, B)
+    L0 = np.full(B, 40)
+    s0 = ostep.accept_resample(lc0, lc0, pending, np.ones(B, dtype=np.int64),
+                               np.full((B, N), -1), L0, 3, 0, N)
+    lc1 = rng.normal(0.0, 1.0, (B, K, V))
+    L1 = L0 + s0["n_commit"]
+    args = (lc1, lc0, s0["next_pending"], s0["next_n"], s0["next_q_row"], L1,
+            3, 1, N)
+    base = ostep.accept_resample(*args)
+    flips = []
+    for b in range(B):
+        a = int(base["accepted"][b])
+        if base["rejected"][b]:
+            flips.append((b, a + 1, "to_accept"))
+        elif a >= 1:
+            flips.append((b, a, "to_reject"))
+    assert len(flips) > 50
+    alt = ostep.accept_resample(*args, flip=[(b, i) for b, i, _ in flips])
+    for b, i, kind in flips:
+        if kind == "to_accept":
+            assert alt["accepted"][b] >= i           # draft i now passes
+            assert alt["n_commit"][b] >= i + 1
+        else:
+            assert alt["rejected"][b] and alt["accepted"][b] == i - 1
+            assert alt["n_commit"][b] == i
+            # Decided the same way before the flipped test: same prefix.
+            assert np.array_equal(alt["commit_tokens"][b, :i],
+                                  base["commit_tokens"][b, :i])
+    # Untouched sequences are unchanged.
+    touched = {b for b, _, _ in flips}
+    for b in range(B):
+        if b not in touched:
+            assert alt["n_commit"][b] == base["n_commit"][b]
+            assert np.array_equal(alt["next_pending"][b],
+                                  base["next_pending"][b])
+
+
+def test_next_q_logz_is_the_draft_rows_logsumexp():
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(12)
+    V, B, N = 50, 20, 3
+    lc = rng.normal(0.0, 2.0, (B, 2 * N, V))
+    pending = np.full((B, N), -1)
+    pending[:, 0] = 1
+    o = ostep.accept_resample(lc, lc, pending, np.ones(B, dtype=np.int64),
+                              np.full((B, N), -1), np.full(B, 5), 0, 0, N)
+    for b in range(B):
+        for j in range(1, N):
+            row = int(o["next_q_row"][b, j])
+            assert row == j                       # R mode: n = 1
+            assert o["next_q_logz"][b, j] == pytest.approx(
+                logsumexp(lc[b, row]), rel=1e-14)

@@ -71,3 +71,66 @@ def test_empirical_distribution():
     draws = np.array([vocab.inverse_cdf(w, x)[0] for x in u[:40000]])
     freq = np.bincount(draws, minlength=5) / draws.size
     np.testing.assert_allclose(freq, w, atol=0.01)
+
+
+def test_tie_alternatives_cross_only_the_near_boundary():
+    # Masses 0.25 each with a zero entry between indices 1 and 3: the
+    # positive-mass neighbour across the boundary at 0.5 is 3, not 2.
+    w = np.array([0.25, 0.25, 0.0, 0.25, 0.25])
+    total = w.sum()
+    # Just below the boundary c[1] = 0.5: the draw is 1, the other side 3.
+    u = (0.5 - 3e-7) / total
+    assert vocab.inverse_cdf(w, u) == (1, True)
+    assert vocab.tie_alternatives(w, u) == [1, 3]
+    # Just above it: the draw is 3, the other side 1.
+    u = (0.5 + 3e-7) / total
+    assert vocab.inverse_cdf(w, u) == (3, True)
+    assert vocab.tie_alternatives(w, u) == [1, 3]
+    # Far from every boundary: the draw alone.
+    assert vocab.tie_alternatives(w, 0.6) == [vocab.inverse_cdf(w, 0.6)[0]]
+    # The first boundary has nothing before index 0.
+    assert vocab.tie_alternatives(w, 1e-9) == [0]
+
+
+def test_tie_alternatives_brute_force():
+    # The alternatives are exactly the draws an inverse CDF makes for every
+    # target within the band, on small vectors with clusters of tiny masses.
+    rng = np.random.default_rng(4)
+    band = 1e-6
+    for _ in range(300):
+        V = int(rng.integers(2, 10))
+        w = rng.random(V)
+        w[rng.random(V) < 0.3] = 0.0
+        tiny = rng.random(V) < 0.3
+        w[tiny] *= 1e-8                     # intervals narrower than the band
+        if w.sum() == 0:
+            w[0] = 1.0
+        c = np.cumsum(w)
+        k = int(rng.integers(0, V))
+        u = float(np.clip((c[k] + rng.uniform(-5e-7, 5e-7) * c[-1]) / c[-1],
+                          0.0, 1.0 - 2.0 ** -24))
+        alts = vocab.tie_alternatives(w, u, band)
+        # Targets across the band: a dense grid plus both sides of every
+        # running-sum boundary inside it (intervals far narrower than any
+        # grid step are still visited).
+        total = c[-1]
+        xs = list(u + np.linspace(-band, band, 401)[1:-1])
+        for cj in c:
+            for x in (cj / total * (1 - 1e-15), cj / total * (1 + 1e-15)):
+                if abs(x - u) < band:
+                    xs.append(x)
+        seen = {vocab.inverse_cdf(w, u)[0]}
+        for x in xs:
+            if 0.0 <= x < 1.0:
+                seen.add(vocab.inverse_cdf(w, float(x))[0])
+        assert set(alts) == seen, (w, u, alts, seen)
+        assert all(w[a] > 0 for a in alts)
+
+
+def test_log_normaliser_is_logsumexp():
+    rng = np.random.default_rng(5)
+    for V in (1, 9, 151936):
+        x = rng.normal(0.0, 3.0, V)
+        x[int(rng.integers(V))] += 18.6
+        assert vocab.log_normaliser(x) == pytest.approx(logsumexp(x),
+                                                        rel=1e-14)

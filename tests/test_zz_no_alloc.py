@@ -11,8 +11,6 @@ of isd_accept_resample with a caller workspace.  The file sorts last so a
 run that stops at the first failure has run every other test first.
 """
 
-import ctypes
-
 import pytest
 import torch
 
@@ -69,12 +67,3 @@ def test_static_scratch_matches_workspace_entry_point():
             assert int((state["n_pending"] == w.N).sum()) > w.B // 2
         state, lp = ref.state_out, lc
         L = L + ref.n_commit
-
-
-def test_static_scratch_rejects_problems_above_its_limit():
-    lib = isd.lib()
-    a = isd.AcceptArgs(B=8192, N=16, K=32, V=151936, dtype=isd.BF16)
-    assert lib.isd_accept_workspace_bytes(ctypes.byref(a)) > \
-        isd.ACCEPT_STATIC_SCRATCH
-    assert lib.isd_accept_resample_static(ctypes.byref(a), None) == \
-        isd.ERR_WORKSPACE
