@@ -9,26 +9,23 @@
 // that rule; the row layout is the stride schedule stated in isd.h.
 //
 // The vocabulary is cut into sub-chunks of 2048 elements, one warp's work
-// (64 elements a lane), so no step needs a block-wide barrier.  Three
-// kernels, one stream, no inter-CTA waiting:
-//   stats   one CTA per SM.  Six producer lanes stream the used rows into
-//           a 12-slot shared-memory ring in 16 KB bulk asynchronous copies
-//           (TMA engine, completion counted on mbarriers); six groups of
-//           four consumer warps take the copies in turn, each warp reducing
-//           one sub-chunk to its max, the first index of that max and the
-//           sum of exp(l - max), in two passes over shared memory.
-//           Rows whose byte length is not a multiple of 16 cannot be bulk
-//           copied and go through a plain-load variant with the same
-//           element order and arithmetic.                         [HBM bound]
-//   decide  one CTA per sequence: warp j merges row j's sub-chunk figures
-//           into the row's (m, s); warp 0 runs the ratio tests, ballots
-//           the first rejection and writes the next state
-//   draw    rejected sequences: one warp per sub-chunk sums max(0, p - q),
-//           and the warp that finishes last (atomic count, no waiting)
-//           draws the replacement; accepted sequences: warp t draws token
-//           t (the bonus, then the drafts).  A draw scans the sub-chunk
-//           masses to pick a sub-chunk, then that sub-chunk's elements,
-//           both in ascending vocabulary order.
+// (64 elements a lane).  Two kernels, one stream, no inter-CTA waiting:
+//   stats  persistent warps stream the used rows sub-chunk by sub-chunk
+//          with 16-byte loads (each lane keeps the next sub-chunk's eight
+//          loads in flight while it reduces the current one) and store each
+//          sub-chunk's max, first index of the max and sum of
+//          exp(l - max).                                        [HBM bound]
+//   draw   grid (sequence, part): every CTA of a sequence merges the
+//          sub-chunk figures of the rows it needs and takes the ratio-test
+//          decision itself (the same inputs and arithmetic in every CTA, so
+//          the same decision); part 0 writes the decision's outputs.  Then
+//          rejected sequences: part y sums max(0, p - q) over sub-chunks
+//          4y .. 4y+3 (two warps each) and the part that finishes last
+//          (atomic count, no waiting) draws the replacement; accepted
+//          sequences: part t draws token t (the bonus, then the drafts).
+//          A draw picks the sub-chunk from a warp scan of the sub-chunk
+//          masses, then scans its 2048 elements with eight warps of 256,
+//          all in ascending vocabulary order.               [latency bound]
 // Element masses are fp32 (MUFU exp2 of exactly formed differences); every
 // sum that places a sampling boundary or normalises a probability is
 // accumulated in fp64 in a fixed order, so draws agree with an fp64
@@ -40,32 +37,16 @@
 
 namespace isd {
 
-constexpr int kSub = 2048;          // vocabulary elements per sub-chunk
-constexpr int kSubPerLane = 4;      // sub-chunks a lane owns in a row scan
+constexpr int kSub = 2048;                 // vocabulary elements per sub-chunk
+constexpr int kSubPerLane = 4;             // sub-chunks a lane owns in a row scan
 constexpr int kMaxSub = 32 * kSubPerLane;  // V <= 262 144 (host check)
-// Stats CTA: a ring of kSlots bulk copies of kCopyBytes (16 KB: 4 bf16 or
-// 2 f32 sub-chunks of a row), filled by kIssuers producer lanes and read by
-// kGroups groups of kGroupWarps consumer warps, warp i of a group taking
-// sub-chunk i of each copy.  kSlots is a multiple of kGroups, so every use
-// of a slot goes to the same group, in order: a warp never waits on a slot
-// whose previous use (another group's) is still pending, which a parity
-// wait could not tell from the use before that.
-constexpr int kCopyBytes = 16 * 1024;
-constexpr int kSlots = 12;
-constexpr int kGroups = 6;
-constexpr int kGroupWarps = 4;
-constexpr int kConsumers = kGroups * kGroupWarps;
-constexpr int kIssuers = 6;
-constexpr uint32_t kIssuerMask = (1u << kIssuers) - 1u;
-constexpr int kStatsThreads = (kConsumers + 1) * 32;  // + producer warp
-static_assert(kStatsThreads <= 1024, "one CTA holds at most 1024 threads");
-static_assert(kSlots % kGroups == 0 && kIssuers <= kSlots, "slot ownership");
-static_assert(kCopyBytes / (kSub * 2) <= kGroupWarps &&
-                  kCopyBytes % (kSub * 4) == 0,
-              "a copy holds whole sub-chunks, at most one per group warp");
-constexpr int kStatsSmem = kSlots * (kCopyBytes + 2 * 8 + 4);
-constexpr int kDrawWarps = 8;
-constexpr uint64_t kAcceptWait = 400000000ull;  // clock cycles, ~0.2 s
+constexpr int kMaxRows = 32;               // K <= 32 (host check: N <= 16)
+constexpr int kStatsWarps = 16;            // stats CTA: 512 threads
+constexpr int kDrawWarps = 8;              // draw CTA: 256 threads
+constexpr int kResidPerCta = 4;            // residual sub-chunks per draw CTA
+constexpr int kWarpElems = kSub / kDrawWarps;   // a draw warp's share: 256
+static_assert(kDrawWarps == 2 * kResidPerCta, "two warps per residual sub-chunk");
+static_assert(kWarpElems == 32 * 8, "a draw lane scans 8 elements");
 
 template <typename T>
 struct AcceptDev {
@@ -93,25 +74,10 @@ struct AcceptDev {
   double* csum;        // [B][RU][C] sub-chunk sum of exp(l - sub-chunk max)
   float* cmax;         // [B][RU][C] sub-chunk max
   int32_t* cidx;       // [B][RU][C] first index of the sub-chunk max
-  double* rsum;        // [B][K] row normaliser s
-  float* rmax;         // [B][K] row max m
   double* resid;       // [B][C] residual sub-chunk mass
-  int32_t* decision;   // [B][4]: valid, rejected, a, n
-  int32_t* count;      // [B] residual sub-chunks finished
+  int32_t* count;      // [B] residual parts finished (zeroed by stats)
   int argmax;          // drafts are argmax q (point-mass proposals)
 };
-
-// Loads elements [idx, idx+8) of a row; out-of-range ones read as -inf.
-template <typename T, bool kVec>
-ISD_DEV void load_row8(const T* row, int idx, int hi, float (&v)[8]) {
-  if (kVec && idx + 8 <= hi) {
-    load8_stream(row + idx, v);
-  } else {
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      v[k] = (idx + k < hi) ? to_f(row[idx + k]) : -INFINITY;
-  }
-}
 
 // Eight consecutive elements kept in their storage format until use
 // (bf16: one 16-byte word, half the registers of eight floats);
@@ -129,6 +95,9 @@ template <> struct Raw8<float> {
   ISD_DEV float at(int e) const { return v[e]; }
 };
 
+// Elements [idx, idx + 8) of a row of `hi` elements.  kVec: the row is
+// 16-byte aligned and holds whole 16-byte units, so one vector load serves
+// when idx + 8 <= hi; otherwise element loads, -inf past the end.
 template <bool kVec>
 ISD_DEV Raw8<__nv_bfloat16> load_raw8(const __nv_bfloat16* row, int idx,
                                       int hi) {
@@ -153,25 +122,17 @@ ISD_DEV Raw8<__nv_bfloat16> load_raw8(const __nv_bfloat16* row, int idx,
 template <bool kVec>
 ISD_DEV Raw8<float> load_raw8(const float* row, int idx, int hi) {
   Raw8<float> r;
-  load_row8<float, kVec>(row, idx, hi, r.v);
-  return r;
-}
-
-// 8 consecutive elements from shared memory (16-byte aligned).
-ISD_DEV void lds8(const __nv_bfloat16* s, float (&v)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4*>(s);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  if (kVec && idx + 8 <= hi) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(row + idx));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(row + idx) + 1);
+    r.v[0] = a.x; r.v[1] = a.y; r.v[2] = a.z; r.v[3] = a.w;
+    r.v[4] = b.x; r.v[5] = b.y; r.v[6] = b.z; r.v[7] = b.w;
+  } else {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = __uint_as_float(w[i] << 16);
-    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    for (int e = 0; e < 8; ++e)
+      r.v[e] = idx + e < hi ? row[idx + e] : -INFINITY;
   }
-}
-ISD_DEV void lds8(const float* s, float (&v)[8]) {
-  const float4 a = *reinterpret_cast<const float4*>(s);
-  const float4 b = *(reinterpret_cast<const float4*>(s) + 1);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  return r;
 }
 
 ISD_DEV double warp_sum_f64(double v) {
@@ -204,26 +165,6 @@ ISD_DEV double warp_scan_f64(double v, double& excl) {
   return x;
 }
 
-// Bounded mbarrier wait: false once ~0.2 s have passed without the phase.
-ISD_DEV bool wait_bounded(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity))
-    if ((uint64_t)(clock64() - t0) > kAcceptWait) return false;
-  return true;
-}
-
-// Bulk asynchronous copy global -> shared (TMA engine), completion counted
-// in bytes on `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.
-ISD_DEV void bulk_load(void* dst, const void* src, uint32_t bytes,
-                       uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
-      "[%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
 template <typename T>
 ISD_DEV uint32_t step_of(const AcceptDev<T>& p) {
   return p.step_dev ? *p.step_dev : p.step;
@@ -236,36 +177,56 @@ ISD_DEV bool state_ok(const AcceptDev<T>& p, int b) {
 }
 
 // ---------------------------------------------------------------------------
-// Sub-chunk figures.  Lane l holds elements lo + (k*32 + l)*8 + e (k, e < 8)
-// of the sub-chunk, -inf past the row end.  Lane 0 stores the max, the sum
-// of exp(l - max) (8 terms in fp32, then fp64) and the first index of the
-// max (exact compares of the same values).
-template <typename T>
-ISD_DEV void finish_sub(const AcceptDev<T>& p, size_t o, int lo,
-                        const float (&v)[8][8]) {
+// Statistics.  Items are the sub-chunks of the used rows, numbered row
+// index first: it = (j * B + b) * C + c (rows j < N are used by every
+// sequence, so warps run out of work together).  Global warp w takes items
+// w, w + W, w + 2W, ... that are in use; lane l holds elements
+// lo + (k*32 + l)*8 + e (k, e < 8) of the sub-chunk, -inf past the row end,
+// and lane 0 stores the max, the sum of exp(l - max) (8 terms in fp32, then
+// fp64) and, for argmax proposals, the first index of the max (exact
+// compares of the same values).
+template <typename T, bool kVec>
+ISD_DEV void load_sub(const AcceptDev<T>& p, int b, int j, int c,
+                      Raw8<T> (&v)[8]) {
   const int lane = threadIdx.x & 31;
-  float m = -INFINITY;
+  const T* row = p.lc + ((size_t)b * p.K + j) * p.V;
+  const int lo = c * kSub;
 #pragma unroll
   for (int k = 0; k < 8; ++k)
+    v[k] = load_raw8<kVec>(row, lo + (k * 32 + lane) * 8, p.V);
+}
+
+template <typename T>
+ISD_DEV void reduce_sub(const AcceptDev<T>& p, int b, int j, int c,
+                        const Raw8<T> (&v)[8]) {
+  const int lane = threadIdx.x & 31;
+  float mk[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) m = fmaxf(m, v[k][e]);
+  for (int k = 0; k < 8; ++k) {
+    mk[k] = fmaxf(fmaxf(fmaxf(v[k].at(0), v[k].at(1)), fmaxf(v[k].at(2), v[k].at(3))),
+                  fmaxf(fmaxf(v[k].at(4), v[k].at(5)), fmaxf(v[k].at(6), v[k].at(7))));
+  }
+  float m = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])),
+                  fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7])));
   m = warp_max(m);
   double s = 0.0;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     float t = 0.0f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) t += ex2((v[k][e] - m) * kLog2e);
+    for (int e = 0; e < 8; ++e) t += ex2((v[k].at(e) - m) * kLog2e);
     s += (double)t;
   }
   s = warp_sum_f64(s);
+  const size_t o = ((size_t)b * p.RU + j) * p.C + c;
   if (p.argmax) {
+    const int lo = c * kSub;
     int first = INT_MAX;
 #pragma unroll
     for (int k = 7; k >= 0; --k)
 #pragma unroll
       for (int e = 7; e >= 0; --e)
-        if (v[k][e] == m) first = lo + (k * 32 + lane) * 8 + e;
+        if (v[k].at(e) == m) first = lo + (k * 32 + lane) * 8 + e;
     first = warp_min_int(first);
     if (lane == 0) p.cidx[o] = first;
   }
@@ -275,319 +236,166 @@ ISD_DEV void finish_sub(const AcceptDev<T>& p, size_t o, int lo,
   }
 }
 
-// Copies are numbered it = (b * RU + j) * CC + cc (chunk cc of row j of
-// sequence b, CC chunks of S sub-chunks per row); sub-chunk c = cc * S + i
-// lands in slot `it`'s i-th kSub elements and its figures at
-// (b * RU + j) * C + c.
-template <typename T>
-__global__ void __launch_bounds__(kStatsThreads, 1)
-    accept_stats_kernel(AcceptDev<T> p) {
-  constexpr int S = kCopyBytes / (kSub * (int)sizeof(T));  // sub-chunks/copy
-  constexpr int kSlotElems = kCopyBytes / (int)sizeof(T);
-  extern __shared__ __align__(128) unsigned char smem[];
-  T* ring = reinterpret_cast<T*>(smem);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kSlots * kCopyBytes);
-  uint64_t* empty = full + kSlots;
-  int* item = reinterpret_cast<int*>(empty + kSlots);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int CC = (p.C + S - 1) / S;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kSlots; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kGroupWarps);
-    }
-    fence_barrier_init();
+// Walks one warp's items it, it + W, it + 2W, ... without divisions:
+// W = (dj * B + db) * C + dc is split once, and (j, b, c) advance by
+// (dj, db, dc) with carries.  `used` gives each sequence's rows in use
+// (0 for a malformed state).
+struct ItemWalk {
+  int B, C, RU, dj, db, dc;
+  int j, b, c;
+  ISD_DEV void init(long long it, long long W, int B_, int C_, int RU_) {
+    B = B_; C = C_; RU = RU_;
+    c = (int)(it % C);
+    const long long jb = it / C;
+    b = (int)(jb % B);
+    j = (int)(jb / B);
+    dc = (int)(W % C);
+    const long long q = W / C;
+    db = (int)(q % B);
+    dj = (int)(q / B);
   }
-  grid_dep_wait();
-  __syncthreads();
+  ISD_DEV void step() {
+    c += dc;
+    int carry = c >= C;
+    c -= carry ? C : 0;
+    b += db + carry;
+    carry = b >= B;
+    b -= carry ? B : 0;
+    j += dj + carry;
+  }
+  // Moves to the next item in use (at or after the current); false when
+  // the items are exhausted.
+  template <typename U>
+  ISD_DEV bool next_used(const U& used) {
+    for (; j < RU; step())
+      if (j < used(b)) return true;
+    return false;
+  }
+};
 
-  if (warp == kConsumers) {
-    // Producers: lanes 0..kIssuers-1 look at kIssuers candidate copies at a
-    // time (this CTA's are blockIdx.x + k * gridDim.x) and each lane whose
-    // copy is of a row in use issues it.  Production q goes to slot
-    // q % kSlots and to consumer group q % kGroups; after the copies comes
-    // one end marker per group.
-    if (lane >= kIssuers) return;
-    const int total = p.B * p.RU * CC;
-    bool failed = false;
-    int q0 = 0;
-    for (int first = blockIdx.x; first < total;
-         first += kIssuers * gridDim.x) {
-      const int it = first + lane * gridDim.x;
-      int b = 0, j = 0, cc = 0;
-      bool use = it < total;
-      if (use) {
-        cc = it % CC;
-        const int bj = it / CC;
-        j = bj % p.RU;
-        b = bj / p.RU;
-        use = state_ok(p, b) && j < p.n_in[b] + p.N - 1;
-      }
-      const uint32_t vote = __ballot_sync(kIssuerMask, use);
-      const int q = q0 + __popc(vote & ((1u << lane) - 1u));
-      q0 += __popc(vote);
-      if (use) {
-        const int s = q % kSlots;
-        if (q >= kSlots && !wait_bounded(&empty[s], ((q / kSlots) - 1) & 1)) {
-          failed = true;
-        } else {
-          const int lo = cc * S * kSub;
-          const uint32_t bytes =
-              (uint32_t)(min(S * kSub, p.V - lo) * (int)sizeof(T));
-          item[s] = it;
-          mbar_arrive_expect_tx(&full[s], bytes);
-          bulk_load(ring + (size_t)s * kSlotElems,
-                    p.lc + ((size_t)b * p.K + j) * p.V + lo, bytes, &full[s]);
-        }
-      }
-      if (__any_sync(kIssuerMask, failed)) {
-        failed = true;
+template <typename T, bool kVec>
+__global__ void __launch_bounds__(kStatsWarps * 32)
+    accept_stats_kernel(AcceptDev<T> p) {
+  grid_dep_wait();
+  // The draw kernel's residual counters start at zero.
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.B;
+       i += gridDim.x * blockDim.x)
+    p.count[i] = 0;
+  auto used = [&](int b) {
+    return state_ok(p, b) ? p.n_in[b] + p.N - 1 : 0;
+  };
+  ItemWalk w;
+  w.init(blockIdx.x * kStatsWarps + (threadIdx.x >> 5),
+         (long long)gridDim.x * kStatsWarps, p.B, p.C, p.RU);
+  bool have = w.next_used(used);
+  Raw8<T> cur[8];
+  if (have) load_sub<T, kVec>(p, w.b, w.j, w.c, cur);
+  while (have) {
+    const int cb = w.b, cj = w.j, cc = w.c;
+    w.step();
+    have = w.next_used(used);
+    Raw8<T> nxt[8];
+    if (have) load_sub<T, kVec>(p, w.b, w.j, w.c, nxt);   // in flight ...
+    reduce_sub(p, cb, cj, cc, cur);                      // ... during this
+#pragma unroll
+    for (int k = 0; k < 8; ++k) cur[k] = nxt[k];
+  }
+}
+
+// The same items and arithmetic for 16-byte aligned bf16 rows, staged
+// through shared memory: each warp owns kStatsStages sub-chunk slots and
+// keeps kStatsStages - 1 sub-chunks in flight with cp.async (16 bytes a
+// lane, 8 per sub-chunk) while it reduces the oldest.  Lane l copies and
+// later reads back exactly its own elements, so a thread's own
+// cp.async.wait_group is the only synchronisation.  A chunk past the row
+// end is not copied; its elements read as -inf.
+constexpr int kStatsStages = 3;
+constexpr int kStatsSmem = kStatsWarps * kStatsStages * kSub * 2;   // 192 KB
+
+ISD_DEV void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int kPending>
+ISD_DEV void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+
+__global__ void __launch_bounds__(kStatsWarps * 32, 1)
+    accept_stats_async_kernel(AcceptDev<__nv_bfloat16> p) {
+  constexpr int S = kStatsStages;
+  extern __shared__ __align__(16) unsigned char stats_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __nv_bfloat16* slots =
+      reinterpret_cast<__nv_bfloat16*>(stats_smem) + (size_t)warp * S * kSub;
+  grid_dep_wait();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.B;
+       i += gridDim.x * blockDim.x)
+    p.count[i] = 0;
+  // Rows in use per sequence, once per CTA (0: malformed state).
+  int* s_used = reinterpret_cast<int*>(stats_smem + kStatsSmem);
+  for (int i = threadIdx.x; i < p.B; i += blockDim.x)
+    s_used[i] = state_ok(p, i) ? p.n_in[i] + p.N - 1 : 0;
+  __syncthreads();
+  auto used = [&](int b) { return s_used[b]; };
+  ItemWalk w;
+  w.init(blockIdx.x * kStatsWarps + warp, (long long)gridDim.x * kStatsWarps,
+         p.B, p.C, p.RU);
+  bool have = w.next_used(used);
+  // Copies this lane's 8 chunks of the walker's item into slot s.
+  auto issue = [&](int s) {
+    const __nv_bfloat16* row = p.lc + ((size_t)w.b * p.K + w.j) * p.V;
+    const int lo = w.c * kSub;
+    const uint32_t dst = smem_u32(slots + (size_t)s * kSub);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int e0 = (k * 32 + lane) * 8;
+      if (lo + e0 < p.V)   // whole 16-byte chunks: V is a multiple of 8
+        cp_async_16(dst + e0 * 2, row + lo + e0, 16u);
+    }
+  };
+  int qb[S], qj[S], qc[S];     // the item in each slot (qb < 0: none)
+#pragma unroll
+  for (int s = 0; s < S; ++s) qb[s] = -1;
+  auto take = [&](int s) {     // the walker's item into slot s, then on
+    if (have) {
+      qb[s] = w.b; qj[s] = w.j; qc[s] = w.c;
+      issue(s);
+      w.step();
+      have = w.next_used(used);
+    } else {
+      qb[s] = -1;
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int s = 0; s < S - 1; ++s) take(s);
+  for (bool more = true; more;) {
+#pragma unroll
+    for (int u = 0; u < S; ++u) {
+      // Refill the slot consumed in the previous round, then reduce slot u.
+      take((u + S - 1) % S);
+      cp_async_wait<S - 1>();
+      if (qb[u] < 0) {
+        more = false;
         break;
       }
-    }
-    // End markers, one per consumer group, kIssuers at a time.
-    for (int m = 0; m < kGroups && !failed; m += kIssuers) {
-      const int q = q0 + lane, s = q % kSlots;
-      if (m + lane < kGroups) {
-        if (q >= kSlots && !wait_bounded(&empty[s], ((q / kSlots) - 1) & 1)) {
-          failed = true;
-        } else {
-          item[s] = -1;
-          mbar_arrive(&full[s]);
-        }
+      const int lo = qc[u] * kSub;
+      const int n_el = min(kSub, p.V - lo);
+      const __nv_bfloat16* src = slots + (size_t)u * kSub;
+      Raw8<__nv_bfloat16> v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int e0 = (k * 32 + lane) * 8;
+        if (e0 < n_el)
+          v[k].u = *reinterpret_cast<const uint4*>(src + e0);
+        else
+          v[k].u = make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u,
+                              0xFF80FF80u);   // -inf
       }
-      failed = __any_sync(kIssuerMask, failed);
-      if (!failed) q0 += min(kIssuers, kGroups - m);
-    }
-    if (lane == 0) {
-      if (failed) report(p.status, ISD_ERR_CUDA);
-      // Copies still in flight land before the CTA's shared memory goes
-      // away (after a failure a slot may never fill: the wait is bounded).
-      for (int k = max(0, q0 - kSlots); k < q0; ++k)
-        if (!wait_bounded(&full[k % kSlots], (k / kSlots) & 1)) break;
-    }
-    return;
-  }
-
-  const int g = warp / kGroupWarps, i = warp % kGroupWarps;
-  for (int t = 0;; ++t) {
-    const int q = g + t * kGroups, s = q % kSlots;
-    if (!wait_bounded(&full[s], (q / kSlots) & 1)) {
-      if (lane == 0) report(p.status, ISD_ERR_CUDA);
-      break;
-    }
-    const int it = item[s];
-    const int c = it < 0 ? p.C : (it % CC) * S + i;
-    if (i >= S || c >= p.C) {  // end marker, or no sub-chunk for this warp
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      if (it < 0) break;
-      continue;
-    }
-    const int lo = c * kSub, n_el = min(kSub, p.V - lo);
-    const T* src = ring + (size_t)s * kSlotElems + i * kSub;
-    // Lane l reads elements (k*32 + l)*8 + e (k, e < 8) of the sub-chunk,
-    // -inf past the row end; the slot is read once per pass, nothing kept.
-    auto group = [&](int k, float (&v)[8]) {
-      const int e0 = (k * 32 + lane) * 8;
-      if (e0 + 8 <= n_el) {
-        lds8(src + e0, v);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          v[e] = e0 + e < n_el ? to_f(src[e0 + e]) : -INFINITY;
-      }
-    };
-    float mk[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      float v[8];
-      group(k, v);
-      mk[k] = fmaxf(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])),
-                    fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7])));
-    }
-    float m = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])),
-                    fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7])));
-    m = warp_max(m);
-    double sum = 0.0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      float v[8];
-      group(k, v);
-      float t8 = 0.0f;  // 8 terms in fp32, then fp64 across groups
-#pragma unroll
-      for (int e = 0; e < 8; ++e) t8 += ex2((v[e] - m) * kLog2e);
-      sum += (double)t8;
-    }
-    int first = INT_MAX;
-    if (p.argmax) {  // first index of the max (exact compares)
-#pragma unroll
-      for (int k = 7; k >= 0; --k) {
-        float v[8];
-        group(k, v);
-#pragma unroll
-        for (int e = 7; e >= 0; --e)
-          if (v[e] == m) first = lo + (k * 32 + lane) * 8 + e;
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);  // this warp no longer reads it
-    sum = warp_sum_f64(sum);
-    const size_t o = (size_t)(it / CC) * p.C + c;
-    if (p.argmax) {
-      first = warp_min_int(first);
-      if (lane == 0) p.cidx[o] = first;
-    }
-    if (lane == 0) {
-      p.cmax[o] = m;
-      p.csum[o] = sum;
+      reduce_sub(p, qb[u], qj[u], qc[u], v);
     }
   }
-}
-
-// Same items, element order and arithmetic, read with plain loads.
-template <typename T>
-__global__ void __launch_bounds__(256) accept_stats_plain_kernel(AcceptDev<T> p) {
-  const int lane = threadIdx.x & 31;
-  grid_dep_wait();
-  const int warps = gridDim.x * (blockDim.x >> 5);
-  const int total = p.B * p.RU * p.C;
-  for (int it = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       it < total; it += warps) {
-    const int c = it % p.C, bj = it / p.C, j = bj % p.RU, b = bj / p.RU;
-    if (!state_ok(p, b) || j >= p.n_in[b] + p.N - 1) continue;
-    const T* row = p.lc + ((size_t)b * p.K + j) * p.V;
-    const int lo = c * kSub, hi = min(p.V, lo + kSub);
-    float v[8][8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      load_row8<T, false>(row, lo + (k * 32 + lane) * 8, hi, v[k]);
-    finish_sub(p, (size_t)it, lo, v);
-  }
-}
-
-// ---------------------------------------------------------------------------
-template <typename T>
-__global__ void __launch_bounds__(1024) accept_decide_kernel(AcceptDev<T> p) {
-  __shared__ float s_m[32];
-  __shared__ double s_s[32];
-  const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int N = p.N, K = p.K;
-  grid_dep_wait();
-  const int n = p.n_in[b];
-  const int L = p.seq_len[b];
-  const int tok = lane < N ? p.pending_in[b * N + lane] : 0;
-  bool ok = (n == 1 || n == N) && L >= 0;
-  if (ok && lane < n) ok = tok >= 0 && tok < p.V;
-  int qr = 0;
-  if (ok && lane >= 1 && lane < n) {
-    qr = p.q_row_in[b * N + lane];
-    ok = qr >= 0 && qr < K;
-  }
-  ok = __all_sync(0xffffffffu, ok);  // every warp reaches the same verdict
-  int32_t* dec = p.decision + b * 4;
-  if (!ok) {
-    if (warp != 0) return;
-    if (lane == 0) {
-      report(p.status, ISD_ERR_BAD_STATE);
-      p.n_commit[b] = 0;
-      p.n_out[b] = n;
-      p.count[b] = 0;
-      dec[0] = 0; dec[1] = 0; dec[2] = -1; dec[3] = n;
-    }
-    if (lane < N) {
-      p.commit_tokens[b * N + lane] = -1;
-      p.pending_out[b * N + lane] = p.pending_in[b * N + lane];
-      p.q_row_out[b * N + lane] = p.q_row_in[b * N + lane];
-      p.q_stats_out[(b * N + lane) * 2] = p.q_stats_in[(b * N + lane) * 2];
-      p.q_stats_out[(b * N + lane) * 2 + 1] =
-          p.q_stats_in[(b * N + lane) * 2 + 1];
-    }
-    return;
-  }
-  // Warp 0 fetches the logits at the drafts first, so that their latency
-  // overlaps the merge.
-  const bool verifies = warp == 0 && lane >= 1 && lane < n;
-  float lx = 0.0f, lqx = 0.0f, zhi = 0.0f, zlo = 0.0f;
-  if (verifies) {
-    lx = to_f(p.lc[((size_t)b * K + lane - 1) * p.V + tok]);
-    if (!p.argmax) {
-      zhi = p.q_stats_in[(b * N + lane) * 2];
-      zlo = p.q_stats_in[(b * N + lane) * 2 + 1];
-      lqx = to_f(p.lp[((size_t)b * K + qr) * p.V + tok]);
-    }
-  }
-  // Row statistics: warp j merges the sub-chunks of row j.
-  const int rows_used = n + N - 1;
-  if (warp < rows_used) {
-    const size_t o = ((size_t)b * p.RU + warp) * p.C;
-    float cm[kSubPerLane];
-    double cs[kSubPerLane];
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < kSubPerLane; ++i) {
-      const int c = lane * kSubPerLane + i;
-      cm[i] = c < p.C ? p.cmax[o + c] : -INFINITY;
-      cs[i] = c < p.C ? p.csum[o + c] : 0.0;
-      m = fmaxf(m, cm[i]);
-    }
-    m = warp_max(m);
-    double s = 0.0;
-#pragma unroll
-    for (int i = 0; i < kSubPerLane; ++i)
-      if (lane * kSubPerLane + i < p.C) s += cs[i] * exp((double)(cm[i] - m));
-    s = warp_sum_f64(s);
-    if (lane == 0) {
-      s_m[warp] = m;
-      s_s[warp] = s;
-      p.rmax[b * K + warp] = m;
-      p.rsum[b * K + warp] = s;
-      if (p.row_stats_out) {
-        p.row_stats_out[(b * K + warp) * 2] = m;
-        p.row_stats_out[(b * K + warp) * 2 + 1] = (float)s;
-      }
-    }
-  }
-  __syncthreads();
-  if (warp != 0) return;
-  // Ratio test of drafts 1..n-1: lane i verifies draft i with row i-1.
-  // l - m is exact in fp32 (both are logits); p, q and the ratio in fp64.
-  bool acc = true;
-  if (verifies) {
-    const double px = exp((double)(lx - s_m[lane - 1])) / s_s[lane - 1];
-    double qx = 1.0;      // argmax drafts: the proposal is a point mass
-    if (!p.argmax) qx = exp(((double)lqx - (double)zhi) - (double)zlo);
-    const double r = qx > 0.0 ? px / qx : INFINITY;
-    const float u = uniform(p.seed, (uint32_t)b, step_of(p),
-                            (uint32_t)(L + lane), ISD_STREAM_ACCEPT);
-    acc = (double)u < r;
-    if (p.ratio_out) p.ratio_out[b * N + lane] = (float)r;
-  }
-  const uint32_t mask = __ballot_sync(0xffffffffu, acc);
-  const uint32_t drafts = ((n >= 32) ? 0xffffffffu : ((1u << n) - 1u)) & ~1u;
-  const uint32_t rej = drafts & ~mask;
-  const bool rejected = rej != 0u;
-  const int a = rejected ? (__ffs(rej) - 2) : (n - 1);
-  if (lane < N) {
-    p.commit_tokens[b * N + lane] = lane <= a ? tok : -1;
-    // Next drafts' q rows and the log-normaliser log sum_v exp(l_v) of
-    // each (lane j: row n + j - 1), stored as a float pair hi + lo.
-    const bool has = !rejected && lane >= 1;
-    const int src = n + lane - 1;
-    p.q_row_out[b * N + lane] = has ? src : -1;
-    const double lz = has ? (double)s_m[src] + log(s_s[src]) : 0.0;
-    const float lz_hi = (float)lz;
-    p.q_stats_out[(b * N + lane) * 2] = lz_hi;
-    p.q_stats_out[(b * N + lane) * 2 + 1] = (float)(lz - (double)lz_hi);
-    // After a rejection only the replacement is pending.
-    if (rejected && lane >= 1) p.pending_out[b * N + lane] = -1;
-  }
-  if (lane == 0) {
-    p.n_commit[b] = a + 1;
-    p.n_out[b] = rejected ? 1 : N;
-    p.count[b] = 0;
-    dec[0] = 1; dec[1] = rejected ? 1 : 0; dec[2] = a; dec[3] = n;
-  }
+  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
@@ -630,14 +438,15 @@ ISD_DEV float resid_w(const ResidRows& r, float lpv, float lqv, int v) {
   return fmaxf(0.0f, w);
 }
 
+// The rows of a rejection at draft a + 1: p from row a of logits_cur (its
+// max and sum `mp`, `sp`), q from the stored row of that draft.
 template <typename T>
-ISD_DEV ResidRows resid_rows(const AcceptDev<T>& p, int b, int a,
-                             const T*& prow, const T*& qrow) {
+ISD_DEV ResidRows resid_rows(const AcceptDev<T>& p, int b, int a, float mp,
+                             double sp, const T*& prow, const T*& qrow) {
   const int N = p.N, K = p.K;
   prow = p.lc + ((size_t)b * K + a) * p.V;
   ResidRows r;
-  r.mp = p.rmax[b * K + a];
-  const double sp = p.rsum[b * K + a];
+  r.mp = mp;
   r.inv_sp = (float)(1.0 / sp);
   if (p.argmax) {
     qrow = prow;                       // not read
@@ -648,7 +457,7 @@ ISD_DEV ResidRows resid_rows(const AcceptDev<T>& p, int b, int a,
     qrow = p.lp + ((size_t)b * K + qr) * p.V;
     r.zq_hi = p.q_stats_in[(b * N + a + 1) * 2];
     r.zq_lo = p.q_stats_in[(b * N + a + 1) * 2 + 1];
-    const double c = ((double)r.mp + log(sp)) - ((double)r.zq_hi + (double)r.zq_lo);
+    const double c = ((double)mp + log(sp)) - ((double)r.zq_hi + (double)r.zq_lo);
     r.c_hi = (float)c;
     r.c_lo = (float)(c - (double)r.c_hi);
     r.x = -1;
@@ -656,241 +465,430 @@ ISD_DEV ResidRows resid_rows(const AcceptDev<T>& p, int b, int a,
   return r;
 }
 
-// One inverse-CDF draw by a warp: the smallest index whose running mass
-// (ascending order) exceeds u * total.  mode 0: the residual of sequence b
-// (rr, prow, qrow; sub-chunk masses from `resid`, written in this kernel);
-// mode 1: row `row` of logits_cur with its statistics.  Returns the token
-// on every lane.
-template <typename T, bool kVec>
-ISD_DEV int warp_draw(const AcceptDev<T>& p, int b, int mode, int row,
-                      const ResidRows& rr, const T* prow, const T* qrow,
-                      float u) {
-  const int lane = threadIdx.x & 31, C = p.C;
-  const float m_row = mode ? p.rmax[b * p.K + row] : 0.0f;
-  const size_t o = ((size_t)b * p.RU + row) * C;
-  // 1. The sub-chunk: lane l owns sub-chunks 4l .. 4l+3.
-  double mc[kSubPerLane];
-  double own = 0.0;
+// What a CTA of the draw kernel shares between its warps.
+struct DrawShared {
+  float m[kMaxRows];           // row max of the merged rows
+  double s[kMaxRows];          // row sum
+  double mass[2][kMaxSub];     // sub-chunk masses of the two candidate draw rows
+  double tot[kDrawWarps];      // per-warp totals of an element scan
+  int lastp[kDrawWarps];       // per-warp last positive element
+  double rem;                  // target left inside the chosen sub-chunk
+  int chosen;                  // chosen sub-chunk
+  int found;                   // warp holding the target (-1: none)
+  int ok, n, rejected, a, last, mode;
+};
+
+// Row statistics from the sub-chunk figures, by one warp: m = max of the
+// sub-chunk maxima, s = sum_c csum_c * exp(cmax_c - m) (fp64, fixed order).
+// With `mass` set, also the sub-chunk masses csum_c * exp(cmax_c - m).
+template <typename T>
+ISD_DEV void merge_row(const AcceptDev<T>& p, int b, int r, float& m_out,
+                       double& s_out, double* mass) {
+  const int lane = threadIdx.x & 31;
+  const size_t o = ((size_t)b * p.RU + r) * p.C;
+  float cm[kSubPerLane];
+  double cs[kSubPerLane];
+  float m = -INFINITY;
 #pragma unroll
   for (int i = 0; i < kSubPerLane; ++i) {
     const int c = lane * kSubPerLane + i;
-    mc[i] = 0.0;
-    if (c < C)
-      mc[i] = mode == 0 ? __ldcg(&p.resid[(size_t)b * C + c])
-                        : p.csum[o + c] * exp((double)(p.cmax[o + c] - m_row));
-    own += mc[i];
+    cm[i] = c < p.C ? p.cmax[o + c] : -INFINITY;
+    cs[i] = c < p.C ? p.csum[o + c] : 0.0;
+    m = fmaxf(m, cm[i]);
   }
-  double excl;
-  const double incl = warp_scan_f64(own, excl);
-  const double target = (double)u * __shfl_sync(0xffffffffu, incl, 31);
-  const uint32_t hit = __ballot_sync(0xffffffffu, incl > target);
-  const uint32_t pos = __ballot_sync(0xffffffffu, own > 0.0);
-  // Rounding can leave the target past every running sum: then the last
-  // sub-chunk with positive mass, scanned to its last positive entry.
-  const int hl = hit ? __ffs(hit) - 1 : (pos ? 31 - __clz(pos) : 0);
-  int chosen = -1;
-  double rem = INFINITY;
-  if (lane == hl) {
-    double run = excl;
-    int lastpos = lane * kSubPerLane;
+  m = warp_max(m);
+  double s = 0.0;
 #pragma unroll
-    for (int i = 0; i < kSubPerLane; ++i) {
-      const int c = lane * kSubPerLane + i;
-      if (c >= C) break;
-      if (mc[i] > 0.0) lastpos = c;
-      const double before = run;
-      run += mc[i];
-      if (hit && chosen < 0 && run > target) {
-        chosen = c;
-        rem = target - before;
-      }
-    }
-    if (chosen < 0) chosen = lastpos;
+  for (int i = 0; i < kSubPerLane; ++i) {
+    const int c = lane * kSubPerLane + i;
+    const double mc = c < p.C ? cs[i] * exp((double)(cm[i] - m)) : 0.0;
+    if (mass && c < kMaxSub) mass[c] = mc;
+    s += mc;
   }
-  chosen = __shfl_sync(0xffffffffu, chosen, hl);
-  rem = __shfl_sync(0xffffffffu, rem, hl);
-  // 2. Inside the sub-chunk, four rounds of 512 elements: in round r lane l
-  //    owns elements lo + 512r + 16l .. +15, so the scan stays ascending.
-  //    Round r + 1 is loaded while round r is scanned.
-  const int lo = chosen * kSub, hi = min(p.V, lo + kSub);
-  const bool with_q = mode == 0 && rr.x < 0;
-  Raw8<T> cp[2], cq[2], np[2], nq[2];
-  auto load_round = [&](int r, Raw8<T> (&rp)[2], Raw8<T> (&rq)[2]) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int idx = lo + r * 512 + lane * 16 + h * 8;
-      rp[h] = load_raw8<kVec>(prow, idx, hi);
-      if (with_q) rq[h] = load_raw8<kVec>(qrow, idx, hi);
-    }
-  };
-  load_round(0, cp, cq);
-  int tok = -1, lastp = -1;
-  bool found = false;
-#pragma unroll 1
-  for (int r = 0; r < 4 && !found; ++r) {
-    if (r < 3) load_round(r + 1, np, nq);
-    const int base = lo + r * 512 + lane * 16;
-    // Element weights are recomputed for the walk (the same operations, so
-    // the same values) rather than kept.
-    auto weight = [&](int h, int e) {
-      return mode == 0
-                 ? resid_w(rr, cp[h].at(e), with_q ? cq[h].at(e) : 0.0f,
-                           base + h * 8 + e)
-                 : ex2((cp[h].at(e) - m_row) * kLog2e);
-    };
-    double lt = 0.0;
-    int lastr = -1;
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float w = weight(h, e);
-        lt += (double)w;
-        if (w > 0.0f) lastr = base + h * 8 + e;
-      }
-    if (lastr >= 0) lastp = lastr;
-    double ex;
-    const double inc = warp_scan_f64(lt, ex);
-    const double tot = __shfl_sync(0xffffffffu, inc, 31);
-    if (rem < tot) {  // the same verdict on every lane
-      const int hl2 = __ffs(__ballot_sync(0xffffffffu, inc > rem)) - 1;
-      if (lane == hl2) {
-        double run = ex;
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            run += (double)weight(h, e);
-            if (tok < 0 && run > rem) tok = base + h * 8 + e;
-          }
-        if (tok < 0) tok = lastr;  // rounding: this lane's last positive
-      }
-      tok = __shfl_sync(0xffffffffu, tok, hl2);
-      found = true;
-    }
-    rem -= tot;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      cp[h] = np[h];
-      cq[h] = nq[h];
-    }
-  }
-  // Rounding left the target past every running sum: the last positive
-  // entry of the sub-chunk.
-  if (tok < 0) {
-    const int lp = warp_max_int(lastp);
-    tok = lp >= 0 ? lp : lo;
-  }
-  return tok;
+  m_out = m;
+  s_out = warp_sum_f64(s);
 }
 
+// One inverse-CDF draw by the whole CTA: the smallest index whose running
+// mass (ascending order) exceeds u * total.  Sub-chunk masses: the
+// residual's from `resid` (mode 0, written by this kernel; if their total
+// is zero, p == q up to rounding, the draw falls back to p of row `row`),
+// or `mass` (mode 1: row `row` of logits_cur, row max m_row).
 template <typename T, bool kVec>
-__global__ void __launch_bounds__(kDrawWarps * 32,
-                                  sizeof(T) == 2 && kVec ? 2 : 1)
-    accept_draw_kernel(AcceptDev<T> p) {
-  // blockIdx.x is the sequence, so that the first block of every sequence
-  // (its draws, or its first residual sub-chunks) is scheduled first.
-  const int b = blockIdx.x, lane = threadIdx.x & 31;
-  const int wi = blockIdx.y * kDrawWarps + (threadIdx.x >> 5);
-  grid_dep_wait();
-  const int32_t* dec = p.decision + b * 4;
-  if (dec[0] == 0) return;  // malformed state: decide copied it through
-  const bool rejected = dec[1] != 0;
-  const int a = dec[2], n = dec[3];
-  const int N = p.N, K = p.K;
-  const int L = p.seq_len[b];
-  // What this warp draws, if anything: mode 0 the residual, 1 a row of p/q.
-  int mode, row, slot;
-  float u;
-  ResidRows rr{};
-  const T* prow = nullptr;
-  const T* qrow = nullptr;
-  if (rejected) {
-    if (wi >= p.C) return;
-    rr = resid_rows(p, b, a, prow, qrow);
-    const int lo = wi * kSub, hi = min(p.V, lo + kSub);
-    // Argmax drafts read no q row (the q row pointer is p's, never used).
-    const T* qsrc = rr.x < 0 ? qrow : prow;
-    Raw8<T> vp[8], vq[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      vp[k] = load_raw8<kVec>(prow, lo + (k * 32 + lane) * 8, hi);
-    if (rr.x < 0) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        vq[k] = load_raw8<kVec>(qsrc, lo + (k * 32 + lane) * 8, hi);
-    }
-    double s = 0.0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int idx = lo + (k * 32 + lane) * 8;
-      float t = 0.0f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        t += resid_w(rr, vp[k].at(e), rr.x < 0 ? vq[k].at(e) : 0.0f, idx + e);
-      s += (double)t;
-    }
-    s = warp_sum_f64(s);
-    int last = 0;
-    if (lane == 0) {
-      p.resid[(size_t)b * p.C + wi] = s;
-      __threadfence();
-      last = atomicAdd(&p.count[b], 1) == p.C - 1;
-    }
-    if (!__shfl_sync(0xffffffffu, last, 0)) return;
-    // Last sub-chunk of this sequence: every resid[b][*] is written.
-    __threadfence();
-    double W = 0.0;
+ISD_DEV int cta_draw(const AcceptDev<T>& p, DrawShared& sh, int b, int mode,
+                     int row, float m_row, const double* mass,
+                     const ResidRows& rr, const T* prow, const T* qrow,
+                     float u) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, C = p.C;
+  // 1. The sub-chunk (warp 0): lane l owns sub-chunks 4l .. 4l+3.
+  if (warp == 0) {
+    double mc[kSubPerLane];
+    double own = 0.0;
 #pragma unroll
     for (int i = 0; i < kSubPerLane; ++i) {
       const int c = lane * kSubPerLane + i;
-      if (c < p.C) W += __ldcg(&p.resid[(size_t)b * p.C + c]);
+      mc[i] = 0.0;
+      if (c < C) mc[i] = mode == 0 ? __ldcg(&p.resid[(size_t)b * C + c]) : mass[c];
+      own += mc[i];
     }
-    W = warp_sum_f64(W);
-    // Zero residual mass (p == q up to rounding): draw from p instead.
-    mode = W > 0.0 ? 0 : 1;
-    row = a;
-    slot = 0;
-    u = uniform(p.seed, (uint32_t)b, step_of(p), (uint32_t)(L + a + 1),
-                ISD_STREAM_RESAMPLE);
+    double excl;
+    double incl = warp_scan_f64(own, excl);
+    double total = __shfl_sync(0xffffffffu, incl, 31);
+    if (mode == 0 && !(total > 0.0)) {
+      // Zero residual mass: draw from p of row `row` instead.
+      mode = 1;
+      const size_t o = ((size_t)b * p.RU + row) * C;
+      own = 0.0;
+#pragma unroll
+      for (int i = 0; i < kSubPerLane; ++i) {
+        const int c = lane * kSubPerLane + i;
+        mc[i] = c < C ? p.csum[o + c] * exp((double)(p.cmax[o + c] - m_row)) : 0.0;
+        own += mc[i];
+      }
+      incl = warp_scan_f64(own, excl);
+      total = __shfl_sync(0xffffffffu, incl, 31);
+    }
+    const double target = (double)u * total;
+    const uint32_t hit = __ballot_sync(0xffffffffu, incl > target);
+    const uint32_t pos = __ballot_sync(0xffffffffu, own > 0.0);
+    // Rounding can leave the target past every running sum: then the last
+    // sub-chunk with positive mass, scanned to its last positive entry.
+    const int hl = hit ? __ffs(hit) - 1 : (pos ? 31 - __clz(pos) : 0);
+    if (lane == hl) {
+      double run = excl;
+      int chosen = -1, lastpos = lane * kSubPerLane;
+      double rem = INFINITY;
+#pragma unroll
+      for (int i = 0; i < kSubPerLane; ++i) {
+        const int c = lane * kSubPerLane + i;
+        if (c >= C) break;
+        if (mc[i] > 0.0) lastpos = c;
+        const double before = run;
+        run += mc[i];
+        if (hit && chosen < 0 && run > target) {
+          chosen = c;
+          rem = target - before;
+        }
+      }
+      sh.chosen = chosen < 0 ? lastpos : chosen;
+      sh.rem = rem;
+      sh.mode = mode;
+    }
+  }
+  __syncthreads();
+  mode = sh.mode;
+  // 2. Inside the sub-chunk: warp w scans elements lo + 256w .. +255, lane
+  //    l elements lo + 256w + 8l .. +7, so warp order and lane order keep
+  //    the scan ascending.  The warps' totals are taken in order from the
+  //    target, which is what one warp scanning all eight parts would do.
+  const int lo = sh.chosen * kSub, hi = min(p.V, lo + kSub);
+  const int base = lo + warp * kWarpElems + lane * 8;
+  const bool with_q = mode == 0 && rr.x < 0;
+  const Raw8<T> cp = load_raw8<kVec>(prow, base, hi);
+  Raw8<T> cq{};
+  if (with_q) cq = load_raw8<kVec>(qrow, base, hi);
+  float wv[8];
+  double lt = 0.0;
+  int lastr = -1;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    wv[e] = mode == 0 ? resid_w(rr, cp.at(e), with_q ? cq.at(e) : 0.0f, base + e)
+                      : ex2((cp.at(e) - m_row) * kLog2e);
+    lt += (double)wv[e];
+    if (wv[e] > 0.0f) lastr = base + e;
+  }
+  double ex;
+  const double inc = warp_scan_f64(lt, ex);
+  const int lastw = warp_max_int(lastr);
+  if (lane == 31) {
+    sh.tot[warp] = inc;
+    sh.lastp[warp] = lastw;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double rem = sh.rem;
+    int f = -1;
+    for (int w = 0; w < kDrawWarps; ++w) {
+      if (rem < sh.tot[w]) {
+        f = w;
+        break;
+      }
+      rem -= sh.tot[w];
+    }
+    sh.found = f;
+    sh.rem = rem;
+  }
+  __syncthreads();
+  int tok = -1;
+  if (sh.found < 0) {
+    // Rounding left the target past every running sum: the last positive
+    // entry of the sub-chunk.
+    int lp = -1;
+    for (int w = 0; w < kDrawWarps; ++w) lp = max(lp, sh.lastp[w]);
+    tok = lp >= 0 ? lp : lo;
+  } else if (warp == sh.found) {
+    const double rem = sh.rem;
+    const int hl2 = __ffs(__ballot_sync(0xffffffffu, inc > rem)) - 1;
+    if (lane == hl2) {
+      double run = ex;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        run += (double)wv[e];
+        if (tok < 0 && run > rem) tok = base + e;
+      }
+      if (tok < 0) tok = lastr;  // rounding: this lane's last positive
+    }
+    tok = __shfl_sync(0xffffffffu, tok, hl2 < 0 ? 0 : hl2);
+    if (hl2 < 0) tok = sh.lastp[warp] >= 0 ? sh.lastp[warp] : lo;
+  }
+  return tok;   // valid on every thread when found < 0, else on warp `found`
+}
+
+// The draw kernel.  Row figures are merged before the sequence's mode is
+// known, for both modes' candidate rows, so the merge loads overlap the
+// state loads: part 0 merges every row (0 .. 2N-2), part y >= 1 the ratio
+// test rows 0 .. N-2 and its two candidate draw rows, y (R mode, n = 1)
+// and N + y - 1 (S mode, n = N); the candidate draw rows also keep their
+// sub-chunk masses in shared memory for the draw.
+template <typename T, bool kVec>
+__global__ void __launch_bounds__(kDrawWarps * 32)
+    accept_draw_kernel(AcceptDev<T> p) {
+  __shared__ DrawShared sh;
+  const int b = blockIdx.x, y = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = p.N, K = p.K;
+  grid_dep_wait();
+  // ---- 0. The sequence's state (warp 0) and the row merges (warps 1..).
+  int n = 0, L = 0, tok = 0, qr = 0;
+  float zhi = 0.0f, zlo = 0.0f;
+  if (warp == 0) {
+    n = p.n_in[b];
+    L = p.seq_len[b];
+    tok = lane < N ? p.pending_in[b * N + lane] : 0;
+    qr = lane < N ? p.q_row_in[b * N + lane] : 0;
+    if (!p.argmax && lane < N) {
+      zhi = p.q_stats_in[(b * N + lane) * 2];
+      zlo = p.q_stats_in[(b * N + lane) * 2 + 1];
+    }
   } else {
-    if (wi >= N) return;
-    slot = wi;                  // 0: the bonus; >= 1: drafts
-    row = n + wi - 1;
-    prow = p.lc + ((size_t)b * K + row) * p.V;
-    if (p.argmax && wi >= 1) {
-      // Argmax draft: the first sub-chunk whose max is the row max holds
-      // the first maximal index (exact compares of the same values).
+    // Merge list: part 0 every row; part y >= 1 rows 0 .. N-2, then its
+    // candidate draw rows (y when it is not already listed, N + y - 1).
+    const int cand_r = (y >= 1 && y < N) ? y : -1;           // R mode
+    const int cand_s = (y >= 1 && y < N) ? N + y - 1 : -1;   // S mode
+    const bool r_listed = cand_r >= 0 && cand_r <= N - 2;
+    const int nlist = y == 0 ? p.RU
+                             : (N - 1) + (cand_r >= 0 && !r_listed ? 1 : 0) +
+                                   (cand_s >= 0 ? 1 : 0);
+    for (int k = warp - 1; k < nlist; k += kDrawWarps - 1) {
+      int r = k;
+      if (y >= 1 && k >= N - 1)
+        r = (k == N - 1 && cand_r >= 0 && !r_listed) ? cand_r : cand_s;
+      // Candidate draw rows keep their masses: slot 0 the R-mode row, slot
+      // 1 the S-mode row (part 0: the bonus rows 0 and N - 1).
+      double* keep = nullptr;
+      if (y == 0) {
+        keep = r == 0 ? sh.mass[0] : (r == N - 1 ? sh.mass[1] : nullptr);
+      } else {
+        keep = r == cand_r ? sh.mass[0] : (r == cand_s ? sh.mass[1] : nullptr);
+      }
+      float m;
+      double s;
+      merge_row(p, b, r, m, s, keep);
+      if (lane == 0) {
+        sh.m[r] = m;
+        sh.s[r] = s;
+      }
+    }
+  }
+  // ---- 1. Validity; R-mode sequences have nothing for parts >= N.
+  float lx = 0.0f, lqx = 0.0f;
+  if (warp == 0) {
+    bool ok = (n == 1 || n == N) && L >= 0;
+    if (ok && lane < n) ok = tok >= 0 && tok < p.V;
+    if (ok && lane >= 1 && lane < n) ok = qr >= 0 && qr < K;
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && lane >= 1 && lane < n) {
+      lx = to_f(p.lc[((size_t)b * K + lane - 1) * p.V + tok]);
+      if (!p.argmax) lqx = to_f(p.lp[((size_t)b * K + qr) * p.V + tok]);
+    }
+    if (lane == 0) {
+      sh.ok = ok;
+      sh.n = n;          // for the other warps
+    }
+  }
+  __syncthreads();
+  n = sh.n;
+  if (!sh.ok) {
+    // Malformed state: reported once, passed through, nothing committed.
+    if (y == 0 && warp == 0) {
+      if (lane == 0) {
+        report(p.status, ISD_ERR_BAD_STATE);
+        p.n_commit[b] = 0;
+        p.n_out[b] = n;
+      }
+      if (lane < N) {
+        const int i = b * N + lane;
+        p.commit_tokens[i] = -1;
+        p.pending_out[i] = p.pending_in[i];
+        p.q_row_out[i] = p.q_row_in[i];
+        p.q_stats_out[2 * i] = p.q_stats_in[2 * i];
+        p.q_stats_out[2 * i + 1] = p.q_stats_in[2 * i + 1];
+      }
+    }
+    return;
+  }
+  if (n == 1 && y >= N) return;   // no drafts: nothing to reject
+  // ---- 2. Ratio tests of drafts 1 .. n-1 (warp 0, lane i verifies draft
+  //         i with row i-1); l - m is exact in fp32; p, q, the ratio fp64.
+  if (warp == 0) {
+    const int rows_used = n + N - 1;
+    const bool verifies = lane >= 1 && lane < n;
+    bool acc = true;
+    double r = 0.0;
+    if (verifies) {
+      const double px = exp((double)(lx - sh.m[lane - 1])) / sh.s[lane - 1];
+      double qx = 1.0;      // argmax drafts: the proposal is a point mass
+      if (!p.argmax) qx = exp(((double)lqx - (double)zhi) - (double)zlo);
+      r = qx > 0.0 ? px / qx : INFINITY;
+      const float u = uniform(p.seed, (uint32_t)b, step_of(p),
+                              (uint32_t)(L + lane), ISD_STREAM_ACCEPT);
+      acc = (double)u < r;
+    }
+    const uint32_t mask = __ballot_sync(0xffffffffu, acc);
+    const uint32_t drafts = ((n >= 32) ? 0xffffffffu : ((1u << n) - 1u)) & ~1u;
+    const uint32_t rej = drafts & ~mask;
+    const bool rejected = rej != 0u;
+    const int a = rejected ? (__ffs(rej) - 2) : (n - 1);
+    if (lane == 0) {
+      sh.rejected = rejected;
+      sh.a = a;
+    }
+    if (y == 0) {
+      // The decision's outputs.
+      if (verifies && p.ratio_out) p.ratio_out[b * N + lane] = (float)r;
+      if (lane < N) {
+        p.commit_tokens[b * N + lane] = lane <= a ? tok : -1;
+        // Next drafts' q rows and the log-normaliser log sum_v exp(l_v) of
+        // each (lane j: row n + j - 1), stored as a float pair hi + lo.
+        const bool has = !rejected && lane >= 1;
+        const int src = n + lane - 1;
+        p.q_row_out[b * N + lane] = has ? src : -1;
+        const double lz = has ? (double)sh.m[src] + log(sh.s[src]) : 0.0;
+        const float lz_hi = (float)lz;
+        p.q_stats_out[(b * N + lane) * 2] = lz_hi;
+        p.q_stats_out[(b * N + lane) * 2 + 1] = (float)(lz - (double)lz_hi);
+        // After a rejection only the replacement is pending.
+        if (rejected && lane >= 1) p.pending_out[b * N + lane] = -1;
+      }
+      if (p.row_stats_out && lane < rows_used) {
+        p.row_stats_out[(b * K + lane) * 2] = sh.m[lane];
+        p.row_stats_out[(b * K + lane) * 2 + 1] = (float)sh.s[lane];
+      }
+      if (lane == 0) {
+        p.n_commit[b] = a + 1;
+        p.n_out[b] = rejected ? 1 : N;
+      }
+    }
+  }
+  __syncthreads();
+  const bool rejected = sh.rejected;
+  const int a = sh.a;
+  if (rejected) {
+    // ---- 3a. Residual sub-chunk sums: part y takes sub-chunks 4y .. 4y+3,
+    //          two warps each (1024 elements, 32 a lane), in fixed order.
+    const int nparts = (p.C + kResidPerCta - 1) / kResidPerCta;
+    if (y >= nparts) return;
+    const T* prow;
+    const T* qrow;
+    const ResidRows rr = resid_rows(p, b, a, sh.m[a], sh.s[a], prow, qrow);
+    const int c = y * kResidPerCta + (warp >> 1), half = warp & 1;
+    double s = 0.0;
+    if (c < p.C) {
+      const int lo = c * kSub + half * (kSub / 2);
+      const int hi = min(p.V, c * kSub + kSub);
+      Raw8<T> vp[4], vq[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        vp[k] = load_raw8<kVec>(prow, lo + (k * 32 + lane) * 8, hi);
+        if (rr.x < 0) vq[k] = load_raw8<kVec>(qrow, lo + (k * 32 + lane) * 8, hi);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int idx = lo + (k * 32 + lane) * 8;
+        float t = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          t += resid_w(rr, vp[k].at(e), rr.x < 0 ? vq[k].at(e) : 0.0f, idx + e);
+        s += (double)t;
+      }
+      s = warp_sum_f64(s);
+    }
+    if (lane == 0) sh.tot[warp] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int i = 0; i < kResidPerCta; ++i) {
+        const int ci = y * kResidPerCta + i;
+        if (ci < p.C) p.resid[(size_t)b * p.C + ci] = sh.tot[2 * i] + sh.tot[2 * i + 1];
+      }
+      __threadfence();
+      sh.last = atomicAdd(&p.count[b], 1) == nparts - 1;
+    }
+    __syncthreads();
+    if (!sh.last) return;
+    // Last part of this sequence: every resid[b][*] is written.
+    __threadfence();
+    const float u = uniform(p.seed, (uint32_t)b, step_of(p),
+                            (uint32_t)(L + a + 1), ISD_STREAM_RESAMPLE);
+    const int t = cta_draw<T, kVec>(p, sh, b, 0, a, sh.m[a], nullptr, rr,
+                                    prow, qrow, u);
+    if (sh.found < 0 ? threadIdx.x == 0 : (warp == sh.found && lane == 0))
+      p.pending_out[b * N] = t;
+    return;
+  }
+  // ---- 3b. All drafts accepted: part y draws token y (0: the bonus from p
+  //          of row n-1; y >= 1: the draft at L + n + y from q of row
+  //          n + y - 1).
+  if (y >= N) return;
+  const int row = n + y - 1;
+  const double* mass = sh.mass[n == 1 ? 0 : 1];
+  if (p.argmax && y >= 1) {
+    // Argmax draft: the first sub-chunk whose max is the row max holds the
+    // first maximal index (exact compares of the same values).
+    if (warp == 0) {
       const size_t o = ((size_t)b * p.RU + row) * p.C;
-      const float m = p.rmax[b * K + row];
+      const float m = sh.m[row];
       int first = INT_MAX;
 #pragma unroll
       for (int i = kSubPerLane - 1; i >= 0; --i) {
-        const int c = lane * kSubPerLane + i;
-        if (c < p.C && p.cmax[o + c] == m) first = c;
+        const int ci = lane * kSubPerLane + i;
+        if (ci < p.C && p.cmax[o + ci] == m) first = ci;
       }
       first = warp_min_int(first);
-      if (lane == 0) p.pending_out[b * N + wi] = first < p.C ? p.cidx[o + first] : -1;
-      return;
+      if (lane == 0) p.pending_out[b * N + y] = first < p.C ? p.cidx[o + first] : -1;
     }
-    mode = 1;
-    u = uniform(p.seed, (uint32_t)b, step_of(p), (uint32_t)(L + n + wi),
-                wi == 0 ? ISD_STREAM_RESAMPLE : ISD_STREAM_DRAFT);
+    return;
   }
-  const int tok = warp_draw<T, kVec>(p, b, mode, row, rr, prow, qrow, u);
-  if (lane == 0) p.pending_out[b * N + slot] = tok;
+  const float u = uniform(p.seed, (uint32_t)b, step_of(p), (uint32_t)(L + n + y),
+                          y == 0 ? ISD_STREAM_RESAMPLE : ISD_STREAM_DRAFT);
+  const ResidRows none{};
+  const T* prow = p.lc + ((size_t)b * K + row) * p.V;
+  const int t = cta_draw<T, kVec>(p, sh, b, 1, row, sh.m[row], mass, none,
+                                  prow, prow, u);
+  if (sh.found < 0 ? threadIdx.x == 0 : (warp == sh.found && lane == 0))
+    p.pending_out[b * N + y] = t;
 }
 
 // ---------------------------------------------------------------------------
 // Host-side launcher (called from the C ABI after validation).
 
 struct AcceptLayout {
-  size_t csum, cmax, cidx, rsum, rmax, resid, decision, count, total;
+  size_t csum, cmax, cidx, resid, count, total;
 };
 
 static AcceptLayout accept_layout(int B, int N, int K, int V) {
   const size_t C = (V + kSub - 1) / kSub;
   const size_t RU = 2 * N - 1;
+  (void)K;
   AcceptLayout l;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -901,10 +899,7 @@ static AcceptLayout accept_layout(int B, int N, int K, int V) {
   l.csum = take((size_t)B * RU * C * 8);
   l.cmax = take((size_t)B * RU * C * 4);
   l.cidx = take((size_t)B * RU * C * 4);
-  l.rsum = take((size_t)B * K * 8);
-  l.rmax = take((size_t)B * K * 4);
   l.resid = take((size_t)B * C * 8);
-  l.decision = take((size_t)B * 4 * 4);
   l.count = take((size_t)B * 4);
   l.total = off;
   return l;
@@ -919,13 +914,82 @@ static int num_sms() {
   return n;
 }
 
+template <typename T, bool kVec>
+static int launch_stats(const AcceptDev<T>& p, int sms, cudaStream_t st) {
+  // As many 512-thread CTAs as fit on every SM at once (the warps loop over
+  // the items), fewer for small problems.
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+          &per_sm, accept_stats_kernel<T, kVec>, kStatsWarps * 32, 0) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return ISD_ERR_CUDA;
+  const long long items = (long long)p.B * p.RU * p.C;
+  const long long ctas = (items + kStatsWarps - 1) / kStatsWarps;
+  const int grid = (int)std::max<long long>(
+      1, std::min<long long>((long long)per_sm * sms, ctas));
+  return launch_pdl(accept_stats_kernel<T, kVec>, dim3(grid),
+                    dim3(kStatsWarps * 32), 0, st, p) == cudaSuccess
+             ? ISD_OK
+             : ISD_ERR_CUDA;
+}
+
+// Aligned bf16 rows: the shared-memory pipeline, one 512-thread CTA per SM.
+template <>
+int launch_stats<__nv_bfloat16, true>(const AcceptDev<__nv_bfloat16>& p,
+                                      int sms, cudaStream_t st) {
+  // Slots, then the rows-in-use table; too many sequences for the table
+  // take the register kernel.
+  const size_t smem = (size_t)kStatsSmem + (size_t)p.B * 4;
+  if (smem > 227 * 1024) {
+    const AcceptDev<__nv_bfloat16>& q = p;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &per_sm, accept_stats_kernel<__nv_bfloat16, true>,
+            kStatsWarps * 32, 0) != cudaSuccess ||
+        per_sm < 1)
+      return ISD_ERR_CUDA;
+    const long long items = (long long)q.B * q.RU * q.C;
+    const long long ctas = (items + kStatsWarps - 1) / kStatsWarps;
+    const int g = (int)std::max<long long>(
+        1, std::min<long long>((long long)per_sm * sms, ctas));
+    return launch_pdl(accept_stats_kernel<__nv_bfloat16, true>, dim3(g),
+                      dim3(kStatsWarps * 32), 0, st, q) == cudaSuccess
+               ? ISD_OK
+               : ISD_ERR_CUDA;
+  }
+  auto kern = accept_stats_async_kernel;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return ISD_ERR_CUDA;
+  const long long items = (long long)p.B * p.RU * p.C;
+  const long long ctas = (items + kStatsWarps - 1) / kStatsWarps;
+  const int grid = (int)std::max<long long>(1, std::min<long long>(sms, ctas));
+  return launch_pdl(kern, dim3(grid), dim3(kStatsWarps * 32), smem, st,
+                    p) == cudaSuccess
+             ? ISD_OK
+             : ISD_ERR_CUDA;
+}
+
+template <typename T, bool kVec>
+static int launch_accept_kernels(const AcceptDev<T>& p, int sms,
+                                 cudaStream_t st) {
+  const int rc = launch_stats<T, kVec>(p, sms, st);
+  if (rc != ISD_OK) return rc;
+  const int parts = std::max((p.C + kResidPerCta - 1) / kResidPerCta, p.N);
+  if (launch_pdl(accept_draw_kernel<T, kVec>, dim3(p.B, parts),
+                 dim3(kDrawWarps * 32), 0, st, p) != cudaSuccess)
+    return ISD_ERR_CUDA;
+  return ISD_OK;
+}
+
 template <typename T>
 static int launch_accept_t(const isd_accept_args* a, cudaStream_t st) {
   AcceptDev<T> p;
   p.B = a->B; p.N = a->N; p.K = a->K; p.V = a->V;
   p.C = (a->V + kSub - 1) / kSub;
   p.RU = 2 * a->N - 1;
-  if (p.C > kMaxSub) return ISD_ERR_UNSUPPORTED;
+  if (p.C > kMaxSub || p.K > kMaxRows) return ISD_ERR_UNSUPPORTED;
   p.step = a->step; p.step_dev = a->step_dev; p.seed = a->seed;
   p.lc = static_cast<const T*>(a->logits_cur);
   p.lp = static_cast<const T*>(a->logits_prev);
@@ -940,46 +1004,16 @@ static int launch_accept_t(const isd_accept_args* a, cudaStream_t st) {
   p.csum = reinterpret_cast<double*>(ws + l.csum);
   p.cmax = reinterpret_cast<float*>(ws + l.cmax);
   p.cidx = reinterpret_cast<int32_t*>(ws + l.cidx);
-  p.rsum = reinterpret_cast<double*>(ws + l.rsum);
-  p.rmax = reinterpret_cast<float*>(ws + l.rmax);
   p.resid = reinterpret_cast<double*>(ws + l.resid);
-  p.decision = reinterpret_cast<int32_t*>(ws + l.decision);
   p.count = reinterpret_cast<int32_t*>(ws + l.count);
   p.argmax = a->proposal == ISD_PROPOSAL_ARGMAX;
-
   const int sms = num_sms();
   if (sms <= 0) return ISD_ERR_CUDA;
-  const long long items = (long long)p.B * p.RU * p.C;
-  // Bulk copies need 16-byte aligned rows (logits_cur itself is checked on
-  // the host) and whole 16-byte multiples.
-  if (((size_t)a->V * sizeof(T)) % 16 == 0) {
-    auto kern = accept_stats_kernel<T>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kStatsSmem) != cudaSuccess)
-      return ISD_ERR_CUDA;
-    const int S = kCopyBytes / (kSub * (int)sizeof(T));
-    const long long copies = (long long)p.B * p.RU * ((p.C + S - 1) / S);
-    const int grid = (int)std::min<long long>(sms, copies);
-    if (launch_pdl(kern, dim3(grid), dim3(kStatsThreads), kStatsSmem, st, p) !=
-        cudaSuccess)
-      return ISD_ERR_CUDA;
-  } else {
-    const int grid = (int)std::min<long long>(8LL * sms, (items + 7) / 8);
-    if (launch_pdl(accept_stats_plain_kernel<T>, dim3(grid), dim3(256), 0, st,
-                   p) != cudaSuccess)
-      return ISD_ERR_CUDA;
-  }
-  if (launch_pdl(accept_decide_kernel<T>, dim3(p.B), dim3(32 * p.RU), 0, st,
-                 p) != cudaSuccess)
-    return ISD_ERR_CUDA;
-  const dim3 g_draw(p.B, (std::max(p.C, p.N) + kDrawWarps - 1) / kDrawWarps);
-  const cudaError_t e =
-      (a->V % 8) == 0
-          ? launch_pdl(accept_draw_kernel<T, true>, g_draw,
-                       dim3(kDrawWarps * 32), 0, st, p)
-          : launch_pdl(accept_draw_kernel<T, false>, g_draw,
-                       dim3(kDrawWarps * 32), 0, st, p);
-  return e == cudaSuccess ? ISD_OK : ISD_ERR_CUDA;
+  // Vector loads need 16-byte aligned rows (logits_cur itself is checked
+  // on the host) of whole 16-byte units.
+  if (((size_t)a->V * sizeof(T)) % 16 == 0)
+    return launch_accept_kernels<T, true>(p, sms, st);
+  return launch_accept_kernels<T, false>(p, sms, st);
 }
 
 size_t accept_workspace_bytes(int B, int N, int K, int V) {
