@@ -21,20 +21,24 @@
 // with S^T, O^T and the per-key partial row sums in TMEM.  No MMA row is
 // padding, and each block costs 16 MMAs whatever M is.
 //
-// Warp roles:
-//   loaders (4 warps)   warp k copies pages k and k + 4 of every block: its
-//                       lane 0 issues the K and V pages through the TMA
-//                       engine (64-column boxes, 128-byte swizzle).  Four
-//                       issuing threads keep enough copies in flight to
-//                       saturate HBM; one does not.  A partial last page
-//                       takes V by cp.async so that its unused slots are
-//                       zero-filled.
-//                       Page ids are read one block ahead.  Also each
-//                       segment's Q rows (cp.async).
-//   MMA warp            one thread issues S^T of block i into a double-
-//                       buffered S in TMEM, then O^T += V^T P^T of block
-//                       i-1, and commits completion to mbarriers.  It also
-//                       allocates and frees TMEM.
+// Warp roles (10 warps):
+//   loaders (4 warps)   two warps copy K tiles, two copy V tiles, each pair
+//                       in its own loop so a V slot in use never holds back
+//                       a K copy; a warp covers 4 pages of every block and
+//                       its lanes 0..7 issue the 8 TMA boxes (64-column
+//                       halves, 128-byte swizzle) in one instruction.  A
+//                       partial last page takes V by cp.async so that its
+//                       unused slots are zero-filled.  Page ids are read
+//                       two blocks ahead.  Warp 0 also loads each segment's
+//                       Q rows by TMA.
+//   QK MMA warp         one thread issues S^T of block i into a double-
+//                       buffered S in TMEM and commits completion.  It
+//                       also allocates and frees TMEM.
+//   P V MMA warp        one thread issues O^T += V^T P^T of block i once
+//                       its P is written.  Two issuing warps: one thread
+//                       issuing both kinds in order made each P V wait for
+//                       the next K tile and capped the issue rate (measured:
+//                       the two-warp split is 10% faster on the C=64 step).
 //   softmax (4 warps)   thread t owns key t of the block (TMEM lane t): it
 //                       masks its scores, writes P = 2^(s c - m_row c) in
 //                       bf16 into P^T, and adds P to its per-row partial
@@ -68,18 +72,23 @@ constexpr int kKH = kKeys * 128;             // one 64-column half of K or V
 constexpr int kTile = 2 * kKH;               // a K or V tile: 32 KB
 constexpr int kSmWarps = 4;
 constexpr int kMmaWarp = 4;
-constexpr int kLoadWarps = 4;
-constexpr int kPagesPerLoader = kNB / kLoadWarps;
-constexpr int kThreads = (kSmWarps + 1 + kLoadWarps) * 32;   // 288
-constexpr int kKStages = 2;                  // K ring
-constexpr int kMaxVStages = 4;               // V ring (fewer if Q, P are big)
+constexpr int kLoadWarps = 4;                // two K and two V warps
+constexpr int kPagesPerLoader = kNB / 2;     // pages of a block per warp
+constexpr int kPvWarp = 5;                   // issues the P V products
+constexpr int kThreads = (kSmWarps + 2 + kLoadWarps) * 32;   // 320
 constexpr int kBarBytes = 32 * 8;            // mbarriers (2 (SK + SV) + 17)
+// Q and P^T tiles in shared memory for N = 32 * nch padded rows.  Two let
+// the next (b, h) segment start (its Q load, its first softmax) while the
+// previous one finishes; the largest row counts keep one where memory is
+// short.
+constexpr int nqb_of(int nch) { return nch == 4 ? 1 : 2; }
+constexpr int npb_of(int nch) { return nch >= 3 ? 1 : 2; }
 constexpr int kStaticSmem = 3072;            // __shared__ arrays, rounded up
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint64_t kWaitCycles = 400000000ull;   // ~0.2 s
 
 struct Params {
-  int B, Hq, Hkv, K, g, M, P, stride, sv;
+  int B, Hq, Hkv, K, g, M, P, stride, sk, sv;
   float scale_log2;
   const __nv_bfloat16* q;
   const __nv_bfloat16* vc;
@@ -406,7 +415,7 @@ template <int NCH>
 __device__ __noinline__ bool store_segment(const EpiIn<NCH>& in, int blk, int code,
                                            int stage_buf, bool failed) {
   constexpr int N = 32 * NCH;
-  constexpr int NPB = NCH >= 3 ? 1 : 2;
+  constexpr int NPB = npb_of(NCH);
   constexpr int NOB = NCH <= 2 ? 2 : 1;
   constexpr int PB = NCH * kKeys * 64;
   constexpr uint32_t kO = 0, kL = NOB * N + 2 * N;
@@ -533,11 +542,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // swizzle), atom a holding rows 32a..32a+31.
   constexpr int PA = kKeys * 64;           // one 32-row atom (8 KB)
   constexpr int PB = NCH * PA;             // one P buffer
-  // Buffers per segment-level resource: two let the next (b, h) segment
-  // start (its Q load, its first P V) while the previous one finishes;
-  // the largest row counts keep one where memory is short.
-  constexpr int NQB = NCH == 4 ? 1 : 2;    // Q tiles (shared memory)
-  constexpr int NPB = NCH >= 3 ? 1 : 2;    // P tiles (shared memory)
+  constexpr int NQB = nqb_of(NCH);         // Q tiles (shared memory)
+  constexpr int NPB = npb_of(NCH);         // P tiles (shared memory)
   // O^T accumulators, row-sum partials (TMEM) and row maxima: with two, a
   // segment's epilogue is deferred until the next segment's first block
   // has been handed to the MMA warp, so the pipeline never waits on it.
@@ -555,8 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // K and V rings: a K tile is consumed by the QK MMAs of its block and
   // freed right after them; a V tile waits for the block's softmax and its
   // P V, so the V ring is deeper.
-  constexpr int SK = kKStages;
-  const int SV = p.sv;
+  const int SK = p.sk, SV = p.sv;
   uint8_t* kr = base;                                  // SK K tiles
   uint8_t* vr = kr + SK * kTile;                       // SV V tiles
   uint8_t* qs = vr + SV * kTile;                       // Q tile [N][128]
@@ -590,11 +595,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     s_bad = 0;
     for (int s = 0; s < SK; ++s) {
-      mbar_init(&k_full[s], kLoadWarps);    // one arrival per loader warp
+      mbar_init(&k_full[s], 2);             // one arrival per K warp
       mbar_init(&k_empty[s], 1);
     }
     for (int s = 0; s < SV; ++s) {
-      mbar_init(&v_full[s], kLoadWarps);
+      mbar_init(&v_full[s], 2);             // one arrival per V warp
       mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -608,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_empty[s], 1);
       mbar_init(&o_free[s], kSmWarps);
     }
-    mbar_init(fin, 1);
+    mbar_init(fin, 2);                      // both MMA warps commit
     fence_barrier_init();
   }
   // Padding rows of Q (M..N-1) stay zero for the whole kernel.
@@ -664,20 +669,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t q_s = smem_u32(qs), p_s = smem_u32(ps);
   bool failed = false;
 
-  if (warp > kMmaWarp) {
+  if (warp > kPvWarp) {
     // ------------------------------------------------------------ loaders
-    // Loader warp lw copies pages lw and lw + 4 of every block; its lane 0
-    // issues their TMA boxes, so four threads keep copies in flight (one
-    // cannot saturate HBM).  Each warp registers its TMA bytes and then
-    // arrives once per block on k_full and on v_full.
-    const int lt = tid - (kMmaWarp + 1) * 32;
+    // Two warps copy K tiles and two copy V tiles, each in its own loop, so
+    // a V slot still in use (its block's softmax and P V pending) never
+    // holds back the next K copy.  Loader warp lw handles pages
+    // 4 (lw & 1) .. 4 (lw & 1) + 3 of every block, and lanes 0..7 issue
+    // their eight TMA boxes (page q = lane / 2, 64-column half lane % 2) in
+    // one instruction: the TMA issue rate, not only the bytes in flight,
+    // bounds the stream.  Each warp registers its TMA bytes, then arrives
+    // once per block on k_full (K warps) or v_full (V warps).
+    const int lt = tid - (kPvWarp + 1) * 32;
     const int lw = lt >> 5;
+    const bool is_k = lw < 2;
+    const int pg0 = (lw & 1) * kPagesPerLoader;    // first page of the block
     BlockWalk w;
     w.init(prefix, B, Hkv, u0, u1);
     // Page ids of this warp's pages (-1: none or the tail), read two blocks
     // ahead: a global load waits microseconds behind the KV stream, and a
     // copy must not wait on one.
-    static_assert(kPagesPerLoader == 2, "two pages per loader warp");
     auto page_id = [&](const BlockWalk& x, int k) {
       const int uidx = x.idx0 + x.k + k;
       return (k < x.nu() && uidx != x.units - 1)
@@ -685,17 +695,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                  : -1;
     };
     BlockWalk wa = w;                 // two blocks ahead of w
-    int pa0 = -1, pa1 = -1, pb0 = -1, pb1 = -1;   // blocks i and i + 1
+    int pa[kPagesPerLoader], pb[kPagesPerLoader];   // blocks i and i + 1
+#pragma unroll
+    for (int q = 0; q < kPagesPerLoader; ++q) pa[q] = pb[q] = -1;
     if (!wa.done()) {
-      pa0 = page_id(wa, lw); pa1 = page_id(wa, lw + kLoadWarps); wa.next();
+#pragma unroll
+      for (int q = 0; q < kPagesPerLoader; ++q) pa[q] = page_id(wa, pg0 + q);
+      wa.next();
     }
     if (!wa.done()) {
-      pb0 = page_id(wa, lw); pb1 = page_id(wa, lw + kLoadWarps); wa.next();
+#pragma unroll
+      for (int q = 0; q < kPagesPerLoader; ++q) pb[q] = page_id(wa, pg0 + q);
+      wa.next();
     }
     int i = 0, t = 0;    // block and segment of this CTA
     while (!w.done()) {
       const int Lb = seqL[w.b];
-      const int pid0 = pa0, pid1 = pa1;
       if (w.first() && lt == 0) {
         // Q rows of (b, h) by TMA: row m = r * g + j holds q[b][r][h*g + j],
         // the box {64, g, K} of the [B][K][Hq][128] tensor, per 64 columns.
@@ -714,11 +729,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int page[kPagesPerLoader], valid[kPagesPerLoader];
 #pragma unroll
       for (int q = 0; q < kPagesPerLoader; ++q) {
-        const int k = lw + q * kLoadWarps;
+        const int k = pg0 + q;
         const int uidx = w.idx0 + w.k + k;
         use[q] = k < w.nu();
         tail[q] = use[q] && uidx == w.units - 1;
-        int pg = q == 0 ? pid0 : pid1;
+        int pg = pa[q];
         const bool bad = use[q] && !tail[q] && (pg < 0 || pg >= p.P);
         if (bad) {
           if (lane == 0) report(p.status, ISD_ERR_BAD_PAGE);
@@ -728,114 +743,107 @@ __global__ void __launch_bounds__(kThreads, 1)
         valid[q] = Lb - uidx * kPage;          // >= 1 for a cached unit
         part[q] = use[q] && !tail[q] && !bad && valid[q] < kPage;
       }
-      // K tiles.  Rows past K of the tail lie outside the staging tensor
-      // and read as zeros.
-      const int ks = i % SK;
-      wait_or_fail(&k_empty[ks], ((i / SK) & 1) ^ 1, failed);
-      if (lane == 0) {
+      // This lane's box: page q = lane / 2 (lanes 0..7), half lane % 2.
+      const int lq = (lane >> 1) & (kPagesPerLoader - 1), hb = lane & 1;
+      bool l_use = false, l_tail = false, l_part = false;
+      int l_page = 0;
+#pragma unroll
+      for (int q = 0; q < kPagesPerLoader; ++q)
+        if (q == lq) {
+          l_use = use[q]; l_tail = tail[q]; l_part = part[q]; l_page = page[q];
+        }
+      l_use = l_use && lane < 2 * kPagesPerLoader;
+      const uint32_t box_off = (pg0 + lq) * 2048 + hb * kKH;
+      if (is_k) {
+        // K tiles.  Rows past K of the tail lie outside the staging tensor
+        // and read as zeros.
+        const int ks = i % SK;
+        int n_use = 0;
+#pragma unroll
+        for (int q = 0; q < kPagesPerLoader; ++q) n_use += use[q] ? 1 : 0;
+        wait_or_fail(&k_empty[ks], ((i / SK) & 1) ^ 1, failed);
+        if (lane == 0) mbar_expect_tx(&k_full[ks], (uint32_t)(n_use * 4096));
+        __syncwarp();
+        if (l_use) {
+          uint8_t* kd = kr + ks * kTile + box_off;
+          if (l_tail)
+            tma_load_4d(kd, &tm_kn, &k_full[ks], hb * 64, w.h, 0, w.b);
+          else
+            tma_load_4d(kd, &tm_kc, &k_full[ks], hb * 64, 0, w.h, l_page);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&k_full[ks]);
+      } else {
+        // V tiles.  A partial last page's V takes cp.async: slots past L_b
+        // are zero-filled, never copied (they may hold any bits, and
+        // 0 * NaN would reach O through P V).  K there is harmless: those
+        // scores are masked.
+        const int vs = i % SV;
+        int n_box = 0;
+        bool partial_v = false;
 #pragma unroll
         for (int q = 0; q < kPagesPerLoader; ++q) {
-          if (!use[q]) continue;
-          uint8_t* kd = kr + ks * kTile + (lw + q * kLoadWarps) * 2048;
-          mbar_expect_tx(&k_full[ks], 2 * 2048);
-          for (int hb = 0; hb < 2; ++hb) {
-            if (tail[q])
-              tma_load_4d(kd + hb * kKH, &tm_kn, &k_full[ks], hb * 64, w.h, 0, w.b);
-            else
-              tma_load_4d(kd + hb * kKH, &tm_kc, &k_full[ks], hb * 64, 0, w.h,
-                          page[q]);
-          }
+          n_box += (use[q] && !part[q]) ? 1 : 0;
+          partial_v = partial_v || part[q];
         }
-        mbar_arrive(&k_full[ks]);
-      }
-      // V tiles.  A partial last page's V takes cp.async: slots past L_b
-      // are zero-filled, never copied (they may hold any bits, and 0 * NaN
-      // would reach O through P V).  K there is harmless: those scores are
-      // masked.
-      const int vs = i % SV;
-      wait_or_fail(&v_empty[vs], ((i / SV) & 1) ^ 1, failed);
-      bool partial_v = false;
+        wait_or_fail(&v_empty[vs], ((i / SV) & 1) ^ 1, failed);
+        if (lane == 0) mbar_expect_tx(&v_full[vs], (uint32_t)(n_box * 4096));
+        __syncwarp();
+        if (l_use && !l_part) {
+          uint8_t* vd = vr + vs * kTile + box_off;
+          if (l_tail)
+            tma_load_4d(vd, &tm_vn, &v_full[vs], hb * 64, w.h, 0, w.b);
+          else
+            tma_load_4d(vd, &tm_vc, &v_full[vs], hb * 64, 0, w.h, l_page);
+        }
+        if (partial_v) {
 #pragma unroll
-      for (int q = 0; q < kPagesPerLoader; ++q) {
-        if (!use[q]) continue;
-        const int k = lw + q * kLoadWarps;
-        uint8_t* vd = vr + vs * kTile + k * 2048;
-        if (!part[q]) {
-          if (lane == 0) {
-            mbar_expect_tx(&v_full[vs], 2 * 2048);
-            for (int hb = 0; hb < 2; ++hb) {
-              if (tail[q])
-                tma_load_4d(vd + hb * kKH, &tm_vn, &v_full[vs], hb * 64, w.h, 0,
-                            w.b);
-              else
-                tma_load_4d(vd + hb * kKH, &tm_vc, &v_full[vs], hb * 64, 0, w.h,
-                            page[q]);
+          for (int q = 0; q < kPagesPerLoader; ++q) {
+            if (!part[q]) continue;
+            const int k = pg0 + q;
+            for (int e = lane; e < kPage * 16; e += 32) {
+              const int row = e >> 4, ch = e & 15;
+              const int key = k * kPage + row;
+              const uint32_t dst = vr_s + vs * kTile + (ch >> 3) * kKH +
+                                   key * 128 + (((ch & 7) ^ (key & 7)) << 4);
+              const bool in = row < valid[q];
+              const __nv_bfloat16* src =
+                  in ? p.vc + (((size_t)page[q] * Hkv + w.h) * kPage + row) * D +
+                           ch * 8
+                     : p.vc;
+              cp_async_16(dst, src, in ? 16u : 0u);
             }
           }
-          continue;
+          asm volatile("cp.async.wait_all;" ::: "memory");
+          proxy_fence();
         }
-        partial_v = true;
-        for (int e = lane; e < kPage * 16; e += 32) {
-          const int row = e >> 4, ch = e & 15;
-          const int key = k * kPage + row;
-          const uint32_t dst = vr_s + vs * kTile + (ch >> 3) * kKH + key * 128 +
-                               (((ch & 7) ^ (key & 7)) << 4);
-          const bool in = row < valid[q];
-          const __nv_bfloat16* src =
-              in ? p.vc + (((size_t)page[q] * Hkv + w.h) * kPage + row) * D +
-                       ch * 8
-                 : p.vc;
-          cp_async_16(dst, src, in ? 16u : 0u);
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&v_full[vs]);
       }
-      if (partial_v) {
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        proxy_fence();
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&v_full[vs]);
       w.next();
-      pa0 = pb0; pa1 = pb1;
-      pb0 = pb1 = -1;
+#pragma unroll
+      for (int q = 0; q < kPagesPerLoader; ++q) {
+        pa[q] = pb[q];
+        pb[q] = -1;
+      }
       if (!wa.done()) {
-        pb0 = page_id(wa, lw); pb1 = page_id(wa, lw + kLoadWarps); wa.next();
+#pragma unroll
+        for (int q = 0; q < kPagesPerLoader; ++q) pb[q] = page_id(wa, pg0 + q);
+        wa.next();
       }
       ++i;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kMmaWarp) {
-    // -------------------------------------------------------------- MMA
+    // ---------------------------------------------------------- QK MMA
     BlockWalk w;
     w.init(prefix, B, Hkv, u0, u1);
     int i = 0, t = -1;   // block and segment of this CTA
-    int prev_nu = 0, prev_pb = 0, prev_t = 0;
-    bool prev_first = false, have_prev = false;
     const uint32_t id_qk = idesc_bf16(128, N, 0, 0);
-    const uint32_t id_pv = idesc_bf16(128, N, 1, 1);
-    auto issue_pv = [&](int j_blk) {
-      // O^T += V^T P^T for block j_blk: one k-step of 16 keys per page.
-      const int vs = j_blk % SV;
-      wait_or_fail(&p_full[prev_pb], (j_blk / NPB) & 1, failed);
-      wait_or_fail(&v_full[vs], (j_blk / SV) & 1, failed);
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t pa = p_s + prev_pb * PB;
-        const uint32_t vb = vr_s + vs * kTile;
-        for (int j = 0; j < prev_nu; ++j)
-          umma(tmem + kO + (prev_t % NOB) * N, sdesc(vb + j * 2048, kKH, 1024),
-               sdesc(pa + j * 1024, PA, 512, 4), id_pv,
-               (prev_first && j == 0) ? 0u : 1u);
-        umma_commit(&v_empty[vs]);
-        umma_commit(&p_empty[prev_pb]);
-      }
-      __syncwarp();
-    };
     while (!w.done()) {
       const int ks = i % SK, sbuf = i & 1;
       if (w.first()) {
         ++t;
-        // Q, K and V arrive by TMA (a partial page's V by cp.async that its
-        // loader warp fences before arriving).
         wait_or_fail(&q_full[t % NQB], (t / NQB) & 1, failed);
       }
       const int qb = t % NQB;
@@ -843,38 +851,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_or_fail(&s_free[sbuf], ((i >> 1) & 1) ^ 1, failed);
       tc_fence_after();
       if (lane == 0) {
-        // S^T = K Q^T over the 128 keys of the tile (rows of pages past
-        // the block's end hold stale data; their scores are masked).
         const uint32_t kb = kr_s + ks * kTile;
         for (int kk = 0; kk < 8; ++kk)
           umma(tmem + kS + sbuf * N,
                sdesc(kb + (kk >> 2) * kKH + (kk & 3) * 32, 16, 1024),
                sdesc(q_s + qb * QB + (kk >> 2) * QH + (kk & 3) * 32, 16, 1024),
-               id_qk,
-               kk > 0 ? 1u : 0u);
+               id_qk, kk > 0 ? 1u : 0u);
         umma_commit(&s_full[sbuf]);
         umma_commit(&k_empty[ks]);
         if (w.last()) umma_commit(&q_empty[qb]);
       }
       __syncwarp();
-      if (have_prev) {
-        // The first P V of segment t overwrites O^T buffer t % NOB: the
-        // epilogue of segment t - NOB must have read it.
-        if (prev_first && prev_t >= NOB)
-          wait_or_fail(&o_free[prev_t % NOB], ((prev_t / NOB) & 1) ^ 1, failed);
-        issue_pv(i - 1);
-      }
-      have_prev = true;
-      prev_nu = w.nu(); prev_pb = i % NPB; prev_first = w.first(); prev_t = t;
       w.next();
       ++i;
     }
-    if (have_prev) {
-      if (prev_first && prev_t >= NOB)
-        wait_or_fail(&o_free[prev_t % NOB], ((prev_t / NOB) & 1) ^ 1, failed);
-      issue_pv(i - 1);
+    if (lane == 0) umma_commit(fin);
+    __syncwarp();
+    bool fin_failed = false;
+    wait_or_fail(fin, 0, fin_failed);
+    failed = failed || fin_failed;
+  } else if (warp == kPvWarp) {
+    // ---------------------------------------------------------- P V MMA
+    BlockWalk w;
+    w.init(prefix, B, Hkv, u0, u1);
+    int i = 0, t = -1;
+    const uint32_t id_pv = idesc_bf16(128, N, 1, 1);
+    while (!w.done()) {
+      const bool first = w.first();
+      if (first) ++t;
+      const int pb = i % NPB, vs = i % SV;
+      // The first P V of segment t overwrites O^T buffer t % NOB: the
+      // epilogue of segment t - NOB must have read it.
+      if (first && t >= NOB)
+        wait_or_fail(&o_free[t % NOB], ((t / NOB) & 1) ^ 1, failed);
+      wait_or_fail(&p_full[pb], (i / NPB) & 1, failed);
+      wait_or_fail(&v_full[vs], (i / SV) & 1, failed);
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t pa = p_s + pb * PB;
+        const uint32_t vb = vr_s + vs * kTile;
+        const int nu = w.nu();
+        for (int j = 0; j < nu; ++j)
+          umma(tmem + kO + (t % NOB) * N, sdesc(vb + j * 2048, kKH, 1024),
+               sdesc(pa + j * 1024, PA, 512, 4), id_pv,
+               (first && j == 0) ? 0u : 1u);
+        umma_commit(&v_empty[vs]);
+        umma_commit(&p_empty[pb]);
+      }
+      __syncwarp();
+      w.next();
+      ++i;
     }
-    // Every MMA this CTA issued has completed before TMEM is released.
     if (lane == 0) umma_commit(fin);
     __syncwarp();
     bool fin_failed = false;
@@ -1134,33 +1161,41 @@ static bool encode_tiled_4d(CUtensorMap* m, const void* base,
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
-// Dynamic shared memory of the kernel for N = 32 * nch rows and a V ring
-// of `sv` tiles (Q and P buffer counts as in the kernel).
-static size_t tc_smem(int B, int nch, int sv) {
+// Dynamic shared memory of the kernel for N = 32 * nch rows, a K ring of
+// `sk` and a V ring of `sv` tiles.
+static size_t tc_smem(int B, int nch, int sk, int sv) {
   const size_t N = 32 * (size_t)nch;
-  const size_t nqb = nch == 4 ? 1 : 2, npb = nch >= 3 ? 1 : 2;
-  return 1024 + (size_t)(tc::kKStages + sv) * tc::kTile + nqb * 2 * N * 128 +
-         npb * 2 * N * 128 + tc::kBarBytes + 16 + (size_t)(2 * B + 1) * 4;
+  return 1024 + (size_t)(sk + sv) * tc::kTile +
+         (size_t)tc::nqb_of(nch) * 2 * N * 128 +
+         (size_t)tc::npb_of(nch) * 2 * N * 128 + tc::kBarBytes + 16 +
+         (size_t)(2 * B + 1) * 4;
 }
 
-// Deepest V ring (at most 4, at least 2 tiles) that fits for M query rows;
-// 0 if none does.
-static int tc_vstages(int B, int M) {
+// K and V ring depths, the first of these that fits next to Q, P and the
+// unit prefix (the deeper a ring, the more bytes each SM keeps in flight;
+// a K tile is held for its QK products, a V tile until its block's
+// softmax and P V are done).
+struct Stages {
+  int sk, sv;
+};
+constexpr Stages kStagePrefs[] = {{2, 4}, {2, 3}, {2, 2}};
+
+static Stages tc_stages(int B, int M) {
   const int nch = (M + 31) / 32;
-  for (int s = tc::kMaxVStages; s >= 2; --s)
-    if (tc_smem(B, nch, s) + tc::kStaticSmem <= kSmemLimit) return s;
-  return 0;
+  for (const Stages& st : kStagePrefs)
+    if (tc_smem(B, nch, st.sk, st.sv) + tc::kStaticSmem <= kSmemLimit) return st;
+  return Stages{0, 0};
 }
 
 size_t attn_tc_smem_bytes(int B, int M) {
-  const int s = tc_vstages(B, M);
-  return s ? tc_smem(B, (M + 31) / 32, s) : (size_t)-1;
+  const Stages st = tc_stages(B, M);
+  return st.sk ? tc_smem(B, (M + 31) / 32, st.sk, st.sv) : (size_t)-1;
 }
 
 bool attn_tc_supported(const isd_attn_args* a) {
   const int M = a->K * (a->Hq / a->Hkv);
   return a->dtype == ISD_BF16 && a->d == 128 && M >= 1 && M <= 128 &&
-         a->K <= kPage && tc_vstages(a->B, M) > 0;
+         a->K <= kPage && tc_stages(a->B, M).sk > 0;
 }
 
 int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
@@ -1168,8 +1203,10 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
   p.B = a->B; p.Hq = a->Hq; p.Hkv = a->Hkv; p.K = a->K;
   p.g = a->Hq / a->Hkv; p.M = a->K * p.g; p.P = a->num_pages;
   p.stride = a->page_table_stride;
-  p.sv = tc_vstages(a->B, p.M);
-  if (p.sv == 0) return ISD_ERR_UNSUPPORTED;
+  const Stages stg = tc_stages(a->B, p.M);
+  if (stg.sk == 0) return ISD_ERR_UNSUPPORTED;
+  p.sk = stg.sk;
+  p.sv = stg.sv;
   p.scale_log2 = a->softmax_scale * kLog2e;
   p.q = static_cast<const __nv_bfloat16*>(a->q);
   p.vc = static_cast<const __nv_bfloat16*>(a->v_cache);
@@ -1238,7 +1275,7 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
       return ISD_ERR_CUDA;
   }
   const int nch = (p.M + 31) / 32;
-  const size_t smem = tc_smem(a->B, nch, p.sv);
+  const size_t smem = tc_smem(a->B, nch, p.sk, p.sv);
   auto kern = nch == 1 ? tc::attn_tc_kernel<1>
             : nch == 2 ? tc::attn_tc_kernel<2>
             : nch == 3 ? tc::attn_tc_kernel<3>
