@@ -45,7 +45,11 @@ constexpr int kStatsWarps = 16;            // stats CTA: 512 threads
 constexpr int kDrawWarps = 8;              // draw CTA: 256 threads
 constexpr int kResidPerCta = 4;            // residual sub-chunks per draw CTA
 constexpr int kWarpElems = kSub / kDrawWarps;   // a draw warp's share: 256
-static_assert(kDrawWarps == 2 * kResidPerCta, "two warps per residual sub-chunk");
+// Warps per residual sub-chunk and the 8-element groups each lane sums.
+constexpr int kResidWarps = kDrawWarps / kResidPerCta;
+constexpr int kResidGroups = kSub / kResidWarps / 256;
+static_assert(kDrawWarps % kResidPerCta == 0 && kResidGroups >= 1,
+              "whole warps per residual sub-chunk");
 static_assert(kWarpElems == 32 * 8, "a draw lane scans 8 elements");
 
 template <typename T>
@@ -794,26 +798,28 @@ __global__ void __launch_bounds__(kDrawWarps * 32)
   const bool rejected = sh.rejected;
   const int a = sh.a;
   if (rejected) {
-    // ---- 3a. Residual sub-chunk sums: part y takes sub-chunks 4y .. 4y+3,
-    //          two warps each (1024 elements, 32 a lane), in fixed order.
+    // ---- 3a. Residual sub-chunk sums: part y takes sub-chunks
+    //          kResidPerCta y .. + kResidPerCta - 1, kResidWarps warps each,
+    //          in fixed order.
     const int nparts = (p.C + kResidPerCta - 1) / kResidPerCta;
     if (y >= nparts) return;
     const T* prow;
     const T* qrow;
     const ResidRows rr = resid_rows(p, b, a, sh.m[a], sh.s[a], prow, qrow);
-    const int c = y * kResidPerCta + (warp >> 1), half = warp & 1;
+    const int c = y * kResidPerCta + warp / kResidWarps;
+    const int part = warp % kResidWarps;
     double s = 0.0;
     if (c < p.C) {
-      const int lo = c * kSub + half * (kSub / 2);
+      const int lo = c * kSub + part * (kSub / kResidWarps);
       const int hi = min(p.V, c * kSub + kSub);
-      Raw8<T> vp[4], vq[4];
+      Raw8<T> vp[kResidGroups], vq[kResidGroups];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < kResidGroups; ++k) {
         vp[k] = load_raw8<kVec>(prow, lo + (k * 32 + lane) * 8, hi);
         if (rr.x < 0) vq[k] = load_raw8<kVec>(qrow, lo + (k * 32 + lane) * 8, hi);
       }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < kResidGroups; ++k) {
         const int idx = lo + (k * 32 + lane) * 8;
         float t = 0.0f;
 #pragma unroll
@@ -828,7 +834,10 @@ __global__ void __launch_bounds__(kDrawWarps * 32)
     if (threadIdx.x == 0) {
       for (int i = 0; i < kResidPerCta; ++i) {
         const int ci = y * kResidPerCta + i;
-        if (ci < p.C) p.resid[(size_t)b * p.C + ci] = sh.tot[2 * i] + sh.tot[2 * i + 1];
+        if (ci >= p.C) continue;
+        double r = 0.0;
+        for (int k = 0; k < kResidWarps; ++k) r += sh.tot[kResidWarps * i + k];
+        p.resid[(size_t)b * p.C + ci] = r;
       }
       __threadfence();
       sh.last = atomicAdd(&p.count[b], 1) == nparts - 1;

@@ -27,10 +27,11 @@
 //                       a K copy; a warp covers 4 pages of every block and
 //                       its lanes 0..7 issue the 8 TMA boxes (64-column
 //                       halves, 128-byte swizzle) in one instruction.  A
-//                       partial last page takes V by cp.async so that its
-//                       unused slots are zero-filled.  Page ids are read
-//                       two blocks ahead.  Warp 0 also loads each segment's
-//                       Q rows by TMA.
+//                       partial last page is loaded from valid - 16 rows
+//                       up, so its slots past L_b read as zeros (from
+//                       outside the tensor) and its keys take the last
+//                       slots.  Page ids are read two blocks ahead.  Warp 0
+//                       also loads each segment's Q rows by TMA.
 //   QK MMA warp         one thread issues S^T of block i into a double-
 //                       buffered S in TMEM and commits completion.  It
 //                       also allocates and frees TMEM.
@@ -65,7 +66,6 @@ void attn_partial_ptrs(const isd_attn_args* a, int G, float** part_o,
 
 namespace tc {
 
-constexpr int D = 128;
 constexpr int kNB = 8;                       // pages per block
 constexpr int kKeys = kNB * kPage;           // 128 keys = TMEM lanes
 constexpr int kKH = kKeys * 128;             // one 64-column half of K or V
@@ -745,12 +745,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // This lane's box: page q = lane / 2 (lanes 0..7), half lane % 2.
       const int lq = (lane >> 1) & (kPagesPerLoader - 1), hb = lane & 1;
-      bool l_use = false, l_tail = false, l_part = false;
-      int l_page = 0;
+      bool l_use = false, l_tail = false;
+      int l_page = 0, l_row = 0;
 #pragma unroll
       for (int q = 0; q < kPagesPerLoader; ++q)
         if (q == lq) {
-          l_use = use[q]; l_tail = tail[q]; l_part = part[q]; l_page = page[q];
+          l_use = use[q]; l_tail = tail[q]; l_page = page[q];
+          // A partial page starts valid - 16 rows up: its slots past L_b
+          // are read from outside the tensor, as zeros, and its keys land
+          // in the last `valid` slots (K and V alike).
+          l_row = part[q] ? valid[q] - kPage : 0;
         }
       l_use = l_use && lane < 2 * kPagesPerLoader;
       const uint32_t box_off = (pg0 + lq) * 2048 + hb * kKH;
@@ -769,53 +773,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (l_tail)
             tma_load_4d(kd, &tm_kn, &k_full[ks], hb * 64, w.h, 0, w.b);
           else
-            tma_load_4d(kd, &tm_kc, &k_full[ks], hb * 64, 0, w.h, l_page);
+            tma_load_4d(kd, &tm_kc, &k_full[ks], hb * 64, l_row, w.h, l_page);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&k_full[ks]);
       } else {
-        // V tiles.  A partial last page's V takes cp.async: slots past L_b
-        // are zero-filled, never copied (they may hold any bits, and
-        // 0 * NaN would reach O through P V).  K there is harmless: those
-        // scores are masked.
+        // V tiles, placed like the K tiles: the zeros a partial page reads
+        // above its first key matter here (its slots past L_b may hold any
+        // bits, and 0 * NaN would reach O through P V).
         const int vs = i % SV;
-        int n_box = 0;
-        bool partial_v = false;
+        int n_use = 0;
 #pragma unroll
-        for (int q = 0; q < kPagesPerLoader; ++q) {
-          n_box += (use[q] && !part[q]) ? 1 : 0;
-          partial_v = partial_v || part[q];
-        }
+        for (int q = 0; q < kPagesPerLoader; ++q) n_use += use[q] ? 1 : 0;
         wait_or_fail(&v_empty[vs], ((i / SV) & 1) ^ 1, failed);
-        if (lane == 0) mbar_expect_tx(&v_full[vs], (uint32_t)(n_box * 4096));
+        if (lane == 0) mbar_expect_tx(&v_full[vs], (uint32_t)(n_use * 4096));
         __syncwarp();
-        if (l_use && !l_part) {
+        if (l_use) {
           uint8_t* vd = vr + vs * kTile + box_off;
           if (l_tail)
             tma_load_4d(vd, &tm_vn, &v_full[vs], hb * 64, w.h, 0, w.b);
           else
-            tma_load_4d(vd, &tm_vc, &v_full[vs], hb * 64, 0, w.h, l_page);
-        }
-        if (partial_v) {
-#pragma unroll
-          for (int q = 0; q < kPagesPerLoader; ++q) {
-            if (!part[q]) continue;
-            const int k = pg0 + q;
-            for (int e = lane; e < kPage * 16; e += 32) {
-              const int row = e >> 4, ch = e & 15;
-              const int key = k * kPage + row;
-              const uint32_t dst = vr_s + vs * kTile + (ch >> 3) * kKH +
-                                   key * 128 + (((ch & 7) ^ (key & 7)) << 4);
-              const bool in = row < valid[q];
-              const __nv_bfloat16* src =
-                  in ? p.vc + (((size_t)page[q] * Hkv + w.h) * kPage + row) * D +
-                           ch * 8
-                     : p.vc;
-              cp_async_16(dst, src, in ? 16u : 0u);
-            }
-          }
-          asm volatile("cp.async.wait_all;" ::: "memory");
-          proxy_fence();
+            tma_load_4d(vd, &tm_vc, &v_full[vs], hb * 64, l_row, w.h, l_page);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&v_full[vs]);
@@ -833,7 +811,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ++i;
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- QK MMA
     BlockWalk w;
@@ -962,7 +939,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int uidx = w.idx0 + w.k + kp;
       const bool in_blk = kp < w.nu();
       const bool tail = in_blk && uidx == w.units - 1;
-      const bool key_all = in_blk && !tail && rr < L - uidx * kPage;
+      // A cached page holding v < 16 keys keeps them in its last v slots.
+      const bool key_all = in_blk && !tail && rr >= kPage - (L - uidx * kPage);
       const int col_min =
           (tail && rr < p.K) ? rr * p.g : (key_all ? 0 : (1 << 30));
       wait_or_fail(&s_full[sbuf], (i >> 1) & 1, failed);

@@ -197,9 +197,12 @@ ISD_DEV int block_exclusive_scan_int(int n, F in, S store, int* sh) {
 // per KV head h: its cached pages, then one tail unit) is cut into G
 // contiguous ranges of equal cost, a unit costing 1 and each (b, h) segment
 // kSegCost more for its fixed work (Q load, first-block max, epilogue), so
-// CTAs that meet many short sequences get fewer pages.
+// CTAs that meet many short sequences get fewer pages.  Measured on the
+// C=64 step: a segment boundary costs about what 30-40 pages of streaming
+// do (per-CTA times fitted against blocks and segments), and costs of 32 to
+// 40 balance the CTAs best (36: attention 4% faster than 16).
 
-constexpr int kSegCost = 16;
+constexpr int kSegCost = 36;
 
 // First unit of CTA c (c = G gives T).  prefix[b] = first unit of sequence
 // b for b < B; T = total units; every segment of b has the same length.
