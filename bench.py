@@ -74,12 +74,13 @@ def parse():
 
 # DRAM traffic of the attention kernel per algorithmic byte, from one ncu
 # capture of the C=64 workload at B = 16 (dram__bytes_read.sum +
-# dram__bytes_write.sum over the launch's algorithmic bytes).  Traffic tracks
-# the algorithmic bytes, so a full launch's traffic is this ratio times its
-# bytes.  Valid only for the kernel source the capture was taken on (None:
-# no capture of the current source).
-TRAFFIC_PER_ALGO_BYTE = None
-TRAFFIC_KERNEL_SHA256 = None
+# dram__bytes_write.sum over the launch's algorithmic bytes; see
+# profiles/attn_tc_kernel_c64_b16_full.md).  Traffic tracks the algorithmic
+# bytes, so a full launch's traffic is this ratio times its bytes.  Valid
+# only for the kernel source the capture was taken on.
+TRAFFIC_PER_ALGO_BYTE = (331.52 + 8.32) / 332.37
+TRAFFIC_KERNEL_SHA256 = (
+    "96f069e3db985f272e1d85995a5c1efd24e57f6e471c16c30d24a1932e37c2ea")
 
 
 def attention_traffic(bytes_per_launch):

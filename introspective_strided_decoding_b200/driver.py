@@ -186,6 +186,6 @@ class Decoder:
     def launches_per_step(self):
         """This library's kernel launches per step: attention (bf16: the
         tcgen05 kernel and the split-segment combine; fp32: one kernel),
-        the three accept kernels (statistics, decide, draws) and the
+        the two accept kernels (statistics; decision and draws) and the
         commit."""
-        return (2 if self.w.dtype == "bf16" else 1) + 3 + 1
+        return (2 if self.w.dtype == "bf16" else 1) + 2 + 1
