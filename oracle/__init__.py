@@ -26,6 +26,8 @@ vocab      softmax statistics, probabilities and the inverse CDF.
 step       the accept / resample / bonus / draft step and the KV commit.
 tpf        the tokens-per-forward closed form, the Markov chain behind it,
            and a finite-horizon expectation.
+lm_head    the LM head that makes the logits, the R-ISD gated LoRA at MASK
+           rows, bfloat16 rounding and sub-chunk vocabulary statistics.
 
 Every floating-point quantity is computed in float64 with plain numpy.
 """
