@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define ISD_ABI_VERSION 3
+#define ISD_ABI_VERSION 4
 #define ISD_PAGE_SIZE 16
 
 /* Return / status codes. */
@@ -176,6 +176,9 @@ int isd_attn_strided(const isd_attn_args* a, void* stream);
  * state is malformed gets ISD_ERR_BAD_STATE in *status (if given),
  * n_commit 0 and its state copied through unchanged.
  * Workspace: isd_accept_workspace_bytes(args) bytes; no initialisation.
+ * vocab_stats (optional, 16-byte aligned): the figures isd_lm_head wrote for
+ * the same logits_cur; the row statistics of step 1 are then merged from
+ * them and logits_cur is read only where the ratio tests and draws need it.
  * ---------------------------------------------------------------------- */
 typedef struct {
   int32_t B, N, K, V;
@@ -204,6 +207,10 @@ typedef struct {
                                   memory instead of `step` (lets one
                                   captured CUDA graph serve every step)    */
   int32_t proposal;            /* ISD_PROPOSAL_SAMPLE or _ARGMAX          */
+  const void* vocab_stats;     /* optional: the sub-chunk statistics of
+                                  logits_cur written by isd_lm_head (M =
+                                  B * K rows); when given, step 1 takes
+                                  them instead of reading logits_cur      */
 } isd_accept_args;
 
 #define ISD_PROPOSAL_SAMPLE 0  /* drafts drawn from q (default)           */
@@ -288,6 +295,63 @@ typedef struct {
 
 size_t isd_commit_workspace_bytes(const isd_commit_args* a);
 int isd_kv_commit(const isd_commit_args* a, void* stream);
+
+/* ------------------------------------------------------------------------
+ * isd_lm_head -- the LM head that makes a step's logits, with the R-ISD
+ * gated LoRA at MASK rows and the vocabulary statistics of every row.
+ *
+ * One forward pass gives every row of the stride its distribution over the
+ * vocabulary, p at the clean rows and q at the MASK rows (summary,
+ * "Inference & ISD"); a row's logits are its final hidden state times the
+ * output embedding.  R-ISD adds a rank-r LoRA (r = 128 on the pages) that
+ * acts only at MASK positions, so the clean rows stay the base model's
+ * (summary, "Speedup Factor Explorer", R-ISD):
+ *
+ *   logits[m][v] = sum_d hidden[m][d] weight[v][d]
+ *                + gate_m sum_j U[m][j] lora_b[v][j],
+ *   U[m][j] = bf16(lora_scale * sum_d hidden[m][d] lora_a[j][d]),
+ *
+ * gate_m = 1 when row m is a MASK row (stride row m % rows_per_seq >=
+ * n_pending[m / rows_per_seq]), else 0.  Sums are accumulated in fp32 on the
+ * tensor cores and the logits are rounded to bf16 (nearest, ties to even).
+ * A sequence whose n_pending lies outside [0, rows_per_seq] gets no LoRA and
+ * ISD_ERR_BAD_STATE in *status.
+ *
+ * vocab_stats (optional): for every row m and vocabulary sub-chunk c of
+ * 2048 entries (C = ceil(V / 2048), the last one ragged), computed from the
+ * bf16 logits as stored: csum f64 [M][C] (sum of exp(l - max)), then cmax
+ * f32 [M][C] (the max), then cidx int32 [M][C] (first index of the max in
+ * the row), packed in that order from vocab_stats; isd_vocab_stats_bytes(M,
+ * V) bytes.  isd_accept_resample takes them through its vocab_stats field.
+ *
+ * Layouts: hidden bf16 [M][D]; weight bf16 [V][D] (one row per vocabulary
+ * entry); logits bf16 [M][V]; lora_a bf16 [r][D]; lora_b bf16 [V][r];
+ * n_pending int32 [M / rows_per_seq].  Sizes: D a multiple of 64; V a
+ * multiple of 8; r = 0 (no LoRA) or a multiple of 64 up to 256; M >= 1.
+ * Every pointer 16-byte aligned.  Workspace: isd_lm_head_workspace_bytes
+ * (args) bytes; no initialisation.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int32_t M, D, V;
+  int32_t dtype;               /* ISD_BF16                                */
+  const void* hidden;
+  const void* weight;
+  void* logits;
+  void* vocab_stats;           /* optional                                */
+  int32_t lora_rank;           /* 0: no LoRA                              */
+  int32_t rows_per_seq;        /* K of the stride (LoRA only)             */
+  const void* lora_a;
+  const void* lora_b;
+  const int32_t* n_pending;    /* LoRA only                               */
+  float lora_scale;
+  int32_t* status;             /* optional                                */
+  void* workspace;
+  size_t workspace_bytes;
+} isd_lm_head_args;
+
+size_t isd_lm_head_workspace_bytes(const isd_lm_head_args* a);
+size_t isd_vocab_stats_bytes(int32_t M, int32_t V);
+int isd_lm_head(const isd_lm_head_args* a, void* stream);
 
 /* Utilities. */
 int isd_abi_version(void);

@@ -55,6 +55,7 @@ static_assert(kWarpElems == 32 * 8, "a draw lane scans 8 elements");
 template <typename T>
 struct AcceptDev {
   int B, N, K, V, C, RU;
+  int SR;              // rows per sequence in the sub-chunk arrays
   uint32_t step;
   const uint32_t* step_dev;  // when set, the step index is read from here
   uint64_t seed;
@@ -75,9 +76,9 @@ struct AcceptDev {
   float* ratio_out;
   int32_t* status;
   // workspace
-  double* csum;        // [B][RU][C] sub-chunk sum of exp(l - sub-chunk max)
-  float* cmax;         // [B][RU][C] sub-chunk max
-  int32_t* cidx;       // [B][RU][C] first index of the sub-chunk max
+  double* csum;        // [B][SR][C] sub-chunk sum of exp(l - sub-chunk max)
+  float* cmax;         // [B][SR][C] sub-chunk max
+  int32_t* cidx;       // [B][SR][C] first index of the sub-chunk max
   double* resid;       // [B][C] residual sub-chunk mass
   int32_t* count;      // [B] residual parts finished (zeroed by stats)
   int argmax;          // drafts are argmax q (point-mass proposals)
@@ -222,7 +223,7 @@ ISD_DEV void reduce_sub(const AcceptDev<T>& p, int b, int j, int c,
     s += (double)t;
   }
   s = warp_sum_f64(s);
-  const size_t o = ((size_t)b * p.RU + j) * p.C + c;
+  const size_t o = ((size_t)b * p.SR + j) * p.C + c;
   if (p.argmax) {
     const int lo = c * kSub;
     int first = INT_MAX;
@@ -489,7 +490,7 @@ template <typename T>
 ISD_DEV void merge_row(const AcceptDev<T>& p, int b, int r, float& m_out,
                        double& s_out, double* mass) {
   const int lane = threadIdx.x & 31;
-  const size_t o = ((size_t)b * p.RU + r) * p.C;
+  const size_t o = ((size_t)b * p.SR + r) * p.C;
   float cm[kSubPerLane];
   double cs[kSubPerLane];
   float m = -INFINITY;
@@ -541,7 +542,7 @@ ISD_DEV int cta_draw(const AcceptDev<T>& p, DrawShared& sh, int b, int mode,
     if (mode == 0 && !(total > 0.0)) {
       // Zero residual mass: draw from p of row `row` instead.
       mode = 1;
-      const size_t o = ((size_t)b * p.RU + row) * C;
+      const size_t o = ((size_t)b * p.SR + row) * C;
       own = 0.0;
 #pragma unroll
       for (int i = 0; i < kSubPerLane; ++i) {
@@ -864,7 +865,7 @@ __global__ void __launch_bounds__(kDrawWarps * 32)
     // Argmax draft: the first sub-chunk whose max is the row max holds the
     // first maximal index (exact compares of the same values).
     if (warp == 0) {
-      const size_t o = ((size_t)b * p.RU + row) * p.C;
+      const size_t o = ((size_t)b * p.SR + row) * p.C;
       const float m = sh.m[row];
       int first = INT_MAX;
 #pragma unroll
@@ -982,9 +983,16 @@ int launch_stats<__nv_bfloat16, true>(const AcceptDev<__nv_bfloat16>& p,
 
 template <typename T, bool kVec>
 static int launch_accept_kernels(const AcceptDev<T>& p, int sms,
-                                 cudaStream_t st) {
-  const int rc = launch_stats<T, kVec>(p, sms, st);
-  if (rc != ISD_OK) return rc;
+                                 cudaStream_t st, bool have_stats) {
+  if (have_stats) {
+    // The sub-chunk figures come from the LM head; only the residual
+    // counters the statistics kernel would have zeroed need clearing.
+    if (cudaMemsetAsync(p.count, 0, (size_t)p.B * 4, st) != cudaSuccess)
+      return ISD_ERR_CUDA;
+  } else {
+    const int rc = launch_stats<T, kVec>(p, sms, st);
+    if (rc != ISD_OK) return rc;
+  }
   const int parts = std::max((p.C + kResidPerCta - 1) / kResidPerCta, p.N);
   if (launch_pdl(accept_draw_kernel<T, kVec>, dim3(p.B, parts),
                  dim3(kDrawWarps * 32), 0, st, p) != cudaSuccess)
@@ -1015,14 +1023,27 @@ static int launch_accept_t(const isd_accept_args* a, cudaStream_t st) {
   p.cidx = reinterpret_cast<int32_t*>(ws + l.cidx);
   p.resid = reinterpret_cast<double*>(ws + l.resid);
   p.count = reinterpret_cast<int32_t*>(ws + l.count);
+  p.SR = p.RU;
+  const bool have_stats = a->vocab_stats != nullptr;
+  if (have_stats) {
+    // isd_lm_head's layout: csum, cmax, cidx, each [B * K][C].
+    const uint8_t* vs = static_cast<const uint8_t*>(a->vocab_stats);
+    const size_t rows = (size_t)a->B * a->K;
+    p.csum = const_cast<double*>(reinterpret_cast<const double*>(vs));
+    p.cmax = const_cast<float*>(
+        reinterpret_cast<const float*>(vs + rows * p.C * 8));
+    p.cidx = const_cast<int32_t*>(
+        reinterpret_cast<const int32_t*>(vs + rows * p.C * 12));
+    p.SR = a->K;
+  }
   p.argmax = a->proposal == ISD_PROPOSAL_ARGMAX;
   const int sms = num_sms();
   if (sms <= 0) return ISD_ERR_CUDA;
   // Vector loads need 16-byte aligned rows (logits_cur itself is checked
   // on the host) of whole 16-byte units.
   if (((size_t)a->V * sizeof(T)) % 16 == 0)
-    return launch_accept_kernels<T, true>(p, sms, st);
-  return launch_accept_kernels<T, false>(p, sms, st);
+    return launch_accept_kernels<T, true>(p, sms, st, have_stats);
+  return launch_accept_kernels<T, false>(p, sms, st, have_stats);
 }
 
 size_t accept_workspace_bytes(int B, int N, int K, int V) {

@@ -14,6 +14,9 @@ size_t attn_workspace_bytes_impl(int B, int M, int D, int G);
 size_t attn_tc_smem_bytes(int B, int M);
 int launch_attn_bf16(const isd_attn_args* a, int G, cudaStream_t st);
 int launch_attn_f32(const isd_attn_args* a, cudaStream_t st);
+size_t lm_head_workspace_bytes(const isd_lm_head_args* a);
+size_t vocab_stats_bytes(int M, int V);
+int launch_lm_head(const isd_lm_head_args* a, cudaStream_t st);
 }  // namespace isd
 
 namespace {
@@ -93,7 +96,8 @@ int accept_validate(const isd_accept_args* a) {
       (const void*)a->q_row_out == (const void*)a->q_row_in ||
       (const void*)a->q_stats_out == (const void*)a->q_stats_in)
     return ISD_ERR_INVALID_ARG;
-  if (!aligned16(a->logits_cur) || !aligned16(a->logits_prev))
+  if (!aligned16(a->logits_cur) || !aligned16(a->logits_prev) ||
+      !aligned16(a->vocab_stats))
     return ISD_ERR_INVALID_ARG;
   return ISD_OK;
 }
@@ -198,6 +202,49 @@ int isd_kv_commit(const isd_commit_args* a, void* stream) {
   if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace))
     return ISD_ERR_WORKSPACE;
   return isd::launch_commit(a, static_cast<cudaStream_t>(stream));
+}
+
+// --------------------------------------------------------------- LM head
+static int lm_head_check(const isd_lm_head_args* a) {
+  if (!a) return ISD_ERR_INVALID_ARG;
+  if (a->M <= 0 || a->D <= 0 || a->V <= 0 || a->lora_rank < 0)
+    return ISD_ERR_INVALID_ARG;
+  if (a->dtype != ISD_BF16) return ISD_ERR_UNSUPPORTED;
+  if (a->D % 64 != 0 || a->V % 8 != 0) return ISD_ERR_UNSUPPORTED;
+  if (a->lora_rank % 64 != 0 || a->lora_rank > 256) return ISD_ERR_UNSUPPORTED;
+  if (a->lora_rank > 0) {
+    if (a->rows_per_seq <= 0 || a->M % a->rows_per_seq != 0)
+      return ISD_ERR_INVALID_ARG;
+  }
+  return ISD_OK;
+}
+
+size_t isd_lm_head_workspace_bytes(const isd_lm_head_args* a) {
+  if (lm_head_check(a) != ISD_OK) return 0;
+  return isd::lm_head_workspace_bytes(a);
+}
+
+size_t isd_vocab_stats_bytes(int32_t M, int32_t V) {
+  if (M <= 0 || V <= 0) return 0;
+  return isd::vocab_stats_bytes(M, V);
+}
+
+int isd_lm_head(const isd_lm_head_args* a, void* stream) {
+  const int rc = lm_head_check(a);
+  if (rc != ISD_OK) return rc;
+  if (!a->hidden || !a->weight || !a->logits) return ISD_ERR_INVALID_ARG;
+  if (a->lora_rank > 0 && (!a->lora_a || !a->lora_b || !a->n_pending))
+    return ISD_ERR_INVALID_ARG;
+  if (!aligned16(a->hidden) || !aligned16(a->weight) ||
+      !aligned16(a->logits) || !aligned16(a->vocab_stats) ||
+      !aligned16(a->lora_a) || !aligned16(a->lora_b))
+    return ISD_ERR_INVALID_ARG;
+  if (a->logits == a->hidden || a->logits == a->weight)
+    return ISD_ERR_INVALID_ARG;
+  const size_t need = isd::lm_head_workspace_bytes(a);
+  if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace))
+    return ISD_ERR_WORKSPACE;
+  return isd::launch_lm_head(a, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -1,0 +1,555 @@
+// isd_lm_head: the LM head that produces a step's logits, on the 5th-
+// generation tensor cores, with the vocabulary statistics the accept step
+// consumes computed in the GEMM's epilogue and the R-ISD gated LoRA at MASK
+// rows.
+//
+// Method: "Introspective Diffusion Language Models", project summary
+// (hada.io).  One forward pass gives p at the clean rows and q at the MASK
+// rows ("Inference & ISD"); the logits of a row are its final hidden state
+// times the output embedding.  R-ISD adds a rank-128 LoRA that acts only at
+// MASK positions, so p stays the base model's ("Speedup Factor Explorer",
+// R-ISD): for a MASK row m
+//   logits[m] = h_m W^T + scale (h_m A^T) B^T,
+// computed as one contraction over the concatenated K axis
+//   [h_m | U_m] . [W | B]^T,  U_m = gate_m * scale * (h_m A^T)  (bf16),
+// with gate_m = 1 at MASK rows and 0 at clean rows, so the clean rows'
+// extra K steps multiply zeros.
+//
+// GEMM layout.  Rows (hidden states) take the MMA's M side and TMEM lanes,
+// vocabulary entries its N side (a tile of 256), so each epilogue thread
+// owns one row and reduces its row's statistics in registers.  A CTA keeps
+// RT = 2 accumulators of 128 rows that share the weight tile (256 rows x
+// 256 entries: 128 B of weight and hidden state loaded per 128 FLOPs
+// instead of per 85 for a single accumulator, which keeps the L2-to-SM
+// stream well under the L2's bandwidth); with 128 rows or fewer RT = 1 and
+// the two TMEM buffers let the epilogue of one tile overlap the next.
+//
+// Warp roles (10 warps): warp 0 issues the TMA loads of the stage ring (one
+// 64-wide K slice of the hidden rows and of the weight tile per stage),
+// warp 1 allocates TMEM and one thread issues the tcgen05 MMAs, warps 2..9
+// (RT = 2; warps 2..5 for RT = 1) drain the accumulators: round to bf16,
+// stage 32 rows x 64 entries in shared memory (128-byte swizzle) and store
+// them by TMA, and fold the rounded values into the row's (max, sum of
+// exp(l - max), first index of the max) of the tile.  A second kernel merges
+// the per-tile figures into the 2048-entry sub-chunk figures the accept
+// step reads.
+//
+// Every mbarrier wait is bounded; after one timeout a thread records
+// ISD_ERR_CUDA (unless an earlier error is recorded) and stops waiting.
+#include "tcgen05.cuh"
+
+namespace isd {
+namespace lm {
+
+using namespace tc;
+
+constexpr int kBK = 64;                  // K elements per stage (128 bytes)
+constexpr int kAccRows = 128;            // MMA M
+constexpr int kMaxTn = 256;              // MMA N (vocabulary entries)
+constexpr int kEpiWarp0 = 2;
+constexpr int kThreads = 10 * 32;
+constexpr int kStoreCols = 64;           // entries per TMA store box
+constexpr int kStoreBuf = 32 * 128;      // one warp's 32 rows x 128 bytes
+constexpr int kSubChunk = 2048;          // accept step's sub-chunk width
+constexpr size_t kSmemLimit = 227 * 1024;
+
+struct Params {
+  int M, V, tn, RTn, VT, kD, kR, ksplit, kps, tiles, stages, mode;
+  // mode 0: logits (+ per-tile statistics when pmax is set)
+  float* pmax;         // [VT][M]
+  double* psum;        // [VT][M]
+  int32_t* pidx;       // [VT][M]
+  // mode 1: fp32 partial products [ksplit][M][tn] of the LoRA down-projection
+  float* part;
+  int32_t* status;
+};
+
+ISD_DEV float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+ISD_DEV float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Tile t -> (row tile, vocabulary tile, first and end K step).
+struct Tile {
+  int rt, vt, k0, k1;
+};
+ISD_DEV Tile tile_of(const Params& p, int t) {
+  Tile x;
+  x.rt = t % p.RTn;
+  if (p.mode == 0) {
+    x.vt = t / p.RTn;
+    x.k0 = 0;
+    x.k1 = p.kD + p.kR;
+  } else {
+    x.vt = 0;
+    const int s = t / p.RTn;
+    x.k0 = s * p.kps;
+    x.k1 = min(p.kD, x.k0 + p.kps);
+  }
+  return x;
+}
+
+template <int RT>
+__global__ void __launch_bounds__(kThreads, 1)
+    lm_gemm_kernel(const __grid_constant__ CUtensorMap tm_h,
+                   const __grid_constant__ CUtensorMap tm_w,
+                   const __grid_constant__ CUtensorMap tm_u,
+                   const __grid_constant__ CUtensorMap tm_b,
+                   const __grid_constant__ CUtensorMap tm_out, Params p) {
+  constexpr int NB = RT == 1 ? 2 : 1;         // accumulator buffers
+  constexpr int kEpiWarps = 4 * RT;
+  constexpr int ABytes = RT * kAccRows * 128;   // hidden rows of a stage
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  const int stage_bytes = ABytes + p.tn * 128;
+  uint8_t* ring = base;
+  uint8_t* stg = ring + (size_t)S * stage_bytes;          // store staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + kEpiWarps * kStoreBuf);
+  uint64_t* full = bars;                  // [S]
+  uint64_t* empty = full + S;             // [S]
+  uint64_t* acc_full = empty + S;         // [NB]
+  uint64_t* acc_empty = acc_full + NB;    // [NB]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + NB);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < NB; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile(
+        "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::
+            "r"(smem_u32(tmem_slot)),
+        "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // The operands may come from the kernel before this one.
+  grid_dep_wait();
+  const int G = gridDim.x, c = blockIdx.x;
+  bool failed = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ loads
+    int s = 0;
+    uint32_t ph = 0;
+    for (int t = c; t < p.tiles; t += G) {
+      const Tile x = tile_of(p, t);
+      for (int k = x.k0; k < x.k1; ++k) {
+        wait_or_fail(&empty[s], ph ^ 1, failed);
+        if (lane == 0 && !failed) {
+          uint8_t* a = ring + (size_t)s * stage_bytes;
+          mbar_arrive_expect_tx(&full[s], stage_bytes);
+          if (k < p.kD) {
+            tma_load_2d(a, &tm_h, &full[s], k * kBK, x.rt * RT * kAccRows);
+            tma_load_2d(a + ABytes, &tm_w, &full[s], k * kBK, x.vt * p.tn);
+          } else {
+            tma_load_2d(a, &tm_u, &full[s], (k - p.kD) * kBK,
+                        x.rt * RT * kAccRows);
+            tma_load_2d(a + ABytes, &tm_b, &full[s], (k - p.kD) * kBK,
+                        x.vt * p.tn);
+          }
+        }
+        __syncwarp();
+        if (++s == S) { s = 0; ph ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMAs
+    const uint32_t id = idesc_bf16(kAccRows, p.tn, 0, 0);
+    int s = 0;
+    uint32_t ph = 0, acc_ph = 0;   // bit b: phase of accumulator buffer b
+    int n = 0;
+    for (int t = c; t < p.tiles; t += G, ++n) {
+      const Tile x = tile_of(p, t);
+      const int buf = NB == 2 ? (n & 1) : 0;
+      wait_or_fail(&acc_empty[buf], ((acc_ph >> buf) & 1) ^ 1, failed);
+      acc_ph ^= 1u << buf;
+      tc_fence_after();
+      for (int k = x.k0; k < x.k1; ++k) {
+        wait_or_fail(&full[s], ph, failed);
+        tc_fence_after();
+        if (lane == 0 && !failed) {
+          const uint32_t a = smem_u32(ring + (size_t)s * stage_bytes);
+          const uint32_t b = a + ABytes;
+#pragma unroll
+          for (int r = 0; r < RT; ++r)
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              umma(tmem + (uint32_t)((buf * RT + r) * kMaxTn),
+                   sdesc(a + r * kAccRows * 128 + kk * 32, 16, 1024),
+                   sdesc(b + kk * 32, 16, 1024), id,
+                   (k > x.k0 || kk > 0) ? 1u : 0u);
+          umma_commit(&empty[s]);
+        }
+        __syncwarp();
+        if (++s == S) { s = 0; ph ^= 1; }
+      }
+      if (lane == 0 && !failed) umma_commit(&acc_full[buf]);
+      __syncwarp();
+    }
+  } else if (warp - kEpiWarp0 < kEpiWarps) {
+    // --------------------------------------------------------- epilogue
+    const int ew = warp - kEpiWarp0;
+    const int q = warp & 3;                  // TMEM lane quarter of the warp
+    const int r = ew >> 2;                   // accumulator of the warp
+    uint8_t* sb = stg + ew * kStoreBuf;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    uint32_t acc_ph = 0;
+    int n = 0;
+    bool stored = false;
+    for (int t = c; t < p.tiles; t += G, ++n) {
+      const Tile x = tile_of(p, t);
+      const int buf = NB == 2 ? (n & 1) : 0;
+      wait_or_fail(&acc_full[buf], (acc_ph >> buf) & 1, failed);
+      acc_ph ^= 1u << buf;
+      tc_fence_after();
+      const int row0 = (x.rt * RT + r) * kAccRows + q * 32;   // warp's rows
+      const int row = row0 + lane;
+      const uint32_t tacc = tmem + lane_off + (uint32_t)((buf * RT + r) * kMaxTn);
+      float run_m = -INFINITY;
+      double run_s = 0.0;
+      int run_i = 0;
+      for (int j = 0; j < p.tn / kStoreCols; ++j) {
+        float v[64];
+        {
+          float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
+          float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
+          tmem_ld32(tacc + j * kStoreCols, v0);
+          tmem_ld32(tacc + j * kStoreCols + 32, v1);
+        }
+        if (p.mode == 1) {
+          // LoRA down-projection partials: fp32, plain stores.
+          if (row < p.M && !failed) {
+            float4* dst = reinterpret_cast<float4*>(
+                p.part + ((size_t)(x.k0 / p.kps) * p.M + row) * p.tn +
+                j * kStoreCols);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2],
+                                   v[4 * e + 3]);
+          }
+          continue;
+        }
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+        const int col0 = x.vt * p.tn + j * kStoreCols;
+        if (p.pmax && col0 < p.V) {
+          // Statistics of the rounded values (what the logits hold).
+          const int nv = min(kStoreCols, p.V - col0);
+          float pm = -INFINITY;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (2 * e < nv) pm = fmaxf(pm, bf_lo(w[e]));
+            if (2 * e + 1 < nv) pm = fmaxf(pm, bf_hi(w[e]));
+          }
+          int pi = 0;
+          float ps = 0.0f;
+#pragma unroll
+          for (int e = 31; e >= 0; --e) {
+            if (2 * e + 1 < nv && bf_hi(w[e]) == pm) pi = col0 + 2 * e + 1;
+            if (2 * e < nv && bf_lo(w[e]) == pm) pi = col0 + 2 * e;
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (2 * e < nv) ps += ex2((bf_lo(w[e]) - pm) * kLog2e);
+            if (2 * e + 1 < nv) ps += ex2((bf_hi(w[e]) - pm) * kLog2e);
+          }
+          if (pm > run_m) {
+            run_s = (run_m == -INFINITY ? 0.0 : run_s * exp((double)run_m - (double)pm)) +
+                    (double)ps;
+            run_m = pm;
+            run_i = pi;
+          } else {
+            run_s += (double)ps * exp((double)pm - (double)run_m);
+          }
+        }
+        // Stage the warp's 32 rows x 64 entries (128-byte swizzle) and store
+        // them (boxes wholly past the last row or entry are skipped); the
+        // previous store from this buffer must have read it.
+        if (col0 >= p.V || row0 >= p.M) continue;
+        if (lane == 0 && stored) bulk_wait_read();
+        __syncwarp();
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          *reinterpret_cast<uint4*>(sb + lane * 128 + ((ch ^ (lane & 7)) << 4)) =
+              make_uint4(w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
+        proxy_fence();
+        __syncwarp();
+        if (lane == 0 && !failed) {
+          tma_store_2d(&tm_out, sb, col0, row0);
+          bulk_commit();
+          stored = true;
+        }
+        __syncwarp();
+      }
+      // This tile's TMEM reads are complete: hand the buffer back.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (p.mode == 0 && p.pmax && row < p.M) {
+        const size_t o = (size_t)x.vt * p.M + row;
+        p.pmax[o] = run_m;
+        p.psum[o] = run_s;
+        p.pidx[o] = run_i;
+      }
+    }
+    if (lane == 0 && stored) bulk_wait_all();
+  }
+  if (failed) report(p.status, ISD_ERR_CUDA);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(
+                     tmem),
+                 "r"(512));
+  }
+}
+
+// U[m][j] = bf16(gate_m * scale * sum over splits of part[s][m][j]), splits
+// summed in order.  gate_m = 1 when row m is a MASK row (its stride row
+// m % K is at or past n_pending of its sequence), else 0; a sequence with
+// n_pending outside [0, K] is reported and gets no LoRA.
+struct ReduceParams {
+  int M, r, ksplit, K;
+  float scale;
+  const float* part;
+  const int32_t* n_pending;
+  __nv_bfloat16* u;
+  int32_t* status;
+};
+
+__global__ void __launch_bounds__(256) lora_reduce_kernel(ReduceParams p) {
+  grid_dep_wait();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= p.M * p.r) return;
+  const int m = i / p.r;
+  const int n = p.n_pending[m / p.K];
+  const bool ok = n >= 0 && n <= p.K;
+  if (!ok && i % p.r == 0 && (m % p.K) == 0) report(p.status, ISD_ERR_BAD_STATE);
+  float g = ok && (m % p.K) >= n ? p.scale : 0.0f;
+  float acc = 0.0f;
+  for (int s = 0; s < p.ksplit; ++s) acc += p.part[(size_t)s * p.M * p.r + i];
+  p.u[i] = __float2bfloat16_rn(g * acc);
+}
+
+// Sub-chunk figures from the per-tile ones: for (row, sub-chunk c) the
+// tiles of c in ascending order give the max, the sum of exp(l - max)
+// (fp64) and the first index of the max.
+struct MergeParams {
+  int M, V, VT, C, per;     // per: tiles per sub-chunk
+  const float* pmax;
+  const double* psum;
+  const int32_t* pidx;
+  double* csum;             // [M][C]
+  float* cmax;
+  int32_t* cidx;
+};
+
+__global__ void __launch_bounds__(256) lm_stats_merge_kernel(MergeParams p) {
+  grid_dep_wait();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= p.M * p.C) return;
+  const int row = i % p.M, c = i / p.M;
+  const int v0 = c * p.per, v1 = min(p.VT, v0 + p.per);
+  float m = -INFINITY;
+  for (int v = v0; v < v1; ++v) m = fmaxf(m, p.pmax[(size_t)v * p.M + row]);
+  double s = 0.0;
+  int idx = -1;
+  for (int v = v0; v < v1; ++v) {
+    const size_t o = (size_t)v * p.M + row;
+    const float pm = p.pmax[o];
+    s += p.psum[o] * exp((double)pm - (double)m);
+    if (idx < 0 && pm == m) idx = p.pidx[o];
+  }
+  const size_t o = (size_t)row * p.C + c;
+  p.csum[o] = s;
+  p.cmax[o] = m;
+  p.cidx[o] = idx;
+}
+
+}  // namespace lm
+
+// ---------------------------------------------------------------------------
+// Host side.
+
+namespace {
+
+struct LmLayout {
+  size_t pmax, psum, pidx, part, u, total;
+};
+
+constexpr int kLoraSplit = 16;
+constexpr int kTn = 256;                 // vocabulary entries per tile
+
+LmLayout lm_layout(const isd_lm_head_args* a) {
+  LmLayout l{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~size_t(255);
+    return o;
+  };
+  const size_t VT = (size_t)(a->V + kTn - 1) / kTn;
+  if (a->vocab_stats) {
+    l.pmax = take(VT * a->M * 4);
+    l.psum = take(VT * a->M * 8);
+    l.pidx = take(VT * a->M * 4);
+  }
+  if (a->lora_rank > 0) {
+    l.part = take((size_t)kLoraSplit * a->M * a->lora_rank * 4);
+    l.u = take((size_t)a->M * a->lora_rank * 2);
+  }
+  l.total = std::max<size_t>(off, 256);
+  return l;
+}
+
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+               uint32_t box_inner, uint32_t box_outer) {
+  const uint64_t dims[2] = {inner, outer};
+  const uint64_t strides[1] = {inner * 2};
+  const uint32_t box[2] = {box_inner, box_outer};
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims,
+                      strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+int stages_for(int RT, int tn) {
+  const size_t stage = (size_t)RT * lm::kAccRows * 128 + (size_t)tn * 128;
+  const size_t fixed = 1024 + (size_t)4 * RT * lm::kStoreBuf + 256;
+  const size_t s = (lm::kSmemLimit - fixed) / stage;
+  return (int)std::min<size_t>(s, 8);
+}
+
+size_t smem_for(int RT, int tn, int S) {
+  return 1024 + (size_t)S * ((size_t)RT * lm::kAccRows * 128 + (size_t)tn * 128) +
+         (size_t)4 * RT * lm::kStoreBuf + 256;
+}
+
+int sms_now() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
+      cudaSuccess)
+    return 0;
+  return n;
+}
+
+template <int RT>
+int launch_gemm(const CUtensorMap& th, const CUtensorMap& tw,
+                const CUtensorMap& tu, const CUtensorMap& tb,
+                const CUtensorMap& tout, lm::Params p, cudaStream_t st) {
+  p.stages = stages_for(RT, p.tn);
+  if (p.stages < 2) return ISD_ERR_UNSUPPORTED;
+  const size_t smem = smem_for(RT, p.tn, p.stages);
+  auto kern = lm::lm_gemm_kernel<RT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return ISD_ERR_CUDA;
+  const int sms = sms_now();
+  if (sms <= 0) return ISD_ERR_CUDA;
+  const int G = std::min(p.tiles, sms);
+  return launch_pdl(kern, dim3(G), dim3(lm::kThreads), smem, st, th, tw, tu,
+                    tb, tout, p) == cudaSuccess
+             ? ISD_OK
+             : ISD_ERR_CUDA;
+}
+
+}  // namespace
+
+size_t lm_head_workspace_bytes(const isd_lm_head_args* a) {
+  return lm_layout(a).total;
+}
+
+size_t vocab_stats_bytes(int M, int V) {
+  const size_t C = (size_t)(V + lm::kSubChunk - 1) / lm::kSubChunk;
+  return std::max<size_t>(((size_t)M * C * 16 + 255) & ~size_t(255), 256);
+}
+
+int launch_lm_head(const isd_lm_head_args* a, cudaStream_t st) {
+  const int M = a->M, D = a->D, V = a->V, r = a->lora_rank;
+  const int RT = M > lm::kAccRows ? 2 : 1;
+  const int rows_box = RT * lm::kAccRows;
+  const int tn = kTn;
+  const LmLayout l = lm_layout(a);
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  CUtensorMap th, tw, tout, tu, tb;
+  if (!encode_2d(&th, a->hidden, D, M, lm::kBK, rows_box) ||
+      !encode_2d(&tw, a->weight, D, V, lm::kBK, tn) ||
+      !encode_2d(&tout, a->logits, V, M, lm::kStoreCols, 32))
+    return ISD_ERR_CUDA;
+  tu = th;
+  tb = tw;
+  __nv_bfloat16* u = nullptr;
+  if (r > 0) {
+    // 1. U = gate * scale * (H A^T): split-K partials, then the ordered sum.
+    CUtensorMap ta;
+    if (!encode_2d(&ta, a->lora_a, D, r, lm::kBK, r)) return ISD_ERR_CUDA;
+    lm::Params q{};
+    q.M = M; q.V = r; q.tn = r; q.RTn = (M + rows_box - 1) / rows_box;
+    q.VT = 1; q.kD = D / lm::kBK; q.kR = 0;
+    q.ksplit = std::min(kLoraSplit, q.kD);
+    q.kps = (q.kD + q.ksplit - 1) / q.ksplit;
+    q.ksplit = (q.kD + q.kps - 1) / q.kps;
+    q.tiles = q.RTn * q.ksplit; q.mode = 1;
+    q.part = reinterpret_cast<float*>(ws + l.part);
+    q.status = a->status;
+    int rc = RT == 2 ? launch_gemm<2>(th, ta, th, ta, tout, q, st)
+                     : launch_gemm<1>(th, ta, th, ta, tout, q, st);
+    if (rc != ISD_OK) return rc;
+    u = reinterpret_cast<__nv_bfloat16*>(ws + l.u);
+    lm::ReduceParams rp;
+    rp.M = M; rp.r = r; rp.ksplit = q.ksplit; rp.K = a->rows_per_seq;
+    rp.scale = a->lora_scale; rp.part = q.part; rp.n_pending = a->n_pending;
+    rp.u = u; rp.status = a->status;
+    const int blocks = (M * r + 255) / 256;
+    if (launch_pdl(lm::lora_reduce_kernel, dim3(blocks), dim3(256), 0, st, rp) !=
+        cudaSuccess)
+      return ISD_ERR_CUDA;
+    if (!encode_2d(&tu, u, r, M, lm::kBK, rows_box) ||
+        !encode_2d(&tb, a->lora_b, r, V, lm::kBK, tn))
+      return ISD_ERR_CUDA;
+  }
+  // 2. logits = [H | U] [W | B]^T with per-tile statistics.
+  lm::Params p{};
+  p.M = M; p.V = V; p.tn = tn; p.RTn = (M + rows_box - 1) / rows_box;
+  p.VT = (V + tn - 1) / tn; p.kD = D / lm::kBK; p.kR = r / lm::kBK;
+  p.ksplit = 1; p.kps = 0; p.tiles = p.RTn * p.VT; p.mode = 0;
+  p.status = a->status;
+  if (a->vocab_stats) {
+    p.pmax = reinterpret_cast<float*>(ws + l.pmax);
+    p.psum = reinterpret_cast<double*>(ws + l.psum);
+    p.pidx = reinterpret_cast<int32_t*>(ws + l.pidx);
+  }
+  int rc = RT == 2 ? launch_gemm<2>(th, tw, tu, tb, tout, p, st)
+                   : launch_gemm<1>(th, tw, tu, tb, tout, p, st);
+  if (rc != ISD_OK || !a->vocab_stats) return rc;
+  // 3. Per-tile figures -> sub-chunk figures in the accept step's layout.
+  lm::MergeParams mp;
+  mp.M = M; mp.V = V; mp.VT = p.VT;
+  mp.C = (V + lm::kSubChunk - 1) / lm::kSubChunk;
+  mp.per = lm::kSubChunk / tn;
+  mp.pmax = p.pmax; mp.psum = p.psum; mp.pidx = p.pidx;
+  uint8_t* vs = static_cast<uint8_t*>(a->vocab_stats);
+  mp.csum = reinterpret_cast<double*>(vs);
+  mp.cmax = reinterpret_cast<float*>(vs + (size_t)M * mp.C * 8);
+  mp.cidx = reinterpret_cast<int32_t*>(vs + (size_t)M * mp.C * 12);
+  const int blocks = (M * mp.C + 255) / 256;
+  return launch_pdl(lm::lm_stats_merge_kernel, dim3(blocks), dim3(256), 0, st,
+                    mp) == cudaSuccess
+             ? ISD_OK
+             : ISD_ERR_CUDA;
+}
+
+}  // namespace isd

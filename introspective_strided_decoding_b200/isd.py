@@ -59,7 +59,8 @@ class AcceptArgs(ctypes.Structure):
                 ("n_commit", _VP), ("commit_tokens", _VP),
                 ("row_stats", _VP), ("ratio", _VP), ("status", _VP),
                 ("workspace", _VP), ("workspace_bytes", ctypes.c_size_t),
-                ("step_dev", _VP), ("proposal", _I32)]
+                ("step_dev", _VP), ("proposal", _I32),
+                ("vocab_stats", _VP)]
 
 
 class CommitArgs(ctypes.Structure):
@@ -69,6 +70,16 @@ class CommitArgs(ctypes.Structure):
                 ("k_new", _VP), ("v_new", _VP), ("k_cache", _VP),
                 ("v_cache", _VP), ("page_table", _VP), ("seq_len", _VP),
                 ("n_commit", _VP), ("free_stack", _VP), ("free_top", _VP),
+                ("status", _VP), ("workspace", _VP),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+class LmHeadArgs(ctypes.Structure):
+    _fields_ = [("M", _I32), ("D", _I32), ("V", _I32), ("dtype", _I32),
+                ("hidden", _VP), ("weight", _VP), ("logits", _VP),
+                ("vocab_stats", _VP), ("lora_rank", _I32),
+                ("rows_per_seq", _I32), ("lora_a", _VP), ("lora_b", _VP),
+                ("n_pending", _VP), ("lora_scale", ctypes.c_float),
                 ("status", _VP), ("workspace", _VP),
                 ("workspace_bytes", ctypes.c_size_t)]
 
@@ -85,6 +96,10 @@ SIGNATURES = {
     "isd_commit_workspace_bytes": (ctypes.c_size_t,
                                    [ctypes.POINTER(CommitArgs)]),
     "isd_kv_commit": (ctypes.c_int, [ctypes.POINTER(CommitArgs), _VP]),
+    "isd_lm_head_workspace_bytes": (ctypes.c_size_t,
+                                    [ctypes.POINTER(LmHeadArgs)]),
+    "isd_vocab_stats_bytes": (ctypes.c_size_t, [_I32, _I32]),
+    "isd_lm_head": (ctypes.c_int, [ctypes.POINTER(LmHeadArgs), _VP]),
     "isd_abi_version": (ctypes.c_int, []),
     "isd_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -239,7 +254,7 @@ def new_state(B, N, device):
 def accept_args(logits_cur, logits_prev, seq_len, state_in, state_out,
                 n_commit, commit_tokens, seed, step, workspace=None,
                 row_stats=None, ratio=None, status=None, step_dev=None,
-                proposal=None):
+                proposal=None, vocab_stats=None):
     B, K, V = logits_cur.shape
     N = K // 2
     dev, dt = logits_cur.device, logits_cur.dtype
@@ -261,6 +276,9 @@ def accept_args(logits_cur, logits_prev, seq_len, state_in, state_out,
         _check(status, "status", (1,), torch.int32, dev)
     if step_dev is not None:
         _check(step_dev, "step_dev", (1,), torch.int32, dev)
+    if vocab_stats is not None:
+        _check(vocab_stats, "vocab_stats", (vocab_stats_bytes(B * K, V),),
+               torch.uint8, dev)
     return AcceptArgs(
         B=B, N=N, K=K, V=V, dtype=_dtype_code(logits_cur),
         step=int(step) & 0xFFFFFFFF, seed=int(seed) & 0xFFFFFFFFFFFFFFFF,
@@ -278,7 +296,8 @@ def accept_args(logits_cur, logits_prev, seq_len, state_in, state_out,
         workspace_bytes=0 if workspace is None else
         workspace.numel() * workspace.element_size(),
         step_dev=_ptr(step_dev),
-        proposal=PROPOSAL_SAMPLE if proposal is None else int(proposal))
+        proposal=PROPOSAL_SAMPLE if proposal is None else int(proposal),
+        vocab_stats=_ptr(vocab_stats))
 
 
 def accept_workspace_bytes(args):
@@ -288,12 +307,14 @@ def accept_workspace_bytes(args):
 def accept_resample(logits_cur, logits_prev, seq_len, state_in, state_out,
                     n_commit, commit_tokens, seed, step, workspace=None,
                     row_stats=None, ratio=None, status=None, stream=None,
-                    proposal=None):
+                    proposal=None, vocab_stats=None):
     """isd_accept_resample on torch tensors (state dicts from new_state).
-    ``proposal``: PROPOSAL_SAMPLE (default) or PROPOSAL_ARGMAX."""
+    ``proposal``: PROPOSAL_SAMPLE (default) or PROPOSAL_ARGMAX;
+    ``vocab_stats``: the statistics buffer ``lm_head`` wrote for
+    ``logits_cur`` (optional)."""
     a = accept_args(logits_cur, logits_prev, seq_len, state_in, state_out,
                     n_commit, commit_tokens, seed, step, workspace, row_stats,
-                    ratio, status, proposal=proposal)
+                    ratio, status, proposal=proposal, vocab_stats=vocab_stats)
     if workspace is None:
         workspace = torch.empty(accept_workspace_bytes(a), dtype=torch.uint8,
                                 device=logits_cur.device)
@@ -366,3 +387,76 @@ def kv_commit(k_new, v_new, k_cache, v_cache, page_table, seq_len, n_commit,
         a.workspace_bytes = workspace.numel()
     _raise(lib().isd_kv_commit(ctypes.byref(a), _stream(stream)),
            "isd_kv_commit")
+
+
+# ----------------------------------------------------------------- LM head
+def vocab_stats_bytes(M, V):
+    return int(lib().isd_vocab_stats_bytes(int(M), int(V)))
+
+
+def new_vocab_stats(M, V, device):
+    """A buffer for the sub-chunk statistics of M rows of V entries."""
+    return torch.empty(vocab_stats_bytes(M, V), dtype=torch.uint8,
+                       device=device)
+
+
+def vocab_stats_view(buf, M, V):
+    """(csum f64 [M][C], cmax f32 [M][C], cidx int32 [M][C]) views of a
+    statistics buffer (its layout in include/isd.h)."""
+    C = (V + 2047) // 2048
+    n = M * C
+    csum = buf[:n * 8].view(torch.float64).view(M, C)
+    cmax = buf[n * 8:n * 12].view(torch.float32).view(M, C)
+    cidx = buf[n * 12:n * 16].view(torch.int32).view(M, C)
+    return csum, cmax, cidx
+
+
+def lm_head_args(hidden, weight, logits, vocab_stats=None, lora_a=None,
+                 lora_b=None, lora_scale=1.0, n_pending=None, rows_per_seq=0,
+                 status=None, workspace=None):
+    M, D = hidden.shape
+    V = weight.shape[0]
+    dev = hidden.device
+    _check(hidden, "hidden", (M, D), torch.bfloat16, dev)
+    _check(weight, "weight", (V, D), torch.bfloat16, dev)
+    _check(logits, "logits", (M, V), torch.bfloat16, dev)
+    r = 0
+    if lora_a is not None:
+        r = lora_a.shape[0]
+        _check(lora_a, "lora_a", (r, D), torch.bfloat16, dev)
+        _check(lora_b, "lora_b", (V, r), torch.bfloat16, dev)
+        _check(n_pending, "n_pending", (M // max(rows_per_seq, 1),),
+               torch.int32, dev)
+    if vocab_stats is not None:
+        _check(vocab_stats, "vocab_stats", (vocab_stats_bytes(M, V),),
+               torch.uint8, dev)
+    if status is not None:
+        _check(status, "status", (1,), torch.int32, dev)
+    return LmHeadArgs(
+        M=M, D=D, V=V, dtype=BF16, hidden=_ptr(hidden), weight=_ptr(weight),
+        logits=_ptr(logits), vocab_stats=_ptr(vocab_stats), lora_rank=r,
+        rows_per_seq=int(rows_per_seq), lora_a=_ptr(lora_a),
+        lora_b=_ptr(lora_b), n_pending=_ptr(n_pending),
+        lora_scale=float(lora_scale), status=_ptr(status),
+        workspace=_ptr(workspace),
+        workspace_bytes=0 if workspace is None else
+        workspace.numel() * workspace.element_size())
+
+
+def lm_head_workspace_bytes(args):
+    return int(lib().isd_lm_head_workspace_bytes(ctypes.byref(args)))
+
+
+def lm_head(hidden, weight, logits, vocab_stats=None, lora_a=None,
+            lora_b=None, lora_scale=1.0, n_pending=None, rows_per_seq=0,
+            status=None, workspace=None, stream=None):
+    """isd_lm_head on torch tensors: logits = hidden . weight^T (+ the gated
+    LoRA at MASK rows), optionally with the vocabulary statistics."""
+    a = lm_head_args(hidden, weight, logits, vocab_stats, lora_a, lora_b,
+                     lora_scale, n_pending, rows_per_seq, status, workspace)
+    if workspace is None:
+        workspace = torch.empty(lm_head_workspace_bytes(a), dtype=torch.uint8,
+                                device=hidden.device)
+        a.workspace = _ptr(workspace)
+        a.workspace_bytes = workspace.numel()
+    _raise(lib().isd_lm_head(ctypes.byref(a), _stream(stream)), "isd_lm_head")

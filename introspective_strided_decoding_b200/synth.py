@@ -67,6 +67,7 @@ class Workload:
     steps: int = 1
     spare_pages: int = 0         # extra free pages beyond growth over steps
     peak: float = 0.0            # logit boost of one keyed token per row
+    D: int = 4096                # hidden size (LM-head inputs)
     meta: dict = field(default_factory=dict, compare=False)
 
     @property
@@ -105,7 +106,8 @@ C64 = Workload("c64_stationary", B=64, Hq=32, Hkv=8, d=128, N=4, L_lo=1024,
                L_hi=8192, V=151936, sigma_p=3.0, target_accept=0.9,
                steps=100)
 SHAPE_32B = Workload("32b_b32", B=32, Hq=64, Hkv=8, d=128, N=8, L_lo=16384,
-                     L_hi=16384, V=151936, sigma_p=3.0, target_accept=0.7)
+                     L_hi=16384, V=151936, sigma_p=3.0, target_accept=0.7,
+                     D=5120)
 
 
 def sweep_workload(B, N, target):
@@ -293,3 +295,107 @@ def initial_state(w, seed, device):
     q_stats = torch.zeros((w.B, w.N, 2), dtype=torch.float32)
     return dict(pending=pending.to(device), n_pending=n_pending.to(device),
                 q_row=q_row.to(device), q_stats=q_stats.to(device))
+
+
+# ---------------------------------------------------------------------------
+# LM-head inputs: final hidden states, the output embedding, LoRA factors.
+#
+# Every tensor is an integer-valued array scaled by a power of two: hidden
+# states h_int * 2^-5 with |h_int| <= 63, weights w_int * 2^-6 with
+# |w_int| <= 31 (both exact in bfloat16).  Every product is then an integer
+# multiple of 2^-11 and any partial sum of up to 8192 of them stays below
+# 2^24 such units, so the contraction is exact in float32 in any summation
+# order, and the float64 oracle and the tensor cores round the same exact
+# value to bfloat16.
+#
+# The hidden state of (sequence b, position t) is keyed like the logits rows
+# above, so a position's verify logits h W^T are the same whenever it is
+# verified; a MASK row adds integer noise keyed by (b, t, step).  The scales
+# follow from the logits model: logit std = sqrt(D) * std(h_int) *
+# std(w_int) * 2^-11 = sigma_p, and the MASK noise gives the logits a
+# Gaussian perturbation of std sigma_q (the acceptance calibration above).
+
+H_SHIFT = 5
+W_SHIFT = 6
+H_LIM = 63
+W_LIM = 31
+W_SIGMA = 8.0
+
+
+def _int_rows(keys, cols, sigma, lim, device):
+    z = keyed_normal(keys, cols, device)
+    return torch.clamp(torch.round(sigma * z), -lim, lim)
+
+
+def lm_weight(seed, V, D, device, rows=None):
+    """Output embedding rows [len(rows) or V][D] (float32, bf16-exact)."""
+    v = torch.arange(V) if rows is None else torch.as_tensor(rows)
+    keys = _row_keys(int(seed) ^ 0x51ED270B, v, 11)
+    out = torch.empty((v.numel(), D), dtype=torch.float32, device=device)
+    for r0 in range(0, v.numel(), 8192):
+        out[r0:r0 + 8192] = _int_rows(keys[r0:r0 + 8192], D, W_SIGMA, W_LIM,
+                                      device)
+    return out * 2.0 ** -W_SHIFT
+
+
+def hidden_scales(w):
+    """(std of h_int, std of the MASK noise before rounding)."""
+    unit = 2.0 ** (H_SHIFT + W_SHIFT) / (math.sqrt(w.D) * W_SIGMA)
+    s_h = w.sigma_p * unit
+    noise = draft_sigma(w) * unit
+    # round(s z) has variance s^2 + 1/12 for the s used here.
+    s_n = math.sqrt(max(noise * noise - 1.0 / 12.0, 0.0))
+    return s_h, s_n
+
+
+def hidden_rows(seed, b, pos, mask_step, D, s_h, s_n, device):
+    """Hidden states for (sequence b, absolute position pos) pairs;
+    ``mask_step`` -1 for a clean row, else the step index.  float32 [R][D],
+    bf16-exact."""
+    b = torch.as_tensor(b, device=device).reshape(-1).to(torch.int64)
+    pos = torch.as_tensor(pos, device=device).reshape(-1).to(torch.int64)
+    ms = torch.as_tensor(mask_step, device=device).reshape(-1).to(torch.int64)
+    ms = ms.expand_as(pos) if ms.numel() == 1 else ms
+    h = torch.round(s_h * keyed_normal(_row_keys(seed ^ 0x2B992DDF, b, pos, 3),
+                                       D, device))
+    noise = torch.round(s_n * keyed_normal(
+        _row_keys(seed ^ 0x68BC21EB, b, pos, ms + 1), D, device))
+    h = h + torch.where(ms[:, None] >= 0, noise, torch.zeros_like(noise))
+    return torch.clamp(h, -H_LIM, H_LIM) * 2.0 ** -H_SHIFT
+
+
+def step_hidden(w, seed, seq_len, n_pending, step, device):
+    """Final hidden states [B][K][D] of one step's strides (bf16): row r of
+    sequence b is the state at position L_b + r + 1, a MASK row when
+    r >= n_b."""
+    B, K = w.B, w.K
+    L = torch.as_tensor(seq_len, device=device).to(torch.int64)
+    n = torch.as_tensor(n_pending, device=device).to(torch.int64)
+    r = torch.arange(K, device=device, dtype=torch.int64)
+    bb = torch.arange(B, device=device, dtype=torch.int64)[:, None].expand(B, K)
+    pos = L[:, None] + r[None, :] + 1
+    ms = torch.where(r[None, :] >= n[:, None],
+                     torch.full_like(pos, int(step)), torch.full_like(pos, -1))
+    s_h, s_n = hidden_scales(w)
+    rows = hidden_rows(seed, bb.reshape(-1), pos.reshape(-1), ms.reshape(-1),
+                       w.D, s_h, s_n, device)
+    return rows.reshape(B, K, w.D).to(torch.bfloat16)
+
+
+def lora_factors(seed, r, D, V, device, sparse=False):
+    """R-ISD LoRA factors A [r][D] and B [V][r] (float32, bf16-exact).
+
+    Dense: integer entries of std 8 scaled by 2^-6 (A) and 2^-6 (B).
+    Sparse: each row j of A holds a single 1 at a keyed column, so
+    (h A^T)_j is one entry of h and stays exact in bfloat16."""
+    rows = torch.arange(r)
+    if sparse:
+        cols = _row_keys(int(seed) ^ 0x3C6EF372, rows, 5) % D
+        A = torch.zeros((r, D), dtype=torch.float32, device=device)
+        A[rows.to(device), cols.to(device)] = 1.0
+    else:
+        A = _int_rows(_row_keys(int(seed) ^ 0x3C6EF372, rows, 6), D, W_SIGMA,
+                      W_LIM, device) * 2.0 ** -W_SHIFT
+    keys = _row_keys(int(seed) ^ 0x1F83D9AB, torch.arange(V), 7)
+    B = _int_rows(keys, r, W_SIGMA, W_LIM, device) * 2.0 ** -W_SHIFT
+    return A, B

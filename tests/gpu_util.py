@@ -124,13 +124,15 @@ class AcceptStep:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
 
-def gpu_accept(lc, lp, seq_len, state_in, seed, step, proposal=None):
+def gpu_accept(lc, lp, seq_len, state_in, seed, step, proposal=None,
+               vocab_stats=None):
     B, K, V = lc.shape
     N = K // 2
     o = AcceptStep(B, N, K, lc.device)
     isd.accept_resample(lc, lp, seq_len, state_in, o.state_out, o.n_commit,
                         o.commit_tokens, seed, step, row_stats=o.row_stats,
-                        ratio=o.ratio, status=o.status, proposal=proposal)
+                        ratio=o.ratio, status=o.status, proposal=proposal,
+                        vocab_stats=vocab_stats)
     return o
 
 

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert isd.abi_version() == 3
+    assert isd.abi_version() == 4
     assert isd.status_string(isd.ERR_POOL_EXHAUSTED) == "KV page pool exhausted"
     assert isd.status_string(12345) == "unknown status"
 
@@ -174,3 +174,53 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(isd, "_LIB_PATH", str(tmp_path / "libisd.so"))
     with pytest.raises(RuntimeError, match="missing"):
         isd.lib()
+
+
+# ----------------------------------------------------------------- LM head
+_FAKE = 1 << 20          # a 16-byte aligned fake device address (never used)
+
+
+def _lm_args(**kw):
+    base = dict(M=512, D=4096, V=151936, dtype=isd.BF16, hidden=_FAKE,
+                weight=_FAKE * 2, logits=_FAKE * 3, lora_rank=0,
+                rows_per_seq=8, lora_scale=1.0)
+    base.update(kw)
+    return isd.LmHeadArgs(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(M=0), isd.ERR_INVALID_ARG),
+    (dict(D=0), isd.ERR_INVALID_ARG),
+    (dict(lora_rank=-64), isd.ERR_INVALID_ARG),
+    (dict(dtype=isd.F32), isd.ERR_UNSUPPORTED),      # bf16 tensor cores only
+    (dict(D=4000), isd.ERR_UNSUPPORTED),             # D a multiple of 64
+    (dict(V=151937), isd.ERR_UNSUPPORTED),           # V a multiple of 8
+    (dict(lora_rank=96), isd.ERR_UNSUPPORTED),       # rank a multiple of 64
+    (dict(lora_rank=320), isd.ERR_UNSUPPORTED),      # rank at most 256
+    (dict(lora_rank=128, rows_per_seq=0), isd.ERR_INVALID_ARG),
+    (dict(lora_rank=128, rows_per_seq=7), isd.ERR_INVALID_ARG),  # M % K
+    (dict(hidden=None), isd.ERR_INVALID_ARG),
+    (dict(lora_rank=128), isd.ERR_INVALID_ARG),      # LoRA pointers missing
+    (dict(hidden=_FAKE + 8), isd.ERR_INVALID_ARG),   # not 16-byte aligned
+    (dict(logits=_FAKE), isd.ERR_INVALID_ARG),       # logits alias hidden
+    (dict(), isd.ERR_WORKSPACE),                     # no workspace
+])
+def test_lm_head_host_validation(lib, kw, code):
+    a = _lm_args(**kw)
+    assert lib.isd_lm_head(ctypes.byref(a), None) == code
+
+
+def test_lm_head_workspace_and_stats_sizes(lib):
+    a = _lm_args()
+    plain = lib.isd_lm_head_workspace_bytes(ctypes.byref(a))
+    a.vocab_stats = _FAKE * 5
+    with_stats = lib.isd_lm_head_workspace_bytes(ctypes.byref(a))
+    # per-256-entry tiles: max (4 B), sum (8 B), first index (4 B) per row
+    assert plain == 256 and with_stats >= 594 * 512 * 16
+    a.lora_rank, a.lora_a, a.lora_b, a.n_pending = 128, _FAKE, _FAKE, _FAKE
+    with_lora = lib.isd_lm_head_workspace_bytes(ctypes.byref(a))
+    assert with_lora - with_stats >= 512 * 128 * 2   # the bf16 U rows
+    # csum f64, cmax f32, cidx i32 for each of M rows x ceil(V / 2048)
+    assert lib.isd_vocab_stats_bytes(512, 151936) >= 512 * 75 * 16
+    assert lib.isd_vocab_stats_bytes(0, 10) == 0
+    assert lib.isd_lm_head_workspace_bytes(ctypes.byref(_lm_args(M=0))) == 0
