@@ -45,7 +45,6 @@ using namespace tc;
 
 constexpr int kBK = 64;                  // K elements per stage (128 bytes)
 constexpr int kAccRows = 128;            // MMA M
-constexpr int kMaxTn = 256;              // MMA N (vocabulary entries)
 constexpr int kEpiWarp0 = 2;
 constexpr int kThreads = 10 * 32;
 constexpr int kStoreCols = 64;           // entries per TMA store box
@@ -67,6 +66,88 @@ struct Params {
 ISD_DEV float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 ISD_DEV float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Running statistics of one row over the 64-entry pieces of a tile: the max
+// m of the rounded values, the sum s of exp(l - m) and the first index i of
+// the max.
+struct RowRun {
+  float m = -INFINITY;
+  double s = 0.0;
+  int i = 0;
+};
+
+// Rounds a row's 64 accumulator values to bf16: w holds the packed pairs
+// (what the logits store), v the rounded values as floats.
+ISD_DEV void round_piece(float (&v)[64], uint32_t (&w)[32]) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+    v[2 * e] = bf_lo(w[e]);
+    v[2 * e + 1] = bf_hi(w[e]);
+  }
+}
+
+// Folds the rounded values of entries col0 .. col0 + 63 (those below V)
+// into the row's running statistics.  The piece is reduced on its own
+// (max, first index of the max, 64-term fp32 sum of exp(l - max)) and then
+// merged in fp64.
+ISD_DEV void fold_piece(const float (&v)[64], int col0, int V, RowRun& rr) {
+  const int nv = V - col0;
+  float pm = -INFINITY;
+  float ps = 0.0f;
+  int pi = 0;
+  if (nv >= 64) {
+#pragma unroll
+    for (int e = 0; e < 64; ++e) pm = fmaxf(pm, v[e]);
+    if (pm > rr.m) {
+#pragma unroll
+      for (int e = 63; e >= 0; --e)
+        if (v[e] == pm) pi = col0 + e;
+    }
+#pragma unroll
+    for (int e = 0; e < 64; ++e) ps += ex2((v[e] - pm) * kLog2e);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 64; ++e)
+      if (e < nv) pm = fmaxf(pm, v[e]);
+#pragma unroll
+    for (int e = 63; e >= 0; --e)
+      if (e < nv && v[e] == pm) pi = col0 + e;
+#pragma unroll
+    for (int e = 0; e < 64; ++e)
+      if (e < nv) ps += ex2((v[e] - pm) * kLog2e);
+  }
+  if (pm > rr.m) {
+    rr.s = (rr.m == -INFINITY ? 0.0 : rr.s * exp((double)rr.m - (double)pm)) +
+           (double)ps;
+    rr.m = pm;
+    rr.i = pi;
+  } else {
+    rr.s += (double)ps * exp((double)pm - (double)rr.m);
+  }
+}
+
+// Stages one warp's 32 rows x 64 entries (128-byte swizzle) and stores them
+// by TMA at (col0, row0); the previous store from this buffer must have
+// read it first.
+ISD_DEV void stage_store(const uint32_t (&w)[32], uint8_t* sb,
+                         const CUtensorMap* tm, int col0, int row0, int lane,
+                         bool failed, bool& stored) {
+  if (lane == 0 && stored) bulk_wait_read();
+  __syncwarp();
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch)
+    *reinterpret_cast<uint4*>(sb + lane * 128 + ((ch ^ (lane & 7)) << 4)) =
+        make_uint4(w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
+  proxy_fence();
+  __syncwarp();
+  if (lane == 0 && !failed) {
+    tma_store_2d(tm, sb, col0, row0);
+    bulk_commit();
+    stored = true;
+  }
+  __syncwarp();
+}
+
 // Tile t -> (row tile, vocabulary tile, first and end K step).
 struct Tile {
   int rt, vt, k0, k1;
@@ -87,14 +168,14 @@ ISD_DEV Tile tile_of(const Params& p, int t) {
   return x;
 }
 
-template <int RT>
+template <int RT, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
     lm_gemm_kernel(const __grid_constant__ CUtensorMap tm_h,
                    const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ CUtensorMap tm_u,
                    const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_out, Params p) {
-  constexpr int NB = RT == 1 ? 2 : 1;         // accumulator buffers
+  // NB accumulator buffers of RT accumulators of tn columns each.
   constexpr int kEpiWarps = 4 * RT;
   constexpr int ABytes = RT * kAccRows * 128;   // hidden rows of a stage
   extern __shared__ uint8_t smem_raw[];
@@ -186,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int r = 0; r < RT; ++r)
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk)
-              umma(tmem + (uint32_t)((buf * RT + r) * kMaxTn),
+              umma(tmem + (uint32_t)((buf * RT + r) * p.tn),
                    sdesc(a + r * kAccRows * 128 + kk * 32, 16, 1024),
                    sdesc(b + kk * 32, 16, 1024), id,
                    (k > x.k0 || kk > 0) ? 1u : 0u);
@@ -216,10 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int row0 = (x.rt * RT + r) * kAccRows + q * 32;   // warp's rows
       const int row = row0 + lane;
-      const uint32_t tacc = tmem + lane_off + (uint32_t)((buf * RT + r) * kMaxTn);
-      float run_m = -INFINITY;
-      double run_s = 0.0;
-      int run_i = 0;
+      const uint32_t tacc = tmem + lane_off + (uint32_t)((buf * RT + r) * p.tn);
+      RowRun rr;
       for (int j = 0; j < p.tn / kStoreCols; ++j) {
         float v[64];
         {
@@ -242,57 +321,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           continue;
         }
         uint32_t w[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
         const int col0 = x.vt * p.tn + j * kStoreCols;
-        if (p.pmax && col0 < p.V) {
-          // Statistics of the rounded values (what the logits hold).
-          const int nv = min(kStoreCols, p.V - col0);
-          float pm = -INFINITY;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (2 * e < nv) pm = fmaxf(pm, bf_lo(w[e]));
-            if (2 * e + 1 < nv) pm = fmaxf(pm, bf_hi(w[e]));
-          }
-          int pi = 0;
-          float ps = 0.0f;
-#pragma unroll
-          for (int e = 31; e >= 0; --e) {
-            if (2 * e + 1 < nv && bf_hi(w[e]) == pm) pi = col0 + 2 * e + 1;
-            if (2 * e < nv && bf_lo(w[e]) == pm) pi = col0 + 2 * e;
-          }
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (2 * e < nv) ps += ex2((bf_lo(w[e]) - pm) * kLog2e);
-            if (2 * e + 1 < nv) ps += ex2((bf_hi(w[e]) - pm) * kLog2e);
-          }
-          if (pm > run_m) {
-            run_s = (run_m == -INFINITY ? 0.0 : run_s * exp((double)run_m - (double)pm)) +
-                    (double)ps;
-            run_m = pm;
-            run_i = pi;
-          } else {
-            run_s += (double)ps * exp((double)pm - (double)run_m);
-          }
-        }
-        // Stage the warp's 32 rows x 64 entries (128-byte swizzle) and store
-        // them (boxes wholly past the last row or entry are skipped); the
-        // previous store from this buffer must have read it.
-        if (col0 >= p.V || row0 >= p.M) continue;
-        if (lane == 0 && stored) bulk_wait_read();
-        __syncwarp();
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          *reinterpret_cast<uint4*>(sb + lane * 128 + ((ch ^ (lane & 7)) << 4)) =
-              make_uint4(w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
-        proxy_fence();
-        __syncwarp();
-        if (lane == 0 && !failed) {
-          tma_store_2d(&tm_out, sb, col0, row0);
-          bulk_commit();
-          stored = true;
-        }
-        __syncwarp();
+        round_piece(v, w);
+        if (p.pmax && col0 < p.V) fold_piece(v, col0, p.V, rr);
+        if (col0 < p.V && row0 < p.M)
+          stage_store(w, sb, &tm_out, col0, row0, lane, failed, stored);
       }
       // This tile's TMEM reads are complete: hand the buffer back.
       tc_fence_before();
@@ -300,9 +333,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
       if (p.mode == 0 && p.pmax && row < p.M) {
         const size_t o = (size_t)x.vt * p.M + row;
-        p.pmax[o] = run_m;
-        p.psum[o] = run_s;
-        p.pidx[o] = run_i;
+        p.pmax[o] = rr.m;
+        p.psum[o] = rr.s;
+        p.pidx[o] = rr.i;
       }
     }
     if (lane == 0 && stored) bulk_wait_all();
@@ -313,6 +346,210 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(
+                     tmem),
+                 "r"(512));
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// The same contraction on CTA pairs (more than 128 rows).  A cluster of two
+// CTAs computes a 256-row x 256-entry tile with cta_group::2 MMAs: each CTA
+// loads its 128 hidden rows and its half (128 entries) of the weight tile,
+// the even CTA issues M = 256, N = 256 MMAs that read both CTAs' shared
+// memory, and each CTA's TMEM receives its 128 rows x 256 entries.  Per SM
+// that is the two-accumulator tile's traffic (64 bytes per 128 FLOPs) with
+// half of its TMEM, so two accumulator buffers fit and the epilogue of one
+// tile overlaps the MMAs of the next.
+//
+// Barriers: the even CTA's full[s] takes one expect-tx arrival (the even
+// CTA's, for both CTAs' bytes) and both CTAs' TMA bytes; empty[s] and acc_full[b] of both CTAs are
+// signalled by the even CTA's commits (multicast); the even CTA's
+// acc_empty[b] counts the epilogue warps of both CTAs.  Before leaving,
+// each CTA's loader waits until every stage it filled has been released
+// (so no commit is still on its way to this CTA), and the pair meets.
+constexpr int kPairThreads = 10 * 32;
+constexpr int kPairEpiWarps = 8;           // two per TMEM lane quarter
+constexpr int kPairRows = 256;             // rows of a pair tile
+constexpr int kPairTn = 256;               // vocabulary entries of a tile
+constexpr int kPairHalf = 128 * 128;       // 128 rows x 64 K (bf16) = 16 KB
+
+__global__ void __launch_bounds__(kPairThreads, 1)
+    lm_pair_kernel(const __grid_constant__ CUtensorMap tm_h,
+                   const __grid_constant__ CUtensorMap tm_w,
+                   const __grid_constant__ CUtensorMap tm_u,
+                   const __grid_constant__ CUtensorMap tm_b,
+                   const __grid_constant__ CUtensorMap tm_out, Params p) {
+  constexpr int kStage = 2 * kPairHalf;    // hidden half + weight half
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  uint8_t* ring = base;
+  uint8_t* stg = ring + (size_t)S * kStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + kPairEpiWarps * kStoreBuf);
+  uint64_t* full = bars;                  // [S] (the even CTA's are used)
+  uint64_t* empty = full + S;             // [S]
+  uint64_t* acc_full = empty + S;         // [2]
+  uint64_t* acc_empty = acc_full + 2;     // [2] (the even CTA's are used)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();   // 0: issues the MMAs
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 2 * kPairEpiWarps);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile(
+        "tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::
+            "r"(smem_u32(tmem_slot)),
+        "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();        // both CTAs' barriers exist before any remote use
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  bool failed = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ loads
+    int s = 0;
+    uint32_t ph = 0;
+    for (int t = pair; t < p.tiles; t += npairs) {
+      const Tile x = tile_of(p, t);
+      const int hrow = x.rt * kPairRows + (int)rank * 128;
+      const int wrow = x.vt * kPairTn + (int)rank * 128;
+      for (int k = x.k0; k < x.k1; ++k) {
+        wait_or_fail(&empty[s], ph ^ 1, failed);
+        if (lane == 0 && !failed) {
+          uint8_t* a = ring + (size_t)s * kStage;
+          const uint32_t fb = cluster_addr(&full[s], 0);
+          // The even CTA arms its barrier for both CTAs' bytes; the odd
+          // CTA's copies count against it too (possibly first: the
+          // transaction count may go below zero until the arming).
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * kStage);
+          if (k < p.kD) {
+            tma_load_2d_pair(a, &tm_h, fb, k * kBK, hrow);
+            tma_load_2d_pair(a + kPairHalf, &tm_w, fb, k * kBK, wrow);
+          } else {
+            tma_load_2d_pair(a, &tm_u, fb, (k - p.kD) * kBK, hrow);
+            tma_load_2d_pair(a + kPairHalf, &tm_b, fb, (k - p.kD) * kBK, wrow);
+          }
+        }
+        __syncwarp();
+        if (++s == S) { s = 0; ph ^= 1; }
+      }
+    }
+    // Every stage this CTA filled has been released by the pair's MMAs.
+    for (int i = 0; i < S; ++i) {
+      wait_or_fail(&empty[s], ph ^ 1, failed);
+      if (++s == S) { s = 0; ph ^= 1; }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMAs (even CTA)
+    if (rank == 0) {
+      const uint32_t id = idesc_bf16(kPairRows, kPairTn, 0, 0);
+      int s = 0;
+      uint32_t ph = 0, acc_ph = 0;
+      int n = 0;
+      for (int t = pair; t < p.tiles; t += npairs, ++n) {
+        const Tile x = tile_of(p, t);
+        const int buf = n & 1;
+        wait_or_fail_cluster(&acc_empty[buf], ((acc_ph >> buf) & 1) ^ 1,
+                             failed);
+        acc_ph ^= 1u << buf;
+        tc_fence_after();
+        for (int k = x.k0; k < x.k1; ++k) {
+          wait_or_fail_cluster(&full[s], ph, failed);
+          tc_fence_after();
+          if (lane == 0 && !failed) {
+            const uint32_t a = smem_u32(ring + (size_t)s * kStage);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              umma_pair(tmem + (uint32_t)(buf * kPairTn),
+                        sdesc(a + kk * 32, 16, 1024),
+                        sdesc(a + kPairHalf + kk * 32, 16, 1024), id,
+                        (k > x.k0 || kk > 0) ? 1u : 0u);
+            umma_pair_commit(&empty[s], 0x3);
+          }
+          __syncwarp();
+          if (++s == S) { s = 0; ph ^= 1; }
+        }
+        if (lane == 0 && !failed) umma_pair_commit(&acc_full[buf], 0x3);
+        __syncwarp();
+      }
+    }
+  } else {
+    // --------------------------------------------------------- epilogue
+    // Warp (q, h): TMEM lane quarter q (rows 32q..32q+31 of this CTA's
+    // 128), entries 128h..128h+127 of the tile.
+    const int ew = warp - kEpiWarp0;
+    const int q = warp & 3;
+    const int h = ew >> 2;
+    uint8_t* sb = stg + ew * kStoreBuf;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    uint32_t acc_ph = 0;
+    int n = 0;
+    bool stored = false;
+    for (int t = pair; t < p.tiles; t += npairs, ++n) {
+      const Tile x = tile_of(p, t);
+      const int buf = n & 1;
+      wait_or_fail(&acc_full[buf], (acc_ph >> buf) & 1, failed);
+      acc_ph ^= 1u << buf;
+      tc_fence_after();
+      const int row0 = x.rt * kPairRows + (int)rank * 128 + q * 32;
+      const int row = row0 + lane;
+      const uint32_t tacc =
+          tmem + lane_off + (uint32_t)(buf * kPairTn + h * 128);
+      RowRun rr;
+#pragma unroll 1
+      for (int j = 0; j < 2; ++j) {
+        float v[64];
+        {
+          float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
+          float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
+          tmem_ld32(tacc + j * kStoreCols, v0);
+          tmem_ld32(tacc + j * kStoreCols + 32, v1);
+        }
+        uint32_t w[32];
+        const int col0 = x.vt * kPairTn + h * 128 + j * kStoreCols;
+        round_piece(v, w);
+        if (p.pmax && col0 < p.V) fold_piece(v, col0, p.V, rr);
+        if (col0 < p.V && row0 < p.M)
+          stage_store(w, sb, &tm_out, col0, row0, lane, failed, stored);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(cluster_addr(&acc_empty[buf], 0));
+      if (p.pmax && row < p.M) {
+        // One record per 128-entry half tile.
+        const size_t o = (size_t)(x.vt * 2 + h) * p.M + row;
+        p.pmax[o] = rr.m;
+        p.psum[o] = rr.s;
+        p.pidx[o] = rr.i;
+      }
+    }
+    if (lane == 0 && stored) bulk_wait_all();
+  }
+  if (failed) report(p.status, ISD_ERR_CUDA);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(
                      tmem),
                  "r"(512));
   }
@@ -392,7 +629,22 @@ struct LmLayout {
 };
 
 constexpr int kLoraSplit = 16;
-constexpr int kTn = 256;                 // vocabulary entries per tile
+
+// Tile shape for M rows.  Up to 128 rows: one CTA per tile, RT = 1
+// accumulator of 128 rows x tn entries, two TMEM buffers.  More rows: CTA
+// pairs with 256-row x 256-entry tiles.  Statistics records cover rec_w
+// entries each (a tile, or the half tile of a pair's epilogue warp).
+struct Shape {
+  int RT, tn, rec_w;
+  bool pair;
+  int nrec(int V) const {
+    return pair ? 2 * ((V + tn - 1) / tn) : (V + tn - 1) / tn;
+  }
+};
+Shape lm_shape(int M) {
+  return M > lm::kAccRows ? Shape{2, lm::kPairTn, 128, true}
+                          : Shape{1, 256, 256, false};
+}
 
 LmLayout lm_layout(const isd_lm_head_args* a) {
   LmLayout l{};
@@ -402,7 +654,7 @@ LmLayout lm_layout(const isd_lm_head_args* a) {
     off += (bytes + 255) & ~size_t(255);
     return o;
   };
-  const size_t VT = (size_t)(a->V + kTn - 1) / kTn;
+  const size_t VT = (size_t)lm_shape(a->M).nrec(a->V);
   if (a->vocab_stats) {
     l.pmax = take(VT * a->M * 4);
     l.psum = take(VT * a->M * 8);
@@ -446,14 +698,16 @@ int sms_now() {
   return n;
 }
 
-template <int RT>
-int launch_gemm(const CUtensorMap& th, const CUtensorMap& tw,
-                const CUtensorMap& tu, const CUtensorMap& tb,
-                const CUtensorMap& tout, lm::Params p, cudaStream_t st) {
+// Two accumulator buffers (the epilogue of one tile overlaps the MMAs of
+// the next) whenever they fit in the 512 TMEM columns.
+template <int RT, int NB>
+int launch_gemm_t(const CUtensorMap& th, const CUtensorMap& tw,
+                  const CUtensorMap& tu, const CUtensorMap& tb,
+                  const CUtensorMap& tout, lm::Params p, cudaStream_t st) {
   p.stages = stages_for(RT, p.tn);
   if (p.stages < 2) return ISD_ERR_UNSUPPORTED;
   const size_t smem = smem_for(RT, p.tn, p.stages);
-  auto kern = lm::lm_gemm_kernel<RT>;
+  auto kern = lm::lm_gemm_kernel<RT, NB>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return ISD_ERR_CUDA;
@@ -464,6 +718,52 @@ int launch_gemm(const CUtensorMap& th, const CUtensorMap& tw,
                     tb, tout, p) == cudaSuccess
              ? ISD_OK
              : ISD_ERR_CUDA;
+}
+
+int launch_pair(const CUtensorMap& th, const CUtensorMap& tw,
+                const CUtensorMap& tu, const CUtensorMap& tb,
+                const CUtensorMap& tout, lm::Params p, cudaStream_t st) {
+  const size_t fixed = 1024 + (size_t)lm::kPairEpiWarps * lm::kStoreBuf + 256;
+  p.stages = (int)std::min<size_t>((lm::kSmemLimit - fixed) /
+                                       (2 * lm::kPairHalf), 8);
+  const size_t smem = fixed + (size_t)p.stages * 2 * lm::kPairHalf;
+  if (cudaFuncSetAttribute(lm::lm_pair_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return ISD_ERR_CUDA;
+  const int sms = sms_now();
+  if (sms < 2) return ISD_ERR_CUDA;
+  const int pairs = std::min(p.tiles, sms / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(lm::kPairThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, lm::lm_pair_kernel, th, tw, tu, tb, tout,
+                            p) == cudaSuccess
+             ? ISD_OK
+             : ISD_ERR_CUDA;
+}
+
+int launch_gemm(int RT, const CUtensorMap& th, const CUtensorMap& tw,
+                const CUtensorMap& tu, const CUtensorMap& tb,
+                const CUtensorMap& tout, const lm::Params& p,
+                cudaStream_t st) {
+  const bool two = 2 * RT * p.tn <= 512;
+  if (RT == 2)
+    return two ? launch_gemm_t<2, 2>(th, tw, tu, tb, tout, p, st)
+               : launch_gemm_t<2, 1>(th, tw, tu, tb, tout, p, st);
+  return two ? launch_gemm_t<1, 2>(th, tw, tu, tb, tout, p, st)
+             : launch_gemm_t<1, 1>(th, tw, tu, tb, tout, p, st);
 }
 
 }  // namespace
@@ -479,23 +779,27 @@ size_t vocab_stats_bytes(int M, int V) {
 
 int launch_lm_head(const isd_lm_head_args* a, cudaStream_t st) {
   const int M = a->M, D = a->D, V = a->V, r = a->lora_rank;
-  const int RT = M > lm::kAccRows ? 2 : 1;
-  const int rows_box = RT * lm::kAccRows;
-  const int tn = kTn;
+  const Shape sh = lm_shape(M);
+  const int RT = sh.RT, tn = sh.tn;
+  const int rows_box = RT * lm::kAccRows;          // single-CTA tiles
+  const int hbox = sh.pair ? 128 : rows_box;       // rows a CTA loads
+  const int wbox = sh.pair ? tn / 2 : tn;          // entries a CTA loads
   const LmLayout l = lm_layout(a);
   uint8_t* ws = static_cast<uint8_t*>(a->workspace);
   CUtensorMap th, tw, tout, tu, tb;
-  if (!encode_2d(&th, a->hidden, D, M, lm::kBK, rows_box) ||
-      !encode_2d(&tw, a->weight, D, V, lm::kBK, tn) ||
+  if (!encode_2d(&th, a->hidden, D, M, lm::kBK, hbox) ||
+      !encode_2d(&tw, a->weight, D, V, lm::kBK, wbox) ||
       !encode_2d(&tout, a->logits, V, M, lm::kStoreCols, 32))
     return ISD_ERR_CUDA;
   tu = th;
   tb = tw;
-  __nv_bfloat16* u = nullptr;
   if (r > 0) {
-    // 1. U = gate * scale * (H A^T): split-K partials, then the ordered sum.
-    CUtensorMap ta;
-    if (!encode_2d(&ta, a->lora_a, D, r, lm::kBK, r)) return ISD_ERR_CUDA;
+    // 1. U = gate * scale * (H A^T): split-K partials on single-CTA tiles
+    // (RT accumulators, r entries), then the ordered sum.
+    CUtensorMap th1, ta;
+    if (!encode_2d(&th1, a->hidden, D, M, lm::kBK, rows_box) ||
+        !encode_2d(&ta, a->lora_a, D, r, lm::kBK, r))
+      return ISD_ERR_CUDA;
     lm::Params q{};
     q.M = M; q.V = r; q.tn = r; q.RTn = (M + rows_box - 1) / rows_box;
     q.VT = 1; q.kD = D / lm::kBK; q.kR = 0;
@@ -505,10 +809,9 @@ int launch_lm_head(const isd_lm_head_args* a, cudaStream_t st) {
     q.tiles = q.RTn * q.ksplit; q.mode = 1;
     q.part = reinterpret_cast<float*>(ws + l.part);
     q.status = a->status;
-    int rc = RT == 2 ? launch_gemm<2>(th, ta, th, ta, tout, q, st)
-                     : launch_gemm<1>(th, ta, th, ta, tout, q, st);
+    int rc = launch_gemm(RT, th1, ta, th1, ta, tout, q, st);
     if (rc != ISD_OK) return rc;
-    u = reinterpret_cast<__nv_bfloat16*>(ws + l.u);
+    __nv_bfloat16* u = reinterpret_cast<__nv_bfloat16*>(ws + l.u);
     lm::ReduceParams rp;
     rp.M = M; rp.r = r; rp.ksplit = q.ksplit; rp.K = a->rows_per_seq;
     rp.scale = a->lora_scale; rp.part = q.part; rp.n_pending = a->n_pending;
@@ -517,13 +820,15 @@ int launch_lm_head(const isd_lm_head_args* a, cudaStream_t st) {
     if (launch_pdl(lm::lora_reduce_kernel, dim3(blocks), dim3(256), 0, st, rp) !=
         cudaSuccess)
       return ISD_ERR_CUDA;
-    if (!encode_2d(&tu, u, r, M, lm::kBK, rows_box) ||
-        !encode_2d(&tb, a->lora_b, r, V, lm::kBK, tn))
+    if (!encode_2d(&tu, u, r, M, lm::kBK, hbox) ||
+        !encode_2d(&tb, a->lora_b, r, V, lm::kBK, wbox))
       return ISD_ERR_CUDA;
   }
   // 2. logits = [H | U] [W | B]^T with per-tile statistics.
   lm::Params p{};
-  p.M = M; p.V = V; p.tn = tn; p.RTn = (M + rows_box - 1) / rows_box;
+  p.M = M; p.V = V; p.tn = tn;
+  p.RTn = (M + (sh.pair ? lm::kPairRows : rows_box) - 1) /
+          (sh.pair ? lm::kPairRows : rows_box);
   p.VT = (V + tn - 1) / tn; p.kD = D / lm::kBK; p.kR = r / lm::kBK;
   p.ksplit = 1; p.kps = 0; p.tiles = p.RTn * p.VT; p.mode = 0;
   p.status = a->status;
@@ -532,14 +837,14 @@ int launch_lm_head(const isd_lm_head_args* a, cudaStream_t st) {
     p.psum = reinterpret_cast<double*>(ws + l.psum);
     p.pidx = reinterpret_cast<int32_t*>(ws + l.pidx);
   }
-  int rc = RT == 2 ? launch_gemm<2>(th, tw, tu, tb, tout, p, st)
-                   : launch_gemm<1>(th, tw, tu, tb, tout, p, st);
+  int rc = sh.pair ? launch_pair(th, tw, tu, tb, tout, p, st)
+                   : launch_gemm(RT, th, tw, tu, tb, tout, p, st);
   if (rc != ISD_OK || !a->vocab_stats) return rc;
-  // 3. Per-tile figures -> sub-chunk figures in the accept step's layout.
+  // 3. Per-record figures -> sub-chunk figures in the accept step's layout.
   lm::MergeParams mp;
-  mp.M = M; mp.V = V; mp.VT = p.VT;
+  mp.M = M; mp.V = V; mp.VT = sh.nrec(V);
   mp.C = (V + lm::kSubChunk - 1) / lm::kSubChunk;
-  mp.per = lm::kSubChunk / tn;
+  mp.per = lm::kSubChunk / sh.rec_w;
   mp.pmax = p.pmax; mp.psum = p.psum; mp.pidx = p.pidx;
   uint8_t* vs = static_cast<uint8_t*>(a->vocab_stats);
   mp.csum = reinterpret_cast<double*>(vs);

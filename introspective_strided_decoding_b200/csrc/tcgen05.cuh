@@ -175,6 +175,93 @@ ISD_DEV void wait_or_fail(uint64_t* bar, uint32_t parity, bool& failed) {
   }
 }
 
+// ---------------------------------------------------------------------
+// CTA pairs (a cluster of two CTAs whose tensor cores work on one tile:
+// tcgen05 with cta_group::2).  The even CTA of the pair issues the MMAs.
+
+ISD_DEV uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+ISD_DEV uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(r)
+               : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+ISD_DEV void cluster_sync() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrival (with transaction bytes) on a barrier anywhere in the cluster.
+ISD_DEV void mbar_arrive_remote(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::
+                   "r"(bar)
+               : "memory");
+}
+ISD_DEV void mbar_arrive_expect_tx_remote(uint32_t bar, uint32_t bytes) {
+  asm volatile(
+      "mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], "
+      "%1;" ::"r"(bar),
+      "r"(bytes)
+      : "memory");
+}
+// Wait whose acquire covers writes made by the other CTA of the cluster.
+ISD_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+ISD_DEV void wait_or_fail_cluster(uint64_t* bar, uint32_t parity, bool& failed) {
+  if (failed) return;
+  if (mbar_try_wait_cluster(bar, parity)) return;
+  const long long t0 = clock64();
+  while (!mbar_try_wait_cluster(bar, parity)) {
+    if ((uint64_t)(clock64() - t0) > kWaitCycles) {
+      failed = true;
+      return;
+    }
+  }
+}
+// 2-D TMA load into this CTA's shared memory whose completion is counted
+// on `bar`, a barrier of either CTA of the pair (cluster address).
+ISD_DEV void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar,
+                              int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+ISD_DEV void umma_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id,
+                       uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(
+          d_tmem),
+      "l"(a), "l"(b), "r"(id), "r"(accumulate)
+      : "memory");
+}
+// Arrives on `bar` (same offset) in every CTA of `mask` once the pair's
+// previously issued MMAs have completed.
+ISD_DEV void umma_pair_commit(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster."
+      "multicast::cluster.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
 }  // namespace tc
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no
