@@ -9,7 +9,8 @@ output, not part of the timed path) are generated between steps, and L2 is
 flushed before every timed step.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl isd|reference]
-                  [--workload c64_stationary|8b_b1|32b_b32|sweep|all]
+                  [--workload c64_stationary|8b_b1|32b_b32|sweep|
+                              c64_lm_head|c64_rlora|all]
                   [--eager]
 
 Prints one JSON line (rank 0) per workload (the default: one).  ``value`` is
@@ -19,6 +20,13 @@ serving path), device-timed with CUDA events around it, max over ranks.
 ``--eager`` times the three calls launched one by one instead.  With N > 1
 every rank runs its own replica (the path shards by sequence; no
 collective on the data path).
+
+``c64_lm_head`` and ``c64_rlora`` put the LM head in the timed step: each
+step starts from the rows' final hidden states (D = 4096), isd_lm_head makes
+the logits and their vocabulary statistics on the tensor cores (with the
+R-ISD gated LoRA of rank 128 at MASK rows for ``c64_rlora``), and the accept
+step takes those statistics; their roofline is the LM head's, against the
+bf16 tensor peak.
 """
 
 import argparse
@@ -40,6 +48,7 @@ sys.path.insert(0, ROOT)
 METRIC = ("ISD accepted tokens/s at B=64,N=4; achieved HBM GB/s as fraction "
           "of B200 peak")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 SWEEP = [(B, N, p) for B in (1, 8, 32, 64) for N in (2, 4, 8)
          for p in (0.5, 0.9)]
 
@@ -52,7 +61,7 @@ def parse():
     ap.add_argument("--impl", default="isd", choices=["isd", "reference"])
     ap.add_argument("--workload", default="c64_stationary",
                     choices=["c64_stationary", "8b_b1", "32b_b32", "sweep",
-                             "all"])
+                             "c64_lm_head", "c64_rlora", "all"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's sequences per GPU (only "
@@ -104,6 +113,18 @@ def peaks():
         return float(j["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 TFLOP/s: the burst figure (the LM head is timed as one
+    call inside the step)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def tpf_closed_form(p, N):
@@ -310,12 +331,15 @@ def workload_list(args):
     from introspective_strided_decoding_b200 import synth
     named = {"c64_stationary": synth.C64, "8b_b1": synth.SHAPE_8B,
              "32b_b32": synth.SHAPE_32B}
+    lm = {"c64_lm_head": synth.C64_LM, "c64_rlora": synth.C64_RLORA}
     if args.workload in named:
         return [named[args.workload]]
+    if args.workload in lm:
+        return [lm[args.workload]]
     sweep = [synth.sweep_workload(B, N, p) for B, N, p in SWEEP]
     if args.workload == "sweep":
         return sweep
-    return list(named.values()) + sweep
+    return list(named.values()) + sweep + list(lm.values())
 
 
 def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
@@ -332,9 +356,23 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
     seed = rank_seed(args.seed, rank)
     cache = synth.make_cache(w, seed, dev)
     st0 = synth.initial_state(w, seed, dev)
+    with_lm = bool(w.meta.get("lm_head"))
+    lm = None
+    lm_flops = 0.0
+    if with_lm:
+        M, r = w.B * w.K, int(w.meta.get("lora_rank", 0))
+        lm = dict(weight=synth.lm_weight(seed, w.V, w.D, dev)
+                  .to(torch.bfloat16))
+        lm_flops = 2.0 * M * w.D * w.V
+        if r:
+            a, b = synth.lora_factors(seed, r, w.D, w.V, dev)
+            lm.update(lora_a=a.to(torch.bfloat16).contiguous(),
+                      lora_b=b.to(torch.bfloat16).contiguous(),
+                      lora_scale=float(w.meta["lora_scale"]))
+            lm_flops += 2.0 * M * w.D * r + 2.0 * M * r * w.V
     dec = Decoder(w, cache, st0, dev, seed,
                   proposal=isd.PROPOSAL_ARGMAX if args.proposal == "argmax"
-                  else isd.PROPOSAL_SAMPLE)
+                  else isd.PROPOSAL_SAMPLE, lm=lm)
     stream = torch.cuda.current_stream(dev)
     use_graph = not args.eager
     if use_graph:
@@ -349,7 +387,10 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
     def prepare(step):
         L = cache["seq_len"]
         n = dec.state["n_pending"]
-        dec.logits_cur.copy_(synth.step_logits(w, seed, L, n, step, dev))
+        if with_lm:
+            dec.hidden.copy_(synth.step_hidden(w, seed, L, n, step, dev))
+        else:
+            dec.logits_cur.copy_(synth.step_logits(w, seed, L, n, step, dev))
         q, k, v = synth.make_stride(w, seed, step, dev)
         dec.q.copy_(q)
         dec.k_new.copy_(k)
@@ -415,9 +456,12 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
     step_bytes = [kv + qo_bytes + r * row_bytes for kv, r in
                   zip(kv_bytes, logit_rows)]
     step_gbs = sum(step_bytes) / (total_ms / 1e3) / 1e9
+    if with_lm:
+        step_gbs = None      # the logits are made in the step, not read
 
     # --------------------------------------- per-phase split (eager calls)
-    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    nev = 5 if with_lm else 4
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)]
            for _ in range(phase_steps)]
     p_kv, p_rows = [], []
     for s in range(phase_steps):
@@ -428,13 +472,17 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
         dec.step(stream, pev[s])
     torch.cuda.synchronize(dev)
     t_attn = [e[0].elapsed_time(e[1]) for e in pev]
-    t_acc = [e[1].elapsed_time(e[2]) for e in pev]
-    t_com = [e[2].elapsed_time(e[3]) for e in pev]
+    t_lm = [e[1].elapsed_time(e[2]) for e in pev] if with_lm else []
+    t_acc = [e[-3].elapsed_time(e[-2]) for e in pev]
+    t_com = [e[-2].elapsed_time(e[-1]) for e in pev]
     attn_bytes = [kv + qo_bytes for kv in p_kv]
     achieved = sum(attn_bytes) / (sum(t_attn) / 1e3) / 1e9
     acc_bytes = sum(r * row_bytes for r in p_rows)
     aa_gbs = (sum(attn_bytes) + acc_bytes) / \
         ((sum(t_attn) + sum(t_acc)) / 1e3) / 1e9
+    lm_ms = sum(t_lm) / phase_steps if with_lm else None
+    if with_lm:
+        aa_gbs = None
 
     # ---------------------------------------------------------------- e2e
     # Host-resident inputs (pinned), H2D copy + the step through the public
@@ -449,8 +497,9 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
     host_in = []
     for s in range(n_e2e):
         prepare(dec.step_idx)
+        first = dec.hidden if with_lm else dec.logits_cur
         host_in.append(tuple(t.to("cpu").pin_memory() for t in
-                             (dec.logits_cur, dec.q, dec.k_new, dec.v_new)))
+                             (first, dec.q, dec.k_new, dec.v_new)))
         run_step()
     torch.cuda.synchronize(dev)
     for k, v in snap.items():
@@ -472,7 +521,8 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
     e0.record(stream)
     for s in range(n_e2e):
         lg, q, k, v = host_in[s]
-        dec.logits_cur.copy_(lg, non_blocking=True)
+        (dec.hidden if with_lm else dec.logits_cur).copy_(lg,
+                                                          non_blocking=True)
         dec.q.copy_(q, non_blocking=True)
         dec.k_new.copy_(k, non_blocking=True)
         dec.v_new.copy_(v, non_blocking=True)
@@ -496,6 +546,24 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
            "steps": n_e2e}
     alpha = accepted / max(tested, 1)
     tpf = tokens / (w.B * steps)
+    calls = ("attention+LM head+accept+commit" if with_lm
+             else "attention+accept+commit")
+    inputs = "hidden-state" if with_lm else "logits"
+    attn_roof = {
+        "kernel": "attn_tc_kernel (+combine)", "bound": "hbm",
+        "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+        "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+        "traffic": attention_traffic(sum(attn_bytes) / len(attn_bytes)),
+        "bytes_per_launch": sum(attn_bytes) / len(attn_bytes)}
+    if with_lm:
+        tpk, tkind = tensor_peak()
+        lm_tf = lm_flops / (lm_ms / 1e3) / 1e12
+        roof = {"kernel": "lm_pair_kernel (+LoRA down, merge)",
+                "bound": "tensor", "achieved": lm_tf, "peak": tpk,
+                "unit": "TFLOP/s", "frac": lm_tf / tpk, "peak_kind": tkind,
+                "traffic": None, "flops_per_launch": lm_flops}
+    else:
+        roof = attn_roof
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": steps, "warmup": warmup,
@@ -509,17 +577,12 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
             "target_accept": w.target_accept, "proposal": args.proposal,
             "l2": "flushed (256 MB write) before every timed step",
             "timing": ("CUDA events around one CUDA-graph replay of "
-                       "attention+accept+commit per step" if use_graph else
-                       "CUDA events around the eager attention+accept+commit "
-                       "calls per step") +
-                      "; logits/Q/K/V generation between steps untimed",
+                       f"{calls} per step" if use_graph else
+                       f"CUDA events around the eager {calls} calls per "
+                       "step") +
+                      f"; {inputs}/Q/K/V generation between steps untimed",
             "parallelism": f"replicas x{world}"},
-        "roofline": {
-            "kernel": "attn_tc_kernel (+combine)", "bound": "hbm",
-            "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-            "frac": achieved / hbm_peak, "peak_kind": peak_kind,
-            "traffic": attention_traffic(sum(attn_bytes) / len(attn_bytes)),
-            "bytes_per_launch": sum(attn_bytes) / len(attn_bytes)},
+        "roofline": roof,
         "e2e": e2e,
         "gpu_launches": dec.launches_per_step * steps,
         "clocks": clk,
@@ -530,14 +593,21 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
             "commit_ms": sum(t_com) / phase_steps,
             "phase_split": f"eager calls, {phase_steps} further steps",
             "steps_per_s": steps / (total_ms / 1e3),
-            "step_gbs": step_gbs, "step_frac": step_gbs / hbm_peak,
+            "step_gbs": step_gbs,
+            "step_frac": None if step_gbs is None else step_gbs / hbm_peak,
             "attn_accept_gbs": aa_gbs,
-            "attn_accept_frac": aa_gbs / hbm_peak,
+            "attn_accept_frac": None if aa_gbs is None else aa_gbs / hbm_peak,
             "tpf": tpf, "accept_rate": alpha,
             "tpf_closed_form_at_rate": tpf_closed_form(alpha, w.N),
             "tokens": tokens},
     }
-    if rank == 0 and with_cpu:
+    if with_lm:
+        line["detail"].update(
+            lm_head_ms=lm_ms, attention_roofline=attn_roof,
+            lora_rank=int(w.meta.get("lora_rank", 0)), D=w.D)
+        line["config"]["D"] = w.D
+        line["config"]["lora_rank"] = int(w.meta.get("lora_rank", 0))
+    if rank == 0 and with_cpu and not with_lm:
         v, cores, desc = oracle_sample(w, args.seed, args.cpu_sample_steps,
                                        proposal=args.proposal,
                                        seqs=args.cpu_sample_seqs)

@@ -9,9 +9,16 @@ three C-ABI calls on one stream:
     isd_attn_strided -> (caller's LM head fills logits) -> isd_accept_resample
     -> isd_kv_commit
 
-The argument structs are built once, so a step costs three ctypes calls on
-the host.  All memory is allocated here, through torch, never by the
-library.
+With an LM head (``lm``: the output embedding and, for R-ISD, the gated
+LoRA factors) the step starts from the rows' final hidden states instead
+of logits:
+
+    isd_attn_strided -> isd_lm_head (logits + vocabulary statistics)
+    -> isd_accept_resample (fed by those statistics) -> isd_kv_commit
+
+The argument structs are built once, so a step costs three or four ctypes
+calls on the host.  All memory is allocated here, through torch, never by
+the library.
 """
 
 import ctypes
@@ -24,7 +31,7 @@ from . import isd
 
 class Decoder:
     def __init__(self, w, cache, state0, device, seed, num_ctas=0,
-                 with_lse=False, record=False, proposal=None):
+                 with_lse=False, record=False, proposal=None, lm=None):
         self.w = w
         self.cache = cache
         self.device = torch.device(device)
@@ -63,6 +70,29 @@ class Decoder:
                                        16), dtype=torch.uint8, device=dev)
         self._attn.workspace = ctypes.c_void_p(self.ws_attn.data_ptr())
         self._attn.workspace_bytes = self.ws_attn.numel()
+        self.lm = lm
+        self.vocab_stats = None
+        self._lm = []
+        if lm is not None:
+            # Hidden states [B][K][D] in, logits and statistics out.
+            M, D = B * K, lm["weight"].shape[1]
+            self.hidden = torch.zeros((B, K, D), dtype=torch.bfloat16,
+                                      device=dev)
+            self.vocab_stats = isd.new_vocab_stats(M, V, dev)
+            for c in range(2):
+                a = isd.lm_head_args(
+                    self.hidden.view(M, D), lm["weight"],
+                    self.logits[c].view(M, V), self.vocab_stats,
+                    lm.get("lora_a"), lm.get("lora_b"),
+                    lm.get("lora_scale", 1.0),
+                    self.states[c]["n_pending"] if lm.get("lora_a")
+                    is not None else None, K, self.status)
+                self._lm.append(a)
+            self.ws_lm = torch.empty(max(isd.lm_head_workspace_bytes(
+                self._lm[0]), 16), dtype=torch.uint8, device=dev)
+            for a in self._lm:
+                a.workspace = ctypes.c_void_p(self.ws_lm.data_ptr())
+                a.workspace_bytes = self.ws_lm.numel()
         self._acc = []
         for c in range(2):
             a = isd.accept_args(self.logits[c], self.logits[1 - c],
@@ -70,7 +100,8 @@ class Decoder:
                                 self.states[1 - c], self.n_commit,
                                 self.commit_tokens, self.seed, 0,
                                 row_stats=self.row_stats, ratio=self.ratio,
-                                status=self.status, proposal=proposal)
+                                status=self.status, proposal=proposal,
+                                vocab_stats=self.vocab_stats)
             self._acc.append(a)
         self.ws_acc = torch.empty(isd.accept_workspace_bytes(self._acc[0]),
                                   dtype=torch.uint8, device=dev)
@@ -104,6 +135,12 @@ class Decoder:
         if rc != isd.OK:
             raise isd.IsdError(rc, "isd_attn_strided")
 
+    def lm_head(self, stream=None):
+        rc = self._lib.isd_lm_head(ctypes.byref(self._lm[self.cur]),
+                                   isd._stream(stream))
+        if rc != isd.OK:
+            raise isd.IsdError(rc, "isd_lm_head")
+
     def accept(self, stream=None):
         a = self._acc[self.cur]
         a.step = self.step_idx & 0xFFFFFFFF  # unused once step_dev is set
@@ -123,20 +160,26 @@ class Decoder:
         self.step_idx += 1
 
     def step(self, stream=None, events=None):
-        """Attention, accept/resample and commit; ``events`` (4 CUDA events)
-        are recorded around the three calls when given."""
+        """Attention, (the LM head,) accept/resample and commit; ``events``
+        (CUDA events) are recorded around the calls when given: before
+        attention, before the LM head or accept, (with 5 events: before
+        accept,) before the commit, after it."""
         s = stream if stream is not None else torch.cuda.current_stream()
         if events:
             events[0].record(s)
         self.attention(s)
         if events:
             events[1].record(s)
+        if self.lm is not None:
+            self.lm_head(s)
+            if events and len(events) == 5:
+                events[2].record(s)
         self.accept(s)
         if events:
-            events[2].record(s)
+            events[-2].record(s)
         self.commit(s)
         if events:
-            events[3].record(s)
+            events[-1].record(s)
         self.advance()
 
     # ------------------------------------------------------ CUDA graphs
@@ -159,6 +202,8 @@ class Decoder:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
                 self.attention()
+                if self.lm is not None:
+                    self.lm_head()
                 self.accept()
                 self.commit()
                 self.step_dev.add_(1)
@@ -186,6 +231,12 @@ class Decoder:
     def launches_per_step(self):
         """This library's kernel launches per step: attention (bf16: the
         tcgen05 kernel and the split-segment combine; fp32: one kernel),
-        the two accept kernels (statistics; decision and draws) and the
-        commit."""
-        return (2 if self.w.dtype == "bf16" else 1) + 2 + 1
+        the accept kernels (statistics, then decision and draws; with an LM
+        head only the second, the statistics coming from the LM head's GEMM
+        and merge kernels, plus the LoRA down-projection and its sum when
+        there is a LoRA) and the commit."""
+        attn = 2 if self.w.dtype == "bf16" else 1
+        if self.lm is None:
+            return attn + 2 + 1
+        lora = 2 if self.lm.get("lora_a") is not None else 0
+        return attn + 2 + lora + 1 + 1

@@ -110,6 +110,14 @@ SHAPE_32B = Workload("32b_b32", B=32, Hq=64, Hkv=8, d=128, N=8, L_lo=16384,
                      D=5120)
 
 
+# The C=64 step with the LM head in the path (hidden states in; D = 4096),
+# and the same with the R-ISD gated LoRA of rank 128 at MASK rows.
+C64_LM = C64.with_(name="c64_lm_head", meta={"lm_head": True})
+C64_RLORA = C64.with_(name="c64_rlora",
+                      meta={"lm_head": True, "lora_rank": 128,
+                            "lora_scale": 2.0 ** -5})
+
+
 def sweep_workload(B, N, target):
     return Workload(f"sweep_b{B}_n{N}_p{target}", B=B, Hq=32, Hkv=8, d=128,
                     N=N, L_lo=512, L_hi=16384, V=151936, sigma_p=3.0,

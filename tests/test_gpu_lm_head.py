@@ -252,3 +252,76 @@ def test_fused_step_matches_oracle():
     print(f"fused: {exact} exact, {rejected} rejected, {accepted_all} "
           "all-accepted")
     assert exact >= 0.9 * w.B * steps
+
+
+@pytest.mark.parametrize("graph", [False, True])
+def test_decoder_with_lm_head_and_lora_matches_oracle(graph):
+    """The decoder's step with the LM head and the R-ISD LoRA (eager calls
+    or CUDA-graph replays), each step checked against the oracle started
+    from the state the GPU carried into it: the LoRA gate must follow that
+    state's pending counts."""
+    from introspective_strided_decoding_b200.driver import Decoder
+    w = synth.Workload("lm_decoder", B=8, Hq=32, Hkv=8, d=128, N=4,
+                       L_lo=100, L_hi=400, V=8200, sigma_p=3.0, sigma_q=0.25,
+                       D=256, steps=6)
+    seed, r = 31, 64
+    W = synth.lm_weight(seed, w.V, w.D, DEV).to(torch.bfloat16).contiguous()
+    A, Bf = synth.lora_factors(seed, r, w.D, w.V, DEV, sparse=True)
+    A = A.to(torch.bfloat16).contiguous()
+    Bf = Bf.to(torch.bfloat16).contiguous()
+    cache = synth.make_cache(w, seed, DEV)
+    dec = Decoder(w, cache, synth.initial_state(w, seed, DEV), DEV, seed,
+                  record=True, lm=dict(weight=W, lora_a=A, lora_b=Bf,
+                                       lora_scale=1.0))
+    if graph:
+        dec.capture()
+    M = w.B * w.K
+    lp_host = np.zeros((w.B, w.K, w.V), dtype=np.float32)
+    exact = 0
+    for s in range(w.steps):
+        st = dec.state
+        ostate = oracle_initial_state(st)
+        L = i64(cache["seq_len"])
+        H = synth.step_hidden(w, seed, cache["seq_len"], st["n_pending"], s,
+                              DEV)
+        dec.hidden.copy_(H)
+        q, k, v = synth.make_stride(w, seed, s, DEV)
+        dec.q.copy_(q)
+        dec.k_new.copy_(k)
+        dec.v_new.copy_(v)
+        if graph:
+            dec.replay()
+        else:
+            dec.step_idx = s
+            dec.step()
+        torch.cuda.synchronize()
+        assert int(dec.status.item()) == isd.OK
+        mask = olm.mask_rows(ostate["n_pending"], w.K)
+        lc_host = olm.round_bf16(_oracle_logits(
+            H.reshape(M, w.D), W, dict(A=f64(A), B=f64(Bf), scale=1.0,
+                                       mask=mask))
+        ).astype(np.float32).reshape(w.B, w.K, w.V)
+        # The logits the step made (the buffer it just used).
+        assert np.array_equal(f64(dec.logits[1 - dec.cur]),
+                              lc_host.astype(np.float64))
+
+        def oracle(flip=(), lc_host=lc_host, lp_host=lp_host, ostate=ostate,
+                   L=L, s=s):
+            return ostep.accept_resample(lc_host, lp_host, ostate["pending"],
+                                         ostate["n_pending"], ostate["q_row"],
+                                         L, seed, s, w.N, flip=flip)
+
+        class View:
+            n_commit = dec.n_commit
+            commit_tokens = dec.commit_tokens
+            state_out = dec.state
+            row_stats = dec.row_stats
+            ratio = dec.ratio
+        c = compare_accept(View, oracle(), ostate["n_pending"],
+                           lambda b, rr: lc_host[b, rr].astype(np.float64),
+                           oracle, ostate["pending"])
+        exact += c["exact"]
+        lp_host = lc_host
+    if graph:
+        dec.release_graphs()
+    assert exact >= 0.9 * w.B * w.steps
