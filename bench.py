@@ -342,6 +342,66 @@ def workload_list(args):
     return list(named.values()) + sweep + list(lm.values())
 
 
+MULTI_STEPS = 8
+
+
+def multi_step_timing(dec, cache, prepare, run_step, flush, stream, dev):
+    """Device time per step of one CUDA graph holding MULTI_STEPS steps
+    (inputs from per-step slots, step index from the device counter), after
+    an L2 flush; the steps' own inputs (weights, KV cache) exceed L2.  The
+    inputs are those of the next MULTI_STEPS single-step replays, recorded
+    and rewound; the multi-step replay must reproduce their lengths."""
+    S = MULTI_STEPS
+    snap = {k: v.clone() for k, v in cache.items()}
+    snap_state = {k: v.clone() for k, v in dec.state.items()}
+    snap_logits = [x.clone() for x in dec.logits]
+    cur, idx = dec.cur, dec.step_idx
+    rec = []
+    for _ in range(S):
+        prepare(dec.step_idx)
+        rec.append(tuple(t.clone() for t in (dec.hidden, dec.q, dec.k_new,
+                                             dec.v_new)))
+        run_step()
+    L_single = cache["seq_len"].clone()
+    torch.cuda.synchronize(dev)
+
+    def rewind():
+        for k, v in snap.items():
+            cache[k].copy_(v)
+        for k, v in snap_state.items():
+            dec.states[cur][k].copy_(v)
+        for x, y in zip(dec.logits, snap_logits):
+            x.copy_(y)
+        dec.set_step(cur, idx)
+
+    rewind()
+    dec.capture_multi(S)
+    times = []
+    for rep in range(3):
+        rewind()
+        dec.step_dev.fill_(idx)
+        for i, (h, q, k, v) in enumerate(rec):
+            dec.slots["first"][i].copy_(h)
+            dec.slots["q"][i].copy_(q)
+            dec.slots["k_new"][i].copy_(k)
+            dec.slots["v_new"][i].copy_(v)
+        flush.fill_(rep & 0xFF)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(100_000)
+        e0.record(stream)
+        dec.replay_multi()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        times.append(e0.elapsed_time(e1))
+        if not torch.equal(cache["seq_len"], L_single):
+            raise RuntimeError("multi-step graph diverged from single steps")
+    rewind()
+    ms = statistics.median(times)
+    return {"steps_per_graph": S, "ms_per_step": ms / S,
+            "replays": len(times), "l2": "flushed before each replay"}
+
+
 def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
     from introspective_strided_decoding_b200 import build, isd, synth
     from introspective_strided_decoding_b200.driver import Decoder
@@ -538,6 +598,8 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
     if int(dec.status.item()) != isd.OK:
         raise RuntimeError("device status after the e2e steps: "
                            f"{isd.status_string(int(dec.status.item()))}")
+    multi = multi_step_timing(dec, cache, prepare, run_step, flush, stream,
+                              dev) if with_lm and use_graph else None
     dec.release_graphs()
     job = job_figures(total_ms, tokens, e2e_ms, e2e_tokens, world, dev)
     total_ms_max, value = job["total_ms_max"], job["value"]
@@ -603,7 +665,7 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
     }
     if with_lm:
         line["detail"].update(
-            lm_head_ms=lm_ms, attention_roofline=attn_roof,
+            lm_head_ms=lm_ms, attention_roofline=attn_roof, multi_step=multi,
             lora_rank=int(w.meta.get("lora_rank", 0)), D=w.D)
         line["config"]["D"] = w.D
         line["config"]["lora_rank"] = int(w.meta.get("lora_rank", 0))

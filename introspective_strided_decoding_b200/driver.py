@@ -180,9 +180,23 @@ class Decoder:
         self.commit(s)
         if events:
             events[-1].record(s)
+        if getattr(self, "step_dev", None) is not None:
+            # Once graphs are captured the accept call reads the step index
+            # from the device counter; eager steps advance it too.
+            with torch.cuda.stream(s):
+                self.step_dev.add_(1)
         self.advance()
 
     # ------------------------------------------------------ CUDA graphs
+    def _step_counter(self):
+        """The device step counter the captured graphs read (one tensor for
+        every graph of this decoder, set to the current step index)."""
+        if getattr(self, "step_dev", None) is None:
+            self.step_dev = torch.full((1,), self.step_idx, dtype=torch.int32,
+                                       device=self.device)
+        else:
+            self.step_dev.fill_(self.step_idx)
+
     def capture(self, stream=None):
         """Capture the step into two CUDA graphs, one per ping-pong parity
         (the pages' serving stack replays a captured decode step; "Serving
@@ -190,8 +204,7 @@ class Decoder:
         accept call then reads the step index from a device counter that
         the graph itself advances, so the same graph serves every step."""
         dev = self.device
-        self.step_dev = torch.full((1,), self.step_idx, dtype=torch.int32,
-                                   device=dev)
+        self._step_counter()
         for a in self._acc:
             a.step_dev = ctypes.c_void_p(self.step_dev.data_ptr())
         cur0 = self.cur
@@ -215,6 +228,90 @@ class Decoder:
         self.graphs[self.cur].replay()
         self.advance()
 
+    # ------------------------------------------- multi-step CUDA graph
+    def capture_multi(self, steps, stream=None):
+        """Capture ``steps`` consecutive steps (an even number, so the
+        ping-pong parity comes back) into one CUDA graph: one replay runs
+        them all, launching nothing from the host in between.  Step i reads
+        its inputs from slot i of ``self.slots`` (hidden states with an LM
+        head, else logits; the stride's Q and staged K/V) and the step
+        index from the device counter.  With logits as inputs, slot i is
+        the step's logits_cur and the stored q rows of step i come from slot
+        i - 1; slot -1 (the previous replay's last step) is ``carry``, which
+        the graph refreshes from slot S - 1 at its end."""
+        if steps < 2 or steps % 2:
+            raise ValueError("steps must be even and >= 2")
+        S, w, dev = steps, self.w, self.device
+        self._step_counter()
+        first = self.hidden if self.lm is not None else self.logits_cur
+        self.slots = dict(
+            first=torch.zeros((S,) + tuple(first.shape), dtype=first.dtype,
+                              device=dev),
+            q=torch.zeros((S,) + tuple(self.q.shape), dtype=self.q.dtype,
+                          device=dev),
+            k_new=torch.zeros((S,) + tuple(self.k_new.shape),
+                              dtype=self.k_new.dtype, device=dev),
+            v_new=torch.zeros((S,) + tuple(self.v_new.shape),
+                              dtype=self.v_new.dtype, device=dev))
+        if self.lm is None:
+            self.carry = self.logits[1 - self.cur].clone()
+
+        def clone_args(a, **ptrs):
+            c = type(a).from_buffer_copy(a)
+            for k, t in ptrs.items():
+                setattr(c, k, ctypes.c_void_p(t.data_ptr()))
+            return c
+
+        attn, lm, acc, com = [], [], [], []
+        for i in range(S):
+            par = (self.cur + i) % 2
+            sq, sk, sv = (self.slots["q"][i], self.slots["k_new"][i],
+                          self.slots["v_new"][i])
+            attn.append(clone_args(self._attn, q=sq, k_new=sk, v_new=sv))
+            com.append(clone_args(self._com, k_new=sk, v_new=sv))
+            if self.lm is not None:
+                lm.append(clone_args(self._lm[par],
+                                     hidden=self.slots["first"][i]))
+                a = clone_args(self._acc[par])
+            else:
+                prev = self.carry if i == 0 else self.slots["first"][i - 1]
+                a = clone_args(self._acc[par],
+                               logits_cur=self.slots["first"][i],
+                               logits_prev=prev)
+            a.step_dev = ctypes.c_void_p(self.step_dev.data_ptr())
+            acc.append(a)
+        self._multi_args = (attn, lm, acc, com)   # kept alive with the graph
+        s = stream if stream is not None else torch.cuda.Stream(dev)
+        g = torch.cuda.CUDAGraph()
+        lib = self._lib
+        with torch.cuda.graph(g, stream=s):
+            cs = torch.cuda.current_stream()
+            for i in range(S):
+                for rc, what in (
+                        (lib.isd_attn_strided(ctypes.byref(attn[i]),
+                                              isd._stream(cs)),
+                         "isd_attn_strided"),
+                        (lib.isd_lm_head(ctypes.byref(lm[i]), isd._stream(cs))
+                         if lm else isd.OK, "isd_lm_head"),
+                        (lib.isd_accept_resample(ctypes.byref(acc[i]),
+                                                 isd._stream(cs)),
+                         "isd_accept_resample"),
+                        (lib.isd_kv_commit(ctypes.byref(com[i]),
+                                           isd._stream(cs)),
+                         "isd_kv_commit")):
+                    if rc != isd.OK:
+                        raise isd.IsdError(rc, what)
+                self.step_dev.add_(1)
+            if self.lm is None:
+                self.carry.copy_(self.slots["first"][S - 1])
+        self.multi_graph = g
+        self.multi_steps = S
+
+    def replay_multi(self):
+        """The captured ``steps`` steps in one graph replay."""
+        self.multi_graph.replay()
+        self.step_idx += self.multi_steps
+
     def set_step(self, cur, step_idx):
         """Rewind (or move) the decoder to ping-pong parity ``cur`` and
         step index ``step_idx``, the device step counter included."""
@@ -226,6 +323,7 @@ class Decoder:
     def release_graphs(self):
         """Drop the captured graphs (before the buffers they use)."""
         self.graphs = []
+        self.multi_graph = None
 
     @property
     def launches_per_step(self):

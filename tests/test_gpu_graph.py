@@ -123,3 +123,77 @@ def test_graph_replay_free_running_matches_oracle(peaked):
     dec.release_graphs()
     print(f"graph free run: {exact} sequence-steps exact, {ties} near-ties")
     assert exact >= 0.9 * w.B * w.steps
+
+
+def _snap(dec, cache):
+    st = {k: v.clone() for k, v in dec.state.items()}
+    return dict(st, **{k: cache[k].clone() for k in
+                       ("seq_len", "page_table", "free_top", "k_cache",
+                        "v_cache")})
+
+
+@pytest.mark.parametrize("with_lm", [False, True])
+def test_multi_step_graph_matches_single_steps(with_lm):
+    """S = 4 steps per graph replay, two replays, against eight eager steps
+    on the same inputs: the state, lengths, page table, free-stack top and
+    cache bytes agree bit for bit after every replay."""
+    S, R = 4, 2
+    if with_lm:
+        w = synth.Workload("multi_lm", B=8, Hq=32, Hkv=8, d=128, N=4,
+                           L_lo=100, L_hi=400, V=8200, sigma_p=3.0,
+                           sigma_q=0.25, D=256, steps=S * R)
+    else:
+        w = synth.C64.with_(name="multi_logits", B=8, steps=S * R)
+    seed = 17
+    lm = None
+    if with_lm:
+        lm = dict(weight=synth.lm_weight(seed, w.V, w.D, DEV)
+                  .to(torch.bfloat16).contiguous())
+
+    def fresh():
+        cache = synth.make_cache(w, seed, DEV)
+        dec = Decoder(w, cache, synth.initial_state(w, seed, DEV), DEV, seed,
+                      lm=lm)
+        return dec, cache
+
+    # Eager reference, recording each step's inputs.
+    dec, cache = fresh()
+    inputs, snaps = [], []
+    for s in range(S * R):
+        st = dec.state
+        if with_lm:
+            first = synth.step_hidden(w, seed, cache["seq_len"],
+                                      st["n_pending"], s, DEV)
+            dec.hidden.copy_(first)
+        else:
+            first = synth.step_logits(w, seed, cache["seq_len"],
+                                      st["n_pending"], s, DEV)
+            dec.logits_cur.copy_(first)
+        q, k, v = synth.make_stride(w, seed, s, DEV)
+        dec.q.copy_(q)
+        dec.k_new.copy_(k)
+        dec.v_new.copy_(v)
+        inputs.append((first, q, k, v))
+        dec.step()
+        if s % S == S - 1:
+            snaps.append(_snap(dec, cache))
+    torch.cuda.synchronize()
+    assert int(dec.status.item()) == isd.OK
+
+    # One graph of S steps, replayed R times.
+    dec2, cache2 = fresh()
+    dec2.capture_multi(S)
+    for r in range(R):
+        for i in range(S):
+            first, q, k, v = inputs[r * S + i]
+            dec2.slots["first"][i].copy_(first)
+            dec2.slots["q"][i].copy_(q)
+            dec2.slots["k_new"][i].copy_(k)
+            dec2.slots["v_new"][i].copy_(v)
+        dec2.replay_multi()
+        torch.cuda.synchronize()
+        assert int(dec2.status.item()) == isd.OK
+        got = _snap(dec2, cache2)
+        for key, ref in snaps[r].items():
+            assert torch.equal(got[key], ref), (r, key)
+    dec2.release_graphs()
