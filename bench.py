@@ -66,6 +66,10 @@ def parse():
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's sequences per GPU (only "
                          "for profiling captures of a smaller case)")
+    ap.add_argument("--vocab", type=int, default=None,
+                    help="override the vocabulary size, keeping the draft "
+                         "noise of the workload's own vocabulary (only for "
+                         "profiling captures of a smaller case)")
     ap.add_argument("--proposal", default="sample", choices=["sample", "argmax"],
                     help="drafts drawn from q (default) or x = argmax q")
     ap.add_argument("--eager", action="store_true",
@@ -413,6 +417,10 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
     w = w.with_(steps=steps + warmup + phase_steps + 2 * n_e2e + 2)
     if args.batch is not None and args.batch != w.B:
         w = w.with_(B=args.batch, name=f"{w.name}_b{args.batch}")
+    if args.vocab is not None and args.vocab != w.V:
+        w = w.with_(V=args.vocab, target_accept=None,
+                    sigma_q=synth.draft_sigma(w),
+                    name=f"{w.name}_v{args.vocab}")
     seed = rank_seed(args.seed, rank)
     cache = synth.make_cache(w, seed, dev)
     st0 = synth.initial_state(w, seed, dev)
