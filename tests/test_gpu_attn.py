@@ -131,6 +131,36 @@ def test_deterministic():
     assert torch.equal(a, b) and torch.equal(la, lb)
 
 
+@pytest.mark.parametrize("num_ctas", [0, 5, 1024])
+def test_workspace_counters_reset_between_calls(num_ctas):
+    """One workspace reused by consecutive calls on different inputs: each
+    call equals a call on a fresh workspace bit for bit (nothing carries
+    over between calls)."""
+    w = _bf(name="reuse", B=3, L_lo=40, L_hi=700)
+    cache = synth.make_cache(w, 4, DEV)
+    a = None
+    ws = None
+    for step in range(3):
+        q, k, v = synth.make_stride(w, 4, step, DEV)
+        out = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=DEV)
+        args = isd.attn_args(q, k, v, cache["k_cache"], cache["v_cache"],
+                             cache["page_table"], cache["seq_len"], out, lse,
+                             None, 1.0 / math.sqrt(w.d), None, num_ctas)
+        if ws is None:
+            ws = torch.zeros(isd.attn_workspace_bytes(args), dtype=torch.uint8,
+                             device=DEV)
+        isd.attn_strided(q, k, v, cache["k_cache"], cache["v_cache"],
+                         cache["page_table"], cache["seq_len"], out=out,
+                         lse=lse, softmax_scale=1.0 / math.sqrt(w.d),
+                         workspace=ws, num_ctas=num_ctas)
+        ref_out, ref_lse = gpu_attention(w, cache, q, k, v, num_ctas=num_ctas)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse), step
+        ref, _ = oracle_attention(w, cache, q, k, v)
+        assert np.abs(f64(out) - ref).max() <= TOL["bf16"]
+
+
 FULL = [synth.SHAPE_8B, synth.C64, synth.SHAPE_32B,
         synth.sweep_workload(8, 2, 0.9), synth.sweep_workload(8, 8, 0.5)]
 
