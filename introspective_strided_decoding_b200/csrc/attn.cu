@@ -30,94 +30,133 @@ struct AttnDev {
 
 // Merges the split-KV partials of each (b, h) segment that straddles CTAs:
 // O = sum_k w_k O_k / sum_k w_k l_k with w_k = 2^((m_k - m*) c) over the
-// CTAs k holding a part (m* = max_k m_k).  One block per (b, h); the CTA
-// ranges come from the starts the attention kernel recorded.  Per 32-row
-// chunk the normalised weights w_k / L are computed once into shared
-// memory, then each thread accumulates float4 columns with independent
-// loads (no dependent load chains per element).
-template <int D>
-__global__ void __launch_bounds__(256) attn_combine_kernel(AttnDev p) {
-  // Shared: [G] partial indices, [G][32] weights, [G + 1] range starts.
+// CTAs k holding a part (m* = max_k m_k).  Block c looks at the boundary
+// between CTAs c and c + 1 and merges the segment that boundary cuts when
+// it is the first boundary inside that segment (so each split segment has
+// one block).  The unit prefix and the CTA range starts come into shared
+// memory in one pass; every later load is independent of the others in its
+// step (the part maxima and sums of a row, the float4 rows of every part).
+constexpr int kCombineThreads = 256;
+constexpr int kCombineChunk = 64;         // parts whose weights are staged
+
+__global__ void __launch_bounds__(kCombineThreads)
+    attn_combine_kernel(AttnDev p) {
   extern __shared__ int s_dyn[];
+  const int B = p.B, G = gridDim.x, c = blockIdx.x, tid = threadIdx.x;
+  const int M = p.M, Hkv = p.Hkv;
+  int* prefix = s_dyn;                    // [B + 1]
+  int* starts = prefix + B + 1;           // [G + 1]
+  int* parts = starts + G + 1;            // [G] part rows
+  float* rowf = reinterpret_cast<float*>(parts + G);   // [2][128]: m* c, 1 / l
+  float* w = rowf + 256;                  // [kCombineChunk][128]
   __shared__ int s_n;
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int B = p.B;
   grid_dep_wait();
-  const int* prefix = p.ws_int;
-  const int G = p.ws_int[B + 1];
-  const int units = (prefix[b + 1] - prefix[b]) / p.Hkv;
-  const int s = prefix[b] + h * units, e = s + units;
-  // The range starts are searched in shared memory: a binary search over
-  // global memory would chain ~log2(G) dependent loads.
-  int* starts = s_dyn + G * 33;
+  for (int i = tid; i <= B; i += blockDim.x) prefix[i] = p.ws_int[i];
   for (int i = tid; i <= G; i += blockDim.x) starts[i] = p.ws_int[B + 2 + i];
   __syncthreads();
-  // CTAs whose range holds unit s and unit e - 1: the last c with
-  // starts[c] <= unit (empty ranges have equal neighbouring starts).
-  auto owner = [&](int u) {
-    int lo = 0, hi = G - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (starts[mid] <= u) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-  };
-  const int cf = owner(s), cl = owner(e - 1);
-  if (cf == cl) return;
-  int* s_part = s_dyn;
-  float* s_w = reinterpret_cast<float*>(s_dyn + G);
-  const int M = p.M, g = p.g, K = p.K, Hq = p.Hq;
+  const int T = starts[G];
+  const int e = starts[c + 1];            // first unit after CTA c
+  if (c + 1 >= G || e >= T) return;
+  int lo = 0, hi = B - 1;                 // the sequence holding unit e
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= e) lo = mid; else hi = mid - 1;
+  }
+  const int b = lo;
+  const int units = (prefix[b + 1] - prefix[b]) / Hkv;
+  const int h = (e - prefix[b]) / units;
+  const int s0 = prefix[b] + h * units, s1 = s0 + units;
+  // No cut at this boundary, or an earlier boundary cuts the segment too.
+  if (e == s0 || starts[c] > s0) return;
   if (tid == 0) {
     int n = 0;
-    for (int cc = cf; cc <= cl; ++cc) {
-      if (starts[cc] == starts[cc + 1]) continue;   // empty range
-      // slot 0: the part that starts at the CTA's own first unit.
-      s_part[n++] = cc * 2 + (starts[cc] < s ? 1 : 0);
+    for (int cc = c; cc < G && starts[cc] < s1; ++cc) {
+      if (starts[cc] == starts[cc + 1]) continue;      // empty range
+      const int slot = cc == c && starts[c] < s0 ? 1 : 0;
+      parts[n++] = (cc * 2 + slot) * M;
     }
     s_n = n;
   }
   __syncthreads();
   const int n = s_n;
   const float c2 = p.scale_log2;
-  for (int r0 = 0; r0 < M; r0 += 32) {
-    const int rows = min(32, M - r0);
-    if (tid < rows) {
-      const int m = r0 + tid;
-      float mstar = -INFINITY;
-      for (int k = 0; k < n; ++k)
-        mstar = fmaxf(mstar, p.part_ml[(size_t)s_part[k] * 2 * M + m]);
-      float l = 0.0f;
-      for (int k = 0; k < n; ++k) {
-        const float* ml = p.part_ml + (size_t)s_part[k] * 2 * M;
-        const float w = ml[m] == -INFINITY ? 0.0f : ex2((ml[m] - mstar) * c2);
-        s_w[k * 32 + tid] = w;
-        l += ml[M + m] * w;
+  // Row m = tid: the maximum and the normaliser over the parts.
+  if (tid < M) {
+    float mstar = -INFINITY;
+    for (int k0 = 0; k0 < n; k0 += 8) {
+      float mk[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        mk[j] = k0 + j < n ? __ldcg(p.part_ml + 2 * (size_t)parts[k0 + j] + tid)
+                           : -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mstar = fmaxf(mstar, mk[j]);
+    }
+    float l = 0.0f;
+    for (int k0 = 0; k0 < n; k0 += 8) {
+      float mk[8], lk[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const bool ok = k0 + j < n;
+        const float* ml = p.part_ml + 2 * (size_t)parts[ok ? k0 + j : 0];
+        mk[j] = ok ? __ldcg(ml + tid) : -INFINITY;
+        lk[j] = ok ? __ldcg(ml + M + tid) : 0.0f;
       }
-      const float inv = 1.0f / l;
-      for (int k = 0; k < n; ++k) s_w[k * 32 + tid] *= inv;
-      if (p.lse) {
-        const int r = m / g, j = m - r * g;
-        p.lse[((size_t)b * K + r) * Hq + h * g + j] =
-            (mstar * c2 + log2f(l)) * kLn2;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (mk[j] != -INFINITY) l += lk[j] * ex2((mk[j] - mstar) * c2);
+    }
+    rowf[tid] = mstar;
+    rowf[128 + tid] = 1.0f / l;
+    if (p.lse) {
+      const int r = tid / p.g, j = tid - r * p.g;
+      p.lse[((size_t)b * p.K + r) * p.Hq + h * p.g + j] =
+          (mstar * c2 + log2f(l)) * kLn2;
+    }
+  }
+  // O: thread (rg, q) owns columns 4q..4q+3 of rows rg + 8i (i < 16).
+  const int q = tid & 31, rg = tid >> 5;
+  float4 acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k0 = 0; k0 < n; k0 += kCombineChunk) {
+    const int kn = min(kCombineChunk, n - k0);
+    __syncthreads();                      // rowf ready / w free again
+    if (tid < M) {
+      for (int j = 0; j < kn; ++j) {
+        const float mk = __ldcg(p.part_ml + 2 * (size_t)parts[k0 + j] + tid);
+        w[j * 128 + tid] = mk == -INFINITY
+                               ? 0.0f
+                               : ex2((mk - rowf[tid]) * c2) * rowf[128 + tid];
       }
     }
     __syncthreads();
-    for (int q = tid; q < rows * (D / 4); q += blockDim.x) {
-      const int rl = q / (D / 4), col = (q - rl * (D / 4)) * 4;
-      const int m = r0 + rl;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int k = 0; k < n; ++k) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(
-            p.part_o + ((size_t)s_part[k] * M + m) * D + col));
-        const float w = s_w[k * 32 + rl];
-        acc.x += v.x * w; acc.y += v.y * w; acc.z += v.z * w; acc.w += v.w * w;
+    for (int j = 0; j < kn; ++j) {
+      const float* po = p.part_o + ((size_t)parts[k0 + j] + rg) * 128 + 4 * q;
+      float4 v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        v[i] = rg + 8 * i < M
+                   ? __ldcg(reinterpret_cast<const float4*>(po + i * 1024))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float wk = w[j * 128 + min(rg + 8 * i, M - 1)];
+        acc[i].x += wk * v[i].x; acc[i].y += wk * v[i].y;
+        acc[i].z += wk * v[i].z; acc[i].w += wk * v[i].w;
       }
-      const int r = m / g, j = m - r * g;
-      __nv_bfloat16* o = p.out + (((size_t)b * K + r) * Hq + h * g + j) * D + col;
-      *reinterpret_cast<uint2*>(o) =
-          make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
     }
-    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int m = rg + 8 * i;
+    if (m < M) {
+      const int r = m / p.g, j = m - r * p.g;
+      *reinterpret_cast<uint2*>(
+          p.out + (((size_t)b * p.K + r) * p.Hq + h * p.g + j) * 128 + 4 * q) =
+          make_uint2(pack_bf16(acc[i].x, acc[i].y),
+                     pack_bf16(acc[i].z, acc[i].w));
+    }
   }
 }
 
@@ -216,15 +255,15 @@ int launch_attn_combine(const isd_attn_args* a, int G, cudaStream_t st) {
   uint8_t* ws = static_cast<uint8_t*>(a->workspace);
   p.ws_int = reinterpret_cast<int32_t*>(ws);
   attn_partial_ptrs(a, G, &p.part_o, &p.part_ml);
-  // Shared memory: G partial indices, G x 32 weights, G + 1 range starts.
-  const size_t smem = (size_t)G * 136 + 4;
-  auto kern = attn_combine_kernel<128>;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  // Shared memory: prefix, starts, part rows, row factors, staged weights.
+  const size_t smem = (size_t)(a->B + 1 + 2 * G + 1) * 4 + 256 * 4 +
+                      (size_t)kCombineChunk * 128 * 4;
+  if (cudaFuncSetAttribute(attn_combine_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return ISD_ERR_CUDA;
-  return launch_pdl(kern, dim3(a->Hkv, a->B), dim3(256), smem, st, p) ==
-                 cudaSuccess
+  return launch_pdl(attn_combine_kernel, dim3(G), dim3(kCombineThreads), smem,
+                    st, p) == cudaSuccess
              ? ISD_OK
              : ISD_ERR_CUDA;
 }
