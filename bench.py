@@ -91,9 +91,9 @@ def parse():
 # profiles/attn_tc_kernel_c64_b16_full.md).  Traffic tracks the algorithmic
 # bytes, so a full launch's traffic is this ratio times its bytes.  Valid
 # only for the kernel source the capture was taken on.
-TRAFFIC_PER_ALGO_BYTE = (331.52 + 8.32) / 332.37
+TRAFFIC_PER_ALGO_BYTE = (331.51 + 7.41) / 332.37
 TRAFFIC_KERNEL_SHA256 = (
-    "96f069e3db985f272e1d85995a5c1efd24e57f6e471c16c30d24a1932e37c2ea")
+    "7ecea19e0e31b5da5e0f02774f322bfaf1f1ceff62ff052288a883029ac02e1f")
 
 
 def attention_traffic(bytes_per_launch):

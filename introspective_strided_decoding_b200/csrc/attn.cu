@@ -80,34 +80,46 @@ __global__ void __launch_bounds__(kCombineThreads)
   __syncthreads();
   const int n = s_n;
   const float c2 = p.scale_log2;
-  // Row m = tid: the maximum and the normaliser over the parts.
+  // Row m = tid: the maximum and the normaliser over the parts.  Up to 8
+  // parts (the usual case) their maxima and sums are loaded once and the
+  // weights come straight from registers.
   if (tid < M) {
-    float mstar = -INFINITY;
-    for (int k0 = 0; k0 < n; k0 += 8) {
-      float mk[8];
+    float mk[8], lk[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        mk[j] = k0 + j < n ? __ldcg(p.part_ml + 2 * (size_t)parts[k0 + j] + tid)
-                           : -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) mstar = fmaxf(mstar, mk[j]);
+    for (int j = 0; j < 8; ++j) {
+      const bool ok = j < n;
+      const float* ml = p.part_ml + 2 * (size_t)parts[ok ? j : 0];
+      mk[j] = ok ? __ldcg(ml + tid) : -INFINITY;
+      lk[j] = ok ? __ldcg(ml + M + tid) : 0.0f;
     }
+    float mstar = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mstar = fmaxf(mstar, mk[j]);
+    for (int k0 = 8; k0 < n; ++k0)
+      mstar = fmaxf(mstar, __ldcg(p.part_ml + 2 * (size_t)parts[k0] + tid));
     float l = 0.0f;
-    for (int k0 = 0; k0 < n; k0 += 8) {
-      float mk[8], lk[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const bool ok = k0 + j < n;
-        const float* ml = p.part_ml + 2 * (size_t)parts[ok ? k0 + j : 0];
-        mk[j] = ok ? __ldcg(ml + tid) : -INFINITY;
-        lk[j] = ok ? __ldcg(ml + M + tid) : 0.0f;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (mk[j] != -INFINITY) l += lk[j] * ex2((mk[j] - mstar) * c2);
+    for (int j = 0; j < 8; ++j) {
+      mk[j] = mk[j] == -INFINITY ? 0.0f : ex2((mk[j] - mstar) * c2);
+      l += lk[j] * mk[j];
+    }
+    for (int k0 = 8; k0 < n; ++k0) {
+      const float* ml = p.part_ml + 2 * (size_t)parts[k0];
+      const float m1 = __ldcg(ml + tid);
+      if (m1 != -INFINITY) l += __ldcg(ml + M + tid) * ex2((m1 - mstar) * c2);
     }
     rowf[tid] = mstar;
     rowf[128 + tid] = 1.0f / l;
+    if (n <= kCombineChunk) {
+      // Weights of the first chunk now (the loop below skips them).
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j < n) w[j * 128 + tid] = mk[j] / l;
+      for (int j = 8; j < n; ++j) {
+        const float m1 = __ldcg(p.part_ml + 2 * (size_t)parts[j] + tid);
+        w[j * 128 + tid] = m1 == -INFINITY ? 0.0f : ex2((m1 - mstar) * c2) / l;
+      }
+    }
     if (p.lse) {
       const int r = tid / p.g, j = tid - r * p.g;
       p.lse[((size_t)b * p.K + r) * p.Hq + h * p.g + j] =
@@ -122,7 +134,7 @@ __global__ void __launch_bounds__(kCombineThreads)
   for (int k0 = 0; k0 < n; k0 += kCombineChunk) {
     const int kn = min(kCombineChunk, n - k0);
     __syncthreads();                      // rowf ready / w free again
-    if (tid < M) {
+    if (tid < M && n > kCombineChunk) {
       for (int j = 0; j < kn; ++j) {
         const float mk = __ldcg(p.part_ml + 2 * (size_t)parts[k0 + j] + tid);
         w[j * 128 + tid] = mk == -INFINITY

@@ -596,20 +596,33 @@ struct MergeParams {
 };
 
 __global__ void __launch_bounds__(256) lm_stats_merge_kernel(MergeParams p) {
+  constexpr int kPer = 16;      // records per sub-chunk at most
   grid_dep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= p.M * p.C) return;
   const int row = i % p.M, c = i / p.M;
-  const int v0 = c * p.per, v1 = min(p.VT, v0 + p.per);
+  const int v0 = c * p.per;
+  // Every record of the sub-chunk is loaded up front (one round trip).
+  float pm[kPer];
+  double ps[kPer];
+  int pi[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const bool ok = k < p.per && v0 + k < p.VT;
+    const size_t o = (size_t)(ok ? v0 + k : v0) * p.M + row;
+    pm[k] = ok ? __ldcg(p.pmax + o) : -INFINITY;
+    ps[k] = ok ? __ldcg(p.psum + o) : 0.0;
+    pi[k] = ok ? __ldcg(p.pidx + o) : 0;
+  }
   float m = -INFINITY;
-  for (int v = v0; v < v1; ++v) m = fmaxf(m, p.pmax[(size_t)v * p.M + row]);
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) m = fmaxf(m, pm[k]);
   double s = 0.0;
   int idx = -1;
-  for (int v = v0; v < v1; ++v) {
-    const size_t o = (size_t)v * p.M + row;
-    const float pm = p.pmax[o];
-    s += p.psum[o] * exp((double)pm - (double)m);
-    if (idx < 0 && pm == m) idx = p.pidx[o];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    if (pm[k] != -INFINITY) s += ps[k] * exp((double)pm[k] - (double)m);
+    if (idx < 0 && pm[k] == m) idx = pi[k];
   }
   const size_t o = (size_t)row * p.C + c;
   p.csum[o] = s;
