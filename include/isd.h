@@ -110,7 +110,10 @@ typedef struct {
   int32_t num_pages, page_table_stride;
   int32_t dtype;
   float softmax_scale;
-  int32_t num_ctas;            /* 0: one CTA per SM; else 1..1024 CTAs    */
+  int32_t num_ctas;            /* 0: one CTA per SM, or fewer for small
+                                  problems (at most one per 40 units of
+                                  the largest work the page table
+                                  admits); else 1..1024 CTAs             */
   const void* q;
   const void* k_new;
   const void* v_new;
