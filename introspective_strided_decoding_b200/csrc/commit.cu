@@ -11,11 +11,13 @@
 //   1. scans the page demand of ALL sequences in sequence order (a few
 //      hundred bytes from L2) and validates the whole commit: lengths and
 //      counts, page-table rows, the pool size, every page id the commit
-//      would write through or pop;
+//      would write through or pop (the free-stack entries below the top are
+//      read while the scan runs);
 //   2. if anything is wrong, writes nothing (the verdict is the same in
 //      every CTA, so the commit is all-or-nothing) and CTA 0 reports it;
 //   3. otherwise records its sequences' new pages in the page table and
-//      copies their committed K/V rows with 16-byte stores;
+//      copies their committed K/V rows with 16-byte stores (the rows' pages
+//      looked up once, eight loads a thread in flight before their stores);
 //   4. counts itself done; the last CTA (a self-resetting counter in the
 //      workspace) grows every seq_len and lowers the free-stack top, once
 //      every CTA has read the old values.
@@ -58,12 +60,18 @@ __global__ void __launch_bounds__(kCommitThreads) commit_kernel(CommitDev p) {
   __shared__ int s_rank;
   __shared__ int s_last;
   __shared__ int s_off[kCommitMaxPer];   // first popped slot of own sequences
+  __shared__ int s_fs[kCommitThreads];   // free_stack[top - 1 - k], k < 256
+  __shared__ int s_pg[2];                // pages of the sequence's new rows
   const int c = blockIdx.x, G = gridDim.x, tid = threadIdx.x;
   if (tid == 0) s_rank = kRankNone;
   grid_dep_wait();
   __syncthreads();
+  // The free-stack top and the first entries below it are read while the
+  // page demand is being scanned (they do not depend on it).
   const int top = *p.free_top;
-  if (tid == 0 && (top < 0 || top > p.P)) atomicMin(&s_rank, kRankBadState);
+  const bool top_ok = top >= 0 && top <= p.P;
+  if (tid == 0 && !top_ok) atomicMin(&s_rank, kRankBadState);
+  s_fs[tid] = top_ok && tid < top ? p.free_stack[top - 1 - tid] : -1;
   // 1. Page demand of every sequence, scanned in sequence order.
   auto need = [&](int b) -> int {
     const int L = p.seq_len[b], n = p.n_commit[b];
@@ -96,7 +104,7 @@ __global__ void __launch_bounds__(kCommitThreads) commit_kernel(CommitDev p) {
   if (rank == kRankNone) {
     // 2. Every page to pop, free_stack[top - total .. top - 1], is an id.
     for (int k = tid; k < total; k += blockDim.x) {
-      const int pg = p.free_stack[top - 1 - k];
+      const int pg = k < kCommitThreads ? s_fs[k] : p.free_stack[top - 1 - k];
       if (pg < 0 || pg >= p.P) atomicMin(&s_rank, kRankBadPage);
     }
     __syncthreads();
@@ -107,6 +115,9 @@ __global__ void __launch_bounds__(kCommitThreads) commit_kernel(CommitDev p) {
     return;   // nothing written; no CTA counts itself, the counter stays 0
   }
   // 3. This CTA's sequences: new pages, then the committed rows.
+  auto popped = [&](int k) {
+    return k < kCommitThreads ? s_fs[k] : p.free_stack[top - 1 - k];
+  };
   const size_t row_bytes = (size_t)p.d * p.esize;   // one head's row
   const int vec_per_head = (int)(row_bytes / 16);
   const int nvec = p.Hkv * vec_per_head;            // per row, K or V
@@ -118,29 +129,55 @@ __global__ void __launch_bounds__(kCommitThreads) commit_kernel(CommitDev p) {
     const int old_pages = (L + kPage - 1) / kPage;
     const int grow = (L + n + kPage - 1) / kPage - old_pages;
     const int off = s_off[k];
-    const int32_t* ptab = p.page_table + (size_t)b * p.stride;
-    if (tid < grow)
-      p.page_table[(size_t)b * p.stride + old_pages + tid] =
-          p.free_stack[top - 1 - (off + tid)];
-    for (int i = tid; i < n * 2 * nvec; i += blockDim.x) {
-      const int r = i / (2 * nvec);
-      const int j2 = i - r * 2 * nvec;
-      const bool is_v = j2 >= nvec;
-      const int j = is_v ? j2 - nvec : j2;
-      const int h = j / vec_per_head, cv = j - h * vec_per_head;
-      const int pos = L + r, lp = pos / kPage;
-      const int page = lp < old_pages
-                           ? ptab[lp]
-                           : p.free_stack[top - 1 - (off + lp - old_pages)];
-      const uint8_t* src = (is_v ? p.v_new : p.k_new) +
-                           (((size_t)b * p.K + r) * p.Hkv + h) * row_bytes +
-                           cv * 16;
-      uint8_t* dst = (is_v ? p.v_cache : p.k_cache) +
-                     (((size_t)page * p.Hkv + h) * kPage + pos % kPage) *
-                         row_bytes +
-                     cv * 16;
-      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+    const int lp0 = L / kPage;                      // first page written
+    // The (at most two) pages the rows land in, and the table entries.
+    if (tid < 2 && lp0 + tid <= (L + n - 1) / kPage) {
+      const int lp = lp0 + tid;
+      s_pg[tid] = lp < old_pages ? p.page_table[(size_t)b * p.stride + lp]
+                                 : popped(off + lp - old_pages);
     }
+    if (tid < grow)
+      p.page_table[(size_t)b * p.stride + old_pages + tid] = popped(off + tid);
+    __syncthreads();
+    // Eight 16-byte vectors a thread in flight before their stores.
+    const int nv = n * 2 * nvec;
+    for (int i0 = 0; i0 < nv; i0 += 8 * blockDim.x) {
+      uint4 val[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * blockDim.x + tid;
+        if (i < nv) {
+          const int r = i / (2 * nvec);
+          const int j2 = i - r * 2 * nvec;
+          const bool is_v = j2 >= nvec;
+          const int j = is_v ? j2 - nvec : j2;
+          const int h = j / vec_per_head, cv = j - h * vec_per_head;
+          const uint8_t* src = (is_v ? p.v_new : p.k_new) +
+                               (((size_t)b * p.K + r) * p.Hkv + h) * row_bytes +
+                               cv * 16;
+          val[u] = __ldg(reinterpret_cast<const uint4*>(src));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * blockDim.x + tid;
+        if (i < nv) {
+          const int r = i / (2 * nvec);
+          const int j2 = i - r * 2 * nvec;
+          const bool is_v = j2 >= nvec;
+          const int j = is_v ? j2 - nvec : j2;
+          const int h = j / vec_per_head, cv = j - h * vec_per_head;
+          const int pos = L + r;
+          const int page = s_pg[pos / kPage - lp0];
+          uint8_t* dst = (is_v ? p.v_cache : p.k_cache) +
+                         (((size_t)page * p.Hkv + h) * kPage + pos % kPage) *
+                             row_bytes +
+                         cv * 16;
+          *reinterpret_cast<uint4*>(dst) = val[u];
+        }
+      }
+    }
+    __syncthreads();                                // s_pg is reused
   }
   // 4. The last CTA publishes the new lengths and the free-stack top.
   __syncthreads();
