@@ -163,12 +163,15 @@ def test_bad_pending_count_is_reported_and_gets_no_lora():
     assert np.array_equal(got[2 * K:3 * K], base[2 * K:3 * K])
 
 
-def test_full_size_sampled():
-    """The C=64 LM head: 512 rows, hidden 4096, vocabulary 151 936, with the
-    rank-128 LoRA (sparse, exact); sampled rows and sub-chunks against the
-    oracle, the rest by properties that hold for any correct result."""
-    B, K, D, V, r = 64, 8, 4096, 151936, 128
-    H, W, A, Bf, n_pending = _lora_inputs(14, B, K, D, V, r, True, [1, 4])
+@pytest.mark.parametrize("B,K,D", [(64, 8, 4096), (32, 16, 5120)])
+def test_full_size_sampled(B, K, D):
+    """The C=64 LM head (512 rows, hidden 4096) and the 32B-shaped one (512
+    rows, hidden 5120), vocabulary 151 936, with the rank-128 LoRA (sparse,
+    exact); sampled rows and sub-chunks against the oracle, the rest by
+    properties that hold for any correct result."""
+    V, r = 151936, 128
+    H, W, A, Bf, n_pending = _lora_inputs(14, B, K, D, V, r, True,
+                                          [1, K // 2])
     logits, vs, st = _gpu(H, W, lora_a=A, lora_b=Bf, lora_scale=1.0,
                           n_pending=n_pending, rows_per_seq=K)
     assert st == isd.OK
@@ -202,10 +205,13 @@ def test_full_size_sampled():
     assert bool(((csum >= 1.0) & (csum <= SUB)).all())
 
 
-def test_fused_step_matches_oracle():
+@pytest.mark.parametrize("proposal", ["sample", "argmax"])
+def test_fused_step_matches_oracle(proposal):
     """Hidden states -> isd_lm_head (logits + statistics) ->
     isd_accept_resample fed by those statistics, in lockstep with the oracle
-    run on its own fp64 logits of the same hidden states."""
+    run on its own fp64 logits of the same hidden states.  With argmax
+    proposals the drafts come straight from the statistics' first-argmax
+    indices."""
     w = synth.Workload("lm_fused", B=8, Hq=32, Hkv=8, d=128, N=4, L_lo=100,
                        L_hi=900, V=151936, target_accept=0.9, D=1024)
     seed, steps = 21, 4
@@ -232,11 +238,14 @@ def test_fused_step_matches_oracle():
                    L=L, s=s):
             return ostep.accept_resample(lc_host, lp_host, ostate["pending"],
                                          ostate["n_pending"], ostate["q_row"],
-                                         L, seed, s, w.N, flip=flip)
+                                         L, seed, s, w.N, proposal=proposal,
+                                         flip=flip)
         ref = oracle()
         o = gpu_accept(lc_dev, lp_dev,
                        torch.as_tensor(L, dtype=torch.int32, device=DEV),
-                       gpu_state_from(ostate, DEV), seed, s, vocab_stats=vs)
+                       gpu_state_from(ostate, DEV), seed, s,
+                       proposal=isd.PROPOSAL_ARGMAX if proposal == "argmax"
+                       else isd.PROPOSAL_SAMPLE, vocab_stats=vs)
         torch.cuda.synchronize()
         assert int(o.status.item()) == isd.OK
         c = compare_accept(o, ref, ostate["n_pending"],
