@@ -70,12 +70,19 @@ constexpr int kNB = 8;                       // pages per block
 constexpr int kKeys = kNB * kPage;           // 128 keys = TMEM lanes
 constexpr int kKH = kKeys * 128;             // one 64-column half of K or V
 constexpr int kTile = 2 * kKH;               // a K or V tile: 32 KB
-constexpr int kSmWarps = 4;
-constexpr int kMmaWarp = 4;
-constexpr int kLoadWarps = 4;                // two K and two V warps
-constexpr int kPagesPerLoader = kNB / 2;     // pages of a block per warp
-constexpr int kPvWarp = 5;                   // issues the P V products
-constexpr int kThreads = (kSmWarps + 2 + kLoadWarps) * 32;   // 320
+// Warp roles for NCH 32-row chunks: softmax warps (warpgroups of four;
+// two for NCH >= 3, splitting the chunks between them), the QK and the P V
+// MMA warps, then the loaders: two K and two V warps, or one of each
+// (covering all 8 pages of a block) next to two softmax warpgroups, which
+// keeps the CTA at 384 threads and 170 registers a thread.  Measured: at
+// 128 rows (the softmax bounds the kernel) two warpgroups are 22% faster;
+// at 64 rows the kernel is near the HBM bound and the single loader warps
+// cost more (16% slower), so 64 rows keep one warpgroup.
+constexpr int sm_warps_of(int nch) { return nch >= 3 ? 8 : 4; }
+constexpr int load_warps_of(int nch) { return nch >= 3 ? 2 : 4; }
+constexpr int threads_of(int nch) {
+  return (sm_warps_of(nch) + 2 + load_warps_of(nch)) * 32;
+}
 constexpr int kBarBytes = 32 * 8;            // mbarriers (2 (SK + SV) + 17)
 // Q and P^T tiles in shared memory for N = 32 * nch padded rows.  Two let
 // the next (b, h) segment start (its Q load, its first softmax) while the
@@ -83,7 +90,8 @@ constexpr int kBarBytes = 32 * 8;            // mbarriers (2 (SK + SV) + 17)
 // short.
 constexpr int nqb_of(int nch) { return nch == 4 ? 1 : 2; }
 constexpr int npb_of(int nch) { return nch >= 3 ? 1 : 2; }
-constexpr int kStaticSmem = 3072;            // __shared__ arrays, rounded up
+// __shared__ arrays of the kernel, rounded up.
+constexpr int static_smem_of(int nch) { return nch >= 3 ? 4096 : 3072; }
 constexpr float kRescaleLog2 = 8.0f;
 
 struct Params {
@@ -139,16 +147,22 @@ ISD_DEV void tmem_scale32(uint32_t taddr, const float* f) {
 }
 
 
-// Named barrier 1 joins the four softmax warps.
-ISD_DEV void sm_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-// OR of `v` over the four softmax warps (also a barrier among them).
-ISD_DEV bool sm_any(bool v) {
+// Named barrier 1 + gi joins the four warps of softmax warpgroup gi;
+// barrier 3 joins every softmax warp (`n` threads).
+ISD_DEV void sm_sync(int gi) {
+  asm volatile("bar.sync %0, 128;" ::"r"(1 + gi) : "memory");
+}
+ISD_DEV void sm_sync_all(int n) {
+  asm volatile("bar.sync 3, %0;" ::"r"(n) : "memory");
+}
+// OR of `v` over the four warps of warpgroup gi (also a barrier among them).
+ISD_DEV bool sm_any(int gi, bool v) {
   uint32_t r;
   asm volatile(
       "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
-      " bar.red.or.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+      " bar.red.or.pred q, %2, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
       : "=r"(r)
-      : "r"((uint32_t)v)
+      : "r"((uint32_t)v), "r"(1 + gi)
       : "memory");
   return r != 0;
 }
@@ -240,16 +254,17 @@ struct EpiIn {
   uint64_t* p_empty;
   uint64_t* o_free;
   const float* m_raw;        // [NOB][N]
-  float* x_red;              // [4][32]
-  float* r_val;              // [32]
+  float* x_red;              // [softmax warps][32]
+  float* r_val;              // [warpgroups][32]
   int g, K, Hq, M, c;
   float c2;
 };
 
 // Stores the finished segment `code` (packed b, h, O buffer, complete,
 // slot) whose last block is `blk`: reduces the per-key row sums over the
-// 128 keys, stages O / l (bf16) or the unnormalised O (fp32, 64 columns
-// at a time) in the P tile of block blk, and writes it with TMA stores
+// 128 keys (each softmax warpgroup its own 32-row chunks), stages O / l
+// (bf16) or the unnormalised O (fp32, 64 columns at a time) in the P tile
+// of block blk, and writes it with TMA stores
 // issued by thread 0; the lse or the partial's max and sum go directly.
 // Runs on the four softmax warps.  Not inlined: its registers would
 // otherwise add to those live across the block loop.  `stage_buf` is a
@@ -262,13 +277,18 @@ __device__ __noinline__ bool store_segment(const EpiIn<NCH>& in, int blk, int co
   constexpr int NOB = NCH <= 2 ? 2 : 1;
   constexpr int PB = NCH * kKeys * 64;
   constexpr uint32_t kO = 0, kL = NOB * N + 2 * N;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, kl = tid;
+  constexpr int kSm = sm_warps_of(NCH), kGroups = kSm / 4;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int kl = tid & 127, gi = tid >> 7, wq = warp & 3;
+  const int ch_lo = gi * ((NCH + kGroups - 1) / kGroups);
+  const int ch_hi = min(NCH, ch_lo + (NCH + kGroups - 1) / kGroups);
+  float* r_val = in.r_val + gi * 32;
   const int b = code >> 12, h = (code >> 3) & 511, tb = (code >> 2) & 1;
   const bool complete = (code >> 1) & 1;
   const int slot = code & 1, M = in.M;
   auto stage_sync = [&]() {    // the earlier store has read its tile
     if (tid == 0) bulk_wait_read();
-    sm_sync();
+    sm_sync_all(kSm * 32);
   };
   // O^T of the segment is complete once the P V of its last block lands:
   // phase blk / NPB of p_empty[blk % NPB], at most one phase past the last
@@ -287,22 +307,23 @@ __device__ __noinline__ bool store_segment(const EpiIn<NCH>& in, int blk, int co
     // one fp32 rows, 64 columns per pass ([M][64] staged).
     if (hb == 1) stage_sync();
 #pragma unroll 1
-    for (int ch = 0; ch < NCH; ++ch) {
+    for (int ch = ch_lo; ch < ch_hi; ++ch) {
       float v[32];
       tmem_ld32(in.tmem_lane + el + ch * 32, v);
       warp_transpose_reduce<false>(v, lane);
       in.x_red[warp * 32 + lane] = v[0];
-      sm_sync();
-      if (warp == 0)
-        in.r_val[lane] = (in.x_red[lane] + in.x_red[32 + lane]) +
-                         (in.x_red[64 + lane] + in.x_red[96 + lane]);
-      sm_sync();
+      sm_sync(gi);
+      if (wq == 0) {
+        const float* xr = in.x_red + gi * 128;
+        r_val[lane] = (xr[lane] + xr[32 + lane]) + (xr[64 + lane] + xr[96 + lane]);
+      }
+      sm_sync(gi);
       float o[32];
       tmem_ld32(in.tmem_lane + eo + ch * 32, o);   // lane = d = kl
       if (complete) {
 #pragma unroll
         for (int q = 0; q < 32; q += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(&in.r_val[q]);
+          const float4 l4 = *reinterpret_cast<const float4*>(&r_val[q]);
           const float inv[4] = {1.0f / l4.x, 1.0f / l4.y, 1.0f / l4.z,
                                 1.0f / l4.w};
 #pragma unroll
@@ -321,13 +342,13 @@ __device__ __noinline__ bool store_segment(const EpiIn<NCH>& in, int blk, int co
             *reinterpret_cast<float*>(stg + col * 256 + (kl & 63) * 4) = o[q];
         }
       }
-      if (warp == 0 && hb == 0) {
+      if (wq == 0 && hb == 0) {
         // lse, or the partial's max and sum: staged for a TMA / bulk store
         // when the layout allows one (plain stores stall behind the KV
         // stream), else written directly.
         const int col = ch * 32 + lane;
         if (col < M) {
-          const float lt = in.r_val[lane], mr = em[col];
+          const float lt = r_val[lane], mr = em[col];
           if (complete) {
             if (in.lse) {
               const float v = (mr * in.c2 + log2f(lt)) * kLn2;
@@ -348,9 +369,9 @@ __device__ __noinline__ bool store_segment(const EpiIn<NCH>& in, int blk, int co
         }
       }
     }
-    // Staged rows -> global through the async proxy.
+    // Staged rows (every warpgroup's) -> global through the async proxy.
     proxy_fence();
-    sm_sync();
+    sm_sync_all(kSm * 32);
     if (tid == 0) {
       if (complete) {
         tma_store_4d(in.tm_out, stg, 0, h * in.g, 0, b);
@@ -370,7 +391,7 @@ __device__ __noinline__ bool store_segment(const EpiIn<NCH>& in, int blk, int co
 
 // NCH: 32-column chunks of the padded query rows (N = 32 * NCH).
 template <int NCH>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_of(NCH), 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kc,
                    const __grid_constant__ CUtensorMap tm_vc,
                    const __grid_constant__ CUtensorMap tm_kn,
@@ -380,6 +401,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_lse, Params p) {
   constexpr int N = 32 * NCH;
+  constexpr int kSm = sm_warps_of(NCH);    // softmax warps
+  constexpr int kGroups = kSm / 4;         // their warpgroups
+  constexpr int kMmaWarp = kSm;            // issues the QK products
+  constexpr int kPvWarp = kSm + 1;         // issues the P V products
+  constexpr int kLoadWarps = load_warps_of(NCH);
+  constexpr int kPagesPerLoader = kNB / (kLoadWarps / 2);   // of a block
   constexpr int QH = N * 128;              // one 64-column half of Q
   // P tile [128 keys][N rows]: 32-row atoms of 128 keys x 64 B (64-byte
   // swizzle), atom a holding rows 32a..32a+31.
@@ -429,8 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int s_bad;
   __shared__ __align__(16) float m_raw[NOB][N];  // reference max per row
   __shared__ __align__(16) float m_sc[N];     // the same times c (-inf kept)
-  __shared__ float x_red[kSmWarps][32];       // cross-warp reduction
-  __shared__ __align__(16) float r_val[32];   // per-row factor of a chunk
+  __shared__ float x_red[kSm][32];            // cross-warp reduction
+  __shared__ __align__(16) float r_val[kGroups][32];  // per-row factors
   __shared__ __align__(128) float ep_small[2 * 128];  // staged lse / max, sum
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -438,23 +465,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     s_bad = 0;
     for (int s = 0; s < SK; ++s) {
-      mbar_init(&k_full[s], 2);             // one arrival per K warp
+      mbar_init(&k_full[s], kLoadWarps / 2);   // one arrival per K warp
       mbar_init(&k_empty[s], 1);
     }
     for (int s = 0; s < SV; ++s) {
-      mbar_init(&v_full[s], 2);             // one arrival per V warp
+      mbar_init(&v_full[s], kLoadWarps / 2);   // one arrival per V warp
       mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], kSmWarps);
-      mbar_init(&p_full[s], kSmWarps);
+      mbar_init(&s_free[s], kSm);
+      mbar_init(&p_full[s], kSm);
       mbar_init(&p_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&q_full[s], 1);             // one expect_tx arrival (TMA)
       mbar_init(&q_empty[s], 1);
-      mbar_init(&o_free[s], kSmWarps);
+      mbar_init(&o_free[s], kSm);
     }
     mbar_init(fin, 2);                      // both MMA warps commit
     fence_barrier_init();
@@ -514,18 +541,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp > kPvWarp) {
     // ------------------------------------------------------------ loaders
-    // Two warps copy K tiles and two copy V tiles, each in its own loop, so
-    // a V slot still in use (its block's softmax and P V pending) never
-    // holds back the next K copy.  Loader warp lw handles pages
-    // 4 (lw & 1) .. 4 (lw & 1) + 3 of every block, and lanes 0..7 issue
-    // their eight TMA boxes (page q = lane / 2, 64-column half lane % 2) in
-    // one instruction: the TMA issue rate, not only the bytes in flight,
-    // bounds the stream.  Each warp registers its TMA bytes, then arrives
+    // K tiles and V tiles are copied by separate warps, each in its own
+    // loop, so a V slot still in use (its block's softmax and P V pending)
+    // never holds back the next K copy.  With two warps of each kind, warp
+    // lw handles pages 4 (lw & 1) .. 4 (lw & 1) + 3 of every block; with one,
+    // all eight.  Lanes 0 .. 2 * pages - 1 issue their TMA boxes (page q =
+    // lane / 2, 64-column half lane % 2) in one instruction: the TMA issue
+    // rate, not only the bytes in flight, bounds the stream.  Each warp registers its TMA bytes, then arrives
     // once per block on k_full (K warps) or v_full (V warps).
     const int lt = tid - (kPvWarp + 1) * 32;
     const int lw = lt >> 5;
-    const bool is_k = lw < 2;
-    const int pg0 = (lw & 1) * kPagesPerLoader;    // first page of the block
+    const bool is_k = lw < kLoadWarps / 2;
+    const int pg0 = (lw % (kLoadWarps / 2)) * kPagesPerLoader;   // first page
     BlockWalk w;
     w.init(prefix, B, Hkv, u0, u1);
     // Page ids of this warp's pages (-1: none or the tail), read two blocks
@@ -729,9 +756,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     failed = failed || fin_failed;
   } else {
     // ---------------------------------------------------------- softmax
-    const int kl = tid;                       // key of the block = TMEM lane
+    // Warpgroup gi (threads 128 gi ..) owns 32-row chunks ch_lo .. ch_hi - 1;
+    // thread kl of a warpgroup owns key kl of the block (TMEM lane kl).
+    const int kl = tid & 127, gi = tid >> 7;
+    const int ch_lo = gi * ((NCH + kGroups - 1) / kGroups);
+    const int ch_hi = min(NCH, ch_lo + (NCH + kGroups - 1) / kGroups);
     const int kp = kl >> 4, rr = kl & 15;     // its page and slot
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float c2 = p.scale_log2;
     BlockWalk w;
     w.init(prefix, B, Hkv, u0, u1);
@@ -752,15 +783,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // stores issued by one thread: per-thread global stores queue behind
     // the KV stream and stall the softmax warps for microseconds.
     int stage_buf = -1;          // P tile a TMA store may still be reading
-    auto stage_sync = [&]() {    // wait for that read (all 128 threads)
+    auto stage_sync = [&]() {    // wait for that read (every softmax warp)
       if (tid == 0) bulk_wait_read();
-      sm_sync();
+      sm_sync_all(kSm * 32);
       stage_buf = -1;
     };
     const EpiIn<NCH> ein{p.out, p.part_o, p.lse, p.part_ml, &tm_out,
                          &tm_part, &tm_lse, ep_small, p.lse_tma, p.ml_bulk,
                          tmem + lane_base, ps, p_empty, o_free, &m_raw[0][0],
-                         &x_red[0][0], r_val, p.g, p.K, p.Hq, M, c, c2};
+                         &x_red[0][0], &r_val[0][0], p.g, p.K, p.Hq, M, c, c2};
     auto epilogue = [&](const Pending& e) {
       failed = store_segment<NCH>(ein, e.blk, e.code, stage_buf, failed);
       stage_buf = e.blk % NPB;
@@ -796,10 +827,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* prow = pt + kl * 64;               // this key's row of P
       const int psw = (kl >> 1) & 3;              // its 64-byte swizzle
 #pragma unroll 1
-      for (int ch = 0; ch < NCH; ++ch) {
+      for (int ch = ch_lo; ch < ch_hi; ++ch) {
         float s[32];
         tmem_ld32(tmem + lane_base + kS + sbuf * N + ch * 32, s);
-        if (ch == NCH - 1) {
+        if (ch == ch_hi - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&s_free[sbuf]);
@@ -853,28 +884,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           load_l();
           need = p_pass() > kRescaleLog2;
         }
-        if (sm_any(need)) {
+        if (sm_any(gi, need)) {
           // Exact block max per row, then move the references.
           float v[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = s[e];
           warp_transpose_reduce<true>(v, lane);
           x_red[warp][lane] = v[0];
-          sm_sync();
-          if (warp == 0) {
+          sm_sync(gi);
+          float* rv = r_val[gi];
+          if ((warp & 3) == 0) {
             const int col = ch * 32 + lane;
-            const float bm = fmaxf(fmaxf(x_red[0][lane], x_red[1][lane]),
-                                   fmaxf(x_red[2][lane], x_red[3][lane]));
+            const int w0 = 4 * gi;
+            const float bm =
+                fmaxf(fmaxf(x_red[w0][lane], x_red[w0 + 1][lane]),
+                      fmaxf(x_red[w0 + 2][lane], x_red[w0 + 3][lane]));
             const float m_old = first ? -INFINITY : m_row[col];
             const float m_new = fmaxf(m_old, bm);
-            r_val[lane] =
-                m_old == -INFINITY ? 0.0f : ex2((m_old - m_new) * c2);
+            rv[lane] = m_old == -INFINITY ? 0.0f : ex2((m_old - m_new) * c2);
             m_row[col] = m_new;
             // Finite stand-in for a row with no key yet, so that masked
             // scores still give 0 and an unmasked one votes.
             m_sc[col] = fmaxf(m_new * c2, -3.0e38f);
           }
-          sm_sync();
+          sm_sync(gi);
           if (!first) {
             // O^T must hold every earlier block's P V before it is scaled.
             // P V of block j completes phase j / NPB of p_empty[j % NPB],
@@ -885,8 +918,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_after();
               o_ready = true;
             }
-            tmem_scale32(tmem + lane_base + o_col + ch * 32, r_val);
-            tmem_scale32(tmem + lane_base + l_col + ch * 32, r_val);
+            tmem_scale32(tmem + lane_base + o_col + ch * 32, rv);
+            tmem_scale32(tmem + lane_base + l_col + ch * 32, rv);
           }
           load_l();
           p_pass();
@@ -958,7 +991,8 @@ constexpr Stages kStagePrefs[] = {{2, 4}, {2, 3}, {2, 2}};
 static Stages tc_stages(int B, int M) {
   const int nch = (M + 31) / 32;
   for (const Stages& st : kStagePrefs)
-    if (tc_smem(B, nch, st.sk, st.sv) + tc::kStaticSmem <= kSmemLimit) return st;
+    if (tc_smem(B, nch, st.sk, st.sv) + tc::static_smem_of(nch) <= kSmemLimit)
+      return st;
   return Stages{0, 0};
 }
 
@@ -1058,7 +1092,7 @@ int launch_attn_tc(const isd_attn_args* a, int G, cudaStream_t st) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return ISD_ERR_CUDA;
-  if (launch_pdl(kern, dim3(G), dim3(tc::kThreads), smem, st, tkc, tvc, tkn,
+  if (launch_pdl(kern, dim3(G), dim3(tc::threads_of(nch)), smem, st, tkc, tvc, tkn,
                  tvn, tout, tpart, tq, tlse, p) != cudaSuccess)
     return ISD_ERR_CUDA;
   return launch_attn_combine(a, G, st);
