@@ -91,9 +91,9 @@ def parse():
 # profiles/attn_tc_kernel_c64_b16_full.md).  Traffic tracks the algorithmic
 # bytes, so a full launch's traffic is this ratio times its bytes.  Valid
 # only for the kernel source the capture was taken on.
-TRAFFIC_PER_ALGO_BYTE = (331.51 + 7.41) / 332.37
+TRAFFIC_PER_ALGO_BYTE = (331.52 + 8.28) / 332.37
 TRAFFIC_KERNEL_SHA256 = (
-    "7ecea19e0e31b5da5e0f02774f322bfaf1f1ceff62ff052288a883029ac02e1f")
+    "36976dbe1f402d9716de47c2f37d0c665acfab2627c5b2b2dfad463b35694446")
 
 
 def attention_traffic(bytes_per_launch):
