@@ -402,6 +402,7 @@ constexpr int kPairEpiWarps = 8;           // two per TMEM lane quarter
 constexpr int kPairRows = 256;             // rows of a pair tile
 constexpr int kPairTn = 256;               // vocabulary entries of a tile
 constexpr int kPairHalf = 128 * 128;       // 128 rows x 64 K (bf16) = 16 KB
+constexpr int kPairAtoms = 2;              // 64-wide K slices per stage
 
 __global__ void __launch_bounds__(kPairThreads, 1)
     lm_pair_kernel(const __grid_constant__ CUtensorMap tm_h,
@@ -409,7 +410,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                    const __grid_constant__ CUtensorMap tm_u,
                    const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_out, Params p) {
-  constexpr int kStage = 2 * kPairHalf;    // hidden half + weight half
+  // A stage: kPairAtoms slices of this CTA's hidden rows, then as many of
+  // its weight rows.
+  constexpr int kStage = 2 * kPairAtoms * kPairHalf;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -460,7 +463,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const Tile x = item(p, pair, npairs, it);
       const int hrow = x.rt * kPairRows + (int)rank * 128;
       const int wrow = x.vt * kPairTn + (int)rank * 128;
-      for (int k = x.k0; k < x.k1; ++k) {
+      for (int k = x.k0; k < x.k1; k += kPairAtoms) {
+        const int na = min(kPairAtoms, x.k1 - k);
         wait_or_fail(&empty[s], ph ^ 1, failed);
         if (lane == 0 && !failed) {
           uint8_t* a = ring + (size_t)s * kStage;
@@ -468,13 +472,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           // The even CTA arms its barrier for both CTAs' bytes; the odd
           // CTA's copies count against it too (possibly first: the
           // transaction count may go below zero until the arming).
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * kStage);
-          if (k < p.kD) {
-            tma_load_2d_pair(a, &tm_h, fb, k * kBK, hrow);
-            tma_load_2d_pair(a + kPairHalf, &tm_w, fb, k * kBK, wrow);
-          } else {
-            tma_load_2d_pair(a, &tm_u, fb, (k - p.kD) * kBK, hrow);
-            tma_load_2d_pair(a + kPairHalf, &tm_b, fb, (k - p.kD) * kBK, wrow);
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 4 * na * kPairHalf);
+          for (int j = 0; j < na; ++j) {
+            const int ka = k + j;
+            uint8_t* aj = a + j * kPairHalf;
+            uint8_t* bj = a + (kPairAtoms + j) * kPairHalf;
+            if (ka < p.kD) {
+              tma_load_2d_pair(aj, &tm_h, fb, ka * kBK, hrow);
+              tma_load_2d_pair(bj, &tm_w, fb, ka * kBK, wrow);
+            } else {
+              tma_load_2d_pair(aj, &tm_u, fb, (ka - p.kD) * kBK, hrow);
+              tma_load_2d_pair(bj, &tm_b, fb, (ka - p.kD) * kBK, wrow);
+            }
           }
         }
         __syncwarp();
@@ -500,17 +509,20 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                              failed);
         acc_ph ^= 1u << buf;
         tc_fence_after();
-        for (int k = x.k0; k < x.k1; ++k) {
+        for (int k = x.k0; k < x.k1; k += kPairAtoms) {
+          const int na = min(kPairAtoms, x.k1 - k);
           wait_or_fail_cluster(&full[s], ph, failed);
           tc_fence_after();
           if (lane == 0 && !failed) {
             const uint32_t a = smem_u32(ring + (size_t)s * kStage);
+            for (int j = 0; j < na; ++j)
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk)
-              umma_pair(tmem + (uint32_t)(buf * kPairTn),
-                        sdesc(a + kk * 32, 16, 1024),
-                        sdesc(a + kPairHalf + kk * 32, 16, 1024), id,
-                        (k > x.k0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < kBK / 16; ++kk)
+                umma_pair(tmem + (uint32_t)(buf * kPairTn),
+                          sdesc(a + j * kPairHalf + kk * 32, 16, 1024),
+                          sdesc(a + (kPairAtoms + j) * kPairHalf + kk * 32, 16,
+                                1024),
+                          id, (k > x.k0 || j > 0 || kk > 0) ? 1u : 0u);
             umma_pair_commit(&empty[s], 0x3);
           }
           __syncwarp();
@@ -916,9 +928,9 @@ int launch_pair(const CUtensorMap& th, const CUtensorMap& tw,
                 const CUtensorMap& tout, lm::Params p, int workers,
                 cudaStream_t st) {
   const size_t fixed = 1024 + (size_t)lm::kPairEpiWarps * lm::kStoreBuf + 256;
-  p.stages = (int)std::min<size_t>((lm::kSmemLimit - fixed) /
-                                       (2 * lm::kPairHalf), 8);
-  const size_t smem = fixed + (size_t)p.stages * 2 * lm::kPairHalf;
+  const size_t stage = (size_t)2 * lm::kPairAtoms * lm::kPairHalf;
+  p.stages = (int)std::min<size_t>((lm::kSmemLimit - fixed) / stage, 8);
+  const size_t smem = fixed + (size_t)p.stages * stage;
   if (cudaFuncSetAttribute(lm::lm_pair_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
