@@ -10,11 +10,11 @@
 //
 // The vocabulary is cut into sub-chunks of 2048 elements, one warp's work
 // (64 elements a lane).  Two kernels, one stream, no inter-CTA waiting:
-//   stats  persistent warps stream the used rows sub-chunk by sub-chunk
-//          with 16-byte loads (each lane keeps the next sub-chunk's eight
-//          loads in flight while it reduces the current one) and store each
+//   stats  persistent warps stream the used rows sub-chunk by sub-chunk,
+//          each warp an equal contiguous range of them, with 16-byte copies
+//          kept in flight ahead of the reduction, and store each
 //          sub-chunk's max, first index of the max and sum of
-//          exp(l - max).                                        [HBM bound]
+//          exp(l - max).                               [HBM and MUFU bound]
 //   draw   grid (sequence, part): every CTA of a sequence merges the
 //          sub-chunk figures of the rows it needs and takes the ratio-test
 //          decision itself (the same inputs and arithmetic in every CTA, so
@@ -241,6 +241,73 @@ ISD_DEV void reduce_sub(const AcceptDev<T>& p, int b, int j, int c,
   }
 }
 
+// bf16 rows: the maximum over packed element pairs (a selection, so the
+// same value as the unpacked compares) and the exponent arguments and sums
+// in paired fp32 arithmetic: (l - m) * log2(e) is formed exactly as in the
+// unpacked path, each sub-chunk group of 8 is summed as two interleaved
+// halves of 4 in fp32, then in fp64.
+ISD_DEV uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+ISD_DEV uint32_t word_of(const uint4& u, int i) {
+  return i == 0 ? u.x : i == 1 ? u.y : i == 2 ? u.z : u.w;
+}
+
+template <>
+ISD_DEV void reduce_sub<__nv_bfloat16>(
+    const AcceptDev<__nv_bfloat16>& p, int b, int j, int c,
+    const Raw8<__nv_bfloat16> (&v)[8]) {
+  const int lane = threadIdx.x & 31;
+  uint32_t mk[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    mk[k] = max_bf16x2(max_bf16x2(v[k].u.x, v[k].u.y),
+                       max_bf16x2(v[k].u.z, v[k].u.w));
+#pragma unroll
+  for (int h = 4; h >= 1; h >>= 1)
+#pragma unroll
+    for (int k = 0; k < h; ++k) mk[k] = max_bf16x2(mk[k], mk[k + h]);
+  float m = fmaxf(__uint_as_float(mk[0] << 16),
+                  __uint_as_float(mk[0] & 0xFFFF0000u));
+  m = warp_max(m);
+  const float2 neg_m = make_float2(-m, -m);
+  const float2 l2e = make_float2(kLog2e, kLog2e);
+  double s = 0.0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t wd = word_of(v[k].u, i);
+      const float2 x = make_float2(__uint_as_float(wd << 16),
+                                   __uint_as_float(wd & 0xFFFF0000u));
+      const float2 d = __fmul2_rn(__fadd2_rn(x, neg_m), l2e);
+      const float2 e = make_float2(ex2(d.x), ex2(d.y));
+      acc = i == 0 ? e : __fadd2_rn(acc, e);
+    }
+    s += (double)(acc.x + acc.y);
+  }
+  s = warp_sum_f64(s);
+  const size_t o = ((size_t)b * p.SR + j) * p.C + c;
+  if (p.argmax) {
+    const int lo = c * kSub;
+    int first = INT_MAX;
+#pragma unroll
+    for (int k = 7; k >= 0; --k)
+#pragma unroll
+      for (int e = 7; e >= 0; --e)
+        if (v[k].at(e) == m) first = lo + (k * 32 + lane) * 8 + e;
+    first = warp_min_int(first);
+    if (lane == 0) p.cidx[o] = first;
+  }
+  if (lane == 0) {
+    p.cmax[o] = m;
+    p.csum[o] = s;
+  }
+}
+
 // Walks one warp's items it, it + W, it + 2W, ... without divisions:
 // W = (dj * B + db) * C + dc is split once, and (j, b, c) advance by
 // (dj, db, dc) with carries.  `used` gives each sequence's rows in use
@@ -307,11 +374,52 @@ __global__ void __launch_bounds__(kStatsWarps * 32)
   }
 }
 
-// The same items and arithmetic for 16-byte aligned bf16 rows, staged
-// through shared memory: each warp owns kStatsStages sub-chunk slots and
-// keeps kStatsStages - 1 sub-chunks in flight with cp.async (16 bytes a
-// lane, 8 per sub-chunk) while it reduces the oldest.  Lane l copies and
-// later reads back exactly its own elements, so a thread's own
+// A warp's share of the used sub-chunks for the shared-memory kernel:
+// items are numbered in memory order (sequence, row, sub-chunk) over the
+// rows in use only, and global warp g of G takes the contiguous range
+// [g T / G, (g + 1) T / G) of the T items, so shares differ by at most one
+// item (a strided walk that skips unused rows leaves some warps a quarter
+// more work than the mean).  pre[b] is the number of rows in use before
+// sequence b, pre[B] the total.
+struct RangeWalk {
+  int b, j, c, left, C;
+  const int* pre;
+  ISD_DEV void init(const int* pre_, int B, int C_, long long g,
+                    long long G) {
+    pre = pre_;
+    C = C_;
+    const long long T = (long long)pre[B] * C;
+    const long long s = g * T / G;
+    left = (int)((g + 1) * T / G - s);
+    const int r = (int)(s / C);
+    c = (int)(s % C);
+    int lo = 0, hi = B;   // the last b with pre[b] <= r
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pre[mid] <= r) lo = mid; else hi = mid;
+    }
+    b = lo;
+    j = r - pre[lo];
+  }
+  // Moves to the next item of the range; the walker stays put once the
+  // range is done, so it never looks past the last row in use.
+  ISD_DEV void step() {
+    if (--left <= 0) return;
+    if (++c < C) return;
+    c = 0;
+    ++j;
+    while (j >= pre[b + 1] - pre[b]) {
+      ++b;
+      j = 0;
+    }
+  }
+};
+
+// The same arithmetic for 16-byte aligned bf16 rows, staged through shared
+// memory: each warp owns kStatsStages sub-chunk slots and keeps
+// kStatsStages - 1 sub-chunks in flight with cp.async (16 bytes a lane, 8
+// per sub-chunk) while it reduces the oldest.  Lane l copies and later
+// reads back exactly its own elements, so a thread's own
 // cp.async.wait_group is the only synchronisation.  A chunk past the row
 // end is not copied; its elements read as -inf.
 constexpr int kStatsStages = 3;
@@ -325,6 +433,12 @@ ISD_DEV void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
 }
 
+// Dynamic shared memory of the kernel below: the slots, then the per-
+// sequence rows in use and their exclusive prefix.
+static inline size_t stats_async_smem(int B) {
+  return (size_t)kStatsSmem + (size_t)(2 * B + 1) * 4;
+}
+
 __global__ void __launch_bounds__(kStatsWarps * 32, 1)
     accept_stats_async_kernel(AcceptDev<__nv_bfloat16> p) {
   constexpr int S = kStatsStages;
@@ -336,16 +450,31 @@ __global__ void __launch_bounds__(kStatsWarps * 32, 1)
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.B;
        i += gridDim.x * blockDim.x)
     p.count[i] = 0;
-  // Rows in use per sequence, once per CTA (0: malformed state).
-  int* s_used = reinterpret_cast<int*>(stats_smem + kStatsSmem);
+  // Rows in use per sequence (0: malformed state), then their prefix.
+  int* s_pre = reinterpret_cast<int*>(stats_smem + kStatsSmem);
+  int* s_used = s_pre + p.B + 1;
   for (int i = threadIdx.x; i < p.B; i += blockDim.x)
     s_used[i] = state_ok(p, i) ? p.n_in[i] + p.N - 1 : 0;
   __syncthreads();
-  auto used = [&](int b) { return s_used[b]; };
-  ItemWalk w;
-  w.init(blockIdx.x * kStatsWarps + warp, (long long)gridDim.x * kStatsWarps,
-         p.B, p.C, p.RU);
-  bool have = w.next_used(used);
+  if (warp == 0) {
+    int carry = 0;
+    if (lane == 0) s_pre[0] = 0;
+    for (int base = 0; base < p.B; base += 32) {
+      int x = base + lane < p.B ? s_used[base + lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (base + lane < p.B) s_pre[base + lane + 1] = carry + x;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+  }
+  __syncthreads();
+  RangeWalk w;
+  w.init(s_pre, p.B, p.C, (long long)blockIdx.x * kStatsWarps + warp,
+         (long long)gridDim.x * kStatsWarps);
+  bool have = w.left > 0;
   // Copies this lane's 8 chunks of the walker's item into slot s.
   auto issue = [&](int s) {
     const __nv_bfloat16* row = p.lc + ((size_t)w.b * p.K + w.j) * p.V;
@@ -366,7 +495,7 @@ __global__ void __launch_bounds__(kStatsWarps * 32, 1)
       qb[s] = w.b; qj[s] = w.j; qc[s] = w.c;
       issue(s);
       w.step();
-      have = w.next_used(used);
+      have = w.left > 0;
     } else {
       qb[s] = -1;
     }
@@ -948,9 +1077,9 @@ static int launch_stats(const AcceptDev<T>& p, int sms, cudaStream_t st) {
 template <>
 int launch_stats<__nv_bfloat16, true>(const AcceptDev<__nv_bfloat16>& p,
                                       int sms, cudaStream_t st) {
-  // Slots, then the rows-in-use table; too many sequences for the table
+  // Slots, then the rows-in-use tables; too many sequences for the tables
   // take the register kernel.
-  const size_t smem = (size_t)kStatsSmem + (size_t)p.B * 4;
+  const size_t smem = stats_async_smem(p.B);
   if (smem > 227 * 1024) {
     const AcceptDev<__nv_bfloat16>& q = p;
     int per_sm = 0;
