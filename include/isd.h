@@ -355,6 +355,11 @@ typedef struct {
 size_t isd_lm_head_workspace_bytes(const isd_lm_head_args* a);
 size_t isd_vocab_stats_bytes(int32_t M, int32_t V);
 int isd_lm_head(const isd_lm_head_args* a, void* stream);
+/* The number of kernels isd_lm_head launches for these arguments on the
+ * current device (the LoRA down-projection and its sum, the GEMM, a split-K
+ * fix-up when the last wave is split, the statistics merge); 0 when the
+ * arguments fail the size checks.  Host only, launches nothing. */
+int isd_lm_head_launches(const isd_lm_head_args* a);
 
 /* Utilities. */
 int isd_abi_version(void);

@@ -18,6 +18,7 @@ int launch_attn_f32(const isd_attn_args* a, cudaStream_t st);
 size_t lm_head_workspace_bytes(const isd_lm_head_args* a);
 size_t vocab_stats_bytes(int M, int V);
 int launch_lm_head(const isd_lm_head_args* a, cudaStream_t st);
+int lm_head_launches(const isd_lm_head_args* a);
 }  // namespace isd
 
 namespace {
@@ -235,6 +236,11 @@ static int lm_head_check(const isd_lm_head_args* a) {
 size_t isd_lm_head_workspace_bytes(const isd_lm_head_args* a) {
   if (lm_head_check(a) != ISD_OK) return 0;
   return isd::lm_head_workspace_bytes(a);
+}
+
+int isd_lm_head_launches(const isd_lm_head_args* a) {
+  if (lm_head_check(a) != ISD_OK) return 0;
+  return isd::lm_head_launches(a);
 }
 
 size_t isd_vocab_stats_bytes(int32_t M, int32_t V) {

@@ -981,6 +981,28 @@ size_t vocab_stats_bytes(int M, int V) {
   return std::max<size_t>(((size_t)M * C * 16 + 255) & ~size_t(255), 256);
 }
 
+// Tiles of the main GEMM and its split-K tail plan (below 64 rows the
+// weight stream bounds the kernel and a lighter last wave gains nothing:
+// measured at M = 8, 2.5% slower with the tail; M = 64 .. 256: 4.5-7%
+// faster).
+int lm_tiles(const isd_lm_head_args* a, const Shape& sh) {
+  const int rows = tile_rows(sh);
+  return ((a->M + rows - 1) / rows) * ((a->V + sh.tn - 1) / sh.tn);
+}
+TailPlan lm_plan(const isd_lm_head_args* a, const Shape& sh, int tiles) {
+  const int Kt = a->D / lm::kBK + a->lora_rank / lm::kBK;
+  return a->M >= 64 ? tail_plan(tiles, lm_workers(sh), Kt)
+                    : tail_plan(tiles, 0, Kt);
+}
+
+int lm_head_launches(const isd_lm_head_args* a) {
+  const Shape sh = lm_shape(a->M);
+  const int tiles = lm_tiles(a, sh);
+  const TailPlan tp = lm_plan(a, sh, tiles);
+  return (a->lora_rank > 0 ? 2 : 0) + 1 + (tp.body < tiles ? 1 : 0) +
+         (a->vocab_stats ? 1 : 0);
+}
+
 int launch_lm_head(const isd_lm_head_args* a, cudaStream_t st) {
   const int M = a->M, D = a->D, V = a->V, r = a->lora_rank;
   const Shape sh = lm_shape(M);
@@ -1032,21 +1054,16 @@ int launch_lm_head(const isd_lm_head_args* a, cudaStream_t st) {
   // 2. logits = [H | U] [W | B]^T with per-tile statistics.
   lm::Params p{};
   p.M = M; p.V = V; p.tn = tn;
-  p.RTn = (M + (sh.pair ? lm::kPairRows : rows_box) - 1) /
-          (sh.pair ? lm::kPairRows : rows_box);
+  p.RTn = (M + tile_rows(sh) - 1) / tile_rows(sh);
   p.VT = (V + tn - 1) / tn; p.kD = D / lm::kBK; p.kR = r / lm::kBK;
-  p.ksplit = 1; p.kps = 0; p.tiles = p.RTn * p.VT; p.mode = 0;
+  p.ksplit = 1; p.kps = 0; p.tiles = lm_tiles(a, sh); p.mode = 0;
   p.status = a->status;
   if (a->vocab_stats) {
     p.pmax = reinterpret_cast<float*>(ws + l.pmax);
     p.psum = reinterpret_cast<double*>(ws + l.psum);
     p.pidx = reinterpret_cast<int32_t*>(ws + l.pidx);
   }
-  // Below 64 rows the weight stream bounds the kernel and a lighter last
-  // wave gains nothing (measured at M = 8: 2.5% slower with the tail;
-  // M = 64 .. 256: 4.5-7% faster).
-  const TailPlan tp = M >= 64 ? tail_plan(p.tiles, lm_workers(sh), p.kD + p.kR)
-                              : tail_plan(p.tiles, 0, p.kD + p.kR);
+  const TailPlan tp = lm_plan(a, sh, p.tiles);
   p.body = tp.body; p.tsplit = tp.tsplit; p.tkps = tp.tkps;
   p.tail = reinterpret_cast<float*>(ws + l.tail);
   int rc = sh.pair ? launch_pair(th, tw, tu, tb, tout, p, tp.workers, st)

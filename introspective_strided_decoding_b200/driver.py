@@ -329,12 +329,11 @@ class Decoder:
     def launches_per_step(self):
         """This library's kernel launches per step: attention (bf16: the
         tcgen05 kernel and the split-segment combine; fp32: one kernel),
-        the accept kernels (statistics, then decision and draws; with an LM
-        head only the second, the statistics coming from the LM head's GEMM
-        and merge kernels, plus the LoRA down-projection and its sum when
-        there is a LoRA) and the commit."""
+        the LM head's kernels when it is part of the step (as the library
+        counts them), the accept kernels (statistics, then decision and
+        draws; with an LM head only the second, the statistics coming from
+        the LM head) and the commit."""
         attn = 2 if self.w.dtype == "bf16" else 1
         if self.lm is None:
             return attn + 2 + 1
-        lora = 2 if self.lm.get("lora_a") is not None else 0
-        return attn + 2 + lora + 1 + 1
+        return attn + isd.lm_head_launches(self._lm[0]) + 1 + 1

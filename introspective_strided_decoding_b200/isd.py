@@ -99,6 +99,7 @@ SIGNATURES = {
     "isd_lm_head_workspace_bytes": (ctypes.c_size_t,
                                     [ctypes.POINTER(LmHeadArgs)]),
     "isd_vocab_stats_bytes": (ctypes.c_size_t, [_I32, _I32]),
+    "isd_lm_head_launches": (ctypes.c_int, [ctypes.POINTER(LmHeadArgs)]),
     "isd_lm_head": (ctypes.c_int, [ctypes.POINTER(LmHeadArgs), _VP]),
     "isd_abi_version": (ctypes.c_int, []),
     "isd_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -445,6 +446,11 @@ def lm_head_args(hidden, weight, logits, vocab_stats=None, lora_a=None,
 
 def lm_head_workspace_bytes(args):
     return int(lib().isd_lm_head_workspace_bytes(ctypes.byref(args)))
+
+
+def lm_head_launches(args):
+    """Kernels isd_lm_head launches for ``args`` on the current device."""
+    return int(lib().isd_lm_head_launches(ctypes.byref(args)))
 
 
 def lm_head(hidden, weight, logits, vocab_stats=None, lora_a=None,

@@ -225,3 +225,16 @@ def test_lm_head_workspace_and_stats_sizes(lib):
     assert lib.isd_vocab_stats_bytes(512, 151936) >= 512 * 75 * 16
     assert lib.isd_vocab_stats_bytes(0, 10) == 0
     assert lib.isd_lm_head_workspace_bytes(ctypes.byref(_lm_args(M=0))) == 0
+
+
+def test_lm_head_launch_count(lib):
+    # Below 64 rows there is never a split-K tail, so the count does not
+    # depend on the device: the GEMM, the statistics merge, the LoRA
+    # down-projection and its sum.
+    a = _lm_args(M=32)
+    assert lib.isd_lm_head_launches(ctypes.byref(a)) == 1
+    a.vocab_stats = _FAKE * 5
+    assert lib.isd_lm_head_launches(ctypes.byref(a)) == 2
+    a.lora_rank, a.lora_a, a.lora_b, a.n_pending = 128, _FAKE, _FAKE, _FAKE
+    assert lib.isd_lm_head_launches(ctypes.byref(a)) == 4
+    assert lib.isd_lm_head_launches(ctypes.byref(_lm_args(M=0))) == 0
