@@ -15,9 +15,13 @@ flushed before every timed step.
 
 Prints one JSON line (rank 0) per workload (the default: one).  ``value`` is
 accepted (committed) tokens per second over all ranks: every step runs as
-one replay of the captured CUDA graph of the three library calls (the
-serving path), device-timed with CUDA events around it, max over ranks.
-``--eager`` times the three calls launched one by one instead.  With N > 1
+one replay of the captured CUDA graph of the library calls (the serving
+path: isd_attn_strided, then isd_accept_commit, the accept step with the KV
+commit running beside its draws), device-timed with CUDA events around it,
+max over ranks.  ``--eager`` times the same calls launched one by one
+instead.  The per-phase split in ``detail`` comes from further eager steps
+with the accept and commit as separate calls (isd_accept_resample,
+isd_kv_commit), events between them.  With N > 1
 every rank runs its own replica (the path shards by sequence; no
 collective on the data path).
 
@@ -616,8 +620,8 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
            "steps": n_e2e}
     alpha = accepted / max(tested, 1)
     tpf = tokens / (w.B * steps)
-    calls = ("attention+LM head+accept+commit" if with_lm
-             else "attention+accept+commit")
+    calls = ("attention+LM head+accept/commit" if with_lm
+             else "attention+accept/commit")
     inputs = "hidden-state" if with_lm else "logits"
     attn_roof = {
         "kernel": "attn_tc_kernel (+combine)", "bound": "hbm",
@@ -661,7 +665,8 @@ def run_workload(w, args, world, rank, local, steps, warmup, with_cpu):
             "attention_ms": sum(t_attn) / phase_steps,
             "accept_ms": sum(t_acc) / phase_steps,
             "commit_ms": sum(t_com) / phase_steps,
-            "phase_split": f"eager calls, {phase_steps} further steps",
+            "phase_split": f"eager calls, {phase_steps} further steps, "
+                           "accept and commit as separate calls",
             "steps_per_s": steps / (total_ms / 1e3),
             "step_gbs": step_gbs,
             "step_frac": None if step_gbs is None else step_gbs / hbm_peak,

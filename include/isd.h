@@ -16,6 +16,8 @@
  *   isd_accept_resample  vocab softmax stats, ratio test, resample / bonus /
  *                        draft sampling
  *   isd_kv_commit        commit of the accepted prefix, rollback of the rest
+ * or two, the last two fused: isd_accept_commit (the same results, with the
+ * commit running beside the draws).
  *
  * Conventions shared by every call
  * --------------------------------
@@ -298,6 +300,21 @@ typedef struct {
 
 size_t isd_commit_workspace_bytes(const isd_commit_args* a);
 int isd_kv_commit(const isd_commit_args* a, void* stream);
+
+/* ------------------------------------------------------------------------
+ * isd_accept_commit -- isd_accept_resample(a) followed by isd_kv_commit(c)
+ * in one call, with the same outputs, state and status as those two calls
+ * in that order.  The KV commit needs only the decisions (n_commit), not
+ * the draws ("Serving (SGLang)": the commit of the accepted prefix), so
+ * after the statistics and the ratio-test decisions the commit runs and the
+ * residual / bonus / draft draws run beside it.  c must describe the same
+ * sequences: c->B == a->B, c->K == a->K, c->n_commit == a->n_commit and
+ * c->seq_len == a->seq_len (else ISD_ERR_INVALID_ARG); every other rule of
+ * the two calls applies unchanged (both workspaces, both checks, checked
+ * before anything is launched).
+ * ---------------------------------------------------------------------- */
+int isd_accept_commit(const isd_accept_args* a, const isd_commit_args* c,
+                      void* stream);
 
 /* ------------------------------------------------------------------------
  * isd_lm_head -- the LM head that makes a step's logits, with the R-ISD

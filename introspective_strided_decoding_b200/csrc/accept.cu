@@ -9,20 +9,20 @@
 // that rule; the row layout is the stride schedule stated in isd.h.
 //
 // The vocabulary is cut into sub-chunks of 2048 elements, one warp's work
-// (64 elements a lane).  Two kernels, one stream, no inter-CTA waiting:
+// (64 elements a lane).  Three kernels, one stream, no inter-CTA waiting:
 //   stats  persistent warps stream the used rows sub-chunk by sub-chunk,
 //          each warp an equal contiguous range of them, with 16-byte copies
 //          kept in flight ahead of the reduction, and store each
 //          sub-chunk's max, first index of the max and sum of
 //          exp(l - max).                               [HBM and MUFU bound]
-//   draw   grid (sequence, part): every CTA of a sequence merges the
-//          sub-chunk figures of the rows it needs and takes the ratio-test
-//          decision itself (the same inputs and arithmetic in every CTA, so
-//          the same decision); part 0 writes the decision's outputs.  Then
-//          rejected sequences: part y sums max(0, p - q) over sub-chunks
-//          4y .. 4y+3 (two warps each) and the part that finishes last
-//          (atomic count, no waiting) draws the replacement; accepted
-//          sequences: part t draws token t (the bonus, then the drafts).
+//   decide one CTA per sequence merges the sub-chunk figures into row
+//          statistics, takes the ratio-test decision, writes its outputs
+//          and leaves a record (decision, row max and sum of every row).
+//   draw   grid (sequence, part) reads the record.  Rejected sequences:
+//          part y sums max(0, p - q) over sub-chunks 4y .. 4y+3 (two warps
+//          each) and the part that finishes last (atomic count, no
+//          waiting) draws the replacement; accepted sequences: part t draws
+//          token t (the bonus, then the drafts); other parts leave at once.
 //          A draw picks the sub-chunk from a warp scan of the sub-chunk
 //          masses, then scans its 2048 elements with eight warps of 256,
 //          all in ascending vocabulary order.               [latency bound]
@@ -80,8 +80,12 @@ struct AcceptDev {
   float* cmax;         // [B][SR][C] sub-chunk max
   int32_t* cidx;       // [B][SR][C] first index of the sub-chunk max
   double* resid;       // [B][C] residual sub-chunk mass
-  int32_t* count;      // [B] residual parts finished (zeroed by stats)
+  int32_t* count;      // [B] residual parts finished (zeroed by decide)
+  int32_t* dec;        // [B][4] decision: flags (1 valid, 2 rejected), a, n, L
+  float* rm;           // [B][RU] row max of every row (decide kernel)
+  double* rs;          // [B][RU] row sum of every row
   int argmax;          // drafts are argmax q (point-mass proposals)
+  int draw_nowait;     // draw launched behind the commit: no wait
 };
 
 // Eight consecutive elements kept in their storage format until use
@@ -349,10 +353,6 @@ template <typename T, bool kVec>
 __global__ void __launch_bounds__(kStatsWarps * 32)
     accept_stats_kernel(AcceptDev<T> p) {
   grid_dep_wait();
-  // The draw kernel's residual counters start at zero.
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.B;
-       i += gridDim.x * blockDim.x)
-    p.count[i] = 0;
   auto used = [&](int b) {
     return state_ok(p, b) ? p.n_in[b] + p.N - 1 : 0;
   };
@@ -447,9 +447,6 @@ __global__ void __launch_bounds__(kStatsWarps * 32, 1)
   __nv_bfloat16* slots =
       reinterpret_cast<__nv_bfloat16*>(stats_smem) + (size_t)warp * S * kSub;
   grid_dep_wait();
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.B;
-       i += gridDim.x * blockDim.x)
-    p.count[i] = 0;
   // Rows in use per sequence (0: malformed state), then their prefix.
   int* s_pre = reinterpret_cast<int*>(stats_smem + kStatsSmem);
   int* s_used = s_pre + p.B + 1;
@@ -573,11 +570,13 @@ ISD_DEV float resid_w(const ResidRows& r, float lpv, float lqv, int v) {
 }
 
 // The rows of a rejection at draft a + 1: p from row a of logits_cur (its
-// max and sum `mp`, `sp`), q from the stored row of that draft.
+// max and sum `mp`, `sp`), q from the stored row of that draft (`x`, `qr`,
+// `zhi` + `zlo`: the draft's token, q row and log-normaliser).
 template <typename T>
 ISD_DEV ResidRows resid_rows(const AcceptDev<T>& p, int b, int a, float mp,
-                             double sp, const T*& prow, const T*& qrow) {
-  const int N = p.N, K = p.K;
+                             double sp, int x, int qr, float zhi, float zlo,
+                             const T*& prow, const T*& qrow) {
+  const int K = p.K;
   prow = p.lc + ((size_t)b * K + a) * p.V;
   ResidRows r;
   r.mp = mp;
@@ -585,12 +584,11 @@ ISD_DEV ResidRows resid_rows(const AcceptDev<T>& p, int b, int a, float mp,
   if (p.argmax) {
     qrow = prow;                       // not read
     r.zq_hi = r.zq_lo = r.c_hi = r.c_lo = 0.0f;
-    r.x = p.pending_in[b * N + a + 1];
+    r.x = x;
   } else {
-    const int qr = p.q_row_in[b * N + a + 1];
     qrow = p.lp + ((size_t)b * K + qr) * p.V;
-    r.zq_hi = p.q_stats_in[(b * N + a + 1) * 2];
-    r.zq_lo = p.q_stats_in[(b * N + a + 1) * 2 + 1];
+    r.zq_hi = zhi;
+    r.zq_lo = zlo;
     const double c = ((double)mp + log(sp)) - ((double)r.zq_hi + (double)r.zq_lo);
     r.c_hi = (float)c;
     r.c_lo = (float)(c - (double)r.c_hi);
@@ -599,25 +597,11 @@ ISD_DEV ResidRows resid_rows(const AcceptDev<T>& p, int b, int a, float mp,
   return r;
 }
 
-// What a CTA of the draw kernel shares between its warps.
-struct DrawShared {
-  float m[kMaxRows];           // row max of the merged rows
-  double s[kMaxRows];          // row sum
-  double mass[2][kMaxSub];     // sub-chunk masses of the two candidate draw rows
-  double tot[kDrawWarps];      // per-warp totals of an element scan
-  int lastp[kDrawWarps];       // per-warp last positive element
-  double rem;                  // target left inside the chosen sub-chunk
-  int chosen;                  // chosen sub-chunk
-  int found;                   // warp holding the target (-1: none)
-  int ok, n, rejected, a, last, mode;
-};
-
 // Row statistics from the sub-chunk figures, by one warp: m = max of the
 // sub-chunk maxima, s = sum_c csum_c * exp(cmax_c - m) (fp64, fixed order).
-// With `mass` set, also the sub-chunk masses csum_c * exp(cmax_c - m).
 template <typename T>
 ISD_DEV void merge_row(const AcceptDev<T>& p, int b, int r, float& m_out,
-                       double& s_out, double* mass) {
+                       double& s_out) {
   const int lane = threadIdx.x & 31;
   const size_t o = ((size_t)b * p.SR + r) * p.C;
   float cm[kSubPerLane];
@@ -635,42 +619,183 @@ ISD_DEV void merge_row(const AcceptDev<T>& p, int b, int r, float& m_out,
 #pragma unroll
   for (int i = 0; i < kSubPerLane; ++i) {
     const int c = lane * kSubPerLane + i;
-    const double mc = c < p.C ? cs[i] * exp((double)(cm[i] - m)) : 0.0;
-    if (mass && c < kMaxSub) mass[c] = mc;
-    s += mc;
+    s += c < p.C ? cs[i] * exp((double)(cm[i] - m)) : 0.0;
   }
   m_out = m;
   s_out = warp_sum_f64(s);
 }
 
+// ---------------------------------------------------------------------------
+// Decide: one CTA per sequence merges the sub-chunk figures of every row
+// into row statistics (warps 1..7), takes the ratio-test decision (warp 0)
+// and writes the decision's outputs, plus a record for the draw kernel:
+// dec[b] = (flags: 1 valid, 2 rejected; a; n; the sequence length L it
+// read) and the row max / sum of every row.  The draw kernel reads L from
+// the record, not from seq_len, so a commit may grow seq_len meanwhile.
+struct DecideShared {
+  float m[kMaxRows];           // row max
+  double s[kMaxRows];          // row sum
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kDrawWarps * 32)
+    accept_decide_kernel(AcceptDev<T> p) {
+  __shared__ DecideShared sh;
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = p.N, K = p.K;
+  grid_dep_wait();
+  // ---- 0. The sequence's state and its drafts' logits (warp 0).
+  int n = 0, L = 0, tok = 0, qr = 0;
+  float zhi = 0.0f, zlo = 0.0f, lx = 0.0f, lqx = 0.0f;
+  bool ok = false;
+  if (warp == 0) {
+    n = p.n_in[b];
+    L = p.seq_len[b];
+    tok = lane < N ? p.pending_in[b * N + lane] : 0;
+    qr = lane < N ? p.q_row_in[b * N + lane] : 0;
+    if (!p.argmax && lane < N) {
+      zhi = p.q_stats_in[(b * N + lane) * 2];
+      zlo = p.q_stats_in[(b * N + lane) * 2 + 1];
+    }
+    ok = (n == 1 || n == N) && L >= 0;
+    if (ok && lane < n) ok = tok >= 0 && tok < p.V;
+    if (ok && lane >= 1 && lane < n) ok = qr >= 0 && qr < K;
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && lane >= 1 && lane < n) {
+      lx = to_f(p.lc[((size_t)b * K + lane - 1) * p.V + tok]);
+      if (!p.argmax) lqx = to_f(p.lp[((size_t)b * K + qr) * p.V + tok]);
+    }
+  }
+  if (threadIdx.x == 0) p.count[b] = 0;   // the draw kernel's residual parts
+  // ---- 1. Row statistics of every row (warps 1..).
+  if (warp > 0) {
+    for (int r = warp - 1; r < p.RU; r += kDrawWarps - 1) {
+      float m;
+      double s;
+      merge_row(p, b, r, m, s);
+      if (lane == 0) {
+        sh.m[r] = m;
+        sh.s[r] = s;
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < p.RU) {
+    p.rm[(size_t)b * p.RU + threadIdx.x] = sh.m[threadIdx.x];
+    p.rs[(size_t)b * p.RU + threadIdx.x] = sh.s[threadIdx.x];
+  }
+  if (warp != 0) return;
+  if (!ok) {
+    // Malformed state: reported once, passed through, nothing committed.
+    if (lane == 0) {
+      report(p.status, ISD_ERR_BAD_STATE);
+      p.n_commit[b] = 0;
+      p.n_out[b] = n;
+      *reinterpret_cast<int4*>(p.dec + 4 * b) = make_int4(0, 0, n, L);
+    }
+    if (lane < N) {
+      const int i = b * N + lane;
+      p.commit_tokens[i] = -1;
+      p.pending_out[i] = p.pending_in[i];
+      p.q_row_out[i] = p.q_row_in[i];
+      p.q_stats_out[2 * i] = p.q_stats_in[2 * i];
+      p.q_stats_out[2 * i + 1] = p.q_stats_in[2 * i + 1];
+    }
+    return;
+  }
+  // ---- 2. Ratio tests of drafts 1 .. n-1 (lane i verifies draft i with
+  //         row i-1); l - m is exact in fp32; p, q, the ratio fp64.
+  const int rows_used = n + N - 1;
+  const bool verifies = lane >= 1 && lane < n;
+  bool acc = true;
+  double r = 0.0;
+  if (verifies) {
+    const double px = exp((double)(lx - sh.m[lane - 1])) / sh.s[lane - 1];
+    double qx = 1.0;      // argmax drafts: the proposal is a point mass
+    if (!p.argmax) qx = exp(((double)lqx - (double)zhi) - (double)zlo);
+    r = qx > 0.0 ? px / qx : INFINITY;
+    const float u = uniform(p.seed, (uint32_t)b, step_of(p),
+                            (uint32_t)(L + lane), ISD_STREAM_ACCEPT);
+    acc = (double)u < r;
+  }
+  const uint32_t mask = __ballot_sync(0xffffffffu, acc);
+  const uint32_t drafts = ((n >= 32) ? 0xffffffffu : ((1u << n) - 1u)) & ~1u;
+  const uint32_t rej = drafts & ~mask;
+  const bool rejected = rej != 0u;
+  const int a = rejected ? (__ffs(rej) - 2) : (n - 1);
+  // The decision's outputs.
+  if (verifies && p.ratio_out) p.ratio_out[b * N + lane] = (float)r;
+  if (lane < N) {
+    p.commit_tokens[b * N + lane] = lane <= a ? tok : -1;
+    // Next drafts' q rows and the log-normaliser log sum_v exp(l_v) of
+    // each (lane j: row n + j - 1), stored as a float pair hi + lo.
+    const bool has = !rejected && lane >= 1;
+    const int src = n + lane - 1;
+    p.q_row_out[b * N + lane] = has ? src : -1;
+    const double lz = has ? (double)sh.m[src] + log(sh.s[src]) : 0.0;
+    const float lz_hi = (float)lz;
+    p.q_stats_out[(b * N + lane) * 2] = lz_hi;
+    p.q_stats_out[(b * N + lane) * 2 + 1] = (float)(lz - (double)lz_hi);
+    // After a rejection only the replacement is pending.
+    if (rejected && lane >= 1) p.pending_out[b * N + lane] = -1;
+  }
+  if (p.row_stats_out && lane < rows_used) {
+    p.row_stats_out[(b * K + lane) * 2] = sh.m[lane];
+    p.row_stats_out[(b * K + lane) * 2 + 1] = (float)sh.s[lane];
+  }
+  if (lane == 0) {
+    p.n_commit[b] = a + 1;
+    p.n_out[b] = rejected ? 1 : N;
+    *reinterpret_cast<int4*>(p.dec + 4 * b) =
+        make_int4(rejected ? 3 : 1, a, n, L);
+  }
+}
+
+// What a CTA of the draw kernel shares between its warps.
+struct DrawShared {
+  float m[kMaxRows];           // row max (from the decide record)
+  double s[kMaxRows];          // row sum
+  int tok[kMaxRows];           // pending tokens (drafts)
+  int qr[kMaxRows];            // their q rows
+  float zq[kMaxRows][2];       // their q log-normalisers (hi, lo)
+  double tot[kDrawWarps];      // per-warp totals of an element scan
+  int lastp[kDrawWarps];       // per-warp last positive element
+  double rem;                  // target left inside the chosen sub-chunk
+  int chosen;                  // chosen sub-chunk
+  int found;                   // warp holding the target (-1: none)
+  int ok, n, rejected, a, last, mode, L;
+};
+
 // One inverse-CDF draw by the whole CTA: the smallest index whose running
 // mass (ascending order) exceeds u * total.  Sub-chunk masses: the
 // residual's from `resid` (mode 0, written by this kernel; if their total
 // is zero, p == q up to rounding, the draw falls back to p of row `row`),
-// or `mass` (mode 1: row `row` of logits_cur, row max m_row).
+// or those of row `row` of logits_cur (mode 1, row max m_row):
+// csum_c * exp(cmax_c - m_row).
 template <typename T, bool kVec>
 ISD_DEV int cta_draw(const AcceptDev<T>& p, DrawShared& sh, int b, int mode,
-                     int row, float m_row, const double* mass,
-                     const ResidRows& rr, const T* prow, const T* qrow,
-                     float u) {
+                     int row, float m_row, const ResidRows& rr,
+                     const T* prow, const T* qrow, float u) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, C = p.C;
   // 1. The sub-chunk (warp 0): lane l owns sub-chunks 4l .. 4l+3.
   if (warp == 0) {
     double mc[kSubPerLane];
     double own = 0.0;
+    double excl = 0.0, incl = 0.0, total = 0.0;
+    if (mode == 0) {
 #pragma unroll
-    for (int i = 0; i < kSubPerLane; ++i) {
-      const int c = lane * kSubPerLane + i;
-      mc[i] = 0.0;
-      if (c < C) mc[i] = mode == 0 ? __ldcg(&p.resid[(size_t)b * C + c]) : mass[c];
-      own += mc[i];
-    }
-    double excl;
-    double incl = warp_scan_f64(own, excl);
-    double total = __shfl_sync(0xffffffffu, incl, 31);
-    if (mode == 0 && !(total > 0.0)) {
+      for (int i = 0; i < kSubPerLane; ++i) {
+        const int c = lane * kSubPerLane + i;
+        mc[i] = c < C ? __ldcg(&p.resid[(size_t)b * C + c]) : 0.0;
+        own += mc[i];
+      }
+      incl = warp_scan_f64(own, excl);
+      total = __shfl_sync(0xffffffffu, incl, 31);
       // Zero residual mass: draw from p of row `row` instead.
-      mode = 1;
+      if (!(total > 0.0)) mode = 1;
+    }
+    if (mode == 1) {
       const size_t o = ((size_t)b * p.SR + row) * C;
       own = 0.0;
 #pragma unroll
@@ -778,12 +903,11 @@ ISD_DEV int cta_draw(const AcceptDev<T>& p, DrawShared& sh, int b, int mode,
   return tok;   // valid on every thread when found < 0, else on warp `found`
 }
 
-// The draw kernel.  Row figures are merged before the sequence's mode is
-// known, for both modes' candidate rows, so the merge loads overlap the
-// state loads: part 0 merges every row (0 .. 2N-2), part y >= 1 the ratio
-// test rows 0 .. N-2 and its two candidate draw rows, y (R mode, n = 1)
-// and N + y - 1 (S mode, n = N); the candidate draw rows also keep their
-// sub-chunk masses in shared memory for the draw.
+// The draw kernel, grid (sequence, part), after the decide kernel: it reads
+// the decision record, then rejected sequences sum the residual over their
+// parts' sub-chunks and the part that finishes last draws the replacement;
+// accepted sequences draw token y in part y (the bonus, then the drafts).
+// Parts with nothing to do leave as soon as the record is read.
 template <typename T, bool kVec>
 __global__ void __launch_bounds__(kDrawWarps * 32)
     accept_draw_kernel(AcceptDev<T> p) {
@@ -791,151 +915,49 @@ __global__ void __launch_bounds__(kDrawWarps * 32)
   const int b = blockIdx.x, y = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = p.N, K = p.K;
-  grid_dep_wait();
-  // ---- 0. The sequence's state (warp 0) and the row merges (warps 1..).
-  int n = 0, L = 0, tok = 0, qr = 0;
-  float zhi = 0.0f, zlo = 0.0f;
+  // Behind the commit (isd_accept_commit) the draws do not wait: the
+  // commit triggered this grid after its own wait, so the decide kernel
+  // and everything before it have finished, and the two kernels touch
+  // disjoint memory.
+  if (!p.draw_nowait) grid_dep_wait();
+  // ---- 0. The sequence's inputs and the decision record.
   if (warp == 0) {
-    n = p.n_in[b];
-    L = p.seq_len[b];
-    tok = lane < N ? p.pending_in[b * N + lane] : 0;
-    qr = lane < N ? p.q_row_in[b * N + lane] : 0;
-    if (!p.argmax && lane < N) {
-      zhi = p.q_stats_in[(b * N + lane) * 2];
-      zlo = p.q_stats_in[(b * N + lane) * 2 + 1];
-    }
-  } else {
-    // Merge list: part 0 every row; part y >= 1 rows 0 .. N-2, then its
-    // candidate draw rows (y when it is not already listed, N + y - 1).
-    const int cand_r = (y >= 1 && y < N) ? y : -1;           // R mode
-    const int cand_s = (y >= 1 && y < N) ? N + y - 1 : -1;   // S mode
-    const bool r_listed = cand_r >= 0 && cand_r <= N - 2;
-    const int nlist = y == 0 ? p.RU
-                             : (N - 1) + (cand_r >= 0 && !r_listed ? 1 : 0) +
-                                   (cand_s >= 0 ? 1 : 0);
-    for (int k = warp - 1; k < nlist; k += kDrawWarps - 1) {
-      int r = k;
-      if (y >= 1 && k >= N - 1)
-        r = (k == N - 1 && cand_r >= 0 && !r_listed) ? cand_r : cand_s;
-      // Candidate draw rows keep their masses: slot 0 the R-mode row, slot
-      // 1 the S-mode row (part 0: the bonus rows 0 and N - 1).
-      double* keep = nullptr;
-      if (y == 0) {
-        keep = r == 0 ? sh.mass[0] : (r == N - 1 ? sh.mass[1] : nullptr);
-      } else {
-        keep = r == cand_r ? sh.mass[0] : (r == cand_s ? sh.mass[1] : nullptr);
-      }
-      float m;
-      double s;
-      merge_row(p, b, r, m, s, keep);
-      if (lane == 0) {
-        sh.m[r] = m;
-        sh.s[r] = s;
-      }
+    if (lane < N) {
+      sh.tok[lane] = p.pending_in[b * N + lane];
+      sh.qr[lane] = p.q_row_in[b * N + lane];
+      sh.zq[lane][0] = p.argmax ? 0.0f : p.q_stats_in[(b * N + lane) * 2];
+      sh.zq[lane][1] = p.argmax ? 0.0f : p.q_stats_in[(b * N + lane) * 2 + 1];
     }
   }
-  // ---- 1. Validity; R-mode sequences have nothing for parts >= N.
-  float lx = 0.0f, lqx = 0.0f;
-  if (warp == 0) {
-    bool ok = (n == 1 || n == N) && L >= 0;
-    if (ok && lane < n) ok = tok >= 0 && tok < p.V;
-    if (ok && lane >= 1 && lane < n) ok = qr >= 0 && qr < K;
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok && lane >= 1 && lane < n) {
-      lx = to_f(p.lc[((size_t)b * K + lane - 1) * p.V + tok]);
-      if (!p.argmax) lqx = to_f(p.lp[((size_t)b * K + qr) * p.V + tok]);
-    }
-    if (lane == 0) {
-      sh.ok = ok;
-      sh.n = n;          // for the other warps
-    }
+  if (threadIdx.x < p.RU) {
+    sh.m[threadIdx.x] = __ldcg(&p.rm[(size_t)b * p.RU + threadIdx.x]);
+    sh.s[threadIdx.x] = __ldcg(&p.rs[(size_t)b * p.RU + threadIdx.x]);
+  }
+  if (threadIdx.x == 32) {
+    const int4 d = __ldcg(reinterpret_cast<const int4*>(p.dec + 4 * b));
+    sh.ok = d.x & 1;
+    sh.rejected = (d.x >> 1) & 1;
+    sh.a = d.y;
+    sh.n = d.z;
+    sh.L = d.w;
   }
   __syncthreads();
-  n = sh.n;
-  if (!sh.ok) {
-    // Malformed state: reported once, passed through, nothing committed.
-    if (y == 0 && warp == 0) {
-      if (lane == 0) {
-        report(p.status, ISD_ERR_BAD_STATE);
-        p.n_commit[b] = 0;
-        p.n_out[b] = n;
-      }
-      if (lane < N) {
-        const int i = b * N + lane;
-        p.commit_tokens[i] = -1;
-        p.pending_out[i] = p.pending_in[i];
-        p.q_row_out[i] = p.q_row_in[i];
-        p.q_stats_out[2 * i] = p.q_stats_in[2 * i];
-        p.q_stats_out[2 * i + 1] = p.q_stats_in[2 * i + 1];
-      }
-    }
-    return;
-  }
+  if (!sh.ok) return;             // malformed: handled by the decide kernel
+  const int n = sh.n, L = sh.L;
   if (n == 1 && y >= N) return;   // no drafts: nothing to reject
-  // ---- 2. Ratio tests of drafts 1 .. n-1 (warp 0, lane i verifies draft
-  //         i with row i-1); l - m is exact in fp32; p, q, the ratio fp64.
-  if (warp == 0) {
-    const int rows_used = n + N - 1;
-    const bool verifies = lane >= 1 && lane < n;
-    bool acc = true;
-    double r = 0.0;
-    if (verifies) {
-      const double px = exp((double)(lx - sh.m[lane - 1])) / sh.s[lane - 1];
-      double qx = 1.0;      // argmax drafts: the proposal is a point mass
-      if (!p.argmax) qx = exp(((double)lqx - (double)zhi) - (double)zlo);
-      r = qx > 0.0 ? px / qx : INFINITY;
-      const float u = uniform(p.seed, (uint32_t)b, step_of(p),
-                              (uint32_t)(L + lane), ISD_STREAM_ACCEPT);
-      acc = (double)u < r;
-    }
-    const uint32_t mask = __ballot_sync(0xffffffffu, acc);
-    const uint32_t drafts = ((n >= 32) ? 0xffffffffu : ((1u << n) - 1u)) & ~1u;
-    const uint32_t rej = drafts & ~mask;
-    const bool rejected = rej != 0u;
-    const int a = rejected ? (__ffs(rej) - 2) : (n - 1);
-    if (lane == 0) {
-      sh.rejected = rejected;
-      sh.a = a;
-    }
-    if (y == 0) {
-      // The decision's outputs.
-      if (verifies && p.ratio_out) p.ratio_out[b * N + lane] = (float)r;
-      if (lane < N) {
-        p.commit_tokens[b * N + lane] = lane <= a ? tok : -1;
-        // Next drafts' q rows and the log-normaliser log sum_v exp(l_v) of
-        // each (lane j: row n + j - 1), stored as a float pair hi + lo.
-        const bool has = !rejected && lane >= 1;
-        const int src = n + lane - 1;
-        p.q_row_out[b * N + lane] = has ? src : -1;
-        const double lz = has ? (double)sh.m[src] + log(sh.s[src]) : 0.0;
-        const float lz_hi = (float)lz;
-        p.q_stats_out[(b * N + lane) * 2] = lz_hi;
-        p.q_stats_out[(b * N + lane) * 2 + 1] = (float)(lz - (double)lz_hi);
-        // After a rejection only the replacement is pending.
-        if (rejected && lane >= 1) p.pending_out[b * N + lane] = -1;
-      }
-      if (p.row_stats_out && lane < rows_used) {
-        p.row_stats_out[(b * K + lane) * 2] = sh.m[lane];
-        p.row_stats_out[(b * K + lane) * 2 + 1] = (float)sh.s[lane];
-      }
-      if (lane == 0) {
-        p.n_commit[b] = a + 1;
-        p.n_out[b] = rejected ? 1 : N;
-      }
-    }
-  }
-  __syncthreads();
   const bool rejected = sh.rejected;
   const int a = sh.a;
   if (rejected) {
-    // ---- 3a. Residual sub-chunk sums: part y takes sub-chunks
+    // ---- 2a. Residual sub-chunk sums: part y takes sub-chunks
     //          kResidPerCta y .. + kResidPerCta - 1, kResidWarps warps each,
     //          in fixed order.
     const int nparts = (p.C + kResidPerCta - 1) / kResidPerCta;
     if (y >= nparts) return;
     const T* prow;
     const T* qrow;
-    const ResidRows rr = resid_rows(p, b, a, sh.m[a], sh.s[a], prow, qrow);
+    const ResidRows rr =
+        resid_rows(p, b, a, sh.m[a], sh.s[a], sh.tok[a + 1], sh.qr[a + 1],
+                   sh.zq[a + 1][0], sh.zq[a + 1][1], prow, qrow);
     const int c = y * kResidPerCta + warp / kResidWarps;
     const int part = warp % kResidWarps;
     double s = 0.0;
@@ -978,18 +1000,16 @@ __global__ void __launch_bounds__(kDrawWarps * 32)
     __threadfence();
     const float u = uniform(p.seed, (uint32_t)b, step_of(p),
                             (uint32_t)(L + a + 1), ISD_STREAM_RESAMPLE);
-    const int t = cta_draw<T, kVec>(p, sh, b, 0, a, sh.m[a], nullptr, rr,
-                                    prow, qrow, u);
+    const int t = cta_draw<T, kVec>(p, sh, b, 0, a, sh.m[a], rr, prow, qrow, u);
     if (sh.found < 0 ? threadIdx.x == 0 : (warp == sh.found && lane == 0))
       p.pending_out[b * N] = t;
     return;
   }
-  // ---- 3b. All drafts accepted: part y draws token y (0: the bonus from p
+  // ---- 2b. All drafts accepted: part y draws token y (0: the bonus from p
   //          of row n-1; y >= 1: the draft at L + n + y from q of row
   //          n + y - 1).
   if (y >= N) return;
   const int row = n + y - 1;
-  const double* mass = sh.mass[n == 1 ? 0 : 1];
   if (p.argmax && y >= 1) {
     // Argmax draft: the first sub-chunk whose max is the row max holds the
     // first maximal index (exact compares of the same values).
@@ -1011,8 +1031,8 @@ __global__ void __launch_bounds__(kDrawWarps * 32)
                           y == 0 ? ISD_STREAM_RESAMPLE : ISD_STREAM_DRAFT);
   const ResidRows none{};
   const T* prow = p.lc + ((size_t)b * K + row) * p.V;
-  const int t = cta_draw<T, kVec>(p, sh, b, 1, row, sh.m[row], mass, none,
-                                  prow, prow, u);
+  const int t = cta_draw<T, kVec>(p, sh, b, 1, row, sh.m[row], none, prow,
+                                  prow, u);
   if (sh.found < 0 ? threadIdx.x == 0 : (warp == sh.found && lane == 0))
     p.pending_out[b * N + y] = t;
 }
@@ -1020,8 +1040,10 @@ __global__ void __launch_bounds__(kDrawWarps * 32)
 // ---------------------------------------------------------------------------
 // Host-side launcher (called from the C ABI after validation).
 
+int launch_commit(const isd_commit_args* a, cudaStream_t st, bool trigger);
+
 struct AcceptLayout {
-  size_t csum, cmax, cidx, resid, count, total;
+  size_t csum, cmax, cidx, resid, count, dec, rm, rs, total;
 };
 
 static AcceptLayout accept_layout(int B, int N, int K, int V) {
@@ -1040,6 +1062,9 @@ static AcceptLayout accept_layout(int B, int N, int K, int V) {
   l.cidx = take((size_t)B * RU * C * 4);
   l.resid = take((size_t)B * C * 8);
   l.count = take((size_t)B * 4);
+  l.dec = take((size_t)B * 16);
+  l.rm = take((size_t)B * RU * 4);
+  l.rs = take((size_t)B * RU * 8);
   l.total = off;
   return l;
 }
@@ -1112,25 +1137,34 @@ int launch_stats<__nv_bfloat16, true>(const AcceptDev<__nv_bfloat16>& p,
 
 template <typename T, bool kVec>
 static int launch_accept_kernels(const AcceptDev<T>& p, int sms,
-                                 cudaStream_t st, bool have_stats) {
-  if (have_stats) {
-    // The sub-chunk figures come from the LM head; only the residual
-    // counters the statistics kernel would have zeroed need clearing.
-    if (cudaMemsetAsync(p.count, 0, (size_t)p.B * 4, st) != cudaSuccess)
-      return ISD_ERR_CUDA;
-  } else {
+                                 cudaStream_t st, bool have_stats,
+                                 const isd_commit_args* commit) {
+  // With the sub-chunk figures from the LM head there is no statistics
+  // kernel.
+  if (!have_stats) {
     const int rc = launch_stats<T, kVec>(p, sms, st);
     if (rc != ISD_OK) return rc;
   }
+  if (launch_pdl(accept_decide_kernel<T>, dim3(p.B), dim3(kDrawWarps * 32), 0,
+                 st, p) != cudaSuccess)
+    return ISD_ERR_CUDA;
+  AcceptDev<T> q = p;
+  if (commit) {
+    // The commit of this step's decisions, then the draws beside it.
+    const int rc = launch_commit(commit, st, true);
+    if (rc != ISD_OK) return rc;
+    q.draw_nowait = 1;
+  }
   const int parts = std::max((p.C + kResidPerCta - 1) / kResidPerCta, p.N);
   if (launch_pdl(accept_draw_kernel<T, kVec>, dim3(p.B, parts),
-                 dim3(kDrawWarps * 32), 0, st, p) != cudaSuccess)
+                 dim3(kDrawWarps * 32), 0, st, q) != cudaSuccess)
     return ISD_ERR_CUDA;
   return ISD_OK;
 }
 
 template <typename T>
-static int launch_accept_t(const isd_accept_args* a, cudaStream_t st) {
+static int launch_accept_t(const isd_accept_args* a, cudaStream_t st,
+                           const isd_commit_args* commit) {
   AcceptDev<T> p;
   p.B = a->B; p.N = a->N; p.K = a->K; p.V = a->V;
   p.C = (a->V + kSub - 1) / kSub;
@@ -1152,6 +1186,9 @@ static int launch_accept_t(const isd_accept_args* a, cudaStream_t st) {
   p.cidx = reinterpret_cast<int32_t*>(ws + l.cidx);
   p.resid = reinterpret_cast<double*>(ws + l.resid);
   p.count = reinterpret_cast<int32_t*>(ws + l.count);
+  p.dec = reinterpret_cast<int32_t*>(ws + l.dec);
+  p.rm = reinterpret_cast<float*>(ws + l.rm);
+  p.rs = reinterpret_cast<double*>(ws + l.rs);
   p.SR = p.RU;
   const bool have_stats = a->vocab_stats != nullptr;
   if (have_stats) {
@@ -1166,22 +1203,27 @@ static int launch_accept_t(const isd_accept_args* a, cudaStream_t st) {
     p.SR = a->K;
   }
   p.argmax = a->proposal == ISD_PROPOSAL_ARGMAX;
+  p.draw_nowait = 0;
   const int sms = num_sms();
   if (sms <= 0) return ISD_ERR_CUDA;
   // Vector loads need 16-byte aligned rows (logits_cur itself is checked
   // on the host) of whole 16-byte units.
   if (((size_t)a->V * sizeof(T)) % 16 == 0)
-    return launch_accept_kernels<T, true>(p, sms, st, have_stats);
-  return launch_accept_kernels<T, false>(p, sms, st, have_stats);
+    return launch_accept_kernels<T, true>(p, sms, st, have_stats, commit);
+  return launch_accept_kernels<T, false>(p, sms, st, have_stats, commit);
 }
 
 size_t accept_workspace_bytes(int B, int N, int K, int V) {
   return accept_layout(B, N, K, V).total;
 }
 
-int launch_accept(const isd_accept_args* a, cudaStream_t st) {
-  if (a->dtype == ISD_BF16) return launch_accept_t<__nv_bfloat16>(a, st);
-  return launch_accept_t<float>(a, st);
+// `commit`: null, or the KV commit of this step's decisions, launched
+// between the decide and draw kernels (isd_accept_commit).
+int launch_accept(const isd_accept_args* a, cudaStream_t st,
+                  const isd_commit_args* commit) {
+  if (a->dtype == ISD_BF16)
+    return launch_accept_t<__nv_bfloat16>(a, st, commit);
+  return launch_accept_t<float>(a, st, commit);
 }
 
 }  // namespace isd

@@ -38,6 +38,7 @@ struct CommitDev {
   int32_t* free_top;
   int32_t* status;
   unsigned int* done;   // workspace: CTAs finished; back to 0 after a call
+  int trigger;          // let the next grid launch once this one has waited
 };
 
 constexpr int kCommitThreads = 256;
@@ -65,6 +66,7 @@ __global__ void __launch_bounds__(kCommitThreads) commit_kernel(CommitDev p) {
   const int c = blockIdx.x, G = gridDim.x, tid = threadIdx.x;
   if (tid == 0) s_rank = kRankNone;
   grid_dep_wait();
+  if (p.trigger) grid_dep_trigger();
   __syncthreads();
   // The free-stack top and the first entries below it are read while the
   // page demand is being scanned (they do not depend on it).
@@ -196,7 +198,7 @@ size_t commit_workspace_bytes(int) { return 256; }
 
 int commit_max_batch() { return kCommitMaxCtas * kCommitMaxPer; }
 
-int launch_commit(const isd_commit_args* a, cudaStream_t st) {
+int launch_commit(const isd_commit_args* a, cudaStream_t st, bool trigger) {
   CommitDev p;
   p.B = a->B; p.K = a->K; p.Hkv = a->Hkv; p.d = a->d;
   p.P = a->num_pages; p.stride = a->page_table_stride;
@@ -211,6 +213,7 @@ int launch_commit(const isd_commit_args* a, cudaStream_t st) {
   p.n_commit = a->n_commit; p.free_stack = a->free_stack;
   p.free_top = a->free_top; p.status = a->status;
   p.done = static_cast<unsigned int*>(a->workspace);
+  p.trigger = trigger ? 1 : 0;
   const int G = (a->B + p.per - 1) / p.per;
   return launch_pdl(commit_kernel, dim3(G), dim3(kCommitThreads), 0, st, p) ==
                  cudaSuccess

@@ -73,6 +73,16 @@ static __device__ __noinline__ void report(int32_t* status, int code) {
 
 ISD_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// The one early trigger: the commit inside isd_accept_commit triggers right
+// after its wait, and the draw kernel launched behind it does not wait at
+// all, so the draws run beside the commit.  Safe because the trigger comes
+// after the commit's own wait (everything ahead of the commit, the decide
+// kernel included, has finished when the draw grid launches) and the two
+// touch disjoint memory.
+ISD_DEV void grid_dep_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Launches `kern` on `st` with programmatic stream serialisation.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block,

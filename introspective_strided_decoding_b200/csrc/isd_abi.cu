@@ -7,10 +7,11 @@
 
 namespace isd {
 size_t accept_workspace_bytes(int B, int N, int K, int V);
-int launch_accept(const isd_accept_args* a, cudaStream_t st);
+int launch_accept(const isd_accept_args* a, cudaStream_t st,
+                  const isd_commit_args* c);
 size_t commit_workspace_bytes(int B);
 int commit_max_batch();
-int launch_commit(const isd_commit_args* a, cudaStream_t st);
+int launch_commit(const isd_commit_args* a, cudaStream_t st, bool trigger);
 size_t attn_workspace_bytes_impl(int B, int M, int D, int G);
 size_t attn_tc_smem_bytes(int B, int M);
 int launch_attn_bf16(const isd_attn_args* a, int G, cudaStream_t st);
@@ -181,7 +182,7 @@ int isd_accept_resample(const isd_accept_args* a, void* stream) {
   const size_t need = isd::accept_workspace_bytes(a->B, a->N, a->K, a->V);
   if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace))
     return ISD_ERR_WORKSPACE;
-  return isd::launch_accept(a, static_cast<cudaStream_t>(stream));
+  return isd::launch_accept(a, static_cast<cudaStream_t>(stream), nullptr);
 }
 
 // ---------------------------------------------------------------- commit
@@ -202,7 +203,7 @@ size_t isd_commit_workspace_bytes(const isd_commit_args* a) {
   return isd::commit_workspace_bytes(a->B);
 }
 
-int isd_kv_commit(const isd_commit_args* a, void* stream) {
+static int commit_validate(const isd_commit_args* a) {
   const int rc = commit_check(a);
   if (rc != ISD_OK) return rc;
   if (!a->k_new || !a->v_new || !a->k_cache || !a->v_cache || !a->page_table ||
@@ -215,7 +216,30 @@ int isd_kv_commit(const isd_commit_args* a, void* stream) {
   const size_t need = isd::commit_workspace_bytes(a->B);
   if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace))
     return ISD_ERR_WORKSPACE;
-  return isd::launch_commit(a, static_cast<cudaStream_t>(stream));
+  return ISD_OK;
+}
+
+int isd_kv_commit(const isd_commit_args* a, void* stream) {
+  const int rc = commit_validate(a);
+  if (rc != ISD_OK) return rc;
+  return isd::launch_commit(a, static_cast<cudaStream_t>(stream), false);
+}
+
+// ------------------------------------------------------ accept + commit
+int isd_accept_commit(const isd_accept_args* a, const isd_commit_args* c,
+                      void* stream) {
+  int rc = isd::accept_validate(a);
+  if (rc != ISD_OK) return rc;
+  const size_t need = isd::accept_workspace_bytes(a->B, a->N, a->K, a->V);
+  if (!a->workspace || a->workspace_bytes < need || !aligned16(a->workspace))
+    return ISD_ERR_WORKSPACE;
+  rc = commit_validate(c);
+  if (rc != ISD_OK) return rc;
+  // The commit consumes this step's decisions on the same sequences.
+  if (c->B != a->B || c->K != a->K || c->n_commit != a->n_commit ||
+      c->seq_len != a->seq_len)
+    return ISD_ERR_INVALID_ARG;
+  return isd::launch_accept(a, static_cast<cudaStream_t>(stream), c);
 }
 
 // --------------------------------------------------------------- LM head

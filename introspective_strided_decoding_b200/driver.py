@@ -155,13 +155,26 @@ class Decoder:
         if rc != isd.OK:
             raise isd.IsdError(rc, "isd_kv_commit")
 
+    def accept_commit(self, stream=None):
+        """The accept step and the commit in one call (isd_accept_commit):
+        the commit runs beside the draws."""
+        a = self._acc[self.cur]
+        a.step = self.step_idx & 0xFFFFFFFF  # unused once step_dev is set
+        rc = self._lib.isd_accept_commit(ctypes.byref(a),
+                                         ctypes.byref(self._com),
+                                         isd._stream(stream))
+        if rc != isd.OK:
+            raise isd.IsdError(rc, "isd_accept_commit")
+
     def advance(self):
         self.cur ^= 1
         self.step_idx += 1
 
     def step(self, stream=None, events=None):
-        """Attention, (the LM head,) accept/resample and commit; ``events``
-        (CUDA events) are recorded around the calls when given: before
+        """Attention, (the LM head,) accept/resample and commit.  Without
+        ``events`` the last two are one isd_accept_commit call; with
+        ``events`` (CUDA events, for a per-phase split) they are separate
+        calls and the events are recorded around the calls: before
         attention, before the LM head or accept, (with 5 events: before
         accept,) before the commit, after it."""
         s = stream if stream is not None else torch.cuda.current_stream()
@@ -174,12 +187,13 @@ class Decoder:
             self.lm_head(s)
             if events and len(events) == 5:
                 events[2].record(s)
-        self.accept(s)
         if events:
+            self.accept(s)
             events[-2].record(s)
-        self.commit(s)
-        if events:
+            self.commit(s)
             events[-1].record(s)
+        else:
+            self.accept_commit(s)
         if getattr(self, "step_dev", None) is not None:
             # Once graphs are captured the accept call reads the step index
             # from the device counter; eager steps advance it too.
@@ -217,8 +231,7 @@ class Decoder:
                 self.attention()
                 if self.lm is not None:
                     self.lm_head()
-                self.accept()
-                self.commit()
+                self.accept_commit()
                 self.step_dev.add_(1)
             self.graphs.append(g)
         self.cur = cur0
@@ -293,12 +306,10 @@ class Decoder:
                          "isd_attn_strided"),
                         (lib.isd_lm_head(ctypes.byref(lm[i]), isd._stream(cs))
                          if lm else isd.OK, "isd_lm_head"),
-                        (lib.isd_accept_resample(ctypes.byref(acc[i]),
-                                                 isd._stream(cs)),
-                         "isd_accept_resample"),
-                        (lib.isd_kv_commit(ctypes.byref(com[i]),
-                                           isd._stream(cs)),
-                         "isd_kv_commit")):
+                        (lib.isd_accept_commit(ctypes.byref(acc[i]),
+                                               ctypes.byref(com[i]),
+                                               isd._stream(cs)),
+                         "isd_accept_commit")):
                     if rc != isd.OK:
                         raise isd.IsdError(rc, what)
                 self.step_dev.add_(1)
@@ -330,10 +341,9 @@ class Decoder:
         """This library's kernel launches per step: attention (bf16: the
         tcgen05 kernel and the split-segment combine; fp32: one kernel),
         the LM head's kernels when it is part of the step (as the library
-        counts them), the accept kernels (statistics, then decision and
-        draws; with an LM head only the second, the statistics coming from
-        the LM head) and the commit."""
+        counts them), the accept kernels (statistics, decide, draw; with an
+        LM head the statistics come from it) and the commit."""
         attn = 2 if self.w.dtype == "bf16" else 1
         if self.lm is None:
-            return attn + 2 + 1
-        return attn + isd.lm_head_launches(self._lm[0]) + 1 + 1
+            return attn + 3 + 1
+        return attn + isd.lm_head_launches(self._lm[0]) + 2 + 1

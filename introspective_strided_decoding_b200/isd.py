@@ -96,6 +96,8 @@ SIGNATURES = {
     "isd_commit_workspace_bytes": (ctypes.c_size_t,
                                    [ctypes.POINTER(CommitArgs)]),
     "isd_kv_commit": (ctypes.c_int, [ctypes.POINTER(CommitArgs), _VP]),
+    "isd_accept_commit": (ctypes.c_int, [ctypes.POINTER(AcceptArgs),
+                                         ctypes.POINTER(CommitArgs), _VP]),
     "isd_lm_head_workspace_bytes": (ctypes.c_size_t,
                                     [ctypes.POINTER(LmHeadArgs)]),
     "isd_vocab_stats_bytes": (ctypes.c_size_t, [_I32, _I32]),
@@ -388,6 +390,15 @@ def kv_commit(k_new, v_new, k_cache, v_cache, page_table, seq_len, n_commit,
         a.workspace_bytes = workspace.numel()
     _raise(lib().isd_kv_commit(ctypes.byref(a), _stream(stream)),
            "isd_kv_commit")
+
+
+def accept_commit(acc_args, com_args, stream=None):
+    """isd_accept_commit on prepared argument structs (from accept_args and
+    commit_args, each with its workspace set): the accept step, then the
+    commit of its decisions with the draws running beside it."""
+    _raise(lib().isd_accept_commit(ctypes.byref(acc_args),
+                                   ctypes.byref(com_args), _stream(stream)),
+           "isd_accept_commit")
 
 
 # ----------------------------------------------------------------- LM head

@@ -238,3 +238,56 @@ def test_lm_head_launch_count(lib):
     a.lora_rank, a.lora_a, a.lora_b, a.n_pending = 128, _FAKE, _FAKE, _FAKE
     assert lib.isd_lm_head_launches(ctypes.byref(a)) == 4
     assert lib.isd_lm_head_launches(ctypes.byref(_lm_args(M=0))) == 0
+
+
+def _fake_pair():
+    """Accept and commit arguments for the fused call, each consistent on
+    its own (fake aligned pointers, workspaces large enough) and describing
+    the same sequences; nothing here is ever launched."""
+    ws = ctypes.c_void_p(0x8000000)
+    a = _fake_accept_args(B=4, N=4, K=8, V=1024, dtype=isd.BF16, workspace=ws,
+                          workspace_bytes=1 << 24)
+    ptr = iter(range(0x4000000, 0x4000000 + 0x10000 * 16, 0x10000))
+    f = {k: ctypes.c_void_p(next(ptr)) for k in (
+        "k_new", "v_new", "k_cache", "v_cache", "page_table", "free_stack",
+        "free_top", "status", "workspace")}
+    c = isd.CommitArgs(B=4, K=8, Hkv=8, d=128, num_pages=64,
+                       page_table_stride=8, dtype=isd.BF16,
+                       seq_len=a.seq_len, n_commit=a.n_commit,
+                       workspace_bytes=256, **f)
+    return a, c
+
+
+def test_accept_commit_host_validation(lib):
+    """The fused call applies both calls' checks and refuses a commit that
+    does not consume this accept step's decisions."""
+    def call(a, c):
+        return lib.isd_accept_commit(ctypes.byref(a), ctypes.byref(c), None)
+
+    a, c = _fake_pair()
+    c.n_commit = ctypes.c_void_p(0x7000000)        # another n_commit
+    assert call(a, c) == isd.ERR_INVALID_ARG
+    a, c = _fake_pair()
+    c.seq_len = ctypes.c_void_p(0x7000000)         # another seq_len
+    assert call(a, c) == isd.ERR_INVALID_ARG
+    a, c = _fake_pair()
+    c.B = 3
+    assert call(a, c) == isd.ERR_INVALID_ARG
+    a, c = _fake_pair()
+    c.K = 16
+    assert call(a, c) == isd.ERR_INVALID_ARG
+    # Each half's own errors, with the codes of the separate calls.
+    a, c = _fake_pair()
+    a.logits_cur = None
+    assert call(a, c) == lib.isd_accept_resample(ctypes.byref(a), None) == \
+        isd.ERR_INVALID_ARG
+    a, c = _fake_pair()
+    a.workspace = None
+    assert call(a, c) == isd.ERR_WORKSPACE
+    a, c = _fake_pair()
+    c.workspace = None
+    assert call(a, c) == lib.isd_kv_commit(ctypes.byref(c), None) == \
+        isd.ERR_WORKSPACE
+    a, c = _fake_pair()
+    c.d = 4                                          # 8-byte rows
+    assert call(a, c) == isd.ERR_UNSUPPORTED
