@@ -419,6 +419,7 @@ __global__ void __launch_bounds__(threads_of(NCH), 1)
   // has been handed to the MMA warp, so the pipeline never waits on it.
   constexpr int NOB = NCH <= 2 ? 2 : 1;
   constexpr bool kDefer = NOB == 2;
+  constexpr bool kLazyP = NCH >= 2;        // see the softmax loop
   constexpr int QB = 2 * QH;               // one Q tile
   // TMEM columns: O^T buffers, two S^T buffers, the row-sum buffers.
   constexpr uint32_t kO = 0, kS = NOB * N, kL = NOB * N + 2 * N;
@@ -820,8 +821,20 @@ __global__ void __launch_bounds__(threads_of(NCH), 1)
       wait_or_fail(&s_full[sbuf], (i >> 1) & 1, failed);
       tc_fence_after();
       const int pbi = i % NPB;
-      wait_or_fail(&p_empty[pbi], ((i / NPB) & 1) ^ 1, failed);
-      if (stage_buf == pbi) stage_sync();   // a TMA store still reads it
+      // The P tile is free once the P V that read it last has completed
+      // (and a TMA store staged in it has read it).  From two chunks up
+      // (kLazyP) this is waited for only just before the first P store, so
+      // that the first chunk's S load and exponentials overlap that P V;
+      // every softmax thread reaches the wait at the same point (its first
+      // chunk), as stage_sync's barrier requires.  With one chunk the S
+      // buffer is released right after its load instead (measured: the
+      // later release costs 4% at B = 1, where the block loop is a latency
+      // chain, while at 64 rows the overlap gains 6%).
+      auto ensure_p = [&]() {
+        wait_or_fail(&p_empty[pbi], ((i / NPB) & 1) ^ 1, failed);
+        if (stage_buf == pbi) stage_sync();   // a TMA store still reads it
+      };
+      if constexpr (!kLazyP) ensure_p();
       bool o_ready = false;
       uint8_t* pt = ps + pbi * PB;
       uint8_t* prow = pt + kl * 64;               // this key's row of P
@@ -829,17 +842,22 @@ __global__ void __launch_bounds__(threads_of(NCH), 1)
 #pragma unroll 1
       for (int ch = ch_lo; ch < ch_hi; ++ch) {
         float s[32];
-        tmem_ld32(tmem + lane_base + kS + sbuf * N + ch * 32, s);
-        if (ch == ch_hi - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s_free[sbuf]);
-        }
-        if (col_min != 0) {
+        auto load_s = [&]() {
+          tmem_ld32(tmem + lane_base + kS + sbuf * N + ch * 32, s);
+          if (col_min != 0) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            s[e] = (ch * 32 + e >= col_min) ? s[e] : -INFINITY;
-        }
+            for (int e = 0; e < 32; ++e)
+              s[e] = (ch * 32 + e >= col_min) ? s[e] : -INFINITY;
+          }
+        };
+        auto free_s = [&]() {    // the block's S has been read (last chunk)
+          if (ch == ch_hi - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[sbuf]);
+          }
+        };
+        load_s();
         // P = 2^(s c - m c) against the current references (masked scores
         // give 0), written as this key's 32 values of the chunk and added
         // to its row sums.  Returns the largest exponent s c - m c.
@@ -876,16 +894,9 @@ __global__ void __launch_bounds__(threads_of(NCH), 1)
             tmem_ld32(tmem + lane_base + l_col + ch * 32, l);
           }
         };
-        // Optimistic pass; the vote asks whether any exponent exceeded 8
-        // (then the references move and the pass is redone).  The first
-        // block of a segment has no references yet.
-        bool need = first;
-        if (!first) {
-          load_l();
-          need = p_pass() > kRescaleLog2;
-        }
-        if (sm_any(gi, need)) {
-          // Exact block max per row, then move the references.
+        // Exact block max per row, then move the references (and rescale
+        // O^T and the row sums).
+        auto move_refs = [&]() {
           float v[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = s[e];
@@ -921,6 +932,72 @@ __global__ void __launch_bounds__(threads_of(NCH), 1)
             tmem_scale32(tmem + lane_base + o_col + ch * 32, rv);
             tmem_scale32(tmem + lane_base + l_col + ch * 32, rv);
           }
+        };
+        if constexpr (!kLazyP) {
+          // Optimistic pass; the vote asks whether any exponent exceeded 8
+          // (then the references move and the pass is redone).  The first
+          // block of a segment has no references yet.
+          free_s();
+          bool need = first;
+          if (!first) {
+            load_l();
+            need = p_pass() > kRescaleLog2;
+          }
+          if (sm_any(gi, need)) {
+            move_refs();
+            load_l();
+            p_pass();
+          }
+          tmem_st32(tmem + lane_base + l_col + ch * 32, l);
+          continue;
+        }
+        // Optimistic pass against the current references, its exponentials
+        // computed in place of the scores (phase A); the vote asks whether
+        // any exponent exceeded 8 (then the references move, the scores are
+        // read again and the pass is redone).  The first block of a segment
+        // has no references yet.
+        bool need = first;
+        if (!first) {
+          load_l();
+          float xmax = -INFINITY;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float4 ma = *reinterpret_cast<const float4*>(&m_sc[ch * 32 + q * 8]);
+            const float4 mb = *reinterpret_cast<const float4*>(&m_sc[ch * 32 + q * 8 + 4]);
+            const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const float x = fmaf(s[q * 8 + u], c2, -mm[u]);
+              xmax = fmaxf(xmax, x);
+              s[q * 8 + u] = ex2(x);
+            }
+          }
+          need = xmax > kRescaleLog2;
+        }
+        need = sm_any(gi, need);
+        if (ch == ch_lo) ensure_p();
+        if (!(need && !first)) free_s();
+        if (!need) {
+          // Phase B: the row sums and the bf16 P of the chunk.
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int e = q * 8 + 2 * u;
+              l[e] += s[e];
+              l[e + 1] += s[e + 1];
+              pk[u] = pack_bf16(s[e], s[e + 1]);
+            }
+            *reinterpret_cast<uint4*>(prow + ch * PA + ((q ^ psw) << 4)) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        } else {
+          if (!first) {
+            load_s();    // phase A replaced the scores
+            free_s();
+          }
+          move_refs();
           load_l();
           p_pass();
         }
