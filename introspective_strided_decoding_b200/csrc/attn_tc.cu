@@ -36,21 +36,24 @@
 //                       buffered S in TMEM and commits completion.  It
 //                       also allocates and frees TMEM.
 //   P V MMA warp        one thread issues O^T += V^T P^T of block i once
-//                       its P is written.  Two issuing warps: one thread
-//                       issuing both kinds in order made each P V wait for
-//                       the next K tile and capped the issue rate (measured:
-//                       the two-warp split is 10% faster on the C=64 step).
+//                       its P is written (from 96 rows up also the row
+//                       sums, a ones tile times the same P^T).  Two issuing
+//                       warps: one thread issuing both kinds in order made
+//                       each P V wait for the next K tile and capped the
+//                       issue rate (measured: the two-warp split is 10%
+//                       faster on the C=64 step).
 //   softmax (4 warps)   thread t owns key t of the block (TMEM lane t): it
 //                       masks its scores, writes P = 2^(s c - m_row c) in
-//                       bf16 into P^T, and adds P to its per-row partial
-//                       sums (TMEM).  The reference max m_row moves only
-//                       when some score of the block exceeds it by more
-//                       than 2^8 (a vote over the 128 threads); then the
-//                       exact block max is reduced across the threads and
-//                       O^T and the sums are rescaled.  At a segment's end
-//                       the sums are reduced over the keys and O^T / l is
-//                       stored (or a partial for the combine kernel when
-//                       the (b, h) straddles CTAs).
+//                       bf16 into P^T, and (up to 64 rows) adds P to its
+//                       per-row partial sums (TMEM).  The reference max
+//                       m_row moves only when some score of the block
+//                       exceeds it by more than 2^8 (a vote over the 128
+//                       threads); then the exact block max is reduced
+//                       across the threads and O^T and the sums are
+//                       rescaled.  At a segment's end the sums (reduced
+//                       over the keys, or read from the ones product) give
+//                       O^T / l, stored (or a partial for the combine
+//                       kernel when the (b, h) straddles CTAs).
 //
 // Every mbarrier wait is bounded; after one timeout a thread records
 // ISD_ERR_CUDA (unless an earlier error is already recorded) and stops
