@@ -95,9 +95,9 @@ def parse():
 # profiles/attn_tc_kernel_c64_b16_full.md).  Traffic tracks the algorithmic
 # bytes, so a full launch's traffic is this ratio times its bytes.  Valid
 # only for the kernel source the capture was taken on.
-TRAFFIC_PER_ALGO_BYTE = (331.52 + 8.28) / 332.37
+TRAFFIC_PER_ALGO_BYTE = (331.50 + 8.13) / 332.37
 TRAFFIC_KERNEL_SHA256 = (
-    "36976dbe1f402d9716de47c2f37d0c665acfab2627c5b2b2dfad463b35694446")
+    "1997e7da6e61d1637e2e96214c47b461c6763b0094e2599cac508beac74df4fb")
 
 
 def attention_traffic(bytes_per_launch):
