@@ -59,6 +59,39 @@ def test_small_cases_every_output(w, num_ctas, sharp):
     assert np.abs(f64(lse) - ref_lse).max() <= tol
 
 
+@pytest.mark.parametrize("w", [SMALL[2], SMALL[4], SMALL[9], SMALL[5]],
+                         ids=lambda w: w.name)
+@pytest.mark.parametrize("num_ctas", [0, 3])
+def test_reference_max_moves_on_later_blocks(w, num_ctas):
+    """Cached keys scaled by 1 + 4i on logical page i, with unscaled queries
+    and 3 to 5 blocks of 128 keys per sequence: each block raises the row
+    maxima by about 7 (natural-log units), more than the 2^8 (5.5) the
+    kernel tolerates against its running reference max, so on every later
+    block the reference moves, O and the row sums are rescaled and the
+    block's pass is redone (at 32, 64, 96 and 128 rows per KV head, with
+    and without split segments)."""
+    w = w.with_(L_lo=300, L_hi=600)
+    cache = synth.make_cache(w, 11, DEV)
+    pt = cache["page_table"].long().cpu()
+    L = cache["seq_len"].long().cpu()
+    kc = cache["k_cache"]
+    with torch.no_grad():
+        for b in range(w.B):
+            for i in range((int(L[b]) + 15) // 16):
+                kc[int(pt[b, i])] *= 1.0 + 4.0 * i
+    q, k, v = synth.make_stride(w, 11, 0, DEV, sharp=True)
+    out, lse = gpu_attention(w, cache, q, k, v, num_ctas=num_ctas)
+    torch.cuda.synchronize()
+    ref, ref_lse = oracle_attention(w, cache, q, k, v)
+    tol = TOL[w.dtype]
+    err = np.abs(f64(out) - ref)
+    assert err.max() <= tol, (err.max(), np.unravel_index(err.argmax(),
+                                                          err.shape))
+    # lse grows to hundreds here: the same bound, relative to its size.
+    lse_err = np.abs(f64(lse) - ref_lse) / np.maximum(1.0, np.abs(ref_lse))
+    assert lse_err.max() <= tol
+
+
 @pytest.mark.parametrize("L", [0, 1, 15, 16, 17, 32])
 def test_edge_lengths(L):
     w = _bf(name="edge", B=2, L_lo=L, L_hi=L)
