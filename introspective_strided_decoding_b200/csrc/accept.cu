@@ -42,6 +42,9 @@ constexpr int kSubPerLane = 4;             // sub-chunks a lane owns in a row sc
 constexpr int kMaxSub = 32 * kSubPerLane;  // V <= 262 144 (host check)
 constexpr int kMaxRows = 32;               // K <= 32 (host check: N <= 16)
 constexpr int kStatsWarps = 16;            // stats CTA: 512 threads
+// The register-staged statistics kernel (two sub-chunks of 8 elements a
+// lane held at once): 256 threads, so its registers are not capped at 128.
+constexpr int kRegStatsWarps = 8;
 constexpr int kDrawWarps = 8;              // draw CTA: 256 threads
 constexpr int kResidPerCta = 4;            // residual sub-chunks per draw CTA
 constexpr int kWarpElems = kSub / kDrawWarps;   // a draw warp's share: 256
@@ -350,15 +353,15 @@ struct ItemWalk {
 };
 
 template <typename T, bool kVec>
-__global__ void __launch_bounds__(kStatsWarps * 32)
+__global__ void __launch_bounds__(kRegStatsWarps * 32)
     accept_stats_kernel(AcceptDev<T> p) {
   grid_dep_wait();
   auto used = [&](int b) {
     return state_ok(p, b) ? p.n_in[b] + p.N - 1 : 0;
   };
   ItemWalk w;
-  w.init(blockIdx.x * kStatsWarps + (threadIdx.x >> 5),
-         (long long)gridDim.x * kStatsWarps, p.B, p.C, p.RU);
+  w.init(blockIdx.x * kRegStatsWarps + (threadIdx.x >> 5),
+         (long long)gridDim.x * kRegStatsWarps, p.B, p.C, p.RU);
   bool have = w.next_used(used);
   Raw8<T> cur[8];
   if (have) load_sub<T, kVec>(p, w.b, w.j, w.c, cur);
@@ -1078,24 +1081,30 @@ static int num_sms() {
   return n;
 }
 
+// The register-staged statistics kernel: as many 256-thread CTAs as fit
+// on every SM at once (the warps loop over the items), fewer for small
+// problems.
 template <typename T, bool kVec>
-static int launch_stats(const AcceptDev<T>& p, int sms, cudaStream_t st) {
-  // As many 512-thread CTAs as fit on every SM at once (the warps loop over
-  // the items), fewer for small problems.
+static int launch_reg_stats(const AcceptDev<T>& p, int sms, cudaStream_t st) {
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-          &per_sm, accept_stats_kernel<T, kVec>, kStatsWarps * 32, 0) !=
+          &per_sm, accept_stats_kernel<T, kVec>, kRegStatsWarps * 32, 0) !=
           cudaSuccess ||
       per_sm < 1)
     return ISD_ERR_CUDA;
   const long long items = (long long)p.B * p.RU * p.C;
-  const long long ctas = (items + kStatsWarps - 1) / kStatsWarps;
+  const long long ctas = (items + kRegStatsWarps - 1) / kRegStatsWarps;
   const int grid = (int)std::max<long long>(
       1, std::min<long long>((long long)per_sm * sms, ctas));
   return launch_pdl(accept_stats_kernel<T, kVec>, dim3(grid),
-                    dim3(kStatsWarps * 32), 0, st, p) == cudaSuccess
+                    dim3(kRegStatsWarps * 32), 0, st, p) == cudaSuccess
              ? ISD_OK
              : ISD_ERR_CUDA;
+}
+
+template <typename T, bool kVec>
+static int launch_stats(const AcceptDev<T>& p, int sms, cudaStream_t st) {
+  return launch_reg_stats<T, kVec>(p, sms, st);
 }
 
 // Aligned bf16 rows: the shared-memory pipeline, one 512-thread CTA per SM.
@@ -1105,23 +1114,7 @@ int launch_stats<__nv_bfloat16, true>(const AcceptDev<__nv_bfloat16>& p,
   // Slots, then the rows-in-use tables; too many sequences for the tables
   // take the register kernel.
   const size_t smem = stats_async_smem(p.B);
-  if (smem > 227 * 1024) {
-    const AcceptDev<__nv_bfloat16>& q = p;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &per_sm, accept_stats_kernel<__nv_bfloat16, true>,
-            kStatsWarps * 32, 0) != cudaSuccess ||
-        per_sm < 1)
-      return ISD_ERR_CUDA;
-    const long long items = (long long)q.B * q.RU * q.C;
-    const long long ctas = (items + kStatsWarps - 1) / kStatsWarps;
-    const int g = (int)std::max<long long>(
-        1, std::min<long long>((long long)per_sm * sms, ctas));
-    return launch_pdl(accept_stats_kernel<__nv_bfloat16, true>, dim3(g),
-                      dim3(kStatsWarps * 32), 0, st, q) == cudaSuccess
-               ? ISD_OK
-               : ISD_ERR_CUDA;
-  }
+  if (smem > 227 * 1024) return launch_reg_stats<__nv_bfloat16, true>(p, sms, st);
   auto kern = accept_stats_async_kernel;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
