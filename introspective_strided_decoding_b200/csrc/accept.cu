@@ -912,16 +912,14 @@ ISD_DEV int cta_draw(const AcceptDev<T>& p, DrawShared& sh, int b, int mode,
 // accepted sequences draw token y in part y (the bonus, then the drafts).
 // Parts with nothing to do leave as soon as the record is read.
 template <typename T, bool kVec>
-__global__ void __launch_bounds__(kDrawWarps * 32)
-    accept_draw_kernel(AcceptDev<T> p) {
-  __shared__ DrawShared sh;
+ISD_DEV void draw_body(const AcceptDev<T>& p, DrawShared& sh) {
   const int b = blockIdx.x, y = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = p.N, K = p.K;
-  // Behind the commit (isd_accept_commit) the draws do not wait: the
-  // commit triggered this grid after its own wait, so the decide kernel
-  // and everything before it have finished, and the two kernels touch
-  // disjoint memory.
+  // Behind the commit (isd_accept_commit) the draws do not wait before
+  // their work: the commit triggered this grid after its own wait, so the
+  // decide kernel and everything before it have finished, and the two
+  // kernels touch disjoint memory (the kernel waits at its end instead).
   if (!p.draw_nowait) grid_dep_wait();
   // ---- 0. The sequence's inputs and the decision record.
   if (warp == 0) {
@@ -1038,6 +1036,19 @@ __global__ void __launch_bounds__(kDrawWarps * 32)
                                   prow, u);
   if (sh.found < 0 ? threadIdx.x == 0 : (warp == sh.found && lane == 0))
     p.pending_out[b * N + y] = t;
+}
+
+template <typename T, bool kVec>
+__global__ void __launch_bounds__(kDrawWarps * 32)
+    accept_draw_kernel(AcceptDev<T> p) {
+  __shared__ DrawShared sh;
+  draw_body<T, kVec>(p, sh);
+  // Behind the commit one CTA waits, after its work, for the commit grid
+  // to complete: the draw grid then completes only after the commit, so a
+  // later kernel's wait on the draw grid covers the commit's writes too.
+  // One is enough (a grid is complete when its last CTA exits); every CTA
+  // waiting held the early-leaving parts' slots (measured: +5 us at C=64).
+  if (p.draw_nowait && blockIdx.x == 0 && blockIdx.y == 0) grid_dep_wait();
 }
 
 // ---------------------------------------------------------------------------

@@ -74,11 +74,12 @@ static __device__ __noinline__ void report(int32_t* status, int code) {
 ISD_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // The one early trigger: the commit inside isd_accept_commit triggers right
-// after its wait, and the draw kernel launched behind it does not wait at
-// all, so the draws run beside the commit.  Safe because the trigger comes
-// after the commit's own wait (everything ahead of the commit, the decide
-// kernel included, has finished when the draw grid launches) and the two
-// touch disjoint memory.
+// after its wait, and the draw kernel launched behind it does not wait
+// before its work, so the draws run beside the commit.  Safe because the
+// trigger comes after the commit's own wait (everything ahead of the
+// commit, the decide kernel included, has finished when the draw grid
+// launches) and the two touch disjoint memory.  One draw CTA waits at its
+// end, so the draw grid completes only after the commit.
 ISD_DEV void grid_dep_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
