@@ -26,6 +26,10 @@
 //          A draw picks the sub-chunk from a warp scan of the sub-chunk
 //          masses, then scans its 2048 elements with eight warps of 256,
 //          all in ascending vocabulary order.               [latency bound]
+// isd_accept_commit launches the KV commit between decide and draw: the
+// commit needs only the decisions, so the draws run beside it (the draw
+// kernel then starts without its grid-dependency wait and one of its CTAs
+// waits at its end; see the draw kernel).
 // Element masses are fp32 (MUFU exp2 of exactly formed differences); every
 // sum that places a sampling boundary or normalises a probability is
 // accumulated in fp64 in a fixed order, so draws agree with an fp64
@@ -189,10 +193,13 @@ ISD_DEV bool state_ok(const AcceptDev<T>& p, int b) {
 }
 
 // ---------------------------------------------------------------------------
-// Statistics.  Items are the sub-chunks of the used rows, numbered row
-// index first: it = (j * B + b) * C + c (rows j < N are used by every
-// sequence, so warps run out of work together).  Global warp w takes items
-// w, w + W, w + 2W, ... that are in use; lane l holds elements
+// Statistics, register-staged (fp32 logits, rows whose byte length is not
+// a multiple of 16, batches too large for the shared-memory kernel's
+// tables).  Items are the sub-chunks of the used rows, numbered row index
+// first: it = (j * B + b) * C + c.  Global warp w takes items w, w + W,
+// w + 2W, ... that are in use (a strided walk: the shared-memory kernel
+// below gives each warp an equal contiguous range instead, which balances
+// better when rows go unused); lane l holds elements
 // lo + (k*32 + l)*8 + e (k, e < 8) of the sub-chunk, -inf past the row end,
 // and lane 0 stores the max, the sum of exp(l - max) (8 terms in fp32, then
 // fp64) and, for argmax proposals, the first index of the max (exact
