@@ -309,9 +309,9 @@ int isd_kv_commit(const isd_commit_args* a, void* stream);
  * after the statistics and the ratio-test decisions the commit runs and the
  * residual / bonus / draft draws run beside it.  c must describe the same
  * sequences: c->B == a->B, c->K == a->K, c->n_commit == a->n_commit and
- * c->seq_len == a->seq_len (else ISD_ERR_INVALID_ARG); every other rule of
- * the two calls applies unchanged (both workspaces, both checks, checked
- * before anything is launched).
+ * c->seq_len == a->seq_len, and the two workspaces must not overlap (else
+ * ISD_ERR_INVALID_ARG); every other rule of the two calls applies unchanged
+ * (both workspaces, both checks, checked before anything is launched).
  * ---------------------------------------------------------------------- */
 int isd_accept_commit(const isd_accept_args* a, const isd_commit_args* c,
                       void* stream);

@@ -239,6 +239,11 @@ int isd_accept_commit(const isd_accept_args* a, const isd_commit_args* c,
   if (c->B != a->B || c->K != a->K || c->n_commit != a->n_commit ||
       c->seq_len != a->seq_len)
     return ISD_ERR_INVALID_ARG;
+  // The two workspaces are in use at the same time: they must not overlap.
+  const uintptr_t wa = reinterpret_cast<uintptr_t>(a->workspace);
+  const uintptr_t wc = reinterpret_cast<uintptr_t>(c->workspace);
+  const size_t need_c = isd::commit_workspace_bytes(c->B);
+  if (wa < wc + need_c && wc < wa + need) return ISD_ERR_INVALID_ARG;
   return isd::launch_accept(a, static_cast<cudaStream_t>(stream), c);
 }
 

@@ -291,3 +291,7 @@ def test_accept_commit_host_validation(lib):
     a, c = _fake_pair()
     c.d = 4                                          # 8-byte rows
     assert call(a, c) == isd.ERR_UNSUPPORTED
+    # The commit's counter inside the accept's workspace.
+    a, c = _fake_pair()
+    c.workspace = ctypes.c_void_p(a.workspace + 256)
+    assert call(a, c) == isd.ERR_INVALID_ARG
